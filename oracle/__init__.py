@@ -1,0 +1,153 @@
+"""fp64 CPU oracle for exact attention, paged gather and paged decode.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package smoke check and the
+benchmark's CPU-baseline / reference leg may import this package.  It shares
+no code with the CUDA library (attn_fwd_04_b200), and the CUDA library never
+imports it.
+
+The arithmetic lives in attn_oracle.c (plain loops, fp64); this module only
+marshals numpy arrays into it.  `method.py` beside it holds the CPU
+restatements of the method's own steps (online softmax, split merge) that
+the pin tests compare with the plain definition.
+
+Inputs are whatever values the GPU receives (bf16 upcast exactly to fp64);
+outputs are fp64.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        L.oracle_attention.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64,
+                                       ctypes.c_int, ctypes.c_double, P, I64]
+        L.oracle_attention.restype = ctypes.c_int
+        L.oracle_attention_probs.argtypes = [P, P, P, I64, I64, ctypes.c_int,
+                                             ctypes.c_double]
+        L.oracle_attention_probs.restype = ctypes.c_int
+        L.oracle_attention_varlen.argtypes = [P, P, P, P, P, P, I64, I64, I64,
+                                              ctypes.c_int, ctypes.c_double, P, I64]
+        L.oracle_attention_varlen.restype = ctypes.c_int
+        L.oracle_gather_paged.argtypes = [P, P, P, P, I64, I64, I64, I64]
+        L.oracle_gather_paged.restype = ctypes.c_int
+        L.oracle_decode_paged.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64]
+        L.oracle_decode_paged.restype = ctypes.c_int
+        L.oracle_num_threads.argtypes = []
+        L.oracle_num_threads.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def _f64(a):
+    """Any array-like (numpy or torch, any float dtype) -> C-contiguous fp64."""
+    if hasattr(a, "detach"):  # torch tensor: upcast on the CPU, exactly
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i64(a):
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def attention(q, k, v, causal: bool, scale: float, rows=None):
+    """Plain fp64 attention over q,k [B,H,N,d] and v [B,H,N,dv].
+
+    Returns (o [B,H,N,dv], lse [B,H,N]).  With `rows` (flat ids
+    (b*H + h)*N + i) only those rows are computed; the other entries of the
+    returned arrays are NaN.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, H, N, d) and v.shape == (B, H, N, dv)
+    o = np.full((B, H, N, dv), np.nan)
+    lse = np.full((B, H, N), np.nan)
+    r = _i64(rows) if rows is not None else None
+    rc = lib().oracle_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                B, H, N, d, dv, int(bool(causal)), float(scale),
+                                _ptr(r), 0 if r is None else r.size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention failed ({rc})")
+    return o, lse
+
+
+def probs(q, k, causal: bool, scale: float):
+    """The full N x N probability matrix of one head; q, k are [N, d]."""
+    q, k = _f64(q), _f64(k)
+    N, d = q.shape
+    p = np.zeros((N, N))
+    lib().oracle_attention_probs(_ptr(q), _ptr(k), _ptr(p), N, d,
+                                 int(bool(causal)), float(scale))
+    return p
+
+
+def attention_varlen(q, k, v, cu_seqlens, causal: bool, scale: float, rows=None):
+    """Plain fp64 attention over packed [total,H,d] sequences.
+
+    Returns (o [total,H,d], lse [H,total]); `rows` are flat ids h*total + g.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu = _i64(cu_seqlens)
+    total, H, d = q.shape
+    B = cu.size - 1
+    assert cu[-1] == total
+    o = np.full((total, H, d), np.nan)
+    lse = np.full((H, total), np.nan)
+    r = _i64(rows) if rows is not None else None
+    rc = lib().oracle_attention_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                       _ptr(cu), B, H, d, int(bool(causal)),
+                                       float(scale), _ptr(r), 0 if r is None else r.size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_varlen failed ({rc})")
+    return o, lse
+
+
+def gather_paged(pages, page_table, seq_lens, page_size: int):
+    """Contiguous [sum(seq_lens), H, d] rows gathered from [P,H,page_size,d] pages."""
+    pages = _f64(pages)
+    pt = _i64(page_table)
+    sl = _i64(seq_lens)
+    _, H, ps, d = pages.shape
+    assert ps == page_size
+    out = np.zeros((int(sl.sum()), H, d))
+    rc = lib().oracle_gather_paged(_ptr(pages), _ptr(pt), _ptr(sl), _ptr(out),
+                                   sl.size, H, d, page_size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_gather_paged failed ({rc})")
+    return out
+
+
+def decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int):
+    """Single-token decode; returns (o [B,H,d], lse [B,H]).  Scale is 1/sqrt(d)."""
+    q = _f64(q)
+    kp, vp = _f64(k_pages), _f64(v_pages)
+    pt, sl = _i64(page_table), _i64(seq_lens)
+    B, H, d = q.shape
+    o = np.zeros((B, H, d))
+    lse = np.zeros((B, H))
+    rc = lib().oracle_decode_paged(_ptr(q), _ptr(kp), _ptr(vp), _ptr(pt), _ptr(sl),
+                                   _ptr(o), _ptr(lse), B, H, d, page_size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_decode_paged failed ({rc})")
+    return o, lse

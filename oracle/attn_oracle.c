@@ -1,0 +1,302 @@
+/*
+ * attn_oracle.c -- plain, slow, fp64 CPU oracle for exact scaled-dot-product
+ * attention, its variable-length form, the paged-KV gather and single-token
+ * paged decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links or calls this
+ * file; only the tests, the package smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header or constant with the CUDA
+ * library.
+ *
+ * What it computes (the plain definition, no tiling, no online update):
+ *
+ *   Standard attention as described on the page "Flash Attention 是什么：
+ *   2026 最新原理、架构演进与实战详解" (ai.lansai.wang), section
+ *   "核心工作机制": scores S = Q K^T, a softmax over each row of S, then the
+ *   product with V.  The same page, section "常见误解澄清" (misconception 1),
+ *   states that the fused method reaches exactly this result up to rounding,
+ *   so this definition is what the GPU path is compared with.
+ *
+ *   For every query row i and its admissible key set A_i:
+ *     s_ij  = scale * sum_k q_ik k_jk          (j in A_i)
+ *     m_i   = max_j s_ij
+ *     l_i   = sum_j exp(s_ij - m_i)
+ *     o_i   = sum_j (exp(s_ij - m_i) / l_i) v_j
+ *     lse_i = m_i + ln l_i
+ *   A_i is every key (non-causal) or keys j <= i (causal, top-left aligned;
+ *   the causal switch is the flash_attn_causal knob on the page
+ *   "为什么“Flash”突然成了AI圈的高频词" (lqnn.cn), section 3.3).  An empty
+ *   A_i gives o_i = 0 and lse_i = -inf.
+ *
+ * Each row of S is materialised in full (a plain array of its scores) before
+ * its max, sum and output are taken; oracle_attention_probs materialises the
+ * whole N x N probability matrix of one head for the small pin tests.
+ *
+ * Paged decode follows the page "“Flash”不是那个被时代淘汰的插件"
+ * (0539edu.com), section 2: the KV cache is a pool of fixed-size pages
+ * (256 tokens by default), each page a contiguous K (or V) slice, and a
+ * sequence owns a list of pages.  The oracle first gathers a sequence's
+ * pages back into a contiguous [len, d] array per head, then applies the
+ * definition above with a single query row and no mask.
+ *
+ * Parallelism: OpenMP over independent output rows.  Each row is computed by
+ * one thread in a fixed order, so results do not depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* One output row of the definition.
+ *   q      : the query row, d values
+ *   kbase  : key row j (d values) starts at kbase + j * kstride
+ *   vbase  : value row j (dv values) starts at vbase + j * vstride
+ *   nkeys  : keys 0 .. nkeys-1 are admissible
+ *   srow   : scratch for the materialised score row, >= nkeys doubles
+ *   o      : dv outputs;  *lse : the row's log-sum-exp
+ */
+static void attention_row(const double *q, const double *kbase, int64_t kstride,
+                          const double *vbase, int64_t vstride, int64_t nkeys,
+                          int64_t d, int64_t dv, double scale, double *srow,
+                          double *o, double *lse) {
+    int64_t j, c;
+    for (c = 0; c < dv; ++c) o[c] = 0.0;
+    if (nkeys <= 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    /* pass 1: the full score row */
+    for (j = 0; j < nkeys; ++j) {
+        const double *kj = kbase + j * kstride;
+        double dot = 0.0;
+        for (c = 0; c < d; ++c) dot += q[c] * kj[c];
+        srow[j] = scale * dot;
+    }
+    /* pass 2: row max and normaliser */
+    double m = srow[0];
+    for (j = 1; j < nkeys; ++j)
+        if (srow[j] > m) m = srow[j];
+    double l = 0.0;
+    for (j = 0; j < nkeys; ++j) l += exp(srow[j] - m);
+    /* pass 3: probabilities times V */
+    for (j = 0; j < nkeys; ++j) {
+        const double p = exp(srow[j] - m) / l;
+        const double *vj = vbase + j * vstride;
+        for (c = 0; c < dv; ++c) o[c] += p * vj[c];
+    }
+    *lse = m + log(l);
+}
+
+/* Fixed-length attention.  q,k are [B,H,N,d] and v,o [B,H,N,dv], contiguous
+ * (the layout the page "为什么“Flash”突然成了AI圈的高频词", section 2.1,
+ * prints as [1, 32, 16384, 128]); lse is [B,H,N].
+ * rows: optional list of nrows flat row ids r = (b*H + h)*N + i; when rows is
+ * NULL every row is computed (nrows ignored).  Outputs for row r go to
+ * o[r*dv ...] and lse[r] in both cases. */
+int oracle_attention(const double *q, const double *k, const double *v,
+                     double *o, double *lse, int64_t B, int64_t H, int64_t N,
+                     int64_t d, int64_t dv, int causal, double scale,
+                     const int64_t *rows, int64_t nrows) {
+    if (B < 0 || H < 0 || N < 0 || d <= 0 || dv <= 0) return -1;
+    const int64_t total = rows ? nrows : B * H * N;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        if (!srow) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = 0; t < total; ++t) {
+                const int64_t r = rows ? rows[t] : t;
+                const int64_t bh = r / N, i = r % N;
+                const double *kb = k + bh * N * d;
+                const double *vb = v + bh * N * dv;
+                const int64_t nk = causal ? (i + 1) : N;
+                attention_row(q + r * d, kb, d, vb, dv, nk, d, dv, scale, srow,
+                              o + r * dv, lse + r);
+            }
+            free(srow);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/* The full probability matrix P = softmax(scale * Q K^T) of one head, with
+ * the causal mask applied (masked entries are exactly 0).  q,k are [N,d];
+ * p is [N,N].  Small inputs only (pin tests). */
+int oracle_attention_probs(const double *q, const double *k, double *p,
+                           int64_t N, int64_t d, int causal, double scale) {
+    int64_t i, j, c;
+    for (i = 0; i < N; ++i) {
+        double *prow = p + i * N;
+        const int64_t nk = causal ? i + 1 : N;
+        for (j = 0; j < N; ++j) prow[j] = 0.0;
+        if (nk == 0) continue;
+        for (j = 0; j < nk; ++j) {
+            double dot = 0.0;
+            for (c = 0; c < d; ++c) dot += q[i * d + c] * k[j * d + c];
+            prow[j] = scale * dot;
+        }
+        double m = prow[0];
+        for (j = 1; j < nk; ++j)
+            if (prow[j] > m) m = prow[j];
+        double l = 0.0;
+        for (j = 0; j < nk; ++j) l += exp(prow[j] - m);
+        for (j = 0; j < nk; ++j) prow[j] = exp(prow[j] - m) / l;
+    }
+    return 0;
+}
+
+/* Variable-length attention over sequences packed back to back.
+ * q,k,v,o are [total,H,d] (row t of sequence b is token cu_seqlens[b] + t);
+ * lse is [H,total].  Attention never crosses a sequence boundary; with
+ * causal set, token t of a sequence sees tokens 0..t of the same sequence.
+ * rows: optional list of flat ids r = h*total + g (g a packed token index);
+ * NULL computes everything. */
+int oracle_attention_varlen(const double *q, const double *k, const double *v,
+                            double *o, double *lse, const int64_t *cu_seqlens,
+                            int64_t B, int64_t H, int64_t d, int causal,
+                            double scale, const int64_t *rows, int64_t nrows) {
+    if (B < 0 || H < 0 || d <= 0) return -1;
+    const int64_t totaltok = cu_seqlens[B];
+    int64_t maxlen = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t len = cu_seqlens[b + 1] - cu_seqlens[b];
+        if (len < 0) return -1;
+        if (len > maxlen) maxlen = len;
+    }
+    const int64_t total = rows ? nrows : H * totaltok;
+    const int64_t rs = H * d; /* stride between consecutive tokens */
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+        double *orow = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!srow || !orow) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = 0; t < total; ++t) {
+                const int64_t r = rows ? rows[t] : t;
+                const int64_t h = r / totaltok, g = r % totaltok;
+                /* the sequence that owns packed token g */
+                int64_t b = 0;
+                while (b + 1 <= B && cu_seqlens[b + 1] <= g) ++b;
+                const int64_t start = cu_seqlens[b];
+                const int64_t len = cu_seqlens[b + 1] - start;
+                const int64_t i = g - start;
+                const int64_t nk = causal ? i + 1 : len;
+                double l;
+                attention_row(q + g * rs + h * d, k + start * rs + h * d, rs,
+                              v + start * rs + h * d, rs, nk, d, d, scale, srow,
+                              orow, &l);
+                for (int64_t c = 0; c < d; ++c) o[g * rs + h * d + c] = orow[c];
+                lse[h * totaltok + g] = l;
+            }
+        }
+        free(srow);
+        free(orow);
+    }
+    return failed ? -2 : 0;
+}
+
+/* Gather of a paged KV cache back into contiguous rows.
+ *   pages      : [P_pool, H, page_size, d]  (one contiguous slice per page
+ *                and head)
+ *   page_table : the pages of every sequence, packed: sequence b's pages are
+ *                entries off_b .. off_b + npages_b - 1, where npages_b is the
+ *                number of page_size-token pages its seq_lens[b] tokens
+ *                occupy and off_b is the sum of npages over earlier
+ *                sequences
+ *   out        : [sum_b seq_lens[b], H, d], sequence b starting at row
+ *                sum_{b'<b} seq_lens[b']
+ * Token t of sequence b lives in page table entry off_b + floor(t/page_size),
+ * at slot t mod page_size of that page. */
+int oracle_gather_paged(const double *pages, const int64_t *page_table,
+                        const int64_t *seq_lens, double *out, int64_t B,
+                        int64_t H, int64_t d, int64_t page_size) {
+    if (page_size <= 0 || d <= 0 || H < 0 || B < 0) return -1;
+    int64_t off = 0, row = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t len = seq_lens[b];
+        if (len < 0) return -1;
+        for (int64_t t = 0; t < len; ++t) {
+            const int64_t page = page_table[off + t / page_size];
+            const int64_t slot = t % page_size;
+            for (int64_t h = 0; h < H; ++h) {
+                const double *src = pages + ((page * H + h) * page_size + slot) * d;
+                double *dst = out + ((row + t) * H + h) * d;
+                for (int64_t c = 0; c < d; ++c) dst[c] = src[c];
+            }
+        }
+        off += (len + page_size - 1) / page_size;
+        row += len;
+    }
+    return 0;
+}
+
+/* Single-token decode over the paged cache: for each sequence b and head h,
+ * the query q[b,h,:] attends (no mask) to all seq_lens[b] cached tokens.
+ * q, o are [B,H,d]; lse (optional, may be NULL) is [B,H]. */
+int oracle_decode_paged(const double *q, const double *k_pages,
+                        const double *v_pages, const int64_t *page_table,
+                        const int64_t *seq_lens, double *o, double *lse,
+                        int64_t B, int64_t H, int64_t d, int64_t page_size) {
+    if (page_size <= 0 || d <= 0 || H < 0 || B < 0) return -1;
+    int64_t off = 0;
+    int rc = 0;
+    for (int64_t b = 0; b < B && rc == 0; ++b) {
+        const int64_t len = seq_lens[b];
+        if (len < 0) return -1;
+        const int64_t np = (len + page_size - 1) / page_size;
+        double *kc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * H * d));
+        double *vc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * H * d));
+        if (!kc || !vc) {
+            free(kc);
+            free(vc);
+            return -2;
+        }
+        /* this sequence alone, as a one-sequence packed table */
+        oracle_gather_paged(k_pages, page_table + off, &len, kc, 1, H, d, page_size);
+        oracle_gather_paged(v_pages, page_table + off, &len, vc, 1, H, d, page_size);
+        int failed = 0;
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+            if (!srow) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+#pragma omp for schedule(static)
+                for (int64_t h = 0; h < H; ++h) {
+                    double l;
+                    attention_row(q + (b * H + h) * d, kc + h * d, H * d, vc + h * d,
+                                  H * d, len, d, d, 1.0 / sqrt((double)d), srow,
+                                  o + (b * H + h) * d, &l);
+                    if (lse) lse[b * H + h] = l;
+                }
+                free(srow);
+            }
+        }
+        if (failed) rc = -2;
+        free(kc);
+        free(vc);
+        off += np;
+    }
+    return rc;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,430 @@
+"""Pins for the fp64 CPU oracle: it is checked against things other than
+itself -- a hand-worked example, high-precision brute force, closed forms,
+invariants and special cases -- chosen so that a plausible slip (a dropped
+max subtraction, a transposed operand, a wrong index, a mask off by one,
+a natural-log / log2 mix-up) fails at least one of them.
+
+The definition pinned here is standard attention, page "Flash Attention
+是什么：2026 最新原理、架构演进与实战详解" (ai.lansai.wang), section
+核心工作机制; the causal switch is flash_attn_causal on the page
+"为什么“Flash”突然成了AI圈的高频词" (lqnn.cn), section 3.3.
+"""
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+
+import oracle
+from oracle import method
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TOL = 1e-12
+
+
+def _num(x):
+    if isinstance(x, str):
+        return math.log(float(x[2:]))  # "lnK"
+    return float(x)
+
+
+def _rand(shape, seed, std=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * std
+
+
+def _mp_attention(q, k, v, causal, scale):
+    """Brute force at 50 significant digits, straight from the definition."""
+    mpmath.mp.dps = 50
+    N, d = q.shape
+    o = np.zeros((N, v.shape[1]))
+    lse = np.zeros(N)
+    for i in range(N):
+        js = range(i + 1) if causal else range(k.shape[0])
+        s = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(float(q[i, c])) * mpmath.mpf(float(k[j, c]))
+                                             for c in range(d)) for j in js]
+        e = [mpmath.exp(x) for x in s]
+        tot = mpmath.fsum(e)
+        for c in range(v.shape[1]):
+            o[i, c] = float(mpmath.fsum(e[t] * mpmath.mpf(float(v[j, c]))
+                                        for t, j in enumerate(js)) / tot)
+        lse[i] = float(mpmath.log(tot))
+    return o, lse
+
+
+def _att(q, k, v, causal, scale):
+    o, lse = oracle.attention(q[None, None], k[None, None], v[None, None], causal, scale)
+    return o[0, 0], lse[0, 0]
+
+
+# -- hand-worked example -----------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_hand_worked_2x2(causal):
+    g = json.load(open(os.path.join(GOLDEN, "hand_worked_2x2.json")))
+    q = np.array([[_num(x) for x in r] for r in g["q"]])
+    k = np.array(g["k"], float)
+    v = np.array(g["v"], float)
+    exp = g["causal" if causal else "noncausal"]
+    o, lse = _att(q, k, v, causal, g["scale"])
+    np.testing.assert_allclose(o, np.array(exp["o"], float), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, [_num(x) for x in exp["lse"]], rtol=0, atol=1e-14)
+
+
+# -- brute force at high precision -------------------------------------------
+
+@pytest.mark.parametrize("N,d,causal", [(1, 1, False), (3, 2, True), (5, 4, False),
+                                        (7, 8, True), (16, 8, False), (16, 5, True)])
+def test_brute_force_mpmath(N, d, causal):
+    q = _rand((N, d), 10 + N)
+    k = _rand((N, d), 20 + N)
+    v = _rand((N, d + 1), 30 + N)  # dv != d catches a q/v shape mix-up
+    v2 = v[:, :d]
+    scale = 0.37 + 0.1 * d
+    o, lse = _att(q, k, v2, causal, scale)
+    ob, lseb = _mp_attention(q, k, v2, causal, scale)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=TOL)
+    np.testing.assert_allclose(lse, lseb, rtol=0, atol=TOL)
+
+
+def test_brute_force_nonsquare_values_catch_transpose():
+    # Q K^T differs from K Q^T here; a transposed operand changes the output
+    N, d = 6, 3
+    q = _rand((N, d), 1)
+    k = _rand((N, d), 2) * 3.0
+    v = _rand((N, d), 3)
+    o, _ = _att(q, k, v, False, 1.0)
+    ob, _ = _mp_attention(q, k, v, False, 1.0)
+    ot, _ = _mp_attention(k, q, v, False, 1.0)
+    np.testing.assert_allclose(o, ob, atol=TOL)
+    assert np.abs(o - ot).max() > 1e-3
+
+
+# -- invariants ---------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_probability_rows_sum_to_one(causal):
+    N, d = 33, 8
+    q, k = _rand((N, d), 4), _rand((N, d), 5)
+    p = oracle.probs(q, k, causal, 1 / math.sqrt(d))
+    np.testing.assert_allclose(p.sum(axis=1), np.ones(N), atol=TOL)
+    assert (p >= 0).all()
+    if causal:
+        assert np.all(np.triu(p, 1) == 0.0)
+        assert np.all(np.diag(p) > 0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v_returns_v(causal):
+    N, d = 40, 16
+    q, k = _rand((N, d), 6, 2.0), _rand((N, d), 7, 2.0)
+    c = _rand((d,), 8)
+    v = np.tile(c, (N, 1))
+    o, _ = _att(q, k, v, causal, 0.5)
+    np.testing.assert_allclose(o, np.tile(c, (N, 1)), atol=TOL)
+
+
+def test_causal_row0_is_v0():
+    N, d = 21, 8
+    q, k, v = _rand((N, d), 9), _rand((N, d), 10), _rand((N, d), 11)
+    scale = 0.3
+    o, lse = _att(q, k, v, True, scale)
+    np.testing.assert_allclose(o[0], v[0], atol=TOL)
+    assert abs(lse[0] - scale * float(q[0] @ k[0])) < TOL
+
+
+def test_causal_last_row_equals_noncausal_last_row():
+    N, d = 19, 4
+    q, k, v = _rand((N, d), 12), _rand((N, d), 13), _rand((N, d), 14)
+    oc, lc = _att(q, k, v, True, 0.7)
+    on, ln = _att(q, k, v, False, 0.7)
+    np.testing.assert_allclose(oc[-1], on[-1], atol=TOL)
+    assert abs(lc[-1] - ln[-1]) < TOL
+    # and the rows before it differ (the mask does something)
+    assert np.abs(oc[:-1] - on[:-1]).max() > 1e-3
+
+
+def test_v_linearity():
+    N, d = 25, 8
+    q, k = _rand((N, d), 15), _rand((N, d), 16)
+    v1, v2 = _rand((N, d), 17), _rand((N, d), 18)
+    a, b = 1.7, -0.4
+    o1, _ = _att(q, k, v1, True, 0.5)
+    o2, _ = _att(q, k, v2, True, 0.5)
+    o12, _ = _att(q, k, a * v1 + b * v2, True, 0.5)
+    np.testing.assert_allclose(o12, a * o1 + b * o2, atol=1e-11)
+
+
+def test_noncausal_key_permutation_invariance():
+    N, d = 30, 8
+    q, k, v = _rand((N, d), 19), _rand((N, d), 20), _rand((N, d), 21)
+    perm = np.random.default_rng(22).permutation(N)
+    o, lse = _att(q, k, v, False, 0.4)
+    # permute keys and values jointly: unchanged
+    op, lsep = _att(q, k[perm], v[perm], False, 0.4)
+    np.testing.assert_allclose(op, o, atol=TOL)
+    np.testing.assert_allclose(lsep, lse, atol=TOL)
+    # permute values only: changed (catches using the wrong index for V)
+    ow, _ = _att(q, k, v[perm], False, 0.4)
+    assert np.abs(ow - o).max() > 1e-3
+
+
+@pytest.mark.parametrize("shift", [3.0, 800.0])
+def test_score_shift_moves_lse_only(shift):
+    """Adding a constant c to every score of a row leaves o unchanged and adds
+    c to the log-sum-exp.  The constant enters through an extra feature:
+    q' = [q, 1], k' = [k, c/scale].  c = 800 overflows exp() unless the row
+    max is subtracted first."""
+    N, d = 17, 8
+    scale = 0.25
+    q, k, v = _rand((N, d), 23), _rand((N, d), 24), _rand((N, d), 25)
+    q2 = np.concatenate([q, np.ones((N, 1))], axis=1)
+    k2 = np.concatenate([k, np.full((N, 1), shift / scale)], axis=1)
+    for causal in (False, True):
+        o, lse = _att(q, k, v, causal, scale)
+        o2, lse2 = _att(q2, k2, v, causal, scale)
+        assert np.all(np.isfinite(o2))
+        np.testing.assert_allclose(o2, o, atol=1e-10)
+        np.testing.assert_allclose(lse2, lse + shift, rtol=0, atol=1e-9)
+
+
+# -- closed forms -------------------------------------------------------------
+
+def test_zero_query_closed_form():
+    N, d = 37, 8
+    q = np.zeros((N, d))
+    k, v = _rand((N, d), 26), _rand((N, d), 27)
+    o, lse = _att(q, k, v, False, 1.0)
+    np.testing.assert_allclose(o, np.tile(v.mean(axis=0), (N, 1)), atol=TOL)
+    np.testing.assert_allclose(lse, np.full(N, math.log(N)), atol=TOL)
+    oc, lsec = _att(q, k, v, True, 1.0)
+    prefix_mean = np.cumsum(v, axis=0) / np.arange(1, N + 1)[:, None]
+    np.testing.assert_allclose(oc, prefix_mean, atol=TOL)
+    np.testing.assert_allclose(lsec, np.log(np.arange(1, N + 1)), atol=TOL)
+
+
+def test_large_scale_is_hard_argmax():
+    N, d = 12, 6
+    q, k, v = _rand((N, d), 28), _rand((N, d), 29), _rand((N, d), 30)
+    scale = 1e4
+    o, lse = _att(q, k, v, False, scale)
+    s = q @ k.T
+    j = s.argmax(axis=1)
+    np.testing.assert_allclose(o, v[j], atol=1e-9)
+    np.testing.assert_allclose(lse, scale * s.max(axis=1), rtol=1e-12)
+
+
+def test_lse_is_natural_log():
+    # two equal scores: lse = s + ln 2 (a log2 slip would give s + 1)
+    q = np.array([[1.0, 0.0], [1.0, 0.0]])
+    k = np.array([[2.0, 0.0], [2.0, 0.0]])
+    v = np.eye(2)
+    _, lse = _att(q, k, v, False, 1.0)
+    assert abs(lse[0] - (2.0 + math.log(2.0))) < 1e-15
+    assert abs(lse[1] - (2.0 + math.log(2.0))) < 1e-15
+
+
+def test_row_subset_matches_full():
+    B, H, N, d = 2, 3, 50, 8
+    q, k, v = _rand((B, H, N, d), 31), _rand((B, H, N, d), 32), _rand((B, H, N, d), 33)
+    o, lse = oracle.attention(q, k, v, True, 0.3)
+    rows = np.array([0, 7, 49, 50, 149, 299])
+    os_, ls = oracle.attention(q, k, v, True, 0.3, rows=rows)
+    fo, fl = o.reshape(-1, d), lse.reshape(-1)
+    np.testing.assert_array_equal(os_.reshape(-1, d)[rows], fo[rows])
+    np.testing.assert_array_equal(ls.reshape(-1)[rows], fl[rows])
+    assert np.isnan(ls.reshape(-1)[1])
+
+
+def test_batch_heads_are_independent():
+    B, H, N, d = 2, 2, 9, 4
+    q, k, v = _rand((B, H, N, d), 34), _rand((B, H, N, d), 35), _rand((B, H, N, d), 36)
+    o, lse = oracle.attention(q, k, v, True, 0.5)
+    for b in range(B):
+        for h in range(H):
+            ob, lb = _mp_attention(q[b, h], k[b, h], v[b, h], True, 0.5)
+            np.testing.assert_allclose(o[b, h], ob, atol=TOL)
+            np.testing.assert_allclose(lse[b, h], lb, atol=TOL)
+
+
+# -- the method's steps reach the definition ---------------------------------
+
+@pytest.mark.parametrize("block", [1, 7, 64, 128, 200])
+@pytest.mark.parametrize("causal", [False, True])
+def test_online_softmax_equals_two_pass(block, causal):
+    N, d = 200, 16
+    q, k, v = _rand((N, d), 40, 2.0), _rand((N, d), 41, 2.0), _rand((N, d), 42)
+    o, lse = _att(q, k, v, causal, 1 / math.sqrt(d))
+    oo, lo = method.online_attention(q, k, v, causal, 1 / math.sqrt(d), block)
+    np.testing.assert_allclose(oo, o, rtol=0, atol=TOL)
+    np.testing.assert_allclose(lo, lse, rtol=0, atol=TOL)
+
+
+def test_online_softmax_without_correction_is_wrong():
+    """Planted slip on the CPU: dropping the correction of earlier partial
+    results (alpha = 1) changes the answer, so the test above is sensitive."""
+    N, d = 64, 8
+    q, k, v = _rand((N, d), 43, 3.0), _rand((N, d), 44, 3.0), _rand((N, d), 45)
+    o, _ = _att(q, k, v, False, 1.0)
+    m = np.full(N, -np.inf)
+    acc = np.zeros((N, d))
+    l = np.zeros(N)
+    for j0 in range(0, N, 8):
+        x = q @ k[j0:j0 + 8].T
+        m = np.maximum(m, x.max(axis=1))
+        p = np.exp(x - m[:, None])
+        l = l + p.sum(axis=1)
+        acc = acc + p @ v[j0:j0 + 8]
+    assert np.abs(acc / l[:, None] - o).max() > 1e-3
+
+
+@pytest.mark.parametrize("nsplit", [1, 2, 3, 8, 40])
+def test_split_merge_equals_unsplit(nsplit):
+    N, d = 300, 16
+    rng = np.random.default_rng(50 + nsplit)
+    q, k, v = rng.standard_normal(d) * 2, rng.standard_normal((N, d)) * 2, rng.standard_normal((N, d))
+    cuts = sorted(rng.integers(0, N + 1, size=nsplit - 1).tolist())
+    edges = [0] + cuts + [N]
+    bounds = list(zip(edges[:-1], edges[1:]))
+    if nsplit >= 3:
+        bounds.append((N, N))  # an empty split must carry no weight
+    o, lse = method.split_merge_attention(q, k, v, 1 / math.sqrt(d), bounds)
+    # the plain definition for this one query: every row of the tiled query
+    # block is the same row
+    ref_o, ref_l = _att(np.tile(q, (N, 1)), k, v, False, 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, ref_o[0], atol=TOL)
+    assert abs(lse - ref_l[0]) < TOL
+
+
+# -- variable length ----------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equals_per_sequence(causal):
+    lens = [5, 1, 17, 9]
+    H, d = 3, 8
+    total = sum(lens)
+    q, k, v = _rand((total, H, d), 60), _rand((total, H, d), 61), _rand((total, H, d), 62)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    o, lse = oracle.attention_varlen(q, k, v, cu, causal, 0.35)
+    for b, L in enumerate(lens):
+        s0 = cu[b]
+        for h in range(H):
+            ob, lb = _mp_attention(q[s0:s0 + L, h], k[s0:s0 + L, h], v[s0:s0 + L, h], causal, 0.35)
+            np.testing.assert_allclose(o[s0:s0 + L, h], ob, atol=TOL)
+            np.testing.assert_allclose(lse[h, s0:s0 + L], lb, atol=TOL)
+
+
+def test_varlen_row_subset_matches_full():
+    lens = [4, 11, 6]
+    H, d = 2, 4
+    total = sum(lens)
+    q, k, v = _rand((total, H, d), 63), _rand((total, H, d), 64), _rand((total, H, d), 65)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    o, lse = oracle.attention_varlen(q, k, v, cu, True, 0.5)
+    rows = np.array([0, 3, 4, 14, 15, 20, 21 + 14])
+    o2, l2 = oracle.attention_varlen(q, k, v, cu, True, 0.5, rows=rows)
+    for r in rows:
+        h, g = divmod(int(r), total)
+        np.testing.assert_array_equal(o2[g, h], o[g, h])
+        assert l2[h, g] == lse[h, g]
+
+
+# -- paged gather and decode --------------------------------------------------
+
+def _append_simulation(seqs, H, d, page_size, n_pool, seed):
+    """Build a paged cache the way a serving loop fills it: tokens arrive one
+    at a time per sequence (round robin); a sequence whose current page is
+    full takes a fresh page from a shuffled free list (page "“Flash”不是那个
+    被时代淘汰的插件", 0539edu.com, section 2: pages come from a fixed pool,
+    a new token goes to a page allocated from the pool).  Returns the pool,
+    the packed page table and the lengths."""
+    rng = np.random.default_rng(seed)
+    free = list(rng.permutation(n_pool))
+    pool = np.full((n_pool, H, page_size, d), np.nan)
+    owned = [[] for _ in seqs]
+    fill = [page_size for _ in seqs]  # current page full -> allocate on first token
+    pos = [0 for _ in seqs]
+    active = True
+    while active:
+        active = False
+        for b, x in enumerate(seqs):
+            if pos[b] >= x.shape[0]:
+                continue
+            active = True
+            if fill[b] == page_size:
+                owned[b].append(free.pop())
+                fill[b] = 0
+            pool[owned[b][-1], :, fill[b], :] = x[pos[b]]
+            fill[b] += 1
+            pos[b] += 1
+    table = np.array([p for o in owned for p in o], dtype=np.int64)
+    return pool, table, np.array([x.shape[0] for x in seqs], dtype=np.int64)
+
+
+@pytest.mark.parametrize("page_size", [4, 256])
+def test_gather_inverts_append(page_size):
+    H, d = 2, 3
+    lens = [1, page_size, page_size + 1, 3 * page_size - 1, 0, 2]
+    seqs = [_rand((L, H, d), 70 + i) for i, L in enumerate(lens)]
+    n_pool = sum((L + page_size - 1) // page_size for L in lens) + 3  # spare pages
+    pool, table, sl = _append_simulation(seqs, H, d, page_size, n_pool, 71)
+    out = oracle.gather_paged(pool, table, sl, page_size)
+    np.testing.assert_array_equal(out, np.concatenate(seqs, axis=0))
+
+
+def test_decode_equals_attention_over_gathered_cache():
+    H, d, page_size = 3, 8, 4
+    lens = [1, 4, 5, 13]
+    kseqs = [_rand((L, H, d), 80 + i) for i, L in enumerate(lens)]
+    vseqs = [_rand((L, H, d), 90 + i) for i, L in enumerate(lens)]
+    n_pool = sum((L + page_size - 1) // page_size for L in lens)
+    kpool, table, sl = _append_simulation(kseqs, H, d, page_size, n_pool, 81)
+    vpool, table2, _ = _append_simulation(vseqs, H, d, page_size, n_pool, 81)
+    assert np.array_equal(table, table2)
+    q = _rand((len(lens), H, d), 82)
+    o, lse = oracle.decode_paged(q, kpool, vpool, table, sl, page_size)
+    assert np.all(np.isfinite(o))  # the NaN-filled spare slots were never read
+    for b, L in enumerate(lens):
+        for h in range(H):
+            ob, lb = _mp_attention(q[b, h][None], kseqs[b][:, h], vseqs[b][:, h], False,
+                                   1 / math.sqrt(d))
+            np.testing.assert_allclose(o[b, h], ob[0], atol=TOL)
+            assert abs(lse[b, h] - lb[0]) < TOL
+
+
+def test_decode_empty_sequence_gives_zero():
+    H, d, page_size = 2, 4, 4
+    kpool = _rand((2, H, page_size, d), 83)
+    vpool = _rand((2, H, page_size, d), 84)
+    q = _rand((2, H, d), 85)
+    o, lse = oracle.decode_paged(q, kpool, vpool, np.array([1, 0]), np.array([0, 5]), page_size)
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(np.isfinite(o[1]))
+
+
+def test_decode_is_last_causal_row():
+    """Decode of the last token equals the last row of causal attention over
+    the same (gathered) keys -- the tie between the two entry points."""
+    H, d, page_size = 2, 8, 4
+    L = 11
+    qs, ks, vs = _rand((L, H, d), 86), _rand((L, H, d), 87), _rand((L, H, d), 88)
+    n_pool = (L + page_size - 1) // page_size
+    kpool, table, sl = _append_simulation([ks], H, d, page_size, n_pool, 89)
+    vpool, _, _ = _append_simulation([vs], H, d, page_size, n_pool, 89)
+    o, lse = oracle.decode_paged(qs[-1][None], kpool, vpool, table, sl, page_size)
+    oc, lc = oracle.attention(qs.transpose(1, 0, 2)[None], ks.transpose(1, 0, 2)[None],
+                              vs.transpose(1, 0, 2)[None], True, 1 / math.sqrt(d))
+    np.testing.assert_allclose(o[0], oc[0, :, -1], atol=TOL)
+    np.testing.assert_allclose(lse[0], lc[0, :, -1], atol=TOL)
+
+
+def test_bf16_inputs_are_upcast_exactly():
+    torch = pytest.importorskip("torch")
+    x = torch.randn(4, 8, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    q = x[None, None]
+    o, _ = oracle.attention(q, q, q, False, 0.5)
+    o2, _ = oracle.attention(x.float().double().numpy()[None, None],
+                             x.float().double().numpy()[None, None],
+                             x.float().double().numpy()[None, None], False, 0.5)
+    np.testing.assert_array_equal(o, o2)
