@@ -1,0 +1,304 @@
+// api.cu -- the extern "C" boundary of libfa.so (declared in include/fa.h):
+// argument checks, TMA tensor maps, the per-GPU decode workspace and the
+// device error word.  No kernel arithmetic lives here.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa_ptx.cuh"
+
+namespace {
+
+// Waits on an mbarrier that nothing ever arrives on, through the same bounded
+// wait the attention kernels use; the wait must give up and record
+// FA_ERR_DEVICE_TIMEOUT instead of spinning forever.
+__global__ void fa_selftest_wait_kernel(unsigned int* err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        fa::mbar_init(&bar, 1);
+        fa::fence_mbar_init();
+        fa::mbar_wait(&bar, 0, err, FA_DEVERR_TIMEOUT, nullptr);
+    }
+}
+
+// First fault recorded by any kernel of this library on a device (see
+// fa_get_device_error).  One copy per device: it lives in the module.
+__device__ unsigned int g_device_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool init = false;
+    int num_sms = 0;
+    int cc_major = 0;
+    unsigned int* err = nullptr;  // device address of g_device_error
+    void* ws = nullptr;           // decode workspace
+    size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int get_encode_fn() {
+    if (g_encode) return FA_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return FA_OK;
+}
+
+// Current device's state, initialised on first use (caller holds g_mu).
+int device_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    DeviceState& s = g_dev[dev];
+    if (!s.init) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FA_ERR_CUDA;
+        s.num_sms = prop.multiProcessorCount;
+        s.cc_major = prop.major;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return FA_ERR_CUDA;
+        s.err = static_cast<unsigned int*>(p);
+        s.init = true;
+    }
+    *out = &s;
+    return FA_OK;
+}
+
+int lookup_device(DeviceState** out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int rc = device_state(out);
+    if (rc != FA_OK) return rc;
+    if ((*out)->cc_major != 10) return FA_ERR_UNSUPPORTED;  // sm_100 family only
+    return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// bf16 tensor map over `dims` (innermost first) with byte strides for dims 1..2
+// and a box of `box` elements; 128-byte swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap* map, const void* base, const cuuint64_t dims[3],
+             const cuuint64_t strides[2], const cuuint32_t box[3]) {
+    if (get_encode_fn() != FA_OK) return FA_ERR_CUDA;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Grow-only per-device workspace, allocated on the caller's stream.
+int ensure_workspace(DeviceState* s, size_t bytes, cudaStream_t stream, void** out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (s->ws_bytes < bytes) {
+        if (s->ws) {
+            if (cudaFreeAsync(s->ws, stream) != cudaSuccess) return FA_ERR_CUDA;
+            s->ws = nullptr;
+            s->ws_bytes = 0;
+        }
+        void* p = nullptr;
+        if (cudaMallocAsync(&p, bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_NOMEM;
+        }
+        s->ws = p;
+        s->ws_bytes = bytes;
+    }
+    *out = s->ws;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, int causal, float scale, fa_stream_t stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * H > 65535) return FA_ERR_SHAPE;
+    if (N > 0x7fffffff - 128) return FA_ERR_SHAPE;
+    if (!std::isfinite(scale)) return FA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    CUtensorMap tq, tk, tv;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(N) * d * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims, strides, box)) != FA_OK) return rc;
+    fa::FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens = nullptr;
+    p.B = B;
+    p.H = H;
+    p.N = N;
+    p.total = 0;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.err = s->err;
+    return fa::launch_fwd(p, tq, tk, tv, d, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens, int B, int H, int total, int max_seqlen, int d,
+                  int causal, float scale, fa_stream_t stream) {
+    if (!q || !k || !v || !o || !lse || !cu_seqlens) return FA_ERR_NULL;
+    if (B < 1 || H < 1 || total < 1 || max_seqlen < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return FA_ERR_SHAPE;
+    if (max_seqlen > 0x7fffffff - 128) return FA_ERR_SHAPE;
+    if (!std::isfinite(scale)) return FA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    CUtensorMap tq, tk, tv;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(total)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(H) * d * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims, strides, box)) != FA_OK) return rc;
+    fa::FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens = cu_seqlens;
+    p.B = B;
+    p.H = H;
+    p.N = max_seqlen;
+    p.total = total;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.err = s->err;
+    return fa::launch_fwd(p, tq, tk, tv, d, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                    int d, int page_size, fa_stream_t stream) {
+    if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !o) return FA_ERR_NULL;
+    if (B < 1 || H < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (page_size != 256) return FA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * H * fa::kDecodeMaxSplits > 0x7fffffff) return FA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits), st,
+                               &ws)) != FA_OK)
+        return rc;
+    return fa::launch_decode(q, k_pages, v_pages, page_table, seq_lens, o, B, H, d, page_size,
+                             fa::kDecodeMaxSplits, ws, s->err, s->num_sms, st);
+}
+
+int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t* seq_lens,
+                    void* out, int B, int H, int d, int page_size, fa_stream_t stream) {
+    if (!pages || !page_table || !seq_lens || !out) return FA_ERR_NULL;
+    if (B < 1 || H < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (page_size != 256) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(pages) || !aligned16(out)) return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H, d, 1), st, &ws)) != FA_OK)
+        return rc;
+    return fa::launch_gather(pages, page_table, seq_lens, out, B, H, d, page_size, ws, s->err,
+                             s->num_sms, st);
+}
+
+int fa_get_device_error(int* code, fa_stream_t stream) {
+    if (!code) return FA_ERR_NULL;
+    DeviceState* s = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int rc = device_state(&s);
+        if (rc != FA_OK) return rc;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int v = 0;
+    const unsigned int zero = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemcpy(&v, s->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemcpy(s->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return FA_ERR_CUDA;
+    *code = -static_cast<int>(v);
+    return FA_OK;
+}
+
+int fa_selftest_bounded_wait(fa_stream_t stream) {
+    DeviceState* s = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int rc = device_state(&s);
+        if (rc != FA_OK) return rc;
+    }
+    fa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(s->err);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_release_workspace(void) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FA_OK;
+    DeviceState& s = g_dev[dev];
+    if (s.ws) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+        if (cudaFree(s.ws) != cudaSuccess) return FA_ERR_CUDA;
+        s.ws = nullptr;
+        s.ws_bytes = 0;
+    }
+    return FA_OK;
+}
+
+const char* fa_status_str(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+        case FA_ERR_SHAPE: return "FA_ERR_SHAPE: a size is out of range";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim, page size or device";
+        case FA_ERR_ALIGN: return "FA_ERR_ALIGN: a tensor pointer is not 16-byte aligned";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call or launch failed";
+        case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+        case FA_ERR_NOMEM: return "FA_ERR_NOMEM: workspace allocation failed";
+        case FA_ERR_DEVICE_BAD_INPUT: return "FA_ERR_DEVICE_BAD_INPUT: invalid device-side input (negative length)";
+        default: return "unknown fa status";
+    }
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// fa_internal.h -- constants and launch entry points shared inside libfa.so.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+
+// A bounded device wait gives up after this much global time.
+#define FA_WAIT_TIMEOUT_NS 2000000000ull
+
+// Values written to the device error word: the magnitude of the FA_ERR_*
+// status the host reports for them.
+#define FA_DEVERR_TIMEOUT (static_cast<unsigned int>(-FA_ERR_DEVICE_TIMEOUT))
+#define FA_DEVERR_BAD_INPUT (static_cast<unsigned int>(-FA_ERR_DEVICE_BAD_INPUT))
+
+namespace fa {
+
+// ---- forward -------------------------------------------------------------
+struct FwdParams {
+    // tensor maps live in the kernel's parameter space (see the launchers)
+    void* o;             // bf16 output
+    float* lse;          // fp32 output
+    const int32_t* cu_seqlens;  // varlen only
+    int B, H, N;         // N: sequence length (fixed) or max_seqlen (varlen)
+    int total;           // varlen: packed rows
+    int causal;
+    float scale_log2;    // scale * log2(e)
+    unsigned int* err;   // device error word
+};
+
+int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+               const CUtensorMap& tv, int d, bool varlen, cudaStream_t stream);
+
+// ---- paged decode ----------------------------------------------------------
+// Number of pages a split covers at least (a split is one CTA work unit) and
+// the most splits one sequence is cut into.
+constexpr int kDecodeChunkPages = 2;
+constexpr int kDecodeMaxSplits = 64;
+
+struct DecodePlan {
+    int32_t* page_off;   // [B+1] prefix of pages per sequence
+    int32_t* tok_off;    // [B+1] prefix of tokens per sequence
+    int32_t* unit_off;   // [B+1] prefix of (split x head) units per sequence
+};
+
+size_t decode_workspace_bytes(int B, int H, int d, int max_splits);
+
+int launch_decode(const void* q, const void* k_pages, const void* v_pages,
+                  const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                  int d, int page_size, int max_splits, void* workspace, unsigned int* err,
+                  int num_sms, cudaStream_t stream);
+
+int launch_gather(const void* pages, const int32_t* page_table, const int32_t* seq_lens,
+                  void* out, int B, int H, int d, int page_size, void* workspace,
+                  unsigned int* err, int num_sms, cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,188 @@
+"""ctypes binding of libfa.so (include/fa.h), one Python function per C entry
+point, same names.  Argument marshalling only: every step of the computation
+runs in the library's CUDA kernels.  PyTorch supplies device memory and the
+stream; there is no fallback -- a missing library or a non-CUDA tensor is an
+error.
+"""
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_OK = 0
+FA_ERR_NULL = -1
+FA_ERR_SHAPE = -2
+FA_ERR_UNSUPPORTED = -3
+FA_ERR_ALIGN = -4
+FA_ERR_CUDA = -5
+FA_ERR_DEVICE_TIMEOUT = -6
+FA_ERR_NOMEM = -7
+FA_ERR_DEVICE_BAD_INPUT = -8
+
+# every symbol include/fa.h declares
+EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_gather_paged",
+           "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
+           "fa_status_str", "fa_version")
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {fa_status_str(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (built in-tree by attn_fwd_04_b200.build); raise if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libfa.so not found at {LIB_PATH}; build it with "
+                              "`python -m attn_fwd_04_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.fa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+        L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+        L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        L.fa_gather_paged.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.fa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
+        L.fa_selftest_bounded_wait.argtypes = [P]
+        L.fa_release_workspace.argtypes = []
+        L.fa_status_str.argtypes = [I]
+        L.fa_status_str.restype = ctypes.c_char_p
+        L.fa_version.argtypes = []
+        for name in ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_gather_paged",
+                     "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
+                     "fa_version"):
+            getattr(L, name).restype = I
+        _lib = L
+    return _lib
+
+
+def fa_status_str(status: int) -> str:
+    return lib().fa_status_str(int(status)).decode()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise_if(status: int, what: str):
+    if status != FA_OK:
+        raise FaError(status, what)
+
+
+def fa_fwd(q, k, v, causal: bool, scale: Optional[float] = None, o=None, lse=None, stream=None):
+    """Fused attention forward over [B,H,N,d] bf16 tensors -> (o, lse [B,H,N] fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same [B,H,N,d] shape")
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(o, "o", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_fwd")
+    return o, lse
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
+                  scale: Optional[float] = None, o=None, lse=None, stream=None):
+    """Forward over packed [total,H,d] sequences -> (o, lse [H,total] fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 3)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    total, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    rc = lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), cu_seqlens.data_ptr(), B, H, total,
+                             int(max_seqlen), d, int(bool(causal)), float(scale),
+                             _stream(stream))
+    _raise_if(rc, "fa_fwd_varlen")
+    return o, lse
+
+
+def fa_decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 256, o=None,
+                    stream=None):
+    """Single-token decode over a paged cache -> o [B,H,d] bf16."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, H, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    rc = lib().fa_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                               page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
+                               B, H, d, int(page_size), _stream(stream))
+    _raise_if(rc, "fa_decode_paged")
+    return o
+
+
+def fa_gather_paged(pages, page_table, seq_lens, total_tokens: int, page_size: int = 256,
+                    out=None, stream=None):
+    """Copy cached tokens out of [P,H,page_size,d] pages -> [total_tokens,H,d]."""
+    _check(pages, "pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _, H, _, d = pages.shape
+    B = seq_lens.numel()
+    if out is None:
+        out = torch.empty((total_tokens, H, d), dtype=torch.bfloat16, device=pages.device)
+    rc = lib().fa_gather_paged(pages.data_ptr(), page_table.data_ptr(), seq_lens.data_ptr(),
+                               out.data_ptr(), B, H, d, int(page_size), _stream(stream))
+    _raise_if(rc, "fa_gather_paged")
+    return out
+
+
+def fa_get_device_error(stream=None) -> int:
+    """Synchronise the stream, read and clear the device error word (FA_* code)."""
+    code = ctypes.c_int(0)
+    rc = lib().fa_get_device_error(ctypes.byref(code), _stream(stream))
+    _raise_if(rc, "fa_get_device_error")
+    return code.value
+
+
+def fa_selftest_bounded_wait(stream=None) -> None:
+    """Launch the bounded-wait self test; read the result with fa_get_device_error."""
+    _raise_if(lib().fa_selftest_bounded_wait(_stream(stream)), "fa_selftest_bounded_wait")
+
+
+def fa_release_workspace() -> None:
+    _raise_if(lib().fa_release_workspace(), "fa_release_workspace")
+
+
+def fa_version() -> int:
+    return lib().fa_version()

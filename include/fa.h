@@ -1,0 +1,186 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact scaled-dot-product attention on B200
+ * (sm_100a).  A fused forward pass (fixed-length and variable-length) and
+ * single-token decode over a paged KV cache.
+ *
+ * What the calls compute.  Standard attention, as the page "Flash Attention
+ * 是什么：2026 最新原理、架构演进与实战详解" (ai.lansai.wang) defines it in its
+ * section 核心工作机制: for each query row i,
+ *     s_ij = scale * q_i . k_j,    p_ij = exp(s_ij - m_i) / l_i,
+ *     o_i  = sum_j p_ij v_j,       lse_i = m_i + ln l_i,
+ * with m_i the row max and l_i = sum_j exp(s_ij - m_i).  The forward pass is
+ * computed the fused way that page describes (tiling into on-chip blocks,
+ * online softmax with a running max and normaliser -- section 关键术语解析,
+ * item 4 -- and one final rescale, as the page at zwxr.cn describes in its
+ * section 3.1), so the N x N score matrix never reaches device memory.  The
+ * same page (section 常见误解澄清, misconception 1) states the result is the
+ * standard one up to floating-point rounding; that is the contract here.
+ *
+ * Conventions shared by every call:
+ *  - Element types: q, k, v, o, pages are bf16 (IEEE binary16-brain, raw
+ *    uint16 storage); lse is fp32; all index arrays are int32.
+ *  - Pointers are DEVICE pointers owned by the caller; the library never
+ *    frees or retains them beyond the call's stream work.  Every tensor base
+ *    pointer must be 16-byte aligned (FA_ERR_ALIGN otherwise).
+ *  - Head dimension d must be 64 or 128 (FA_ERR_UNSUPPORTED otherwise).
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream) and
+ *    never synchronise, except fa_get_device_error.  Argument errors are
+ *    returned before anything is launched.  FA_ERR_CUDA means a CUDA launch
+ *    or runtime call failed (cudaGetLastError is left as CUDA set it).
+ *  - Faults found on the device (a bounded wait that ran out, a negative
+ *    sequence length) do not trap: the kernel records a code in the library's
+ *    device error word and returns; fa_get_device_error reads it.
+ *  - The library holds one device workspace per GPU for the decode split
+ *    partials (grown on demand with cudaMallocAsync on the caller's stream,
+ *    freed by fa_release_workspace).  Calls that use it (fa_decode_paged,
+ *    fa_gather_paged) on different streams of the same GPU must not overlap:
+ *    order them on one stream or with events.
+ *  - Thread safety: the host entry points may be called from several host
+ *    threads; the workspace bookkeeping is guarded by a mutex.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported from libfa.so (which is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* fa_stream_t;
+
+enum fa_status {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,           /* a required pointer is NULL */
+    FA_ERR_SHAPE = -2,          /* a size is out of range (negative, zero where not allowed, too large) */
+    FA_ERR_UNSUPPORTED = -3,    /* d not in {64,128}, page_size != 256, or not an sm_100 device */
+    FA_ERR_ALIGN = -4,          /* a tensor base pointer is not 16-byte aligned */
+    FA_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
+    FA_ERR_DEVICE_TIMEOUT = -6, /* reported through fa_get_device_error: a bounded device wait ran out */
+    FA_ERR_NOMEM = -7,          /* the decode workspace could not be allocated */
+    FA_ERR_DEVICE_BAD_INPUT = -8 /* reported through fa_get_device_error: e.g. a negative seq_lens entry */
+};
+
+/*
+ * fa_fwd -- fused attention forward pass over fixed-length sequences.
+ *
+ * Computes, for every batch b, head h and query row i < N,
+ *   o[b,h,i,:] = sum_j softmax_j(scale * q[b,h,i,:] . k[b,h,j,:]) v[b,h,j,:]
+ *   lse[b,h,i] = natural log of sum_j exp(scale * q[b,h,i,:] . k[b,h,j,:])
+ * over keys j < N, or j <= i when `causal` is non-zero (the flash_attn_causal
+ * knob of the page "为什么“Flash”突然成了AI圈的高频词" (lqnn.cn), section 3.3,
+ * top-left aligned).  `scale` is the softmax scale (that section's
+ * softmax_scale; callers normally pass 1/sqrt(d)); any finite value.
+ *
+ * Layout: q, k, v, o are [B, H, N, d] contiguous bf16 (the [1, 32, 16384, 128]
+ * layout of that page's section 2.1); lse is [B, H, N] fp32.
+ * Any N >= 1 (no padding to a multiple of the tile is required).
+ * Limits: B*H <= 65535, N <= 2^31 - 1 - 128.
+ * Returns FA_OK, or an FA_ERR_* code before launching anything.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, int causal, float scale, fa_stream_t stream);
+
+/*
+ * fa_fwd_varlen -- the forward pass over B sequences of different lengths
+ * packed back to back (the variable-length batches of the page "Flash
+ * Attention 是什么", section 典型应用场景).
+ *
+ * Sequence b owns packed rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (cu_seqlens
+ * is a DEVICE int32 array of B+1 non-decreasing offsets, cu_seqlens[0] = 0).
+ * Attention never crosses a sequence; with `causal`, row t of a sequence sees
+ * rows 0..t of the same sequence.
+ * Layout: q, k, v, o are [total, H, d] bf16; lse is [H, total] fp32.
+ * `total` (the packed row count, = cu_seqlens[B]) is passed from the host so
+ * that the call never has to read device memory; `max_seqlen` must be >= every
+ * sequence length (it sizes the launch).  A cu_seqlens entry that breaks
+ * these rules (decreasing, past `total`, a sequence longer than max_seqlen) is
+ * clamped on the device and reported as FA_ERR_DEVICE_BAD_INPUT; no access
+ * leaves the [total, H, d] tensors.
+ */
+FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens, int B, int H, int total, int max_seqlen, int d,
+                  int causal, float scale, fa_stream_t stream);
+
+/*
+ * fa_decode_paged -- single-token decode over a paged KV cache, split over
+ * the cache pages and merged by log-sum-exp.
+ *
+ * The cache is the fixed-size page pool of the page "“Flash”不是那个被时代淘汰
+ * 的插件" (0539edu.com), section 2: every page holds page_size (= 256)
+ * consecutive tokens of one sequence.
+ *   q          : [B, H, d] bf16, the new token's query of each sequence
+ *   k_pages,
+ *   v_pages    : [P, H, page_size, d] bf16 -- page p, head h is one contiguous
+ *                page_size x d slice
+ *   page_table : int32, the pages of all sequences packed back to back:
+ *                sequence b's pages are entries off_b .. off_b + n_b - 1 with
+ *                n_b = ceil(seq_lens[b] / page_size) and off_b = sum of n over
+ *                earlier sequences; token t of sequence b is in page
+ *                page_table[off_b + t / page_size], slot t % page_size
+ *   seq_lens   : [B] int32, tokens cached per sequence (the new token's k/v
+ *                already appended); 0 gives o = 0; a negative entry is treated
+ *                as 0 and reported as FA_ERR_DEVICE_BAD_INPUT
+ *   o          : [B, H, d] bf16 output
+ * The query attends, without a mask, to all seq_lens[b] cached tokens, with
+ * softmax scale 1/sqrt(d) (the default of the lqnn.cn page, section 3.3; the
+ * call has no scale argument).  page_size must be 256.
+ * Uses the library's per-GPU workspace (see the conventions above).
+ */
+FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* seq_lens, void* o,
+                    int B, int H, int d, int page_size, fa_stream_t stream);
+
+/*
+ * fa_gather_paged -- copy the cached tokens of every sequence out of the page
+ * pool into contiguous rows (a checking aid for the decode path's address
+ * arithmetic; same page_table / seq_lens conventions as fa_decode_paged).
+ *   pages : [P, H, page_size, d] bf16
+ *   out   : [sum_b seq_lens[b], H, d] bf16, sequence b starting at row
+ *           sum_{b' < b} seq_lens[b']
+ * page_size must be 256.  Uses the library's per-GPU workspace.
+ */
+FA_API int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t* seq_lens,
+                    void* out, int B, int H, int d, int page_size, fa_stream_t stream);
+
+/*
+ * fa_get_device_error -- synchronise `stream`, then read and clear the
+ * current GPU's device error word.  *code receives FA_OK or the FA_ERR_*
+ * value of the first fault a kernel recorded since the last read.
+ * Returns FA_OK, FA_ERR_NULL or FA_ERR_CUDA.
+ */
+FA_API int fa_get_device_error(int* code, fa_stream_t stream);
+
+/*
+ * fa_selftest_bounded_wait -- launch one tiny kernel that waits on a device
+ * barrier nothing ever signals, using the same bounded wait as every
+ * attention kernel.  The wait gives up after about two seconds and records
+ * FA_ERR_DEVICE_TIMEOUT, which fa_get_device_error then returns.  This checks
+ * the failure-detection path without hanging or faulting the GPU.
+ * Returns FA_OK once launched, or FA_ERR_CUDA.
+ */
+FA_API int fa_selftest_bounded_wait(fa_stream_t stream);
+
+/* Free the current GPU's decode workspace (synchronises the device first).
+ * Returns FA_OK or FA_ERR_CUDA. */
+FA_API int fa_release_workspace(void);
+
+/* A static, human-readable name for a status code. */
+FA_API const char* fa_status_str(int status);
+
+/* Library ABI version: 100 * major + minor. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

@@ -1,0 +1,50 @@
+"""Shared comparison helpers for the GPU parity tests.
+
+Tolerances (fixed by the accuracy target for bf16 inputs with fp32
+accumulation): O within max-abs 2e-2 and relative RMS 5e-3 of the fp64
+oracle, the log-sum-exp within 1e-3 absolute.
+"""
+import numpy as np
+import torch
+
+O_MAX_ABS = 2e-2
+O_REL_RMS = 5e-3
+LSE_MAX_ABS = 1e-3
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").double().numpy()
+
+
+def o_errors(o_gpu: np.ndarray, o_ref: np.ndarray):
+    diff = o_gpu - o_ref
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    denom = float(np.sqrt(np.sum(o_ref * o_ref)))
+    rel_rms = float(np.sqrt(np.sum(diff * diff)) / denom) if denom > 0 else float(np.sqrt(np.sum(diff * diff)))
+    return max_abs, rel_rms
+
+
+def assert_o_close(o_gpu, o_ref, what=""):
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
+    max_abs, rel_rms = o_errors(o_gpu, o_ref)
+    assert max_abs <= O_MAX_ABS, f"{what}: O max-abs {max_abs:.3e} > {O_MAX_ABS}"
+    assert rel_rms <= O_REL_RMS, f"{what}: O rel-RMS {rel_rms:.3e} > {O_REL_RMS}"
+    return max_abs, rel_rms
+
+
+def assert_lse_close(lse_gpu, lse_ref, what=""):
+    assert np.all(np.isfinite(lse_gpu)), f"{what}: non-finite lse"
+    err = float(np.max(np.abs(lse_gpu - lse_ref))) if np.size(lse_ref) else 0.0
+    assert err <= LSE_MAX_ABS, f"{what}: LSE max-abs {err:.3e} > {LSE_MAX_ABS}"
+    return err
+
+
+def sample_rows(N: int, count: int, seed: int, tile: int = 128):
+    """Query rows to check at full size: the first and last rows, both sides
+    of every few tile boundaries, and seeded random rows."""
+    g = torch.Generator().manual_seed(seed)
+    fixed = {0, 1, N - 1, N - 2}
+    for t in range(tile, N, max(tile, (N // 8) // tile * tile)):
+        fixed.update({t - 1, t})
+    rand = torch.randint(0, N, (max(0, count - len(fixed)),), generator=g).tolist()
+    return sorted({r for r in fixed | set(rand) if 0 <= r < N})

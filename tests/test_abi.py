@@ -1,0 +1,128 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+header declares, names its status codes, and rejects bad arguments before
+touching CUDA.  No compute call runs here."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import attn_fwd_04_b200 as fa
+from attn_fwd_04_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    fa_build.build()
+    return fa.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]*?\b(fa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(fa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    codes = [fa.FA_OK, fa.FA_ERR_NULL, fa.FA_ERR_SHAPE, fa.FA_ERR_UNSUPPORTED, fa.FA_ERR_ALIGN,
+             fa.FA_ERR_CUDA, fa.FA_ERR_DEVICE_TIMEOUT, fa.FA_ERR_NOMEM, fa.FA_ERR_DEVICE_BAD_INPUT]
+    names = [fa.fa_status_str(c) for c in codes]
+    assert names[0] == "FA_OK"
+    assert len(set(names)) == len(names)
+    assert fa.fa_status_str(12345) == "unknown fa status"
+    assert fa.fa_version() == 100
+
+
+# Fake, never-dereferenced device addresses: validation rejects the calls
+# before any CUDA call is made.
+A = 1 << 20          # 16-byte aligned
+MIS = A + 8          # not 16-byte aligned
+S = None             # default stream
+
+
+def fwd(L, q=A, k=A, v=A, o=A, lse=A, B=1, H=2, N=256, d=64, causal=0, scale=0.125):
+    return L.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, S)
+
+
+def varlen(L, q=A, k=A, v=A, o=A, lse=A, cu=A, B=2, H=2, total=100, maxlen=60, d=128,
+           causal=1, scale=0.1):
+    return L.fa_fwd_varlen(q, k, v, o, lse, cu, B, H, total, maxlen, d, causal, scale, S)
+
+
+def decode(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=2, d=128, ps=256):
+    return L.fa_decode_paged(q, kp, vp, pt, sl, o, B, H, d, ps, S)
+
+
+def gather(L, pages=A, pt=A, sl=A, out=A, B=4, H=2, d=128, ps=256):
+    return L.fa_gather_paged(pages, pt, sl, out, B, H, d, ps, S)
+
+
+def test_fwd_argument_errors(L):
+    assert fwd(L, q=None) == fa.FA_ERR_NULL
+    assert fwd(L, lse=None) == fa.FA_ERR_NULL
+    assert fwd(L, N=0) == fa.FA_ERR_SHAPE
+    assert fwd(L, B=0) == fa.FA_ERR_SHAPE
+    assert fwd(L, H=-1) == fa.FA_ERR_SHAPE
+    assert fwd(L, B=256, H=256) == fa.FA_ERR_SHAPE       # B*H > 65535
+    assert fwd(L, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert fwd(L, d=256) == fa.FA_ERR_UNSUPPORTED
+    assert fwd(L, scale=float("nan")) == fa.FA_ERR_SHAPE
+    assert fwd(L, scale=float("inf")) == fa.FA_ERR_SHAPE
+    assert fwd(L, k=MIS) == fa.FA_ERR_ALIGN
+    assert fwd(L, o=MIS) == fa.FA_ERR_ALIGN
+
+
+def test_varlen_argument_errors(L):
+    assert varlen(L, cu=None) == fa.FA_ERR_NULL
+    assert varlen(L, total=0) == fa.FA_ERR_SHAPE
+    assert varlen(L, maxlen=0) == fa.FA_ERR_SHAPE
+    assert varlen(L, d=32) == fa.FA_ERR_UNSUPPORTED
+    assert varlen(L, v=MIS) == fa.FA_ERR_ALIGN
+
+
+def test_decode_argument_errors(L):
+    assert decode(L, pt=None) == fa.FA_ERR_NULL
+    assert decode(L, sl=None) == fa.FA_ERR_NULL
+    assert decode(L, B=0) == fa.FA_ERR_SHAPE
+    assert decode(L, ps=128) == fa.FA_ERR_UNSUPPORTED
+    assert decode(L, ps=16) == fa.FA_ERR_UNSUPPORTED
+    assert decode(L, d=80) == fa.FA_ERR_UNSUPPORTED
+    assert decode(L, kp=MIS) == fa.FA_ERR_ALIGN
+    assert gather(L, out=None) == fa.FA_ERR_NULL
+    assert gather(L, ps=255) == fa.FA_ERR_UNSUPPORTED
+    assert gather(L, pages=MIS) == fa.FA_ERR_ALIGN
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_call_without_gpu_reports_cuda_error(L):
+    # arguments pass validation; the device lookup then fails cleanly
+    assert fwd(L) == fa.FA_ERR_CUDA
+    assert decode(L) == fa.FA_ERR_CUDA
+    code = ctypes.c_int(7)
+    assert L.fa_get_device_error(ctypes.byref(code), S) == fa.FA_ERR_CUDA
+
+
+def test_binding_refuses_cpu_tensors():
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        fa.fa_fwd(x, x, x, causal=False)
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    from attn_fwd_04_b200 import fa as binding
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", "/nonexistent/libfa.so")
+    with pytest.raises(ImportError):
+        binding.lib()

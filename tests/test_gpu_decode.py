@@ -1,0 +1,172 @@
+"""GPU parity of paged decode (fa_decode_paged) and of the paged gather
+(fa_gather_paged) against the fp64 CPU oracle, through the C ABI.
+
+The gather is integer/byte work and must match the oracle's gather bit for
+bit.  Decode is compared within the floating-point tolerances, element by
+element on small caches and on sampled sequences of the full-size workload.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import attn_fwd_04_b200 as fa
+import oracle
+from attn_fwd_04_b200 import workloads as W
+from helpers import assert_lse_close, assert_o_close, to64
+
+pytestmark = pytest.mark.gpu
+
+PS = 256
+
+
+def _on_gpu(c: W.PagedCache) -> W.PagedCache:
+    return W.PagedCache(c.q.cuda(), c.k_pages.cuda(), c.v_pages.cuda(), c.page_table.cuda(),
+                        c.seq_lens.cuda(), c.page_size, c.pages_per_seq)
+
+
+def _decode(c: W.PagedCache):
+    o = torch.full_like(c.q, float("nan"))
+    fa.fa_decode_paged(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, c.page_size, o=o)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return o
+
+
+def _mini(c: W.PagedCache, b: int):
+    """Sequence b alone: its pages (in table order) as a small pool, with the
+    identity page table -- so the oracle can gather and decode it on the host."""
+    off = sum(c.pages_per_seq[:b])
+    n = c.pages_per_seq[b]
+    idx = c.page_table[off:off + n].long()
+    kp = c.k_pages.index_select(0, idx.to(c.k_pages.device)).cpu()
+    vp = c.v_pages.index_select(0, idx.to(c.v_pages.device)).cpu()
+    return kp, vp, torch.arange(n, dtype=torch.int32), c.seq_lens[b:b + 1].cpu()
+
+
+LENS_SMALL = [1, 2, 255, 256, 257, 511, 512, 513, 1000, 4103]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_gather_bit_exact_small(d):
+    c = W.paged_inputs(len(LENS_SMALL) + 1, 3, d, LENS_SMALL + [0], seed=21, device="cpu")
+    g = _on_gpu(c)
+    total = int(c.seq_lens.sum())
+    out = torch.full((total, 3, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    fa.fa_gather_paged(g.k_pages, g.page_table, g.seq_lens, total, PS, out=out)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    ref = oracle.gather_paged(c.k_pages, c.page_table, c.seq_lens, PS)
+    ref_bf16 = torch.from_numpy(ref).to(torch.bfloat16)  # exact: values are bf16
+    assert torch.equal(out.cpu().view(torch.int16), ref_bf16.view(torch.int16))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_small_full_compare(d):
+    c = W.paged_inputs(len(LENS_SMALL), 4, d, LENS_SMALL, seed=22, device="cpu")
+    o = _decode(_on_gpu(c))
+    o_ref, _ = oracle.decode_paged(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
+    assert_o_close(to64(o), o_ref, f"decode d={d}")
+
+
+def test_decode_long_sequence_bigger_splits():
+    # more pages than splits x chunk: each split covers more than the minimum
+    lens = [256 * 130 + 17, 300]
+    c = W.paged_inputs(2, 2, 128, lens, seed=23, device="cpu")
+    o = _decode(_on_gpu(c))
+    o_ref, _ = oracle.decode_paged(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
+    assert_o_close(to64(o), o_ref, "long decode")
+
+
+def test_decode_empty_sequence_is_zero():
+    c = W.paged_inputs(3, 2, 128, [0, 700, 0], seed=24, device="cpu")
+    o = _decode(_on_gpu(c))
+    assert torch.all(o[0] == 0) and torch.all(o[2] == 0)
+    o_ref, _ = oracle.decode_paged(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
+    assert_o_close(to64(o[1]), o_ref[1], "middle sequence")
+
+
+def test_decode_negative_length_reported():
+    c = W.paged_inputs(2, 2, 64, [300, 5], seed=25, device="cpu")
+    g = _on_gpu(c)
+    bad = torch.tensor([300, -5], dtype=torch.int32, device="cuda")
+    o = torch.full_like(g.q, float("nan"))
+    fa.fa_decode_paged(g.q, g.k_pages, g.v_pages, g.page_table, bad, PS, o=o)
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_BAD_INPUT
+    assert torch.all(o[1] == 0)
+    o_ref, _ = oracle.decode_paged(c.q[:1], c.k_pages, c.v_pages, c.page_table, c.seq_lens[:1], PS)
+    assert_o_close(to64(o[0:1]), o_ref, "valid sequence")
+
+
+def test_decode_deterministic_and_pool_order_invariant():
+    lens = [3000, 77, 1025]
+    H, d = 4, 128
+    c = W.paged_inputs(3, H, d, lens, seed=26, device="cpu", poison_unused=False)
+    g = _on_gpu(c)
+    o1 = _decode(g)
+    o2 = _decode(g)
+    assert torch.equal(o1, o2)
+    # move every page to another pool slot; same content through the table
+    P = c.k_pages.shape[0]
+    perm = torch.randperm(P, generator=torch.Generator().manual_seed(27))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(P)
+    k2 = c.k_pages[perm].contiguous()   # new slot s holds old page perm[s]
+    v2 = c.v_pages[perm].contiguous()
+    pt2 = inv[c.page_table.long()].to(torch.int32)
+    g2 = W.PagedCache(g.q, k2.cuda(), v2.cuda(), pt2.cuda(), g.seq_lens, PS, c.pages_per_seq)
+    o3 = _decode(g2)
+    assert torch.equal(o1, o3)
+
+
+def test_decode_equals_last_causal_row_of_fwd():
+    """Decode of a sequence's last token equals the last row of the causal
+    forward pass over the same keys, gathered into contiguous memory."""
+    H, d, L = 4, 128, 1500
+    c = W.paged_inputs(1, H, d, [L], seed=28, device="cpu")
+    g = _on_gpu(c)
+    kc = fa.fa_gather_paged(g.k_pages, g.page_table, g.seq_lens, L, PS)  # [L,H,d]
+    vc = fa.fa_gather_paged(g.v_pages, g.page_table, g.seq_lens, L, PS)
+    qf = torch.randn((1, H, L, d), generator=torch.Generator().manual_seed(29)).to(torch.bfloat16).cuda()
+    qf[0, :, L - 1] = g.q[0]
+    kf = kc.permute(1, 0, 2).contiguous()[None]
+    vf = vc.permute(1, 0, 2).contiguous()[None]
+    of, _ = fa.fa_fwd(qf, kf, vf, True, 1 / math.sqrt(d))
+    od = _decode(g)
+    # both are within tolerance of the oracle, so within 2x of each other
+    diff = (of[0, :, L - 1].float() - od[0].float()).abs().max().item()
+    assert diff <= 4e-2
+
+
+def test_paged_decode_workload_sampled():
+    w = W.PAGED_DECODE
+    c = W.decode_workload_inputs(w, device="cuda")
+    c = W.PagedCache(c.q, c.k_pages, c.v_pages, c.page_table.cuda(), c.seq_lens.cuda(),
+                     c.page_size, c.pages_per_seq)
+    o = _decode(c)
+    assert bool(torch.isfinite(o).all())
+    lens = c.seq_lens.cpu().tolist()
+    order = sorted(range(w.B), key=lambda b: lens[b])
+    picks = sorted({order[0], order[-1], order[w.B // 2], 0, w.B - 1, 17})
+    got, ref = [], []
+    for b in picks:
+        kp, vp, pt, sl = _mini(c, b)
+        o_ref, _ = oracle.decode_paged(c.q[b:b + 1].cpu(), kp, vp, pt, sl, PS)
+        got.append(to64(o[b:b + 1]))
+        ref.append(o_ref)
+    assert_o_close(np.concatenate(got), np.concatenate(ref), w.name)
+
+
+def test_paged_gather_workload_sampled_bit_exact():
+    w = W.PAGED_DECODE
+    c = W.decode_workload_inputs(w, device="cuda")
+    pt, sl = c.page_table.cuda(), c.seq_lens.cuda()
+    total = int(c.seq_lens.sum())
+    out = fa.fa_gather_paged(c.k_pages, pt, sl, total, PS)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    starts = np.concatenate([[0], np.cumsum(c.seq_lens.numpy())])
+    for b in (0, 31, w.B - 1):
+        kp, _, ptb, slb = _mini(c, b)
+        ref = oracle.gather_paged(kp, ptb, slb, PS)
+        got = out[int(starts[b]):int(starts[b + 1])].cpu()
+        assert torch.equal(got.view(torch.int16),
+                           torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16))

@@ -1,0 +1,223 @@
+"""GPU parity of the fused forward pass (fa_fwd, fa_fwd_varlen) against the
+fp64 CPU oracle, through the C ABI.
+
+Small shapes are compared element by element over every output; the
+full-size workloads (long prefill, batched prefill, varlen, 128K context) run
+the same launch the benchmark times and are compared on sampled query rows
+the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import attn_fwd_04_b200 as fa
+import oracle
+from attn_fwd_04_b200 import workloads as W
+from helpers import assert_lse_close, assert_o_close, sample_rows, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd_gpu(q, k, v, causal, scale):
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    B, H, N, d = q.shape
+    o = torch.full_like(qc, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda")
+    fa.fa_fwd(qc, kc, vc, causal, scale, o=o, lse=lse)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_workload(causal):
+    w = W.TINY_CAUSAL if causal else W.TINY
+    q, k, v, _fp32 = W.fwd_inputs(w, device="cpu")
+    scale = 1 / math.sqrt(w.d)
+    o, lse = _fwd_gpu(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention(q, k, v, causal, scale)
+    assert_o_close(to64(o), o_ref, w.name)
+    assert_lse_close(to64(lse), lse_ref, w.name)
+
+
+SHAPES = [(1, 1, 1, 64), (1, 1, 1, 128), (1, 2, 127, 128), (2, 3, 129, 64), (1, 2, 255, 128),
+          (1, 1, 1000, 128), (2, 2, 384, 64), (1, 4, 1024, 128), (1, 2, 2049, 64)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_shapes_full_compare(shape, causal):
+    B, H, N, d = shape
+    q, k, v = W.custom_fwd_inputs(B, H, N, d, seed=100 + N + d)
+    scale = 1 / math.sqrt(d)
+    o, lse = _fwd_gpu(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention(q, k, v, causal, scale)
+    assert_o_close(to64(o), o_ref, str(shape))
+    assert_lse_close(to64(lse), lse_ref, str(shape))
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.3, -0.1])
+def test_other_scales(scale):
+    q, k, v = W.custom_fwd_inputs(1, 2, 300, 128, seed=7)
+    for causal in (False, True):
+        o, lse = _fwd_gpu(q, k, v, causal, scale)
+        o_ref, lse_ref = oracle.attention(q, k, v, causal, scale)
+        assert_o_close(to64(o), o_ref, f"scale {scale}")
+        assert_lse_close(to64(lse), lse_ref, f"scale {scale}")
+
+
+def test_large_magnitude_scores_stay_finite():
+    # scores up to ~+-200: the running max must be subtracted before exp
+    q, k, v = W.custom_fwd_inputs(1, 1, 512, 64, seed=8, std=4.0)
+    o, lse = _fwd_gpu(q, k, v, True, 1.0)
+    o_ref, lse_ref = oracle.attention(q, k, v, True, 1.0)
+    assert_o_close(to64(o), o_ref, "large scores")
+    # lse magnitudes are in the hundreds here; compare relative to them
+    np.testing.assert_allclose(to64(lse), lse_ref, rtol=2e-6, atol=1e-3)
+
+
+def test_deterministic():
+    q, k, v = W.custom_fwd_inputs(1, 3, 700, 128, seed=9)
+    o1, l1 = _fwd_gpu(q, k, v, True, 0.1)
+    o2, l2 = _fwd_gpu(q, k, v, True, 0.1)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def _sampled_parity(q, k, v, causal, scale, o, lse, rows_per_head, seed):
+    """Oracle on sampled rows, one head at a time (keeps host memory small)."""
+    B, H, N, d = q.shape
+    g = torch.Generator().manual_seed(seed)
+    pairs = [(int(b), int(h)) for b, h in zip(torch.randint(0, B, (8,), generator=g),
+                                             torch.randint(0, H, (8,), generator=g))]
+    pairs = sorted(set(pairs) | {(0, 0), (B - 1, H - 1)})
+    got_o, ref_o, got_l, ref_l = [], [], [], []
+    for (b, h) in pairs:
+        rows = sample_rows(N, rows_per_head, seed + 31 * b + h)
+        qh, kh, vh = q[b, h][None, None], k[b, h][None, None], v[b, h][None, None]
+        o_ref, lse_ref = oracle.attention(qh, kh, vh, causal, scale, rows=rows)
+        got_o.append(to64(o[b, h, rows]))
+        ref_o.append(o_ref[0, 0, rows])
+        got_l.append(to64(lse[b, h, rows]))
+        ref_l.append(lse_ref[0, 0, rows])
+    assert_o_close(np.concatenate(got_o), np.concatenate(ref_o), "sampled")
+    assert_lse_close(np.concatenate(got_l), np.concatenate(ref_l), "sampled")
+
+
+@pytest.mark.parametrize("w", [W.LONG_PREFILL, W.BATCHED], ids=lambda w: w.name)
+def test_full_size_sampled(w):
+    q, k, v = W.fwd_inputs(w, device="cuda")
+    scale = 1 / math.sqrt(w.d)
+    o, lse = fa.fa_fwd(q, k, v, w.causal, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(lse).all())
+    _sampled_parity(q.cpu(), k.cpu(), v.cpu(), w.causal, scale, o.cpu(), lse.cpu(), 24, w.seed)
+
+
+def test_ctx128k_sampled():
+    """128K context: 256 query rows in total, seeded, across heads (the first
+    and last row of head 0 always included); K/V of each head copied to the
+    host one at a time."""
+    w = W.CTX128K
+    q, k, v = W.fwd_inputs(w, device="cuda")
+    scale = 1 / math.sqrt(w.d)
+    o, lse = fa.fa_fwd(q, k, v, w.causal, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    g = torch.Generator().manual_seed(4)
+    hs = torch.randint(0, w.H, (254,), generator=g).tolist()
+    rs = torch.randint(0, w.N, (254,), generator=g).tolist()
+    picks = {}
+    for h, r in [(0, 0), (0, w.N - 1)] + list(zip(hs, rs)):
+        picks.setdefault(h, set()).add(r)
+    got_o, ref_o, got_l, ref_l = [], [], [], []
+    for h, rows in sorted(picks.items()):
+        rows = sorted(rows)
+        qh, kh, vh = q[0, h].cpu(), k[0, h].cpu(), v[0, h].cpu()
+        o_ref, lse_ref = oracle.attention(qh[None, None], kh[None, None], vh[None, None],
+                                          True, scale, rows=rows)
+        got_o.append(to64(o[0, h, rows]))
+        ref_o.append(o_ref[0, 0, rows])
+        got_l.append(to64(lse[0, h, rows]))
+        ref_l.append(lse_ref[0, 0, rows])
+    assert_o_close(np.concatenate(got_o), np.concatenate(ref_o), w.name)
+    assert_lse_close(np.concatenate(got_l), np.concatenate(ref_l), w.name)
+
+
+# -- variable length -----------------------------------------------------------
+
+def _varlen_gpu(q, k, v, cu, maxlen, causal, scale):
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    total, H, d = q.shape
+    o = torch.full_like(qc, float("nan"))
+    lse = torch.full((H, total), float("nan"), device="cuda")
+    fa.fa_fwd_varlen(qc, kc, vc, cu.cuda(), maxlen, causal, scale, o=o, lse=lse)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_small_full_compare(d, causal):
+    lens = [1, 127, 128, 129, 300, 5, 256]
+    q, k, v, cu = W.varlen_inputs(3, d, lens, seed=11)
+    scale = 1 / math.sqrt(d)
+    o, lse = _varlen_gpu(q, k, v, cu, max(lens), causal, scale)
+    o_ref, lse_ref = oracle.attention_varlen(q, k, v, cu, causal, scale)
+    assert_o_close(to64(o), o_ref, f"varlen d={d}")
+    assert_lse_close(to64(lse), lse_ref, f"varlen d={d}")
+
+
+def test_varlen_equals_fixed_per_sequence():
+    """Each packed sequence gives bit-identical results to a fixed-length call
+    on that sequence alone (same tiles, same arithmetic)."""
+    lens = [200, 64, 513]
+    H, d = 2, 128
+    q, k, v, cu = W.varlen_inputs(H, d, lens, seed=12)
+    o, lse = _varlen_gpu(q, k, v, cu, max(lens), True, 0.125)
+    for b, L in enumerate(lens):
+        s0 = int(cu[b])
+        sl = slice(s0, s0 + L)
+        qf = q[sl].permute(1, 0, 2).contiguous()[None]
+        kf = k[sl].permute(1, 0, 2).contiguous()[None]
+        vf = v[sl].permute(1, 0, 2).contiguous()[None]
+        of, lf = _fwd_gpu(qf, kf, vf, True, 0.125)
+        assert torch.equal(of[0].permute(1, 0, 2), o[sl])
+        assert torch.equal(lf[0], lse[:, sl])
+
+
+def test_varlen_workload_sampled():
+    w = W.BATCHED_VARLEN
+    q, k, v, cu = W.varlen_workload_inputs(w, device="cuda")
+    lens = (cu[1:] - cu[:-1]).tolist()
+    scale = 1 / math.sqrt(w.d)
+    o, lse = fa.fa_fwd_varlen(q, k, v, cu.cuda(), max(lens), w.causal, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    total = q.shape[0]
+    g = torch.Generator().manual_seed(w.seed)
+    rows = []
+    for b, L in enumerate(lens):
+        s0 = int(cu[b])
+        for r in {0, L - 1, min(127, L - 1), min(128, L - 1)} | set(torch.randint(0, L, (6,), generator=g).tolist()):
+            h = int(torch.randint(0, w.H, (1,), generator=g))
+            rows.append(h * total + s0 + r)
+    rows = sorted(set(rows))
+    o_ref, lse_ref = oracle.attention_varlen(q.cpu(), k.cpu(), v.cpu(), cu, True, scale, rows=rows)
+    hs = [r // total for r in rows]
+    gs = [r % total for r in rows]
+    oc, lc = o.cpu(), lse.cpu()
+    assert_o_close(np.stack([to64(oc[g_, h_]) for h_, g_ in zip(hs, gs)]),
+                   np.stack([o_ref[g_, h_] for h_, g_ in zip(hs, gs)]), w.name)
+    assert_lse_close(np.array([float(lc[h_, g_]) for h_, g_ in zip(hs, gs)]),
+                     np.array([lse_ref[h_, g_] for h_, g_ in zip(hs, gs)]), w.name)
+
+
+def test_bounded_wait_reports_timeout():
+    assert fa.fa_get_device_error() == fa.FA_OK
+    fa.fa_selftest_bounded_wait()
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_TIMEOUT
+    assert fa.fa_get_device_error() == fa.FA_OK  # read clears it
+    # the context is still usable afterwards
+    q, k, v = W.custom_fwd_inputs(1, 1, 130, 64, seed=13)
+    o, lse = _fwd_gpu(q, k, v, True, 0.125)
+    o_ref, lse_ref = oracle.attention(q, k, v, True, 0.125)
+    assert_o_close(to64(o), o_ref, "after timeout")
