@@ -68,8 +68,10 @@ def test_other_scales(scale):
 
 
 def test_large_magnitude_scores_stay_finite():
-    # scores up to ~+-200: the running max must be subtracted before exp
-    q, k, v = W.custom_fwd_inputs(1, 1, 512, 64, seed=8, std=4.0)
+    # scores up to ~+-200: the running max must be subtracted before exp.
+    # V stays unit-scale so the absolute O tolerance keeps its meaning.
+    q, k, _ = W.custom_fwd_inputs(1, 1, 512, 64, seed=8, std=4.0)
+    _, _, v = W.custom_fwd_inputs(1, 1, 512, 64, seed=18)
     o, lse = _fwd_gpu(q, k, v, True, 1.0)
     o_ref, lse_ref = oracle.attention(q, k, v, True, 1.0)
     assert_o_close(to64(o), o_ref, "large scores")
