@@ -1,0 +1,511 @@
+"""Benchmark of the attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic
+input: the fused causal forward pass on the long-prefill workload
+(B=1, H=32, N=16384, d=128, bf16) followed by paged decode on the
+paged-decode workload (64 sequences, H=32, d=128, KV lengths uniform in
+[1024, 32768], 256-token pages).  Inputs are resident in HBM before the timed
+region; both working sets are larger than the 126 MB L2 (384 MB and ~17.7 GB),
+so no flush runs between steps.
+
+Printed: one JSON line (rank 0).  `value` is forward TFLOP/s (FLOPs counted as
+4*B*H*N^2*d, halved for causal) from CUDA events around the forward launches;
+`decode` carries the paged-decode GB/s (algorithmic K/V + q + o + table bytes).
+With N GPUs (torchrun, one process per GPU) every rank runs an independent
+replica of the step ("replicas only": the path has no exchange step); times
+are the max over ranks and `value` counts the work of all ranks.
+
+--impl reference times the fp64 CPU oracle as it stands, on a bounded sample
+of the same workload, on this machine's host cores (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from attn_fwd_04_b200 import workloads as W  # noqa: E402
+
+METRIC = "attn fwd TFLOPS & % of BF16 tensor peak; paged-decode HBM GB/s (1×B200)"
+FWD = W.LONG_PREFILL
+DEC = W.PAGED_DECODE
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# helpers shared by both arms
+# ---------------------------------------------------------------------------
+def fwd_flops(w=FWD) -> float:
+    f = 4.0 * w.B * w.H * w.N * w.N * w.d
+    return f / 2 if w.causal else f
+
+
+def decode_bytes(seq_lens, H, d, B) -> float:
+    """Algorithmic bytes of one decode launch: every cached K and V element
+    once, q and o, the page table and the lengths."""
+    tokens = float(sum(int(x) for x in seq_lens))
+    pages = float(sum((int(x) + 255) // 256 for x in seq_lens))
+    return tokens * H * d * 2 * 2 + 2 * B * H * d * 2 + pages * 4 + B * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        d = dict(FALLBACK_PEAKS)
+        d["source"] = "fallback"
+        return d
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "attn_fwd_04_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, sha: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic_per_launch.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        parts = dict(x.split("=", 1) for x in line.split() if "=" in x)
+        if parts.get("kernel") == kernel and parts.get("src_sha") == sha:
+            try:
+                return float(parts["dram_bytes"])
+            except (KeyError, ValueError):
+                return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def reduce_max(values, world):
+    """Element-wise max of a list of floats over ranks."""
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle samples (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_fwd_sample(q, k, v, target_s: float, seed: int, n_heads: int = 2):
+    """Time the oracle on seeded random query rows of the forward workload,
+    growing the sample until it has run about target_s seconds.  Rows come
+    from `n_heads` seeded heads, converted to fp64 once outside the timing.
+    Returns (TFLOP/s under the workload's FLOP convention, rows, seconds)."""
+    import numpy as np
+
+    import oracle
+    B, H, N, d = q.shape
+    scale = 1 / math.sqrt(d)
+    g = torch.Generator().manual_seed(seed)
+    heads = torch.randperm(H, generator=g)[:n_heads].tolist()
+    f64 = {h: tuple(np.ascontiguousarray(t[0, h].double().cpu().numpy())[None, None]
+                    for t in (q, k, v)) for h in heads}
+    per_row = (4.0 * N * d) / (2 if FWD.causal else 1)
+    done_rows, spent, count = 0, 0.0, 32
+    while spent < target_s:
+        for h in heads:
+            rows = sorted(set(torch.randint(0, N, (count,), generator=g).tolist()))
+            qh, kh, vh = f64[h]
+            t0 = time.perf_counter()
+            oracle.attention(qh, kh, vh, FWD.causal, scale, rows=rows)
+            spent += time.perf_counter() - t0
+            done_rows += len(rows)
+        count = min(count * 2, 4096)
+    return per_row * done_rows / spent / 1e12, done_rows, spent
+
+
+def oracle_decode_sample(cache: W.PagedCache, target_s: float):
+    """Time the oracle's paged decode on whole sequences of the decode
+    workload (shortest first) for about target_s seconds -> GB/s."""
+    import oracle
+    lens = cache.seq_lens.tolist()
+    order = sorted(range(len(lens)), key=lambda b: lens[b])
+    H, d = cache.q.shape[1], cache.q.shape[2]
+    spent, nbytes, seqs = 0.0, 0.0, 0
+    for b in order:
+        off = sum(cache.pages_per_seq[:b])
+        n = cache.pages_per_seq[b]
+        idx = cache.page_table[off:off + n].long().to(cache.k_pages.device)
+        kp = cache.k_pages.index_select(0, idx).cpu()
+        vp = cache.v_pages.index_select(0, idx).cpu()
+        t0 = time.perf_counter()
+        oracle.decode_paged(cache.q[b:b + 1].cpu(), kp, vp, torch.arange(n, dtype=torch.int32),
+                            cache.seq_lens[b:b + 1].cpu(), cache.page_size)
+        spent += time.perf_counter() - t0
+        nbytes += decode_bytes([lens[b]], H, d, 1)
+        seqs += 1
+        if spent >= target_s:
+            break
+    return nbytes / spent / 1e9, seqs, spent
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+def decode_cache(batch: int) -> W.PagedCache:
+    if batch >= DEC.B:
+        return W.decode_workload_inputs(DEC, device="cuda")
+    lengths = W.varlen_lengths(DEC.B, DEC.len_lo, DEC.len_hi, DEC.seed)[:batch]
+    return W.paged_inputs(batch, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda")
+
+
+def run_native(args, world, rank, local):
+    import attn_fwd_04_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+    do_fwd = args.only in ("all", "fwd")
+    do_dec = args.only in ("all", "decode")
+
+    scale = 1 / math.sqrt(FWD.d)
+    if do_fwd:
+        q, k, v = W.fwd_inputs(FWD, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty((FWD.B, FWD.H, FWD.N), dtype=torch.float32, device=dev)
+    if do_dec:
+        cache = decode_cache(args.decode_batch)
+        dpt, dsl = cache.page_table.to(dev), cache.seq_lens.to(dev)
+        do = torch.empty_like(cache.q)
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        if do_fwd:
+            fa.fa_fwd(q, k, v, FWD.causal, scale, o=o, lse=lse, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if do_dec:
+            fa.fa_decode_paged(cache.q, cache.k_pages, cache.v_pages, dpt, dsl, DEC.page_size,
+                               o=do, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("device error during the timed steps")
+
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_sum, dec_sum, total_ms = reduce_max([sum(fwd_ms), sum(dec_ms), total_ms], world)
+
+    flops = fwd_flops()
+    fwd_tflops = world * flops * args.steps / (fwd_sum * 1e-3) / 1e12 if do_fwd else None
+    per_launch_tf = flops / (fwd_sum / args.steps * 1e-3) / 1e12 if do_fwd else None
+    if do_dec:
+        dbytes = decode_bytes(cache.seq_lens.tolist(), DEC.H, DEC.d, cache.q.shape[0])
+        dec_gbs = world * dbytes * args.steps / (dec_sum * 1e-3) / 1e9
+        per_launch_gbs = dbytes / (dec_sum / args.steps * 1e-3) / 1e9
+
+    # ---- end to end through the public API, host buffers ------------------
+    e2e = None
+    if do_fwd and not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 5))
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            dq2.copy_(hq, non_blocking=True)
+            dk2.copy_(hk, non_blocking=True)
+            dv2.copy_(hv, non_blocking=True)
+            fa.fa_fwd(dq2, dk2, dv2, FWD.causal, scale, o=o, lse=lse, stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        (e2e_ms,) = reduce_max([e0.elapsed_time(e1)], world)
+        e2e = {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
+               "steps": e2e_steps,
+               "what": "fa_fwd through the Python binding, q/k/v copied from pinned host "
+                       "memory and o/lse copied back inside the timed region"}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and do_fwd:
+        import oracle
+        tf, rows, secs = oracle_fwd_sample(q, k, v, args.cpu_seconds, seed=2)
+        cpu_baseline = {"value": tf, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                        "kind": "oracle",
+                        "sample": f"{rows} seeded random query rows of two seeded heads of the "
+                                  f"long-prefill workload, {secs:.1f} s, FLOPs counted like "
+                                  f"the GPU number (2*N*d per causal row)"}
+        if do_dec:
+            gbs, seqs, dsecs = oracle_decode_sample(cache, args.cpu_seconds / 2)
+            cpu_baseline["decode"] = {"value": gbs, "unit": "GB/s",
+                                      "sample": f"{seqs} whole sequences (shortest first) of "
+                                                f"the paged-decode workload, {dsecs:.1f} s"}
+
+    if rank != 0:
+        return None
+    fwd_sha = kernel_source_sha(["fwd_sm100.cu", "fa_ptx.cuh"])
+    dec_sha = kernel_source_sha(["decode_sm100.cu", "fa_ptx.cuh"])
+    peak_tf = peaks["bf16_tflops"]
+    out = {
+        "metric": METRIC,
+        "value": fwd_tflops if do_fwd else dec_gbs,
+        "unit": "TFLOP/s" if do_fwd else "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded torch.randn, N(0,1) bf16; lengths uniform; shuffled page pool)",
+        "config": {
+            "workload": " + ".join(([FWD.name] if do_fwd else []) + ([DEC.name] if do_dec else [])),
+            "l2": "inputs larger than L2 (fwd 384 MiB, decode ~17.7 GB); no flush",
+            "parallelism": f"replicas x{world}",
+        },
+        "gpu_launches": args.steps * ((1 if do_fwd else 0) + (3 if do_dec else 0)),
+        "clocks": clocks,
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+    }
+    if do_fwd:
+        out["config"]["fwd"] = {"B": FWD.B, "H": FWD.H, "N": FWD.N, "d": FWD.d,
+                                "causal": FWD.causal, "scale": scale, "seed": FWD.seed}
+        out["pct_of_bf16_peak"] = {
+            "datasheet_2250": 100 * per_launch_tf / DATASHEET_BF16_TFLOPS,
+            "measured_burst": 100 * per_launch_tf / peak_tf,
+            "measured_sustained": 100 * per_launch_tf / peaks["bf16_tflops_sustained"]}
+        out["fwd_ms_per_launch"] = fwd_sum / args.steps
+        out["roofline"] = {"bound": "tensor", "kernel": "fa_fwd_kernel", "achieved": per_launch_tf,
+                           "peak": peak_tf, "unit": "TFLOP/s", "frac": per_launch_tf / peak_tf,
+                           "peak_source": f"{peaks['source']} bf16 burst",
+                           "traffic": recorded_traffic("fa_fwd_kernel", fwd_sha),
+                           "algorithmic_flops_per_launch": flops}
+    if do_dec:
+        out["config"]["decode"] = {"B": int(cache.q.shape[0]), "H": DEC.H, "d": DEC.d,
+                                   "page_size": DEC.page_size,
+                                   "len_range": [DEC.len_lo, DEC.len_hi], "seed": DEC.seed,
+                                   "tokens": int(cache.seq_lens.sum())}
+        out["decode"] = {"value": dec_gbs, "unit": "GB/s", "ms_per_launch": dec_sum / args.steps,
+                         "bytes_per_launch": dbytes,
+                         "pct_of_hbm": {"datasheet_8000": 100 * per_launch_gbs / 8000.0,
+                                        "measured": 100 * per_launch_gbs / peaks["hbm_gbs"]}}
+        out["roofline_decode"] = {
+            "bound": "hbm", "kernel": "fa_decode_split_kernel (+plan, merge)",
+            "achieved": per_launch_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": per_launch_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy",
+            "traffic": recorded_traffic("fa_decode_split_kernel", dec_sha),
+            "algorithmic_bytes_per_launch": dbytes}
+    return out
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle, timed as it stands
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    # inputs on the host (the oracle is CPU code); same seeded recipe, drawn on
+    # the CPU generator so no GPU is needed for this arm
+    q, k, v = W.fwd_inputs(FWD, device="cpu")
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for i in range(args.warmup):
+        oracle_fwd_sample(q, k, v, per_step, seed=100 + i)
+    tfs, rows_total, secs_total = [], 0, 0.0
+    for i in range(args.steps):
+        tf, rows, secs = oracle_fwd_sample(q, k, v, per_step, seed=200 + i)
+        tfs.append(tf)
+        rows_total += rows
+        secs_total += secs
+    per_row = (4.0 * FWD.N * FWD.d) / (2 if FWD.causal else 1)
+    value = rows_total * per_row / secs_total / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs_total / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (same seeded recipe as the native arm, drawn on the CPU)",
+        "config": {"workload": FWD.name, "fwd": {"B": FWD.B, "H": FWD.H, "N": FWD.N, "d": FWD.d,
+                                                 "causal": FWD.causal, "seed": FWD.seed},
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows_total} seeded random query rows over {args.steps} "
+                                   f"steps of ~{per_step:.1f} s each"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time budget of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
+                    help="profiling aid: run one entry point only (the JSON line then "
+                         "reports that part alone)")
+    ap.add_argument("--decode-batch", type=int, default=DEC.B,
+                    help="profiling aid: decode over the first B sequences only")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "native":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # CPU only: rank 0 runs the oracle, any other rank exits at once
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        out = run_reference(args, world, int(os.environ.get("RANK", "0")))
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        out = run_native(args, world, rank, local)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
