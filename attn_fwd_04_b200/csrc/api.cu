@@ -124,6 +124,17 @@ int ensure_workspace(DeviceState* s, size_t bytes, cudaStream_t stream, void** o
 
 }  // namespace
 
+namespace fa {
+int device_error_word(unsigned int** err, int* num_sms) {
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    *err = s->err;
+    *num_sms = s->num_sms;
+    return FA_OK;
+}
+}  // namespace fa
+
 extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,

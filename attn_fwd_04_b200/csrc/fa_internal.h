@@ -51,6 +51,9 @@ int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   int d, int page_size, int max_splits, void* workspace, unsigned int* err,
                   int num_sms, cudaStream_t stream);
 
+// The current device's error word and SM count (sm_100 devices only).
+int device_error_word(unsigned int** err, int* num_sms);
+
 int launch_gather(const void* pages, const int32_t* page_table, const int32_t* seq_lens,
                   void* out, int B, int H, int d, int page_size, void* workspace,
                   unsigned int* err, int num_sms, cudaStream_t stream);

@@ -24,7 +24,8 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_gather_paged",
+EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_noalloc",
+           "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
            "fa_status_str", "fa_version")
 
@@ -49,6 +50,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_gather_paged.argtypes = [P, P, P, P, I, I, I, I, P]
         L.fa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
         L.fa_selftest_bounded_wait.argtypes = [P]
@@ -56,7 +58,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_gather_paged",
+        for name in ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_noalloc",
+                     "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
                      "fa_version"):
             getattr(L, name).restype = I
@@ -148,6 +151,26 @@ def fa_decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 
                                page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
                                B, H, d, int(page_size), _stream(stream))
     _raise_if(rc, "fa_decode_paged")
+    return o
+
+
+def fa_decode_paged_noalloc(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 256,
+                            o=None, stream=None):
+    """fa_decode_paged without any device allocation by the library (its scratch
+    is a fixed 16 MiB device array).  `o` should be preallocated by callers that
+    cannot allocate; it is created here only as a convenience."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, H, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    rc = lib().fa_decode_paged_noalloc(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                       page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
+                                       B, H, d, int(page_size), _stream(stream))
+    _raise_if(rc, "fa_decode_paged_noalloc")
     return o
 
 

@@ -152,6 +152,38 @@ FA_API int fa_gather_paged(const void* pages, const int32_t* page_table, const i
                     void* out, int B, int H, int d, int page_size, fa_stream_t stream);
 
 /*
+ * fa_decode_paged_noalloc -- the same decode as fa_decode_paged, for callers
+ * that must not allocate device memory (the pages have no counterpart: this
+ * is a deployment variant of the decode entry point).
+ *
+ * Who needs it: code that runs while a CUDA graph is being captured, serving
+ * loops that reserve all device memory up front, and hosts with their own
+ * device allocator that forbid other allocations cannot let the library call
+ * cudaMalloc, which fa_decode_paged does on its first call (and whenever it
+ * needs a larger workspace).
+ *
+ * Arguments, layouts and results are those of fa_decode_paged.  The scratch
+ * (split offsets and per-split partial outputs) lives in one fixed 16 MiB
+ * device array inside the library instead of a workspace; each GPU that
+ * loads the library holds it until the process exits.  Nothing is allocated
+ * and no allocating routine is called.
+ *  - Limit: the partials of at least one split per (sequence, head) must fit,
+ *    i.e. roughly 4*B*H*(d+1) bytes <= 16 MiB (B*H <= 32,000 at d = 128);
+ *    larger calls return FA_ERR_SHAPE before launching.  Within the limit the
+ *    call uses as many splits per sequence (up to fa_decode_paged's) as fit,
+ *    so its output can differ from fa_decode_paged's by rounding only.
+ *  - The first call on each GPU looks up the array's device address (with
+ *    that GPU current) and caches it; make that first call before any stream
+ *    capture.
+ *  - All calls share the array and it keeps the last call's contents (no part
+ *    of it needs to start at zero).  Calls whose kernels overlap on the GPU
+ *    race on it: order them on one stream or with events.
+ */
+FA_API int fa_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* page_table, const int32_t* seq_lens, void* o,
+                                   int B, int H, int d, int page_size, fa_stream_t stream);
+
+/*
  * fa_get_device_error -- synchronise `stream`, then read and clear the
  * current GPU's device error word.  *code receives FA_OK or the FA_ERR_*
  * value of the first fault a kernel recorded since the last read.
