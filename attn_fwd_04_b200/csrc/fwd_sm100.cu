@@ -10,64 +10,111 @@
 // last block (page at zwxr.cn, section 3.1).
 //
 // B200 mapping (not the pages' design, which targets older GPUs):
-//   * one CTA per 128-row query tile; K/V tiles of 128 keys stream through a
-//     2-stage shared-memory ring filled by TMA (128-byte swizzle);
-//   * the two products run on the 5th-generation tensor cores: S = Q K^T
-//     (both operands in shared memory) and O += P V (P read from tensor
-//     memory), with S, P and the O accumulator held in TMEM;
-//   * warp roles: warps 0-3 do the softmax (one thread per query row, scores
-//     read with tcgen05.ld), the O correction and the epilogue; warp 4 issues
-//     TMA loads; warp 5 allocates TMEM and issues the MMAs;
-//   * exp is evaluated as exp2 with scale*log2(e) folded into the scores.
+//   * one CTA per 256-row query block, processed as two 128-row tiles that
+//     share every K/V tile; K and V tiles of 128 keys stream through a 4-slot
+//     shared-memory ring filled by TMA (128-byte swizzle);
+//   * both products run on the 5th-generation tensor cores: S = Q K^T (both
+//     operands in shared memory) and O += P V (P read from tensor memory);
+//     S, P and both O accumulators live in TMEM (all 512 columns);
+//   * warp roles (512 threads): warpgroup 0 and 1 run the softmax of tile 0
+//     and tile 1 (one thread per query row); their exponential phases take
+//     turns, so one tile's softmax overlaps the other tile's MMAs; warpgroup
+//     2 rescales O when the running max
+//     grows, and writes the epilogue; in warpgroup 3, warp 12 issues the MMAs
+//     and warp 13 the TMA loads.  Registers are moved to the softmax
+//     warpgroups with setmaxnreg (2 x 192 + 80 + 48 = 4 x 128 per thread);
+//   * exp is exp2 with scale*log2(e) folded in; O is rescaled only when the
+//     running max has grown by more than 2^8 (the stale max is used for both
+//     the numerator and l, so the result is unchanged up to rounding).
 //
-// TMEM columns: S double buffer [0,128) and [128,256), O [256, 256+D),
-// P (bf16 pairs) [384, 448).
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
+// P_t (bf16 pairs) overwrites the first 64 columns of S_t; the next S_t is
+// issued behind P_t V in the same in-order MMA stream.
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "fa_ptx.cuh"
 
 namespace fa {
 namespace {
 
-constexpr int BM = 128;      // query rows per tile (MMA M)
-constexpr int BN = 128;      // keys per K/V tile (MMA N of Q K^T, K of P V)
-constexpr int kStages = 2;   // K/V ring depth
-constexpr int kThreads = 192;
+constexpr int BM = 128;       // query rows per tile (MMA M)
+constexpr int BN = 128;       // keys per K/V tile
+constexpr int kSlots = 4;     // K/V ring slots (each holds one K or one V tile)
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }  // O_t
 constexpr int kBoxBytes = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16
+constexpr float kRescaleLog2 = 8.0f;     // rescale O when the max grows by > 2^8
 
 template <int D>
 struct alignas(1024) FwdSmem {
-    uint8_t q[BM * D * 2];
-    uint8_t k[kStages][BN * D * 2];
-    uint8_t v[kStages][BN * D * 2];
-    uint64_t bar_q;
-    uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], s_free[2];
-    uint64_t p_full, pv_done, drain;
+    uint8_t q[2][BM * D * 2];
+    uint8_t kv[kSlots][BN * D * 2];
+    float alpha[2][BM];   // per-row O correction factor of the current step
+    float row_m[2][BM];   // final running max (log2 domain) per row
+    float row_l[2][BM];   // final normaliser per row
+    uint64_t q_full[2];
+    uint64_t kv_full[kSlots], kv_empty[kSlots];
+    uint64_t s_full[2], p_full[2], a_full[2], o_ready[2], pv_done[2], stats_full[2];
+    uint64_t turn[2];  // exp phases of the two softmax warpgroups take turns
+    uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
 
-// All lanes wait; the warp proceeds only if every lane saw the phase.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
                                           volatile int* abort) {
     bool ok = mbar_wait(bar, parity, err, FA_DEVERR_TIMEOUT, abort);
     return __all_sync(0xffffffffu, ok);
 }
 
+// K/V ring position of tile j's K (v = 0) or V (v = 1)
+__device__ __forceinline__ int ring_slot(int j, int v) { return (2 * j + v) % kSlots; }
+__device__ __forceinline__ uint32_t ring_phase(int j, int v) { return ((2 * j + v) / kSlots) & 1; }
+
+// Max (or, for a negative scale, min) of the 128 raw scores of a row.
+__device__ __forceinline__ float row_extreme(const uint32_t (&s)[BN], bool neg) {
+    float a[43];
+    if (!neg) {
+#pragma unroll
+        for (int i = 0; i < 42; ++i)
+            a[i] = max3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]),
+                         __uint_as_float(s[3 * i + 2]));
+        a[42] = fmaxf(__uint_as_float(s[126]), __uint_as_float(s[127]));
+#pragma unroll
+        for (int i = 0; i < 14; ++i) a[i] = max3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        a[14] = a[42];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) a[i] = max3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        return max3f(fmaxf(a[0], a[1]), a[2], fmaxf(a[3], a[4]));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 42; ++i)
+            a[i] = min3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]),
+                         __uint_as_float(s[3 * i + 2]));
+        a[42] = fminf(__uint_as_float(s[126]), __uint_as_float(s[127]));
+#pragma unroll
+        for (int i = 0; i < 14; ++i) a[i] = min3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        a[14] = a[42];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) a[i] = min3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        return min3f(fminf(a[0], a[1]), a[2], fminf(a[3], a[4]));
+    }
+}
+
 template <int D, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
-    // ---- the work unit: (sequence/head, query tile) --------------------------
+    // ---- the work unit: (sequence/head, 256-row query block) --------------
     int len, seq_start = 0, bh = 0, h = 0;
     if constexpr (VARLEN) {
         const int b = blockIdx.z;
         h = blockIdx.y;
-        int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
+        const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
         // keep every access inside the [total, H, d] tensors whatever the offsets say
         const int c0 = min(max(s0, 0), p.total), c1 = min(max(s1, c0), p.total);
         const int c1m = min(c1, c0 + p.N);
@@ -79,12 +126,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         bh = blockIdx.y;
         len = p.N;
     }
-    const int nq = (len + BM - 1) / BM;
-    // causal tiles near the end of the sequence carry the most work: start them first
-    const int t = p.causal ? (nq - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-    if (t < 0 || t >= nq) return;
+    const int nblk = (len + 2 * BM - 1) / (2 * BM);
+    // causal blocks near the end of the sequence carry the most work: start them first
+    const int blk = p.causal ? (nblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+    if (blk < 0 || blk >= nblk) return;
+    const int row0 = blk * 2 * BM;
     const int nkv_all = (len + BN - 1) / BN;
-    const int n_kv = p.causal ? min(t + 1, nkv_all) : nkv_all;
+    int n_t[2];
+    n_t[0] = p.causal ? min(2 * blk + 1, nkv_all) : nkv_all;
+    n_t[1] = (row0 + BM < len) ? (p.causal ? min(2 * blk + 2, nkv_all) : nkv_all) : 0;
+    const int n = max(n_t[0], n_t[1]);
 
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
@@ -92,28 +143,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t warp = warp_id_uniform();
     const uint32_t lane = lane_id();
+    const uint32_t wg = warp / 4;
     unsigned int* err = p.err;
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.k_full[s], 1);
-            mbar_init(&sm.k_empty[s], 1);
-            mbar_init(&sm.v_full[s], 1);
-            mbar_init(&sm.v_empty[s], 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&sm.q_full[t], 1);
+            mbar_init(&sm.s_full[t], 1);
+            mbar_init(&sm.p_full[t], BM);
+            mbar_init(&sm.a_full[t], BM);
+            mbar_init(&sm.o_ready[t], BM);
+            mbar_init(&sm.pv_done[t], 1);
+            mbar_init(&sm.stats_full[t], BM);
+            mbar_init(&sm.turn[t], BM);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.s_full[s], 1);
-            mbar_init(&sm.s_free[s], BM);
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
         }
-        mbar_init(&sm.p_full, BM);
-        mbar_init(&sm.pv_done, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 12) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -122,11 +175,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    const int q_row0 = t * BM;
-
-    if (warp == 4) {
-        // ================= TMA producer =================
-        if (lane == 0) {
+    if (wg == 3) {
+        regs_dec<48>();
+        if (warp == 13 && lane == 0) {
+            // ================= TMA producer =================
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
@@ -139,160 +191,243 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, row, bh);
                 }
             };
-            mbar_arrive_expect_tx(&sm.bar_q, BM * D * 2);
-            load_tile(sm.q, &tq, &sm.bar_q, q_row0);
-            int issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                if (!mbar_wait(&sm.k_empty[st], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
-                mbar_arrive_expect_tx(&sm.k_full[st], BN * D * 2);
-                load_tile(sm.k[st], &tk, &sm.k_full[st], j * BN);
-                if (!mbar_wait(&sm.v_empty[st], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) {
-                    issued = j;  // K of tile j is in flight, V is not
-                    mbar_wait(&sm.k_full[st], ph, err, FA_DEVERR_TIMEOUT, nullptr);
-                    break;
+            for (int t = 0; t < 2; ++t) {
+                if (n_t[t] > 0) {
+                    mbar_arrive_expect_tx(&sm.q_full[t], BM * D * 2);
+                    load_tile(sm.q[t], &tq, &sm.q_full[t], row0 + t * BM);
                 }
-                mbar_arrive_expect_tx(&sm.v_full[st], BN * D * 2);
-                load_tile(sm.v[st], &tv, &sm.v_full[st], j * BN);
-                issued = j + 1;
             }
-            // Before the CTA may exit, every copy it started must have landed.
-            // On the normal path the MMA warp has consumed them all already.
-            mbar_wait(&sm.bar_q, 0, err, FA_DEVERR_TIMEOUT, nullptr);
-            for (int j = max(0, issued - kStages); j < issued; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                mbar_wait(&sm.k_full[st], ph, err, FA_DEVERR_TIMEOUT, nullptr);
-                mbar_wait(&sm.v_full[st], ph, err, FA_DEVERR_TIMEOUT, nullptr);
+            int issued = 0;  // ring uses issued so far
+            for (int u = 0; u < 2 * n; ++u) {
+                const int slot = u % kSlots;
+                const uint32_t ph = (u / kSlots) & 1;
+                if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
+                mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
+                load_tile(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], (u >> 1) * BN);
+                issued = u + 1;
             }
-        }
-        __syncwarp();
-    } else if (warp == 5) {
-        // ================= MMA issuer =================
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
+            // every copy this CTA started must land before it exits
+            for (int t = 0; t < 2; ++t)
+                if (n_t[t] > 0) mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, nullptr);
+            for (int u = max(0, issued - kSlots); u < issued; ++u)
+                mbar_wait(&sm.kv_full[u % kSlots], (u / kSlots) & 1, err, FA_DEVERR_TIMEOUT,
+                          nullptr);
+        } else if (warp == 12 && lane == 0) {
+            // ================= MMA issuer =================
+            // The tensor pipe runs this thread's MMAs in issue order, so
+            // S_t(j+1), which overwrites the TMEM columns holding P_t(j), is
+            // issued right behind P_t(j) V_j without waiting: P_t is read first.
+            constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
-            const uint32_t q_base = smem_u32(sm.q);
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % kStages;
-                const int sb = j & 1;
-                if (!mbar_wait(&sm.k_full[st], (j / kStages) & 1, err, FA_DEVERR_TIMEOUT, abort))
-                    return false;
-                if (!mbar_wait(&sm.s_free[sb], ((j >> 1) & 1) ^ 1, err, FA_DEVERR_TIMEOUT, abort))
-                    return false;
-                tc_fence_after();
-                const uint32_t k_base = smem_u32(sm.k[st]);
+            // descriptor words: high = SBO 1024 B | version 1 | 128-byte swizzle;
+            // low = LBO (16 B for K-major, the 64-column block stride for V) | addr>>4
+            constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+            constexpr uint32_t kLboK = (16u >> 4) << 16;
+            constexpr uint32_t kLboV = (static_cast<uint32_t>(kBoxBytes) >> 4) << 16;
+            constexpr uint32_t kTile16 = (BN * D * 2) >> 4;  // one ring slot, in 16-byte units
+            const uint32_t q_lo0 = smem_u32(sm.q[0]) >> 4;
+            const uint32_t q_lo1 = smem_u32(sm.q[1]) >> 4;
+            const uint32_t kv_lo = smem_u32(sm.kv[0]) >> 4;
+            auto issue_s = [&](int t, int j) {
+                const uint32_t qa = t ? q_lo1 : q_lo0;
+                const uint32_t kb = kv_lo + ring_slot(j, 0) * kTile16;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    const uint64_t da = smem_desc_sw128(q_base + off, 16, 1024);
-                    const uint64_t db = smem_desc_sw128(k_base + off, 16, 1024);
-                    mma_ss(tmem + kColS + sb * BN, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint32_t o = (kk >> 2) * (kBoxBytes >> 4) + (kk & 3) * 2;
+                    mma_ss(tmem + col_s(t),
+                           (static_cast<uint64_t>(kDescHi) << 32) | (kLboK | (qa + o)),
+                           (static_cast<uint64_t>(kDescHi) << 32) | (kLboK | (kb + o)), idesc_s,
+                           kk > 0 ? 1u : 0u);
                 }
-                tc_commit(&sm.s_full[sb]);
-                tc_commit(&sm.k_empty[st]);
-                return true;
             };
-            bool ok = mbar_wait(&sm.bar_q, 0, err, FA_DEVERR_TIMEOUT, abort);
-            if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < n_kv; ++j) {
-                if (j + 1 < n_kv && !issue_s(j + 1)) break;
-                const int st = j % kStages;
-                if (!mbar_wait(&sm.p_full, j & 1, err, FA_DEVERR_TIMEOUT, abort)) break;
-                if (!mbar_wait(&sm.v_full[st], (j / kStages) & 1, err, FA_DEVERR_TIMEOUT, abort))
-                    break;
-                tc_fence_after();
-                const uint32_t v_base = smem_u32(sm.v[st]);
+            auto issue_pv = [&](int t, int j) {
+                const uint32_t vb = kv_lo + ring_slot(j, 1) * kTile16;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    // 16 keys = 16 rows of 128 bytes in each 64-column block
-                    const uint64_t db = smem_desc_sw128(v_base + kk * 16 * 128, kBoxBytes, 1024);
-                    mma_ts(tmem + kColO, tmem + kColP + kk * 8, db, idesc_pv,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 16 rows of 128 bytes
+                    mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                           (static_cast<uint64_t>(kDescHi) << 32) | (kLboV | (vb + kk * 128)),
+                           idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = true;
+            for (int t = 0; t < 2 && ok; ++t)
+                if (n_t[t] > 0) ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort);
+            ok = ok && mbar_wait(&sm.kv_full[ring_slot(0, 0)], ring_phase(0, 0), err,
+                                 FA_DEVERR_TIMEOUT, abort);
+            if (ok) {
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t) {
+                    if (n_t[t] > 0) {
+                        issue_s(t, 0);
+                        tc_commit(&sm.s_full[t]);
+                    }
                 }
-                tc_commit(&sm.pv_done);
-                tc_commit(&sm.v_empty[st]);
+                tc_commit(&sm.kv_empty[ring_slot(0, 0)]);
+            }
+            for (int j = 0; ok && j < n; ++j) {
+                if (!mbar_wait(&sm.kv_full[ring_slot(j, 1)], ring_phase(j, 1), err,
+                               FA_DEVERR_TIMEOUT, abort)) break;
+                const bool next_k = j + 1 < n;
+                if (next_k && !mbar_wait(&sm.kv_full[ring_slot(j + 1, 0)], ring_phase(j + 1, 0),
+                                         err, FA_DEVERR_TIMEOUT, abort)) break;
+                for (int t = 0; t < 2; ++t) {
+                    if (j >= n_t[t]) continue;
+                    if (!mbar_wait(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort) ||
+                        !mbar_wait(&sm.o_ready[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv(t, j);
+                    tc_commit(&sm.pv_done[t]);
+                    if (j + 1 < n_t[t]) {
+                        issue_s(t, j + 1);
+                        tc_commit(&sm.s_full[t]);
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&sm.kv_empty[ring_slot(j, 1)]);
+                if (next_k) tc_commit(&sm.kv_empty[ring_slot(j + 1, 0)]);
             }
             // every MMA this thread issued must be complete before TMEM is freed
             tc_commit(&sm.drain);
             mbar_wait(&sm.drain, 0, err, FA_DEVERR_TIMEOUT, nullptr);
         }
         __syncwarp();
-    } else {
-        // ================= softmax / correction / epilogue (warps 0-3) =================
-        const int r = threadIdx.x;  // query row within the tile == TMEM lane
-        const uint32_t lane_off = (warp * 32u) << 16;
-        const int qrow = q_row0 + r;
+    } else if (wg < 2) {
+        // ================= softmax of tile t (warpgroups 0 and 1) =================
+        regs_inc<192>();
+        const int t = wg;
+        const int r = threadIdx.x - t * BM;          // row within the tile == TMEM lane
+        const uint32_t lane_off = ((warp & 3) * 32u) << 16;
+        const uint32_t s_addr = tmem + lane_off + col_s(t);
+        const int row_first = row0 + t * BM;
+        const int qrow = row_first + r;
         const float sl = p.scale_log2;
-        float m = -INFINITY, l = 0.f;
+        const bool neg = sl < 0.f;
+        const uint64_t sl2 = f2_pack(sl, sl);
+        float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            const int sb = j & 1;
-            if (!warp_wait(&sm.s_full[sb], (j >> 1) & 1, err, abort)) { ok = false; break; }
+        for (int j = 0; j < n_t[t]; ++j) {
+            if (!warp_wait(&sm.s_full[t], j & 1, err, abort)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[BN];
+            uint32_t s[BN];
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c)
-                tmem_ld32(tmem + lane_off + kColS + sb * BN + c * 32,
-                          *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+                tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.s_free[sb]);
 
-            // scaled scores in the log2 domain, masked entries -> -inf
-            float x[BN];
-            int limit = len - j * BN;                        // keys past the sequence end
-            if (p.causal) limit = min(limit, qrow - j * BN + 1);  // keys after this row
+            // masked keys: past the sequence end, or after this row (causal)
+            const int kbase = j * BN;
+            const bool need_mask = (kbase + BN > len) || (p.causal && kbase + BN - 1 > row_first);
+            int lim = BN;
+            if (need_mask) {
+                lim = min(BN, len - kbase);
+                if (p.causal) lim = min(lim, qrow - kbase + 1);
+                const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const float s = __uint_as_float(sr[c]) * sl;
-                x[c] = (c < limit) ? s : -INFINITY;
+                for (int c = 0; c < BN; ++c) s[c] = (c < lim) ? s[c] : fill;
             }
-            float mt = x[0];
-#pragma unroll
-            for (int c = 1; c < BN; ++c) mt = fmaxf(mt, x[c]);
-            const float m_new = fmaxf(m, mt);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            const float alpha = ex2_approx(m - m_use);  // m = -inf -> 0
+            const float mt = row_extreme(s, neg) * sl;  // = max over keys of scale*log2e*s
+            float alpha = 1.f;
+            if (j == 0) {
+                m_used = mt;
+            } else if (mt > m_used + kRescaleLog2) {
+                alpha = ex2_approx(m_used - mt);
+                m_used = mt;
+            }
+            sm.alpha[t][r] = alpha;
+            mbar_arrive(&sm.a_full[t]);
 
-            if (j > 0) {
-                // O and the P buffer are free once P V of the previous tile is done
-                if (!warp_wait(&sm.pv_done, (j - 1) & 1, err, abort)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t orr[32];
-                        tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                        tmem_st32(tmem + lane_off + kColO + c * 32, orr);
-                    }
-                }
-            }
-            float rs = 0.f;
+            const float mb = (m_used == -INFINITY) ? 0.f : m_used;
+            const uint64_t nm2 = f2_pack(-mb, -mb);
+            uint64_t acc[4] = {0, 0, 0, 0};  // partial row sums (pairs)
             uint32_t pk[BN / 2];
+            // p = 2^(scale*log2e*s - m); masked keys give exactly 0
+            auto exp_row = [&](auto masked, int lim) {
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-                const float p0 = ex2_approx(x[c] - m_use);
-                const float p1 = ex2_approx(x[c + 1] - m_use);
-                rs += p0 + p1;
-                pk[c / 2] = pack_bf16x2(p0, p1);
-            }
-            l = l * alpha + rs;
-            m = m_new;
-            tmem_st32(tmem + lane_off + kColP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tmem + lane_off + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+                for (int c = 0; c < BN; c += 2) {
+                    const uint64_t x = f2_fma(
+                        f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, nm2);
+                    float p0 = ex2_approx(f2_lo(x));
+                    float p1 = ex2_approx(f2_hi(x));
+                    if constexpr (decltype(masked)::value) {
+                        p0 = (c < lim) ? p0 : 0.f;
+                        p1 = (c + 1 < lim) ? p1 : 0.f;
+                    }
+                    acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], f2_pack(p0, p1));
+                    pk[c / 2] = pack_bf16x2(p0, p1);
+                }
+            };
+            // The exp unit is the scarce resource: tile 0's step j, then tile
+            // 1's step j, then tile 0's step j+1 ...  so that one tile's
+            // exponentials overlap the other tile's MMAs instead of competing.
+            const bool my_turn_wait = (t == 0) ? (j > 0 && j - 1 < n_t[1]) : (j < n_t[0]);
+            if (my_turn_wait &&
+                !warp_wait(&sm.turn[t], (t == 0 ? j - 1 : j) & 1, err, abort)) { ok = false; break; }
+            if (need_mask)
+                exp_row(std::true_type{}, lim);
+            else
+                exp_row(std::false_type{}, BN);
+            mbar_arrive(&sm.turn[1 - t]);
+            const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+            l = l * alpha + (f2_lo(acc2) + f2_hi(acc2));
+            tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.p_full);
+            mbar_arrive(&sm.p_full[t]);
         }
-        if (ok && warp_wait(&sm.pv_done, (n_kv - 1) & 1, err, abort)) {
+        if (ok && n_t[t] > 0) {
+            sm.row_m[t][r] = m_used;
+            sm.row_l[t][r] = l;
+            mbar_arrive(&sm.stats_full[t]);
+        }
+    } else {
+        // ================= O correction and epilogue (warpgroup 2) =================
+        regs_dec<80>();
+        const int r = threadIdx.x - 2 * BM;
+        const uint32_t lane_off = ((warp & 3) * 32u) << 16;
+        bool ok = true;
+        for (int j = 0; ok && j < n; ++j) {
+            for (int t = 0; t < 2; ++t) {
+                if (j >= n_t[t]) continue;
+                if (!warp_wait(&sm.a_full[t], j & 1, err, abort)) { ok = false; break; }
+                const float a = sm.alpha[t][r];
+                if (j > 0 && __any_sync(0xffffffffu, a != 1.f)) {
+                    // O_t must hold P_t V_{j-1} before it is scaled
+                    if (!warp_wait(&sm.pv_done[t], (j - 1) & 1, err, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t a2 = f2_pack(a, a);
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        const uint32_t addr = tmem + lane_off + col_o(t) + c * 32;
+                        tmem_ld32(addr, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const uint64_t v = f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+                            o[e] = __float_as_uint(f2_lo(v));
+                            o[e + 1] = __float_as_uint(f2_hi(v));
+                        }
+                        tmem_st32(addr, o);
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.o_ready[t]);
+            }
+        }
+        // epilogue: O / l -> bf16, log-sum-exp
+        for (int t = 0; ok && t < 2; ++t) {
+            if (n_t[t] == 0) continue;
+            if (!warp_wait(&sm.stats_full[t], 0, err, abort) ||
+                !warp_wait(&sm.pv_done[t], (n_t[t] - 1) & 1, err, abort))
+                break;
             tc_fence_after();
+            const int qrow = row0 + t * BM + r;
             const bool store = qrow < len;
+            const float m = sm.row_m[t][r], l = sm.row_l[t][r];
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16* orow;
             if constexpr (VARLEN)
@@ -303,22 +438,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                        (static_cast<int64_t>(bh) * p.N + qrow) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t orr[32];
-                tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + col_o(t) + c * 32, o);
                 tmem_wait_ld();
                 if (store) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(orr[e * 8 + 0]) * inv_l,
-                                          __uint_as_float(orr[e * 8 + 1]) * inv_l);
-                        w.y = pack_bf16x2(__uint_as_float(orr[e * 8 + 2]) * inv_l,
-                                          __uint_as_float(orr[e * 8 + 3]) * inv_l);
-                        w.z = pack_bf16x2(__uint_as_float(orr[e * 8 + 4]) * inv_l,
-                                          __uint_as_float(orr[e * 8 + 5]) * inv_l);
-                        w.w = pack_bf16x2(__uint_as_float(orr[e * 8 + 6]) * inv_l,
-                                          __uint_as_float(orr[e * 8 + 7]) * inv_l);
+                        w.x = pack_bf16x2(__uint_as_float(o[e * 8 + 0]) * inv_l,
+                                          __uint_as_float(o[e * 8 + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(o[e * 8 + 2]) * inv_l,
+                                          __uint_as_float(o[e * 8 + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(o[e * 8 + 4]) * inv_l,
+                                          __uint_as_float(o[e * 8 + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(o[e * 8 + 6]) * inv_l,
+                                          __uint_as_float(o[e * 8 + 7]) * inv_l);
                         dst[e] = w;
                     }
                 }
@@ -337,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 12) tmem_dealloc(tmem, kTmemCols);
 }
 
 template <int D, bool VARLEN>
@@ -352,11 +487,11 @@ int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
     dim3 grid;
-    const int tiles = (p.N + BM - 1) / BM;
+    const int blocks = (p.N + 2 * BM - 1) / (2 * BM);
     if constexpr (VARLEN)
-        grid = dim3(tiles, p.H, p.B);
+        grid = dim3(blocks, p.H, p.B);
     else
-        grid = dim3(tiles, p.B * p.H, 1);
+        grid = dim3(blocks, p.B * p.H, 1);
     kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

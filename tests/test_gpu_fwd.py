@@ -57,7 +57,7 @@ def test_shapes_full_compare(shape, causal):
     assert_lse_close(to64(lse), lse_ref, str(shape))
 
 
-@pytest.mark.parametrize("scale", [0.02, 0.3, -0.1])
+@pytest.mark.parametrize("scale", [0.0, 0.02, 0.3, -0.1])
 def test_other_scales(scale):
     q, k, v = W.custom_fwd_inputs(1, 2, 300, 128, seed=7)
     for causal in (False, True):
