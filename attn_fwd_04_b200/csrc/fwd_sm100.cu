@@ -16,16 +16,18 @@
 //   * both products run on the 5th-generation tensor cores: S = Q K^T (both
 //     operands in shared memory) and O += P V (P read from tensor memory);
 //     S, P and both O accumulators live in TMEM (all 512 columns);
-//   * warp roles (512 threads): warpgroup 0 and 1 run the softmax of tile 0
-//     and tile 1 (one thread per query row); their exponential phases take
-//     turns, so one tile's softmax overlaps the other tile's MMAs; warpgroup
-//     2 rescales O when the running max
-//     grows, and writes the epilogue; in warpgroup 3, warp 12 issues the MMAs
-//     and warp 13 the TMA loads.  Registers are moved to the softmax
-//     warpgroups with setmaxnreg (2 x 192 + 80 + 48 = 4 x 128 per thread);
-//   * exp is exp2 with scale*log2(e) folded in; O is rescaled only when the
-//     running max has grown by more than 2^8 (the stale max is used for both
-//     the numerator and l, so the result is unchanged up to rounding).
+//   * warp roles (512 threads): warpgroups 0 and 1 run the softmax of tile 0
+//     and tile 1 (one thread per query row), so one tile's softmax overlaps
+//     the other tile's MMAs; each also rescales its own O accumulator when
+//     the running max grows; warpgroup 2 writes the epilogue; in warpgroup 3,
+//     warp 12 issues the MMAs and warp 13 the TMA loads.  Registers are moved
+//     to the softmax warpgroups with setmaxnreg (2 x 192 + 80 + 48 = 4 x 128
+//     per thread);
+//   * exp is exp2 with scale*log2(e) folded in (the polynomial path below can
+//     take a share of the exponentials off the special-function unit; it is
+//     switched off because it measured slower here); O is rescaled only when
+//     the running max has grown by more than 2^8 (the stale max is used for
+//     both the numerator and l, so the result is unchanged up to rounding).
 //
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
 // P_t (bf16 pairs) overwrites the first 64 columns of S_t; the next S_t is
@@ -48,18 +50,23 @@ __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }  // O_t
 constexpr int kBoxBytes = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16
 constexpr float kRescaleLog2 = 8.0f;     // rescale O when the max grows by > 2^8
+// Exponentials of pairs (c/2) % 8 in [0, kPolyPairs) are evaluated with the
+// FMA-pipe polynomial below, the rest with the special-function unit.
+constexpr int kPolyPairs = 0;
+// 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by
+// the Remez exchange in exp2_poly_remez.py beside this file.
+constexpr float kExp2P0 = 0.9999280571937561f, kExp2P1 = 0.6932609677314758f,
+                kExp2P2 = 0.2426111251115799f, kExp2P3 = 0.0551716685295105f;
 
 template <int D>
 struct alignas(1024) FwdSmem {
     uint8_t q[2][BM * D * 2];
     uint8_t kv[kSlots][BN * D * 2];
-    float alpha[2][BM];   // per-row O correction factor of the current step
     float row_m[2][BM];   // final running max (log2 domain) per row
     float row_l[2][BM];   // final normaliser per row
     uint64_t q_full[2];
     uint64_t kv_full[kSlots], kv_empty[kSlots];
-    uint64_t s_full[2], p_full[2], a_full[2], o_ready[2], pv_done[2], stats_full[2];
-    uint64_t turn[2];  // exp phases of the two softmax warpgroups take turns
+    uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -103,6 +110,26 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&s)[BN], bool neg) 
         for (int i = 0; i < 5; ++i) a[i] = min3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
         return min3f(fminf(a[0], a[1]), a[2], fminf(a[3], a[4]));
     }
+}
+
+// 2^x for a pair of x values on the FMA pipe: x = j + f with j = round(x)
+// (adding 1.5 * 2^23 leaves j in the low mantissa bits), 2^f from the
+// polynomial, and j added straight into the exponent field.  x is clamped to
+// >= -125 so that the result stays a normal number (2^-125 is 0 for every
+// practical purpose next to the row's leading term 2^0).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    const float x0 = fmaxf(f2_lo(x), -125.f), x1 = fmaxf(f2_hi(x), -125.f);
+    const uint64_t xc = f2_pack(x0, x1);
+    const uint64_t big = f2_pack(12582912.f, 12582912.f);
+    const uint64_t y = f2_add(xc, big);
+    const uint64_t jf = f2_add(y, f2_pack(-12582912.f, -12582912.f));
+    const uint64_t f = f2_add(xc, f2_pack(-f2_lo(jf), -f2_hi(jf)));
+    uint64_t q = f2_fma(f2_pack(kExp2P3, kExp2P3), f, f2_pack(kExp2P2, kExp2P2));
+    q = f2_fma(q, f, f2_pack(kExp2P1, kExp2P1));
+    q = f2_fma(q, f, f2_pack(kExp2P0, kExp2P0));
+    const uint32_t r0 = static_cast<uint32_t>(q) + (static_cast<uint32_t>(y) << 23);
+    const uint32_t r1 = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(y >> 32) << 23);
+    return (static_cast<uint64_t>(r1) << 32) | r0;
 }
 
 template <int D, bool VARLEN>
@@ -152,11 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.q_full[t], 1);
             mbar_init(&sm.s_full[t], 1);
             mbar_init(&sm.p_full[t], BM);
-            mbar_init(&sm.a_full[t], BM);
-            mbar_init(&sm.o_ready[t], BM);
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
-            mbar_init(&sm.turn[t], BM);
         }
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sm.kv_full[s], 1);
@@ -271,8 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          err, FA_DEVERR_TIMEOUT, abort)) break;
                 for (int t = 0; t < 2; ++t) {
                     if (j >= n_t[t]) continue;
-                    if (!mbar_wait(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort) ||
-                        !mbar_wait(&sm.o_ready[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+                    if (!mbar_wait(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
                         ok = false;
                         break;
                     }
@@ -300,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = threadIdx.x - t * BM;          // row within the tile == TMEM lane
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         const uint32_t s_addr = tmem + lane_off + col_s(t);
+        const uint32_t o_addr = tmem + lane_off + col_o(t);
         const int row_first = row0 + t * BM;
         const int qrow = row_first + r;
         const float sl = p.scale_log2;
@@ -335,9 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 alpha = ex2_approx(m_used - mt);
                 m_used = mt;
             }
-            sm.alpha[t][r] = alpha;
-            mbar_arrive(&sm.a_full[t]);
-
             const float mb = (m_used == -INFINITY) ? 0.f : m_used;
             const uint64_t nm2 = f2_pack(-mb, -mb);
             uint64_t acc[4] = {0, 0, 0, 0};  // partial row sums (pairs)
@@ -348,8 +369,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < BN; c += 2) {
                     const uint64_t x = f2_fma(
                         f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, nm2);
-                    float p0 = ex2_approx(f2_lo(x));
-                    float p1 = ex2_approx(f2_hi(x));
+                    float p0, p1;
+                    if ((c / 2) % 8 < kPolyPairs) {
+                        const uint64_t e = exp2_poly2(x);
+                        p0 = f2_lo(e);
+                        p1 = f2_hi(e);
+                    } else {
+                        p0 = ex2_approx(f2_lo(x));
+                        p1 = ex2_approx(f2_hi(x));
+                    }
                     if constexpr (decltype(masked)::value) {
                         p0 = (c < lim) ? p0 : 0.f;
                         p1 = (c + 1 < lim) ? p1 : 0.f;
@@ -358,21 +386,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
             };
-            // The exp unit is the scarce resource: tile 0's step j, then tile
-            // 1's step j, then tile 0's step j+1 ...  so that one tile's
-            // exponentials overlap the other tile's MMAs instead of competing.
-            const bool my_turn_wait = (t == 0) ? (j > 0 && j - 1 < n_t[1]) : (j < n_t[0]);
-            if (my_turn_wait &&
-                !warp_wait(&sm.turn[t], (t == 0 ? j - 1 : j) & 1, err, abort)) { ok = false; break; }
             if (need_mask)
                 exp_row(std::true_type{}, lim);
             else
                 exp_row(std::false_type{}, BN);
-            mbar_arrive(&sm.turn[1 - t]);
             const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
             l = l * alpha + (f2_lo(acc2) + f2_hi(acc2));
             tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
             tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+            // O_t holds P_t V_0..j-1 and is idle: S_t(j) was issued behind
+            // P_t V_{j-1} in the MMA stream, so that product has completed.
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    const uint32_t addr = o_addr + c * 32;
+                    tmem_ld32(addr, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const uint64_t v = f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+                        o[e] = static_cast<uint32_t>(v);
+                        o[e + 1] = static_cast<uint32_t>(v >> 32);
+                    }
+                    tmem_st32(addr, o);
+                }
+            }
+
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[t]);
@@ -383,41 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sm.stats_full[t]);
         }
     } else {
-        // ================= O correction and epilogue (warpgroup 2) =================
+        // ================= epilogue (warpgroup 2) =================
         regs_dec<80>();
         const int r = threadIdx.x - 2 * BM;
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
-        for (int j = 0; ok && j < n; ++j) {
-            for (int t = 0; t < 2; ++t) {
-                if (j >= n_t[t]) continue;
-                if (!warp_wait(&sm.a_full[t], j & 1, err, abort)) { ok = false; break; }
-                const float a = sm.alpha[t][r];
-                if (j > 0 && __any_sync(0xffffffffu, a != 1.f)) {
-                    // O_t must hold P_t V_{j-1} before it is scaled
-                    if (!warp_wait(&sm.pv_done[t], (j - 1) & 1, err, abort)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t a2 = f2_pack(a, a);
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        const uint32_t addr = tmem + lane_off + col_o(t) + c * 32;
-                        tmem_ld32(addr, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const uint64_t v = f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
-                            o[e] = __float_as_uint(f2_lo(v));
-                            o[e + 1] = __float_as_uint(f2_hi(v));
-                        }
-                        tmem_st32(addr, o);
-                    }
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                mbar_arrive(&sm.o_ready[t]);
-            }
-        }
         // epilogue: O / l -> bf16, log-sum-exp
         for (int t = 0; ok && t < 2; ++t) {
             if (n_t[t] == 0) continue;
