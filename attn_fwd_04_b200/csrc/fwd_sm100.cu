@@ -21,7 +21,7 @@
 //     the other tile's MMAs; each also rescales its own O accumulator when
 //     the running max grows; warpgroup 2 writes the epilogue; in warpgroup 3,
 //     warp 12 issues the MMAs and warp 13 the TMA loads.  Registers are moved
-//     to the softmax warpgroups with setmaxnreg (2 x 192 + 80 + 48 = 4 x 128
+//     to the softmax warpgroups with setmaxnreg (2 x 192 + 72 + 56 = 4 x 128
 //     per thread);
 //   * exp is exp2 with scale*log2(e) folded in (the polynomial path below can
 //     take a share of the exponentials off the special-function unit; it is
@@ -49,7 +49,10 @@ constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }  // O_t
 constexpr int kBoxBytes = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16
-constexpr float kRescaleLog2 = 8.0f;     // rescale O when the max grows by > 2^8
+// P is computed against the running max of earlier steps; only when a row's
+// sum of P exceeds 2^16 (so some score beat that max by more than 2^16 / 128)
+// is the row's true max taken, O and l rescaled and P recomputed.
+constexpr float kLazySum = 65536.f;
 // Exponentials of pairs (c/2) % 8 in [0, kPolyPairs) are evaluated with the
 // FMA-pipe polynomial below, the rest with the special-function unit.
 constexpr int kPolyPairs = 0;
@@ -132,6 +135,39 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
     return (static_cast<uint64_t>(r1) << 32) | r0;
 }
 
+// p = 2^(scale*log2e*s - m) for the 128 scores of a row, packed to bf16 pairs
+// in pk; returns the row sum of p.  With MASKED, keys from `lim` on give
+// exactly 0.
+template <bool MASKED>
+__device__ __forceinline__ float exp_pairs(const uint32_t (&s)[BN], uint32_t (&pk)[BN / 2],
+                                           uint64_t sl2, float m, int lim) {
+    const float mb = (m == -INFINITY) ? 0.f : m;
+    const uint64_t nm2 = f2_pack(-mb, -mb);
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int c = 0; c < BN; c += 2) {
+        const uint64_t x =
+            f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, nm2);
+        float p0, p1;
+        if ((c / 2) % 8 < kPolyPairs) {
+            const uint64_t e = exp2_poly2(x);
+            p0 = f2_lo(e);
+            p1 = f2_hi(e);
+        } else {
+            p0 = ex2_approx(f2_lo(x));
+            p1 = ex2_approx(f2_hi(x));
+        }
+        if constexpr (MASKED) {
+            p0 = (c < lim) ? p0 : 0.f;
+            p1 = (c + 1 < lim) ? p1 : 0.f;
+        }
+        acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], f2_pack(p0, p1));
+        pk[c / 2] = pack_bf16x2(p0, p1);
+    }
+    const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+    return f2_lo(a2) + f2_hi(a2);
+}
+
 template <int D, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -200,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = sm.tmem_base;
 
     if (wg == 3) {
-        regs_dec<48>();
+        regs_dec<56>();
         if (warp == 13 && lane == 0) {
             // ================= TMA producer =================
             tma_prefetch_desc(&tq);
@@ -334,12 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < n_t[t]; ++j) {
             if (!warp_wait(&sm.s_full[t], j & 1, err, abort)) { ok = false; break; }
             tc_fence_after();
-            uint32_t s[BN];
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c)
-                tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
-            tmem_wait_ld();
-
             // masked keys: past the sequence end, or after this row (causal)
             const int kbase = j * BN;
             const bool need_mask = (kbase + BN > len) || (p.causal && kbase + BN - 1 > row_first);
@@ -347,51 +377,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (need_mask) {
                 lim = min(BN, len - kbase);
                 if (p.causal) lim = min(lim, qrow - kbase + 1);
-                const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
-#pragma unroll
-                for (int c = 0; c < BN; ++c) s[c] = (c < lim) ? s[c] : fill;
             }
-            const float mt = row_extreme(s, neg) * sl;  // = max over keys of scale*log2e*s
-            float alpha = 1.f;
-            if (j == 0) {
-                m_used = mt;
-            } else if (mt > m_used + kRescaleLog2) {
-                alpha = ex2_approx(m_used - mt);
-                m_used = mt;
-            }
-            const float mb = (m_used == -INFINITY) ? 0.f : m_used;
-            const uint64_t nm2 = f2_pack(-mb, -mb);
-            uint64_t acc[4] = {0, 0, 0, 0};  // partial row sums (pairs)
+            uint32_t s[BN];
             uint32_t pk[BN / 2];
-            // p = 2^(scale*log2e*s - m); masked keys give exactly 0
-            auto exp_row = [&](auto masked, int lim) {
+            float alpha = 1.f, rs = 0.f;
+            // Pass 1 uses the running max of earlier steps; if that leaves a
+            // row sum above kLazySum anywhere in the warp (or on the first
+            // step), pass 2 reloads the scores and uses the true row max.
+            for (int pass = (j == 0) ? 1 : 0; pass < 2; ++pass) {
 #pragma unroll
-                for (int c = 0; c < BN; c += 2) {
-                    const uint64_t x = f2_fma(
-                        f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, nm2);
-                    float p0, p1;
-                    if ((c / 2) % 8 < kPolyPairs) {
-                        const uint64_t e = exp2_poly2(x);
-                        p0 = f2_lo(e);
-                        p1 = f2_hi(e);
-                    } else {
-                        p0 = ex2_approx(f2_lo(x));
-                        p1 = ex2_approx(f2_hi(x));
-                    }
-                    if constexpr (decltype(masked)::value) {
-                        p0 = (c < lim) ? p0 : 0.f;
-                        p1 = (c + 1 < lim) ? p1 : 0.f;
-                    }
-                    acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], f2_pack(p0, p1));
-                    pk[c / 2] = pack_bf16x2(p0, p1);
+                for (int c = 0; c < BN / 32; ++c)
+                    tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+                tmem_wait_ld();
+                if (need_mask) {
+                    const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) s[c] = (c < lim) ? s[c] : fill;
                 }
-            };
-            if (need_mask)
-                exp_row(std::true_type{}, lim);
-            else
-                exp_row(std::false_type{}, BN);
-            const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-            l = l * alpha + (f2_lo(acc2) + f2_hi(acc2));
+                if (pass == 1) {
+                    const float mt = row_extreme(s, neg) * sl;  // max over keys of scale*log2e*s
+                    if (j == 0) {
+                        m_used = mt;
+                    } else if (mt > m_used) {
+                        alpha = ex2_approx(m_used - mt);
+                        m_used = mt;
+                    }
+                }
+                rs = need_mask ? exp_pairs<true>(s, pk, sl2, m_used, lim)
+                               : exp_pairs<false>(s, pk, sl2, m_used, BN);
+                if (pass == 1 || !__any_sync(0xffffffffu, !(rs <= kLazySum))) break;
+            }
+            l = l * alpha + rs;
             tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
             tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             // O_t holds P_t V_0..j-1 and is idle: S_t(j) was issued behind
@@ -425,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================= epilogue (warpgroup 2) =================
-        regs_dec<80>();
+        regs_dec<72>();
         const int r = threadIdx.x - 2 * BM;
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
