@@ -12,11 +12,15 @@
 // Decode runs as three launches on the caller's stream:
 //   plan   -- one CTA: prefix sums over the sequences of pages, tokens and
 //             work units (a unit is one head of one split of one sequence);
-//   split  -- a persistent grid over the units; a unit attends its query to
-//             the tokens of a few consecutive pages with the online softmax
-//             (running max and normaliser, page "Flash Attention 是什么",
-//             section 关键术语解析, item 4) and writes a normalised partial
-//             output and its log-sum-exp;
+//   split  -- a persistent grid, one CTA per SM, over the units; a unit
+//             attends its query to the tokens of a few consecutive pages with
+//             the online softmax (running max and normaliser, page "Flash
+//             Attention 是什么", section 关键术语解析, item 4) and writes a
+//             normalised partial output and its log-sum-exp.  A producer warp
+//             streams each (page, head) slice -- contiguous in the pool --
+//             into a 6-stage shared-memory ring with bulk copies, so each SM
+//             keeps ~200 KB of reads in flight; eight consumer warps compute
+//             from shared memory;
 //   merge  -- per (sequence, head), the log-sum-exp merge of the partials:
 //             lse = M + log sum_s 2^(lse_s - M), o = sum_s 2^(lse_s - lse) o_s.
 // All logs and exponents are base 2 inside the path (scale * log2 e folded
@@ -29,8 +33,6 @@ namespace fa {
 namespace {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kSplitThreads = 128;
-constexpr int kUnroll = 4;  // tokens in flight per half-warp and step
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -157,10 +159,63 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
     return r;
 }
 
-// One CTA (4 warps = 8 groups of LPT lanes) per work unit at a time.
-// LPT = D / 8 lanes hold one token's row (8 bf16 = 16 bytes each).
+constexpr int kDecTok = 64;           // tokens per ring stage (a quarter of a page)
+constexpr int kDecStages = 6;         // ring depth
+constexpr int kDecConsumerWarps = 8;
+constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;  // + one producer warp
+
 template <int D>
-__global__ void __launch_bounds__(kSplitThreads)
+struct DecSmem {
+    static constexpr int LPT = D / 8;                              // lanes per token
+    static constexpr int G = kDecConsumerWarps * 32 / LPT;         // token groups
+    alignas(128) uint8_t k[kDecStages][kDecTok * D * 2];
+    alignas(128) uint8_t v[kDecStages][kDecTok * D * 2];
+    float cm[2][G], cl[2][G];          // per-group partial state, by unit parity
+    float co[2][G][D];
+    uint64_t full[kDecStages], empty[kDecStages], cmb[2];
+    int abort;
+};
+
+// Walks the units u = first, first + stride, ... in increasing order and keeps
+// track of the owning sequence without a search per unit.
+struct UnitCursor {
+    int b = 0, next_off = 0;
+    __device__ __forceinline__ void seek(const int32_t* unit_off, int B, int u) {
+        while (b + 1 < B && u >= next_off) {
+            ++b;
+            next_off = __ldg(unit_off + b + 1);
+        }
+    }
+};
+
+struct UnitShape {
+    int b, s, h, tok0, ntok, cp, pt_base;
+};
+
+__device__ __forceinline__ UnitShape unit_shape(int u, UnitCursor& cur,
+                                                const int32_t* __restrict__ unit_off,
+                                                const int32_t* __restrict__ page_off,
+                                                const int32_t* __restrict__ seq_lens, int B,
+                                                int H, int page_size, int max_splits) {
+    cur.seek(unit_off, B, u);
+    UnitShape us;
+    us.b = cur.b;
+    const int r = u - __ldg(unit_off + us.b);
+    us.s = r / H;
+    us.h = r % H;
+    int len = __ldg(seq_lens + us.b);
+    if (len < 0) len = 0;
+    const int np = (len + page_size - 1) / page_size;
+    int ns;
+    split_shape(np, max_splits, ns, us.cp);
+    us.tok0 = us.s * us.cp * page_size;
+    us.ntok = min(len, us.tok0 + us.cp * page_size) - us.tok0;
+    us.pt_base = __ldg(page_off + us.b) + us.s * us.cp;
+    return us;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_split_kernel(const __nv_bfloat16* __restrict__ q,
                            const __nv_bfloat16* __restrict__ k_pages,
                            const __nv_bfloat16* __restrict__ v_pages,
@@ -168,117 +223,169 @@ __global__ void __launch_bounds__(kSplitThreads)
                            const int32_t* __restrict__ seq_lens, int B, int H, int page_size,
                            int max_splits, const int32_t* __restrict__ page_off,
                            const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
-                           float* __restrict__ part_o, float scale_log2) {
-    constexpr int LPT = D / 8;               // lanes per token
-    constexpr int GPW = 32 / LPT;            // token groups per warp
-    constexpr int G = (kSplitThreads / 32) * GPW;  // token groups per CTA
-    __shared__ float sh_m[G], sh_l[G];
-    __shared__ float sh_o[G][D];
-
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int sub = lane / LPT;              // group within the warp
-    const int gl = lane % LPT;               // lane within the group
-    const int grp = warp * GPW + sub;        // group within the CTA
-    const unsigned gmask = (LPT == 32) ? 0xffffffffu : (((1u << LPT) - 1u) << (sub * LPT));
-
+                           float* __restrict__ part_o, float scale_log2, unsigned int* err) {
+    using Sm = DecSmem<D>;
+    constexpr int LPT = Sm::LPT, G = Sm::G;
+    constexpr int GPW = 32 / LPT;  // token groups per warp
+    constexpr uint32_t kChunkBytes = kDecTok * D * 2;
+    extern __shared__ uint8_t dec_smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 127) &
+                                    ~static_cast<uintptr_t>(127));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort = &sm.abort;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDecStages; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kDecConsumerWarps);
+        }
+        mbar_init(&sm.cmb[0], kDecConsumerWarps * 32);
+        mbar_init(&sm.cmb[1], kDecConsumerWarps * 32);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
     const int total_units = __ldg(unit_off + B);
-    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-        const int b = find_owner(unit_off, B, u);
-        const int r = u - __ldg(unit_off + b);
-        const int s = r / H, h = r % H;
-        int len = __ldg(seq_lens + b);
-        if (len < 0) len = 0;
-        const int np = (len + page_size - 1) / page_size;
-        int ns, cp;
-        split_shape(np, max_splits, ns, cp);
-        const int tok0 = s * cp * page_size;
-        const int tok1 = min(len, tok0 + cp * page_size);
-        const int32_t* pt = page_table + __ldg(page_off + b);
+    UnitCursor cur;
+    cur.next_off = (B > 1) ? __ldg(unit_off + 1) : 0x7fffffff;
 
-        // this lane's 8 query values, pre-scaled into the log2 domain
-        float qf[8];
-        {
-            const uint4 qu = *reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * H + h) * D + gl * 8);
-            bf16x8_to_f32(qu, qf);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) qf[i] *= scale_log2;
-        }
-        float m = -INFINITY, l = 0.f, acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-
-        for (int t0 = tok0 + grp; t0 < tok1; t0 += G * kUnroll) {
-            uint4 kr[kUnroll], vr[kUnroll];
-            bool valid[kUnroll];
-#pragma unroll
-            for (int x = 0; x < kUnroll; ++x) {
-                const int t = t0 + x * G;
-                valid[x] = t < tok1;
-                if (valid[x]) {
-                    const int page = __ldg(pt + t / page_size);
-                    const int slot = t % page_size;
-                    const int64_t row = (static_cast<int64_t>(page) * H + h) * page_size + slot;
-                    kr[x] = ld_stream(k_pages + row * D + gl * 8);
-                    vr[x] = ld_stream(v_pages + row * D + gl * 8);
+    if (warp == kDecConsumerWarps) {
+        // ================= producer: bulk copies of (page, head) slices =================
+        int g = 0;  // ring uses so far
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
+                                            page_size, max_splits);
+            const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
+            constexpr int per_page = 256 / kDecTok;  // page_size is 256
+            int page = 0;
+            for (int c = 0; c < nchunks; ++c, ++g) {
+                if (c % per_page == 0) page = __ldg(page_table + us.pt_base + c / per_page);
+                const int slot = g % kDecStages;
+                if (lane == 0) {
+                    if (!mbar_wait(&sm.empty[slot], ((g / kDecStages) & 1) ^ 1, err,
+                                   FA_DEVERR_TIMEOUT, abort)) {
+                        ok = false;
+                    } else {
+                        const int64_t row = (static_cast<int64_t>(page) * H + us.h) * page_size +
+                                            (c % per_page) * kDecTok;
+                        mbar_arrive_expect_tx(&sm.full[slot], 2 * kChunkBytes);
+                        bulk_load(sm.k[slot], k_pages + row * D, kChunkBytes, &sm.full[slot]);
+                        bulk_load(sm.v[slot], v_pages + row * D, kChunkBytes, &sm.full[slot]);
+                    }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
             }
-            float sc[kUnroll];
+        }
+        // every copy this CTA started must land before it exits
+        if (lane == 0)
+            for (int i = max(0, g - kDecStages); i < g; ++i)
+                mbar_wait(&sm.full[i % kDecStages], (i / kDecStages) & 1, err, FA_DEVERR_TIMEOUT,
+                          nullptr);
+        __syncwarp();
+    } else {
+        // ================= consumers =================
+        const int sub = lane / LPT;            // group within the warp
+        const int gl = lane % LPT;             // lane within the group
+        const int grp = warp * GPW + sub;      // group within the CTA
+        const unsigned gmask = (LPT == 32) ? 0xffffffffu : (((1u << LPT) - 1u) << (sub * LPT));
+        int g = 0, k = 0;  // ring uses, units done
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
+                                            page_size, max_splits);
+            float qf[8];
+            {
+                const uint4 qu = *reinterpret_cast<const uint4*>(
+                    q + (static_cast<int64_t>(us.b) * H + us.h) * D + gl * 8);
+                bf16x8_to_f32(qu, qf);
 #pragma unroll
-            for (int x = 0; x < kUnroll; ++x) {
-                float kf[8];
-                bf16x8_to_f32(kr[x], kf);
-                float dot = 0.f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) dot = fmaf(qf[i], kf[i], dot);
-#pragma unroll
-                for (int o = LPT / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(gmask, dot, o);
-                sc[x] = valid[x] ? dot : -INFINITY;
+                for (int i = 0; i < 8; ++i) qf[i] *= scale_log2;
             }
-            float mb = sc[0];
+            float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
-            for (int x = 1; x < kUnroll; ++x) mb = fmaxf(mb, sc[x]);
-            const float m_new = fmaxf(m, mb);  // finite: sc[0] is always a valid token
-            const float alpha = ex2_approx(m - m_new);
-            l *= alpha;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] *= alpha;
-#pragma unroll
-            for (int x = 0; x < kUnroll; ++x) {
-                if (valid[x]) {
-                    const float pw = ex2_approx(sc[x] - m_new);
-                    l += pw;
-                    float vf[8];
-                    bf16x8_to_f32(vr[x], vf);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] = fmaf(pw, vf[i], acc[i]);
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
+            for (int c = 0; c < nchunks; ++c, ++g) {
+                const int slot = g % kDecStages;
+                if (!mbar_wait(&sm.full[slot], (g / kDecStages) & 1, err, FA_DEVERR_TIMEOUT,
+                               abort)) {
+                    ok = false;
+                    break;
                 }
+                constexpr int TPG = kDecTok / G;  // tokens per group per chunk
+                float sc[TPG];
+                const int base = c * kDecTok;
+#pragma unroll
+                for (int x = 0; x < TPG; ++x) {
+                    const int t = grp + x * G;
+                    const uint4 kr = *reinterpret_cast<const uint4*>(sm.k[slot] + t * D * 2 + gl * 16);
+                    float kf[8];
+                    bf16x8_to_f32(kr, kf);
+                    float dot = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dot = fmaf(qf[i], kf[i], dot);
+#pragma unroll
+                    for (int o = LPT / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(gmask, dot, o);
+                    sc[x] = (base + t < us.ntok) ? dot : -INFINITY;
+                }
+                float mb = sc[0];
+#pragma unroll
+                for (int x = 1; x < TPG; ++x) mb = fmaxf(mb, sc[x]);
+                const float m_new = fmaxf(m, mb);
+                if (m_new != -INFINITY) {
+                    const float alpha = ex2_approx(m - m_new);  // m = -inf -> 0
+                    l *= alpha;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] *= alpha;
+#pragma unroll
+                    for (int x = 0; x < TPG; ++x) {
+                        const int t = grp + x * G;
+                        if (base + t < us.ntok) {
+                            const float pw = ex2_approx(sc[x] - m_new);
+                            l += pw;
+                            const uint4 vr =
+                                *reinterpret_cast<const uint4*>(sm.v[slot] + t * D * 2 + gl * 16);
+                            float vf[8];
+                            bf16x8_to_f32(vr, vf);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[i] = fmaf(pw, vf[i], acc[i]);
+                        }
+                    }
+                    m = m_new;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.empty[slot]);
             }
-            m = m_new;
-        }
-        // combine the G groups of this CTA
-        if (gl == 0) {
-            sh_m[grp] = m;
-            sh_l[grp] = l;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sh_o[grp][gl * 8 + i] = acc[i];
-        __syncthreads();
-        if (threadIdx.x < D) {
-            float M = -INFINITY;
-#pragma unroll
-            for (int g = 0; g < G; ++g) M = fmaxf(M, sh_m[g]);
-            float L = 0.f, o = 0.f;
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float w = (sh_m[g] == -INFINITY) ? 0.f : ex2_approx(sh_m[g] - M);
-                L += w * sh_l[g];
-                o += w * sh_o[g][threadIdx.x];
+            if (!ok) break;
+            // combine the G groups of this unit (buffers double-buffered by unit parity)
+            const int par = k & 1;
+            if (gl == 0) {
+                sm.cm[par][grp] = m;
+                sm.cl[par][grp] = l;
             }
-            part_o[static_cast<int64_t>(u) * D + threadIdx.x] = o / L;
-            if (threadIdx.x == 0) part_lse[u] = M + __log2f(L);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sm.co[par][grp][gl * 8 + i] = acc[i];
+            mbar_arrive(&sm.cmb[par]);
+            if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+                ok = false;
+                break;
+            }
+            if (threadIdx.x < D) {
+                float M = -INFINITY;
+#pragma unroll
+                for (int gi = 0; gi < G; ++gi) M = fmaxf(M, sm.cm[par][gi]);
+                float L = 0.f, o = 0.f;
+#pragma unroll
+                for (int gi = 0; gi < G; ++gi) {
+                    const float w = (sm.cm[par][gi] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][gi] - M);
+                    L += w * sm.cl[par][gi];
+                    o += w * sm.co[par][gi][threadIdx.x];
+                }
+                part_o[static_cast<int64_t>(u) * D + threadIdx.x] = o / L;
+                if (threadIdx.x == 0) part_lse[u] = M + __log2f(L);
+            }
         }
-        __syncthreads();
     }
 }
 
@@ -370,11 +477,20 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
     fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, H, page_size, max_splits,
                                                           page_off, tok_off, unit_off, err);
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-    const int grid = num_sms * 16;
-    fa_decode_split_kernel<D><<<grid, kSplitThreads, 0, stream>>>(
+    const size_t smem = sizeof(DecSmem<D>) + 128;
+    if (cudaFuncSetAttribute(fa_decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    // a persistent grid of the CTAs that are resident at once
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fa_decode_split_kernel<D>,
+                                                      kDecThreads, smem) != cudaSuccess ||
+        occ < 1)
+        return FA_ERR_CUDA;
+    fa_decode_split_kernel<D><<<num_sms * occ, kDecThreads, smem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pages),
         static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, page_size,
-        max_splits, page_off, unit_off, part_lse, part_o, scale_log2);
+        max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
         seq_lens, B, H, page_size, max_splits, unit_off, part_lse, part_o,
