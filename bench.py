@@ -235,6 +235,53 @@ def oracle_decode_sample(cache: W.PagedCache, target_s: float):
 # ---------------------------------------------------------------------------
 # native arm
 # ---------------------------------------------------------------------------
+def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
+    """TFLOP/s of the forward pass on the other workloads (tiny, batched,
+    variable-length, 128K context), timed with CUDA events; reported beside
+    the headline number, not part of the timed step."""
+    out = {}
+
+    def timed(fn, flops, name, extra=None):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if fa.fa_get_device_error() != fa.FA_OK:
+            raise RuntimeError(f"device error on {name}")
+        ms = e0.elapsed_time(e1) / steps
+        d = {"ms_per_launch": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+             "pct_of_2250": 100 * flops / (ms * 1e-3) / 1e12 / DATASHEET_BF16_TFLOPS}
+        d.update(extra or {})
+        out[name] = d
+
+    for w in (W.TINY_CAUSAL, W.BATCHED, W.CTX128K):
+        q, k, v = W.fwd_inputs(w, device="cuda")[:3]
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        sc = 1 / math.sqrt(w.d)
+        timed(lambda: fa.fa_fwd(q, k, v, w.causal, sc, o=o, lse=lse, stream=stream),
+              fwd_flops(w), w.name)
+        del q, k, v, o, lse
+    w = W.BATCHED_VARLEN
+    q, k, v, cu = W.varlen_workload_inputs(w, device="cuda")
+    lens = (cu[1:] - cu[:-1]).tolist()
+    cud = cu.cuda()
+    o = torch.empty_like(q)
+    lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=q.device)
+    flops = sum(4.0 * w.H * L * L * w.d / (2 if w.causal else 1) for L in lens)
+    sc = 1 / math.sqrt(w.d)
+    timed(lambda: fa.fa_fwd_varlen(q, k, v, cud, max(lens), w.causal, sc, o=o, lse=lse,
+                                   stream=stream),
+          flops, w.name, {"lengths": lens})
+    torch.cuda.empty_cache()
+    return out
+
+
 def decode_cache(batch: int) -> W.PagedCache:
     if batch >= DEC.B:
         return W.decode_workload_inputs(DEC, device="cuda")
@@ -349,6 +396,10 @@ def run_native(args, world, rank, local):
                "what": "fa_fwd through the Python binding, q/k/v copied from pinned host "
                        "memory and o/lse copied back inside the timed region"}
 
+    secondary = None
+    if do_fwd and not args.no_secondary:
+        secondary = secondary_workloads(fa, stream)
+
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and do_fwd:
         import oracle
@@ -391,6 +442,7 @@ def run_native(args, world, rank, local):
         "clocks": clocks,
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
+        "other_workloads": secondary,
     }
     if do_fwd:
         out["config"]["fwd"] = {"B": FWD.B, "H": FWD.H, "N": FWD.N, "d": FWD.d,
@@ -481,6 +533,8 @@ def main(argv=None):
                     help="CPU time budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the forward pass on the other workloads")
     ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
                     help="profiling aid: run one entry point only (the JSON line then "
                          "reports that part alone)")
