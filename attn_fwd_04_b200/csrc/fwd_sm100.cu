@@ -173,25 +173,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
     // ---- the work unit: (sequence/head, 256-row query block) --------------
+    // CTAs are numbered by rank first: rank r is the r-th 256-row block counted
+    // from the end of its sequence, so under a causal mask every head's (and
+    // sequence's) heaviest block is dispatched before any second-heaviest one
+    // and the last CTAs to start are the lightest.
+    const int units = p.B * p.H;
+    const int rank = static_cast<int>(blockIdx.x) / units;
+    const int unit = static_cast<int>(blockIdx.x) - rank * units;
     int len, seq_start = 0, bh = 0, h = 0;
     if constexpr (VARLEN) {
-        const int b = blockIdx.z;
-        h = blockIdx.y;
+        const int b = unit / p.H;
+        h = unit - b * p.H;
         const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
         // keep every access inside the [total, H, d] tensors whatever the offsets say
         const int c0 = min(max(s0, 0), p.total), c1 = min(max(s1, c0), p.total);
         const int c1m = min(c1, c0 + p.N);
-        if ((c0 != s0 || c1m != s1) && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        if ((c0 != s0 || c1m != s1) && rank == 0 && h == 0 && threadIdx.x == 0)
             record_error(p.err, FA_DEVERR_BAD_INPUT);
         seq_start = c0;
         len = c1m - c0;
     } else {
-        bh = blockIdx.y;
+        bh = unit;
         len = p.N;
     }
     const int nblk = (len + 2 * BM - 1) / (2 * BM);
-    // causal blocks near the end of the sequence carry the most work: start them first
-    const int blk = p.causal ? (nblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+    const int blk = p.causal ? (nblk - 1 - rank) : rank;
     if (blk < 0 || blk >= nblk) return;
     const int row0 = blk * 2 * BM;
     const int nkv_all = (len + BN - 1) / BN;
@@ -513,13 +519,11 @@ int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
-    dim3 grid;
-    const int blocks = (p.N + 2 * BM - 1) / (2 * BM);
-    if constexpr (VARLEN)
-        grid = dim3(blocks, p.H, p.B);
-    else
-        grid = dim3(blocks, p.B * p.H, 1);
-    kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+    // one CTA per (rank, sequence/head); rank-major order, see the kernel
+    const long long blocks = (p.N + 2 * BM - 1) / (2 * BM);
+    const long long ctas = blocks * p.B * p.H;
+    if (ctas > 0x7fffffffLL) return FA_ERR_SHAPE;
+    kern<<<dim3(static_cast<unsigned>(ctas)), kThreads, smem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
