@@ -43,6 +43,11 @@ def lib():
         L.oracle_gather_paged.restype = ctypes.c_int
         L.oracle_decode_paged.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64]
         L.oracle_decode_paged.restype = ctypes.c_int
+        L.oracle_attention_gqa.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64, I64,
+                                           ctypes.c_int, ctypes.c_double, P, I64]
+        L.oracle_attention_gqa.restype = ctypes.c_int
+        L.oracle_decode_paged_gqa.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64]
+        L.oracle_decode_paged_gqa.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         _LIB = L
@@ -89,6 +94,26 @@ def attention(q, k, v, causal: bool, scale: float, rows=None):
                                 _ptr(r), 0 if r is None else r.size)
     if rc != 0:
         raise RuntimeError(f"oracle_attention failed ({rc})")
+    return o, lse
+
+
+def attention_gqa(q, k, v, causal: bool, scale: float, rows=None):
+    """Grouped-query attention: q [B,H,N,d], k [B,Hkv,N,d], v [B,Hkv,N,dv];
+    query head h reads K/V head h // (H // Hkv).  Returns (o [B,H,N,dv],
+    lse [B,H,N]); `rows` as in attention()."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    dv = v.shape[-1]
+    assert k.shape == (B, Hkv, N, d) and v.shape == (B, Hkv, N, dv) and H % Hkv == 0
+    o = np.full((B, H, N, dv), np.nan)
+    lse = np.full((B, H, N), np.nan)
+    r = _i64(rows) if rows is not None else None
+    rc = lib().oracle_attention_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                    B, H, Hkv, N, d, dv, int(bool(causal)), float(scale),
+                                    _ptr(r), 0 if r is None else r.size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_gqa failed ({rc})")
     return o, lse
 
 
@@ -150,4 +175,22 @@ def decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int):
                                    _ptr(o), _ptr(lse), B, H, d, page_size)
     if rc != 0:
         raise RuntimeError(f"oracle_decode_paged failed ({rc})")
+    return o, lse
+
+
+def decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: int):
+    """Single-token decode with grouped K/V heads: q [B,H,d], pages
+    [P,Hkv,page_size,d]; returns (o [B,H,d], lse [B,H]).  Scale 1/sqrt(d)."""
+    q = _f64(q)
+    kp, vp = _f64(k_pages), _f64(v_pages)
+    pt, sl = _i64(page_table), _i64(seq_lens)
+    B, H, d = q.shape
+    Hkv = kp.shape[1]
+    assert H % Hkv == 0
+    o = np.zeros((B, H, d))
+    lse = np.zeros((B, H))
+    rc = lib().oracle_decode_paged_gqa(_ptr(q), _ptr(kp), _ptr(vp), _ptr(pt), _ptr(sl),
+                                       _ptr(o), _ptr(lse), B, H, Hkv, d, page_size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_decode_paged_gqa failed ({rc})")
     return o, lse

@@ -293,6 +293,98 @@ int oracle_decode_paged(const double *q, const double *k_pages,
     return rc;
 }
 
+/* Grouped-query attention (multi-query when Hkv = 1): H query heads share
+ * Hkv key/value heads, query head h reading K/V head h / (H / Hkv) (integer
+ * division), the variant the page "Flash Attention 是什么" names in its
+ * section 进阶学习路径 (item 4).  q is [B,H,N,d], k is [B,Hkv,N,d], v is
+ * [B,Hkv,N,dv], o is [B,H,N,dv], lse is [B,H,N]; the definition per row is
+ * the one above.  rows: optional flat query row ids (b*H + h)*N + i. */
+int oracle_attention_gqa(const double *q, const double *k, const double *v,
+                         double *o, double *lse, int64_t B, int64_t H, int64_t Hkv,
+                         int64_t N, int64_t d, int64_t dv, int causal, double scale,
+                         const int64_t *rows, int64_t nrows) {
+    if (B < 0 || H < 0 || N < 0 || d <= 0 || dv <= 0 || Hkv <= 0 || H % Hkv != 0) return -1;
+    const int64_t group = H / Hkv;
+    const int64_t total = rows ? nrows : B * H * N;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        if (!srow) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = 0; t < total; ++t) {
+                const int64_t r = rows ? rows[t] : t;
+                const int64_t bh = r / N, i = r % N;
+                const int64_t b = bh / H, h = bh % H;
+                const int64_t g = h / group;
+                const double *kb = k + (b * Hkv + g) * N * d;
+                const double *vb = v + (b * Hkv + g) * N * dv;
+                const int64_t nk = causal ? (i + 1) : N;
+                attention_row(q + r * d, kb, d, vb, dv, nk, d, dv, scale, srow,
+                              o + r * dv, lse + r);
+            }
+            free(srow);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/* Single-token decode with grouped K/V heads: q, o are [B,H,d]; the pages
+ * are [P_pool, Hkv, page_size, d]; query head h of sequence b attends to K/V
+ * head h / (H / Hkv) of its cached tokens.  lse (optional) is [B,H]. */
+int oracle_decode_paged_gqa(const double *q, const double *k_pages,
+                            const double *v_pages, const int64_t *page_table,
+                            const int64_t *seq_lens, double *o, double *lse,
+                            int64_t B, int64_t H, int64_t Hkv, int64_t d,
+                            int64_t page_size) {
+    if (page_size <= 0 || d <= 0 || H < 0 || B < 0 || Hkv <= 0 || H % Hkv != 0) return -1;
+    const int64_t group = H / Hkv;
+    int64_t off = 0;
+    int rc = 0;
+    for (int64_t b = 0; b < B && rc == 0; ++b) {
+        const int64_t len = seq_lens[b];
+        if (len < 0) return -1;
+        const int64_t np = (len + page_size - 1) / page_size;
+        double *kc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * Hkv * d));
+        double *vc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * Hkv * d));
+        if (!kc || !vc) {
+            free(kc);
+            free(vc);
+            return -2;
+        }
+        oracle_gather_paged(k_pages, page_table + off, &len, kc, 1, Hkv, d, page_size);
+        oracle_gather_paged(v_pages, page_table + off, &len, vc, 1, Hkv, d, page_size);
+        int failed = 0;
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+            if (!srow) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+#pragma omp for schedule(static)
+                for (int64_t h = 0; h < H; ++h) {
+                    const int64_t g = h / group;
+                    double l;
+                    attention_row(q + (b * H + h) * d, kc + g * d, Hkv * d, vc + g * d,
+                                  Hkv * d, len, d, d, 1.0 / sqrt((double)d), srow,
+                                  o + (b * H + h) * d, &l);
+                    if (lse) lse[b * H + h] = l;
+                }
+                free(srow);
+            }
+        }
+        if (failed) rc = -2;
+        free(kc);
+        free(vc);
+        off += np;
+    }
+    return rc;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

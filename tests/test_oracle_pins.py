@@ -428,3 +428,67 @@ def test_bf16_inputs_are_upcast_exactly():
                              x.float().double().numpy()[None, None],
                              x.float().double().numpy()[None, None], False, 0.5)
     np.testing.assert_array_equal(o, o2)
+
+
+# -- grouped-query attention (MQA/GQA: page "Flash Attention 是什么",
+#    section 进阶学习路径, item 4) --------------------------------------------
+
+@pytest.mark.parametrize("H,Hkv,causal", [(4, 2, True), (6, 3, False), (4, 1, True)])
+def test_gqa_brute_force_mpmath(H, Hkv, causal):
+    """Query head h against K/V head h // (H // Hkv), brute force per head;
+    a mapping by h % Hkv (the plausible slip) fails the (4, 2) and (6, 3)
+    cases, where the two mappings differ."""
+    N, d = 6, 4
+    q, k, v = _rand((1, H, N, d), 130), _rand((1, Hkv, N, d), 131), _rand((1, Hkv, N, d), 132)
+    o, lse = oracle.attention_gqa(q, k, v, causal, 0.6)
+    g = H // Hkv
+    for h in range(H):
+        ob, lb = _mp_attention(q[0, h], k[0, h // g], v[0, h // g], causal, 0.6)
+        np.testing.assert_allclose(o[0, h], ob, atol=TOL)
+        np.testing.assert_allclose(lse[0, h], lb, atol=TOL)
+
+
+def test_gqa_equals_attention_with_repeated_heads():
+    """GQA is ordinary attention after repeating each K/V head H // Hkv times
+    (np.repeat puts copies of head g at h = g*G .. g*G + G - 1)."""
+    B, H, Hkv, N, d = 2, 8, 2, 37, 8
+    q, k, v = _rand((B, H, N, d), 133), _rand((B, Hkv, N, d), 134), _rand((B, Hkv, N, d), 135)
+    for causal in (False, True):
+        o, lse = oracle.attention_gqa(q, k, v, causal, 0.4)
+        o2, l2 = oracle.attention(q, np.repeat(k, H // Hkv, axis=1),
+                                  np.repeat(v, H // Hkv, axis=1), causal, 0.4)
+        np.testing.assert_allclose(o, o2, atol=1e-15)
+        np.testing.assert_allclose(lse, l2, atol=1e-15)
+
+
+def test_mqa_zero_query_closed_form():
+    """Hkv = 1, q = 0: every head of every row averages the shared V (prefix
+    means when causal) and lse = ln(#keys)."""
+    B, H, N, d = 1, 3, 9, 4
+    k, v = _rand((B, 1, N, d), 136), _rand((B, 1, N, d), 137)
+    q = np.zeros((B, H, N, d))
+    o, lse = oracle.attention_gqa(q, k, v, True, 1.0)
+    for h in range(H):
+        for i in range(N):
+            np.testing.assert_allclose(o[0, h, i], v[0, 0, :i + 1].mean(axis=0), atol=1e-14)
+            assert abs(lse[0, h, i] - math.log(i + 1)) < 1e-14
+
+
+def test_decode_gqa_equals_brute_force():
+    H, Hkv, d, page_size = 6, 2, 8, 4
+    lens = [1, 5, 12]
+    kseqs = [_rand((L, Hkv, d), 140 + i) for i, L in enumerate(lens)]
+    vseqs = [_rand((L, Hkv, d), 150 + i) for i, L in enumerate(lens)]
+    n_pool = sum((L + page_size - 1) // page_size for L in lens) + 1
+    kpool, table, sl = _append_simulation(kseqs, Hkv, d, page_size, n_pool, 141)
+    vpool, _, _ = _append_simulation(vseqs, Hkv, d, page_size, n_pool, 141)
+    q = _rand((len(lens), H, d), 142)
+    o, lse = oracle.decode_paged_gqa(q, kpool, vpool, table, sl, page_size)
+    assert np.all(np.isfinite(o))
+    g = H // Hkv
+    for b in range(len(lens)):
+        for h in range(H):
+            ob, lb = _mp_attention(q[b, h][None], kseqs[b][:, h // g], vseqs[b][:, h // g],
+                                   False, 1 / math.sqrt(d))
+            np.testing.assert_allclose(o[b, h], ob[0], atol=TOL)
+            assert abs(lse[b, h] - lb[0]) < TOL
