@@ -135,12 +135,14 @@ int device_error_word(unsigned int** err, int* num_sms) {
 }
 }  // namespace fa
 
-extern "C" {
+namespace {
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-           int d, int causal, float scale, fa_stream_t stream) {
+// Fixed-length forward pass with H query heads and H_kv K/V heads.
+int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+              int H_kv, int N, int d, int causal, float scale, fa_stream_t stream) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
-    if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+    if (B < 1 || H < 1 || H_kv < 1 || N < 1) return FA_ERR_SHAPE;
+    if (H % H_kv != 0) return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(B) * H > 65535) return FA_ERR_SHAPE;
     if (N > 0x7fffffff - 128) return FA_ERR_SHAPE;
@@ -151,26 +153,43 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     int rc = lookup_device(&s);
     if (rc != FA_OK) return rc;
     CUtensorMap tq, tk, tv;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                                static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t dims_q[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                  static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t dims_kv[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                   static_cast<cuuint64_t>(B) * H_kv};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                    static_cast<cuuint64_t>(N) * d * 2};
     const cuuint32_t box[3] = {64, 128, 1};
-    if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tk, k, dims, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tv, v, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tq, q, dims_q, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims_kv, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims_kv, strides, box)) != FA_OK) return rc;
     fa::FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.cu_seqlens = nullptr;
     p.B = B;
     p.H = H;
+    p.H_kv = H_kv;
     p.N = N;
     p.total = 0;
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
     return fa::launch_fwd(p, tq, tk, tv, d, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, int causal, float scale, fa_stream_t stream) {
+    return fwd_fixed(q, k, v, o, lse, B, H, H, N, d, causal, scale, stream);
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int H_kv, int N, int d, int causal, float scale, fa_stream_t stream) {
+    return fwd_fixed(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, stream);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -202,6 +221,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
     p.cu_seqlens = cu_seqlens;
     p.B = B;
     p.H = H;
+    p.H_kv = H;
     p.N = max_seqlen;
     p.total = total;
     p.causal = causal ? 1 : 0;
@@ -210,13 +230,17 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
     return fa::launch_fwd(p, tq, tk, tv, d, true, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
-                    const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                    int d, int page_size, fa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+int decode_impl(const void* q, const void* k_pages, const void* v_pages,
+                const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                int H_kv, int d, int page_size, fa_stream_t stream) {
     if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !o) return FA_ERR_NULL;
-    if (B < 1 || H < 1) return FA_ERR_SHAPE;
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0) return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (page_size != 256) return FA_ERR_UNSUPPORTED;
+    if (!fa::decode_group_supported(H, H_kv)) return FA_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(B) * H * fa::kDecodeMaxSplits > 0x7fffffff) return FA_ERR_SHAPE;
     if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
         return FA_ERR_ALIGN;
@@ -228,8 +252,25 @@ int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
     if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits), st,
                                &ws)) != FA_OK)
         return rc;
-    return fa::launch_decode(q, k_pages, v_pages, page_table, seq_lens, o, B, H, d, page_size,
-                             fa::kDecodeMaxSplits, ws, s->err, s->num_sms, st);
+    return fa::launch_decode(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H_kv, d,
+                             page_size, fa::kDecodeMaxSplits, ws, s->err, s->num_sms, st);
+}
+}  // namespace
+
+extern "C" {
+
+int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                    int d, int page_size, fa_stream_t stream) {
+    return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H, d, page_size,
+                       stream);
+}
+
+int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v_pages,
+                        const int32_t* page_table, const int32_t* seq_lens, void* o, int B,
+                        int H, int H_kv, int d, int page_size, fa_stream_t stream) {
+    return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H_kv, d, page_size,
+                       stream);
 }
 
 int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t* seq_lens,

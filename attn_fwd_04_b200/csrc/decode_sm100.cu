@@ -160,19 +160,29 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 }
 
 constexpr int kDecTok = 64;           // tokens per ring stage (a quarter of a page)
-constexpr int kDecStages = 6;         // ring depth
 constexpr int kDecConsumerWarps = 8;
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;  // + one producer warp
 
-template <int D>
+// GH: query heads served by each K/V head (1 = multi-head attention).  A
+// unit's K/V chunks are staged once in shared memory and every query head of
+// the group is evaluated against them: each consumer warp carries HW =
+// min(GH, 4) query heads, and the consumer warps form GH / HW teams, each
+// team covering all tokens of a chunk for its heads.
+template <int D, int GH>
 struct DecSmem {
     static constexpr int LPT = D / 8;                              // lanes per token
     static constexpr int G = kDecConsumerWarps * 32 / LPT;         // token groups
-    alignas(128) uint8_t k[kDecStages][kDecTok * D * 2];
-    alignas(128) uint8_t v[kDecStages][kDecTok * D * 2];
-    float cm[2][G], cl[2][G];          // per-group partial state, by unit parity
-    float co[2][G][D];
-    uint64_t full[kDecStages], empty[kDecStages], cmb[2];
+    static constexpr int STAGES = 6;                               // ring depth
+    static constexpr int HW = GH < 4 ? GH : 4;                     // query heads per warp
+    static constexpr int TEAM = kDecConsumerWarps / (GH / HW);     // warps per team
+    // combine slots per head: one per token group (GH = 1), or one per warp
+    // of the head's team once the groups of a warp are merged with shuffles
+    static constexpr int C = GH == 1 ? G : TEAM;
+    alignas(128) uint8_t k[STAGES][kDecTok * D * 2];
+    alignas(128) uint8_t v[STAGES][kDecTok * D * 2];
+    float cm[2][GH][C], cl[2][GH][C];  // per-slot partial state, by unit parity
+    float co[2][GH][C][D];
+    uint64_t full[STAGES], empty[STAGES], cmb[2];
     int abort;
 };
 
@@ -189,20 +199,22 @@ struct UnitCursor {
 };
 
 struct UnitShape {
-    int b, s, h, tok0, ntok, cp, pt_base;
+    int b, s, h, tok0, ntok, cp, pt_base;  // h: the unit's K/V head
 };
 
+// Units of a sequence are (split, K/V head) pairs, split-major; Hk is the
+// number of K/V heads.
 __device__ __forceinline__ UnitShape unit_shape(int u, UnitCursor& cur,
                                                 const int32_t* __restrict__ unit_off,
                                                 const int32_t* __restrict__ page_off,
                                                 const int32_t* __restrict__ seq_lens, int B,
-                                                int H, int page_size, int max_splits) {
+                                                int Hk, int page_size, int max_splits) {
     cur.seek(unit_off, B, u);
     UnitShape us;
     us.b = cur.b;
     const int r = u - __ldg(unit_off + us.b);
-    us.s = r / H;
-    us.h = r % H;
+    us.s = r / Hk;
+    us.h = r % Hk;
     int len = __ldg(seq_lens + us.b);
     if (len < 0) len = 0;
     const int np = (len + page_size - 1) / page_size;
@@ -214,18 +226,21 @@ __device__ __forceinline__ UnitShape unit_shape(int u, UnitCursor& cur,
     return us;
 }
 
-template <int D>
+// H query heads, Hk = H / GH K/V heads.  Partial outputs are indexed by
+// (unit, query head within the group): u * GH + gi.
+template <int D, int GH>
 __global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_split_kernel(const __nv_bfloat16* __restrict__ q,
                            const __nv_bfloat16* __restrict__ k_pages,
                            const __nv_bfloat16* __restrict__ v_pages,
                            const int32_t* __restrict__ page_table,
-                           const int32_t* __restrict__ seq_lens, int B, int H, int page_size,
-                           int max_splits, const int32_t* __restrict__ page_off,
+                           const int32_t* __restrict__ seq_lens, int B, int H, int Hk,
+                           int page_size, int max_splits, const int32_t* __restrict__ page_off,
                            const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                            float* __restrict__ part_o, float scale_log2, unsigned int* err) {
-    using Sm = DecSmem<D>;
+    using Sm = DecSmem<D, GH>;
     constexpr int LPT = Sm::LPT, G = Sm::G;
+    constexpr int kDecStages = Sm::STAGES;
     constexpr int GPW = 32 / LPT;  // token groups per warp
     constexpr uint32_t kChunkBytes = kDecTok * D * 2;
     extern __shared__ uint8_t dec_smem_raw[];
@@ -253,7 +268,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         int g = 0;  // ring uses so far
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
-            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk,
                                             page_size, max_splits);
             const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
             constexpr int per_page = 256 / kDecTok;  // page_size is 256
@@ -266,7 +281,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                    FA_DEVERR_TIMEOUT, abort)) {
                         ok = false;
                     } else {
-                        const int64_t row = (static_cast<int64_t>(page) * H + us.h) * page_size +
+                        const int64_t row = (static_cast<int64_t>(page) * Hk + us.h) * page_size +
                                             (c % per_page) * kDecTok;
                         mbar_arrive_expect_tx(&sm.full[slot], 2 * kChunkBytes);
                         bulk_load(sm.k[slot], k_pages + row * D, kChunkBytes, &sm.full[slot]);
@@ -291,8 +306,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const unsigned gmask = (LPT == 32) ? 0xffffffffu : (((1u << LPT) - 1u) << (sub * LPT));
         int g = 0, k = 0;  // ring uses, units done
         bool ok = true;
+        if constexpr (GH == 1) {
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
-            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk,
                                             page_size, max_splits);
             float qf[8];
             {
@@ -361,11 +377,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             // combine the G groups of this unit (buffers double-buffered by unit parity)
             const int par = k & 1;
             if (gl == 0) {
-                sm.cm[par][grp] = m;
-                sm.cl[par][grp] = l;
+                sm.cm[par][0][grp] = m;
+                sm.cl[par][0][grp] = l;
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sm.co[par][grp][gl * 8 + i] = acc[i];
+            for (int i = 0; i < 8; ++i) sm.co[par][0][grp][gl * 8 + i] = acc[i];
             mbar_arrive(&sm.cmb[par]);
             if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) {
                 ok = false;
@@ -374,26 +390,207 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             if (threadIdx.x < D) {
                 float M = -INFINITY;
 #pragma unroll
-                for (int gi = 0; gi < G; ++gi) M = fmaxf(M, sm.cm[par][gi]);
+                for (int gi = 0; gi < G; ++gi) M = fmaxf(M, sm.cm[par][0][gi]);
                 float L = 0.f, o = 0.f;
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
-                    const float w = (sm.cm[par][gi] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][gi] - M);
-                    L += w * sm.cl[par][gi];
-                    o += w * sm.co[par][gi][threadIdx.x];
+                    const float w = (sm.cm[par][0][gi] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][0][gi] - M);
+                    L += w * sm.cl[par][0][gi];
+                    o += w * sm.co[par][0][gi][threadIdx.x];
                 }
                 part_o[static_cast<int64_t>(u) * D + threadIdx.x] = o / L;
                 if (threadIdx.x == 0) part_lse[u] = M + __log2f(L);
             }
         }
+        } else {
+        // ---- grouped query heads: GH queries against each staged chunk ----
+        // Warp w serves query heads HW * (w / TEAM) + {0 .. HW-1} of the
+        // unit's group.  A token row is spread over LG lanes holding NP packed
+        // fp32 pairs (8 dims, one 16-byte shared-memory load) each, as in the
+        // single-head path; products use the paired fp32 FMA.
+        constexpr int HW = Sm::HW;                      // query heads per warp
+        constexpr int TEAM = Sm::TEAM;                  // warps per team
+        constexpr int LG = D / 8;                       // lanes per token
+        constexpr int NP = D / LG / 2;                  // fp32 pairs per lane
+        constexpr int GW = 32 / LG;                     // token groups per warp
+        constexpr int GG = TEAM * GW;                   // token groups per team
+        constexpr int TPG = kDecTok / GG;               // tokens per group per chunk
+        static_assert(GH % HW == 0 && TPG >= 1 && kDecTok % GG == 0, "chunk split");
+        const int team = warp / TEAM, wt = warp - team * TEAM;
+        const int gsub = lane / LG, glane = lane % LG;
+        const int ggrp = wt * GW + gsub;
+        const unsigned gm = (LG == 32) ? 0xffffffffu : (((1u << LG) - 1u) << (gsub * LG));
+        // bf16 pairs (low element in the low half) -> packed fp32 pairs
+        auto widen = [](const uint4* src, uint64_t (&dst)[NP]) {
+#pragma unroll
+            for (int v = 0; v < NP / 4; ++v) {
+                const uint4 u4 = src[v];
+                const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[v * 4 + i] = (static_cast<uint64_t>(w[i] & 0xffff0000u) << 32) | (w[i] << 16);
+            }
+        };
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk,
+                                            page_size, max_splits);
+            uint64_t q2[HW][NP];
+#pragma unroll
+            for (int hi = 0; hi < HW; ++hi) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    q + (static_cast<int64_t>(us.b) * H + us.h * GH + team * HW + hi) * D +
+                    glane * 2 * NP);
+                widen(src, q2[hi]);
+                const uint64_t s2 = f2_pack(scale_log2, scale_log2);
+#pragma unroll
+                for (int i = 0; i < NP; ++i) q2[hi][i] = f2_mul(q2[hi][i], s2);
+            }
+            float m[HW], l[HW];
+            uint64_t acc[HW][NP];
+#pragma unroll
+            for (int hi = 0; hi < HW; ++hi) {
+                m[hi] = -INFINITY;
+                l[hi] = 0.f;
+#pragma unroll
+                for (int i = 0; i < NP; ++i) acc[hi][i] = 0;
+            }
+            const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
+            for (int c = 0; c < nchunks; ++c, ++g) {
+                const int slot = g % kDecStages;
+                if (!mbar_wait(&sm.full[slot], (g / kDecStages) & 1, err, FA_DEVERR_TIMEOUT,
+                               abort)) {
+                    ok = false;
+                    break;
+                }
+                float sc[HW][TPG];
+                const int base = c * kDecTok;
+#pragma unroll
+                for (int x = 0; x < TPG; ++x) {
+                    const int t = ggrp + x * GG;
+                    uint64_t k2[NP];
+                    widen(reinterpret_cast<const uint4*>(sm.k[slot] + t * D * 2 + glane * 4 * NP),
+                          k2);
+#pragma unroll
+                    for (int hi = 0; hi < HW; ++hi) {
+                        uint64_t d2 = f2_mul(q2[hi][0], k2[0]);
+#pragma unroll
+                        for (int i = 1; i < NP; ++i) d2 = f2_fma(q2[hi][i], k2[i], d2);
+                        float dot = f2_lo(d2) + f2_hi(d2);
+#pragma unroll
+                        for (int o = LG / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(gm, dot, o);
+                        sc[hi][x] = (base + t < us.ntok) ? dot : -INFINITY;
+                    }
+                }
+                float mn[HW];
+#pragma unroll
+                for (int hi = 0; hi < HW; ++hi) {
+                    float mb = sc[hi][0];
+#pragma unroll
+                    for (int x = 1; x < TPG; ++x) mb = fmaxf(mb, sc[hi][x]);
+                    mn[hi] = fmaxf(m[hi], mb);
+                    if (mn[hi] != -INFINITY && mn[hi] != m[hi]) {
+                        const float alpha = ex2_approx(m[hi] - mn[hi]);  // m = -inf -> 0
+                        l[hi] *= alpha;
+                        const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+                        for (int i = 0; i < NP; ++i) acc[hi][i] = f2_mul(acc[hi][i], a2);
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < TPG; ++x) {
+                    const int t = ggrp + x * GG;
+                    if (base + t < us.ntok) {
+                        uint64_t v2[NP];
+                        widen(reinterpret_cast<const uint4*>(sm.v[slot] + t * D * 2 +
+                                                             glane * 4 * NP),
+                              v2);
+#pragma unroll
+                        for (int hi = 0; hi < HW; ++hi) {
+                            const float pw = ex2_approx(sc[hi][x] - mn[hi]);
+                            l[hi] += pw;
+                            const uint64_t p2 = f2_pack(pw, pw);
+#pragma unroll
+                            for (int i = 0; i < NP; ++i) acc[hi][i] = f2_fma(p2, v2[i], acc[hi][i]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int hi = 0; hi < HW; ++hi)
+                    if (mn[hi] != -INFINITY) m[hi] = mn[hi];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.empty[slot]);
+            }
+            if (!ok) break;
+            // merge the token groups of this warp (their lanes glane hold the
+            // same columns) with shuffles, then the team's warps through
+            // shared memory
+            const int par = k & 1;
+#pragma unroll
+            for (int hi = 0; hi < HW; ++hi) {
+                const int hq = team * HW + hi;  // query head within the group
+                float mm = m[hi], ll = l[hi];
+#pragma unroll
+                for (int o = LG; o < 32; o <<= 1) {
+                    const float m2 = __shfl_xor_sync(0xffffffffu, mm, o);
+                    const float l2 = __shfl_xor_sync(0xffffffffu, ll, o);
+                    const float M = fmaxf(mm, m2);
+                    const float w1 = (mm == -INFINITY) ? 0.f : ex2_approx(mm - M);
+                    const float w2 = (m2 == -INFINITY) ? 0.f : ex2_approx(m2 - M);
+                    ll = ll * w1 + l2 * w2;
+                    const uint64_t w1p = f2_pack(w1, w1), w2p = f2_pack(w2, w2);
+#pragma unroll
+                    for (int i = 0; i < NP; ++i) {
+                        const float a_lo = __shfl_xor_sync(0xffffffffu, f2_lo(acc[hi][i]), o);
+                        const float a_hi = __shfl_xor_sync(0xffffffffu, f2_hi(acc[hi][i]), o);
+                        acc[hi][i] = f2_fma(acc[hi][i], w1p, f2_mul(f2_pack(a_lo, a_hi), w2p));
+                    }
+                    mm = M;
+                }
+                if (gsub == 0) {
+                    if (glane == 0) {
+                        sm.cm[par][hq][wt] = mm;
+                        sm.cl[par][hq][wt] = ll;
+                    }
+#pragma unroll
+                    for (int i = 0; i < NP; ++i) {
+                        sm.co[par][hq][wt][glane * 2 * NP + 2 * i] = f2_lo(acc[hi][i]);
+                        sm.co[par][hq][wt][glane * 2 * NP + 2 * i + 1] = f2_hi(acc[hi][i]);
+                    }
+                }
+            }
+            mbar_arrive(&sm.cmb[par]);
+            if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+                ok = false;
+                break;
+            }
+            for (int idx = threadIdx.x; idx < GH * D; idx += kDecConsumerWarps * 32) {
+                const int hi = idx / D, x = idx - hi * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < TEAM; ++w) M = fmaxf(M, sm.cm[par][hi][w]);
+                float L = 0.f, o = 0.f;
+#pragma unroll
+                for (int w = 0; w < TEAM; ++w) {
+                    const float wt = (sm.cm[par][hi][w] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][hi][w] - M);
+                    L += wt * sm.cl[par][hi][w];
+                    o += wt * sm.co[par][hi][w][x];
+                }
+                const int64_t pu = static_cast<int64_t>(u) * GH + hi;
+                part_o[pu * D + x] = o / L;
+                if (x == 0) part_lse[pu] = M + __log2f(L);
+            }
+        }
+        }
     }
 }
 
-// One warp per (sequence, head).
+
+// One warp per (sequence, query head).  Sequence b's partials start at
+// unit_off[b] * GH and are split-major with H per split.
 template <int D>
 __global__ void __launch_bounds__(128)
-    fa_decode_merge_kernel(const int32_t* __restrict__ seq_lens, int B, int H, int page_size,
-                           int max_splits, const int32_t* __restrict__ unit_off,
+    fa_decode_merge_kernel(const int32_t* __restrict__ seq_lens, int B, int H, int GH,
+                           int page_size, int max_splits, const int32_t* __restrict__ unit_off,
                            const float* __restrict__ part_lse, const float* __restrict__ part_o,
                            __nv_bfloat16* __restrict__ o) {
     constexpr int PER = D / 32;
@@ -406,7 +603,7 @@ __global__ void __launch_bounds__(128)
     const int np = (len + page_size - 1) / page_size;
     int ns, cp;
     split_shape(np, max_splits, ns, cp);
-    const int base = __ldg(unit_off + b);
+    const int base = __ldg(unit_off + b) * GH;
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32) M = fmaxf(M, part_lse[base + s * H + h]);
 #pragma unroll
@@ -462,11 +659,12 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <int D>
+template <int D, int GH>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
                        int num_sms, cudaStream_t stream) {
+    const int Hk = H / GH;
     const WorkspaceLayout L = layout_of(B, H, D, max_splits);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* page_off = reinterpret_cast<int32_t*>(ws);
@@ -474,26 +672,28 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
     int32_t* unit_off = tok_off + (B + 1);
     float* part_lse = reinterpret_cast<float*>(ws + L.lse_off);
     float* part_o = reinterpret_cast<float*>(ws + L.o_off);
-    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, H, page_size, max_splits,
+    // units are (split, K/V head) pairs
+    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, Hk, page_size, max_splits,
                                                           page_off, tok_off, unit_off, err);
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-    const size_t smem = sizeof(DecSmem<D>) + 128;
-    if (cudaFuncSetAttribute(fa_decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto split = fa_decode_split_kernel<D, GH>;
+    const size_t smem = sizeof(DecSmem<D, GH>) + 128;
+    if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
     // a persistent grid of the CTAs that are resident at once
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fa_decode_split_kernel<D>,
-                                                      kDecThreads, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, split, kDecThreads, smem) !=
+            cudaSuccess ||
         occ < 1)
         return FA_ERR_CUDA;
-    fa_decode_split_kernel<D><<<num_sms * occ, kDecThreads, smem, stream>>>(
+    split<<<num_sms * occ, kDecThreads, smem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pages),
-        static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, page_size,
+        static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, Hk, page_size,
         max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
-        seq_lens, B, H, page_size, max_splits, unit_off, part_lse, part_o,
+        seq_lens, B, H, GH, page_size, max_splits, unit_off, part_lse, part_o,
         static_cast<__nv_bfloat16*>(o));
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -519,16 +719,44 @@ size_t decode_workspace_bytes(int B, int H, int d, int max_splits) {
     return layout_of(B, H, d, max_splits).total;
 }
 
+namespace {
+template <int D>
+int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                    int Hk, int page_size, int max_splits, void* workspace, unsigned int* err,
+                    int num_sms, cudaStream_t stream) {
+    switch (H / Hk) {
+#define FA_DECODE_GH(GH)                                                                        \
+    case GH:                                                                                    \
+        return launch_decode_impl<D, GH>(q, k_pages, v_pages, page_table, seq_lens, o, B, H,   \
+                                         page_size, max_splits, workspace, err, num_sms, stream);
+        FA_DECODE_GH(1)
+        FA_DECODE_GH(2)
+        FA_DECODE_GH(4)
+        FA_DECODE_GH(8)
+#undef FA_DECODE_GH
+        default: return FA_ERR_UNSUPPORTED;
+    }
+}
+}  // namespace
+
+bool decode_group_supported(int H, int Hk) {
+    if (Hk < 1 || H % Hk != 0) return false;
+    const int g = H / Hk;
+    return g == 1 || g == 2 || g == 4 || g == 8;
+}
+
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                  int d, int page_size, int max_splits, void* workspace, unsigned int* err,
-                  int num_sms, cudaStream_t stream) {
+                  int Hk, int d, int page_size, int max_splits, void* workspace,
+                  unsigned int* err, int num_sms, cudaStream_t stream) {
+    if (!decode_group_supported(H, Hk)) return FA_ERR_UNSUPPORTED;
     if (d == 128)
-        return launch_decode_impl<128>(q, k_pages, v_pages, page_table, seq_lens, o, B, H,
-                                       page_size, max_splits, workspace, err, num_sms, stream);
+        return launch_decode_d<128>(q, k_pages, v_pages, page_table, seq_lens, o, B, H, Hk,
+                                    page_size, max_splits, workspace, err, num_sms, stream);
     if (d == 64)
-        return launch_decode_impl<64>(q, k_pages, v_pages, page_table, seq_lens, o, B, H,
-                                      page_size, max_splits, workspace, err, num_sms, stream);
+        return launch_decode_d<64>(q, k_pages, v_pages, page_table, seq_lens, o, B, H, Hk,
+                                   page_size, max_splits, workspace, err, num_sms, stream);
     return FA_ERR_UNSUPPORTED;
 }
 

@@ -23,6 +23,7 @@ struct FwdParams {
     float* lse;          // fp32 output
     const int32_t* cu_seqlens;  // varlen only
     int B, H, N;         // N: sequence length (fixed) or max_seqlen (varlen)
+    int H_kv;            // K/V heads; query head h reads K/V head h / (H / H_kv)
     int total;           // varlen: packed rows
     int causal;
     float scale_log2;    // scale * log2(e)
@@ -46,10 +47,12 @@ struct DecodePlan {
 
 size_t decode_workspace_bytes(int B, int H, int d, int max_splits);
 
+// H query heads over Hk K/V heads (H / Hk in {1, 2, 4, 8}).
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                  int d, int page_size, int max_splits, void* workspace, unsigned int* err,
-                  int num_sms, cudaStream_t stream);
+                  int Hk, int d, int page_size, int max_splits, void* workspace,
+                  unsigned int* err, int num_sms, cudaStream_t stream);
+bool decode_group_supported(int H, int Hk);
 
 // The current device's error word and SM count (sm_100 devices only).
 int device_error_word(unsigned int** err, int* num_sms);

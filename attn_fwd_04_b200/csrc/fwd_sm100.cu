@@ -176,11 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // CTAs are numbered by rank first: rank r is the r-th 256-row block counted
     // from the end of its sequence, so under a causal mask every head's (and
     // sequence's) heaviest block is dispatched before any second-heaviest one
-    // and the last CTAs to start are the lightest.
+    // and the last CTAs to start are the lightest.  With grouped K/V heads
+    // (H_kv < H) query head h reads K/V head h / (H / H_kv).
     const int units = p.B * p.H;
     const int rank = static_cast<int>(blockIdx.x) / units;
     const int unit = static_cast<int>(blockIdx.x) - rank * units;
-    int len, seq_start = 0, bh = 0, h = 0;
+    int len, seq_start = 0, bh = 0, h = 0, bkv = 0;
     if constexpr (VARLEN) {
         const int b = unit / p.H;
         h = unit - b * p.H;
@@ -194,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         len = c1m - c0;
     } else {
         bh = unit;
+        const int b = bh / p.H;
+        bkv = b * p.H_kv + (bh - b * p.H) / (p.H / p.H_kv);
         len = p.N;
     }
     const int nblk = (len + 2 * BM - 1) / (2 * BM);
@@ -248,19 +251,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row) {
+            // head: the fixed-length maps' outer coordinate (flat sequence/head)
+            auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row,
+                                 int head) {
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb) {
                     if constexpr (VARLEN)
                         tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, h, seq_start + row);
                     else
-                        tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, row, bh);
+                        tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, row, head);
                 }
             };
             for (int t = 0; t < 2; ++t) {
                 if (n_t[t] > 0) {
                     mbar_arrive_expect_tx(&sm.q_full[t], BM * D * 2);
-                    load_tile(sm.q[t], &tq, &sm.q_full[t], row0 + t * BM);
+                    load_tile(sm.q[t], &tq, &sm.q_full[t], row0 + t * BM, bh);
                 }
             }
             int issued = 0;  // ring uses issued so far
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (u / kSlots) & 1;
                 if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
                 mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
-                load_tile(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], (u >> 1) * BN);
+                load_tile(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], (u >> 1) * BN, bkv);
                 issued = u + 1;
             }
             // every copy this CTA started must land before it exits

@@ -24,7 +24,8 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_noalloc",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
+           "fa_decode_paged_noalloc",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
            "fa_status_str", "fa_version")
@@ -48,8 +49,10 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+        L.fa_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_gather_paged.argtypes = [P, P, P, P, I, I, I, I, P]
         L.fa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
@@ -58,7 +61,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_noalloc",
+        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen", "fa_decode_paged",
+                     "fa_decode_paged_gqa", "fa_decode_paged_noalloc",
                      "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
                      "fa_version"):
@@ -114,6 +118,30 @@ def fa_fwd(q, k, v, causal: bool, scale: Optional[float] = None, o=None, lse=Non
     return o, lse
 
 
+def fa_fwd_gqa(q, k, v, causal: bool, scale: Optional[float] = None, o=None, lse=None,
+               stream=None):
+    """Grouped-query forward: q [B,H,N,d], k/v [B,H_kv,N,d] bf16 with H a
+    multiple of H_kv -> (o [B,H,N,d], lse [B,H,N] fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    if k.shape != (B, H_kv, N, d) or v.shape != k.shape:
+        raise ValueError("k, v must be [B,H_kv,N,d] with q's B, N, d")
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(o, "o", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    rc = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, H, H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_fwd_gqa")
+    return o, lse
+
+
 def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
                   scale: Optional[float] = None, o=None, lse=None, stream=None):
     """Forward over packed [total,H,d] sequences -> (o, lse [H,total] fp32)."""
@@ -151,6 +179,26 @@ def fa_decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 
                                page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
                                B, H, d, int(page_size), _stream(stream))
     _raise_if(rc, "fa_decode_paged")
+    return o
+
+
+def fa_decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 256, o=None,
+                        stream=None):
+    """Decode with grouped K/V heads: q [B,H,d], pages [P,H_kv,page_size,d]
+    -> o [B,H,d] bf16."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, H, d = q.shape
+    H_kv = k_pages.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    rc = lib().fa_decode_paged_gqa(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                   page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
+                                   B, H, H_kv, d, int(page_size), _stream(stream))
+    _raise_if(rc, "fa_decode_paged_gqa")
     return o
 
 

@@ -124,6 +124,18 @@ def custom_fwd_inputs(B, H, N, d, seed, std=1.0, device="cpu"):
     return fwd_inputs(FwdWorkload("custom", B, H, N, d, False, seed, std), device)
 
 
+def gqa_fwd_inputs(B, H, H_kv, N, d, seed, std=1.0, device=None):
+    """q [B,H,N,d] and k, v [B,H_kv,N,d] (grouped-query attention), same
+    recipe: q, then k, then v from one seeded generator."""
+    n = B * H * N * d
+    dev = _device_for(n, device)
+    g = _gen(seed, dev)
+    q = _randn_bf16((B, H, N, d), g, std, dev)
+    k = _randn_bf16((B, H_kv, N, d), g, std, dev)
+    v = _randn_bf16((B, H_kv, N, d), g, std, dev)
+    return q, k, v
+
+
 def varlen_lengths(B: int, lo: int, hi: int, seed: int) -> List[int]:
     g = _gen(seed, "cpu")
     return [int(x) for x in torch.randint(lo, hi + 1, (B,), generator=g)]
@@ -166,7 +178,7 @@ class PagedCache:
 
 def paged_inputs(B: int, H: int, d: int, lengths: List[int], seed: int,
                  page_size: int = PAGE_SIZE, device: Optional[str] = None,
-                 poison_unused: bool = True) -> PagedCache:
+                 poison_unused: bool = True, H_kv: Optional[int] = None) -> PagedCache:
     """A paged KV cache holding `lengths[b]` tokens for sequence b.
 
     The pool holds exactly the pages the sequences need; the pages are
@@ -174,21 +186,23 @@ def paged_inputs(B: int, H: int, d: int, lengths: List[int], seed: int,
     a sequence sit at unrelated pool slots.  The page table lists every
     sequence's pages in order, sequences back to back.  With poison_unused,
     the slots past a sequence's last token in its last page hold NaN, so any
-    read of them shows up in the output.
+    read of them shows up in the output.  H_kv (default H) is the number of
+    K/V heads the pages hold (grouped-query caches); q keeps H heads.
     """
+    Hk = H if H_kv is None else H_kv
     pages_per_seq = [(int(L) + page_size - 1) // page_size for L in lengths]
     P = sum(pages_per_seq)
-    n = max(P, 1) * H * page_size * d
+    n = max(P, 1) * Hk * page_size * d
     dev = _device_for(n, device)
     g = _gen(seed, dev)
     q = _randn_bf16((B, H, d), g, 1.0, dev)
-    k_pages = torch.empty((P, H, page_size, d), dtype=torch.bfloat16, device=dev)
-    v_pages = torch.empty((P, H, page_size, d), dtype=torch.bfloat16, device=dev)
-    chunk = max(1, (1 << 26) // (H * page_size * d))
+    k_pages = torch.empty((P, Hk, page_size, d), dtype=torch.bfloat16, device=dev)
+    v_pages = torch.empty((P, Hk, page_size, d), dtype=torch.bfloat16, device=dev)
+    chunk = max(1, (1 << 26) // (Hk * page_size * d))
     for dst in (k_pages, v_pages):
         for p0 in range(0, P, chunk):
             p1 = min(P, p0 + chunk)
-            dst[p0:p1] = _randn_bf16((p1 - p0, H, page_size, d), g, 1.0, dev)
+            dst[p0:p1] = _randn_bf16((p1 - p0, Hk, page_size, d), g, 1.0, dev)
     gperm = _gen(seed + 1, "cpu")
     perm = torch.randperm(P, generator=gperm).to(torch.int32)
     if poison_unused:

@@ -90,6 +90,23 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
            int B, int H, int N, int d, int causal, float scale, fa_stream_t stream);
 
 /*
+ * fa_fwd_gqa -- fa_fwd with fewer K/V heads than query heads (grouped-query
+ * attention; multi-query attention is H_kv = 1).  The page "Flash Attention
+ * 是什么" names adapting the fused method to MQA and GQA as the next step
+ * (section 进阶学习路径, item 4); the arithmetic per head is fa_fwd's.
+ *
+ * Query head h reads K/V head h / (H / H_kv):
+ *   o[b,h,i,:] = sum_j softmax_j(scale * q[b,h,i,:] . k[b,g,j,:]) v[b,g,j,:],
+ *   g = h / (H / H_kv) (integer division), same mask and lse as fa_fwd.
+ * Layout: q, o are [B, H, N, d] bf16; k, v are [B, H_kv, N, d] bf16; lse is
+ * [B, H, N] fp32.  H must be a multiple of H_kv (else FA_ERR_SHAPE).
+ * fa_fwd is this call with H_kv = H.  Other limits, ownership and errors as
+ * fa_fwd.
+ */
+FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int H_kv, int N, int d, int causal, float scale, fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- the forward pass over B sequences of different lengths
  * packed back to back (the variable-length batches of the page "Flash
  * Attention 是什么", section 典型应用场景).
@@ -138,6 +155,24 @@ FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, f
 FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                     const int32_t* page_table, const int32_t* seq_lens, void* o,
                     int B, int H, int d, int page_size, fa_stream_t stream);
+
+/*
+ * fa_decode_paged_gqa -- fa_decode_paged with grouped K/V heads (grouped- or
+ * multi-query attention, the variants named by the page "Flash Attention
+ * 是什么", section 进阶学习路径, item 4).
+ *   q, o       : [B, H, d] bf16
+ *   k_pages,
+ *   v_pages    : [P, H_kv, page_size, d] bf16 -- the cache holds H_kv heads
+ * Query head h attends to K/V head h / (H / H_kv) of its sequence's cached
+ * tokens; everything else (page table, lengths, scale 1/sqrt(d), no mask,
+ * workspace) as fa_decode_paged.  H / H_kv must be 1, 2, 4 or 8
+ * (FA_ERR_UNSUPPORTED otherwise; FA_ERR_SHAPE if H is not a multiple of
+ * H_kv).  Each (page, K/V head) slice is read from device memory once and
+ * serves all H / H_kv query heads of its group.
+ */
+FA_API int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* seq_lens, void* o,
+                    int B, int H, int H_kv, int d, int page_size, fa_stream_t stream);
 
 /*
  * fa_gather_paged -- copy the cached tokens of every sequence out of the page

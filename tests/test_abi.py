@@ -56,6 +56,11 @@ def fwd(L, q=A, k=A, v=A, o=A, lse=A, B=1, H=2, N=256, d=64, causal=0, scale=0.1
     return L.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, S)
 
 
+def fwd_gqa(L, q=A, k=A, v=A, o=A, lse=A, B=1, H=8, H_kv=2, N=256, d=128, causal=1,
+            scale=0.1):
+    return L.fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, S)
+
+
 def varlen(L, q=A, k=A, v=A, o=A, lse=A, cu=A, B=2, H=2, total=100, maxlen=60, d=128,
            causal=1, scale=0.1):
     return L.fa_fwd_varlen(q, k, v, o, lse, cu, B, H, total, maxlen, d, causal, scale, S)
@@ -63,6 +68,10 @@ def varlen(L, q=A, k=A, v=A, o=A, lse=A, cu=A, B=2, H=2, total=100, maxlen=60, d
 
 def decode(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=2, d=128, ps=256):
     return L.fa_decode_paged(q, kp, vp, pt, sl, o, B, H, d, ps, S)
+
+
+def decode_gqa(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=8, H_kv=2, d=128, ps=256):
+    return L.fa_decode_paged_gqa(q, kp, vp, pt, sl, o, B, H, H_kv, d, ps, S)
 
 
 def gather(L, pages=A, pt=A, sl=A, out=A, B=4, H=2, d=128, ps=256):
@@ -84,6 +93,15 @@ def test_fwd_argument_errors(L):
     assert fwd(L, o=MIS) == fa.FA_ERR_ALIGN
 
 
+def test_fwd_gqa_argument_errors(L):
+    assert fwd_gqa(L, k=None) == fa.FA_ERR_NULL
+    assert fwd_gqa(L, H_kv=0) == fa.FA_ERR_SHAPE
+    assert fwd_gqa(L, H_kv=3) == fa.FA_ERR_SHAPE        # H not a multiple of H_kv
+    assert fwd_gqa(L, H=4, H_kv=8) == fa.FA_ERR_SHAPE
+    assert fwd_gqa(L, d=80) == fa.FA_ERR_UNSUPPORTED
+    assert fwd_gqa(L, v=MIS) == fa.FA_ERR_ALIGN
+
+
 def test_varlen_argument_errors(L):
     assert varlen(L, cu=None) == fa.FA_ERR_NULL
     assert varlen(L, total=0) == fa.FA_ERR_SHAPE
@@ -100,6 +118,13 @@ def test_decode_argument_errors(L):
     assert decode(L, ps=16) == fa.FA_ERR_UNSUPPORTED
     assert decode(L, d=80) == fa.FA_ERR_UNSUPPORTED
     assert decode(L, kp=MIS) == fa.FA_ERR_ALIGN
+    assert decode_gqa(L, vp=None) == fa.FA_ERR_NULL
+    assert decode_gqa(L, H_kv=0) == fa.FA_ERR_SHAPE
+    assert decode_gqa(L, H_kv=3) == fa.FA_ERR_SHAPE       # 8 is not a multiple of 3
+    assert decode_gqa(L, H=24, H_kv=8) == fa.FA_ERR_UNSUPPORTED  # group of 3
+    assert decode_gqa(L, H=32, H_kv=2) == fa.FA_ERR_UNSUPPORTED  # group of 16
+    assert decode_gqa(L, ps=128) == fa.FA_ERR_UNSUPPORTED
+    assert decode_gqa(L, o=MIS) == fa.FA_ERR_ALIGN
     assert gather(L, out=None) == fa.FA_ERR_NULL
     assert gather(L, ps=255) == fa.FA_ERR_UNSUPPORTED
     assert gather(L, pages=MIS) == fa.FA_ERR_ALIGN
@@ -109,7 +134,9 @@ def test_decode_argument_errors(L):
 def test_valid_call_without_gpu_reports_cuda_error(L):
     # arguments pass validation; the device lookup then fails cleanly
     assert fwd(L) == fa.FA_ERR_CUDA
+    assert fwd_gqa(L) == fa.FA_ERR_CUDA
     assert decode(L) == fa.FA_ERR_CUDA
+    assert decode_gqa(L) == fa.FA_ERR_CUDA
     code = ctypes.c_int(7)
     assert L.fa_get_device_error(ctypes.byref(code), S) == fa.FA_ERR_CUDA
 

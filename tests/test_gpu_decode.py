@@ -170,3 +170,50 @@ def test_paged_gather_workload_sampled_bit_exact():
         got = out[int(starts[b]):int(starts[b + 1])].cpu()
         assert torch.equal(got.view(torch.int16),
                            torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16))
+
+
+# -- grouped K/V heads (fa_decode_paged_gqa) ---------------------------------------
+
+def _decode_gqa(c: W.PagedCache):
+    o = torch.full_like(c.q, float("nan"))
+    fa.fa_decode_paged_gqa(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, c.page_size,
+                           o=o)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return o
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (8, 1), (16, 2), (3, 3)])
+def test_decode_gqa_small_full_compare(d, H, H_kv):
+    lens = [1, 255, 257, 1000, 4103, 0]
+    c = W.paged_inputs(len(lens), H, d, lens, seed=40 + H + H_kv, device="cpu", H_kv=H_kv)
+    o = _decode_gqa(_on_gpu(c))
+    o_ref, _ = oracle.decode_paged_gqa(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
+    assert torch.all(o[-1] == 0)  # the empty sequence
+    assert_o_close(to64(o), o_ref, f"decode gqa d={d} H={H} H_kv={H_kv}")
+
+
+def test_decode_gqa_group1_equals_decode():
+    """With one query head per K/V head the grouped entry point is decode."""
+    lens = [700, 3, 2049]
+    c = W.paged_inputs(3, 4, 128, lens, seed=48, device="cpu")
+    g = _on_gpu(c)
+    assert torch.equal(_decode_gqa(g), _decode(g))
+
+
+def test_decode_gqa_workload_sampled():
+    """The paged-decode workload's lengths with 8 K/V heads for 32 query heads."""
+    w = W.PAGED_DECODE
+    lengths = W.varlen_lengths(w.B, w.len_lo, w.len_hi, w.seed)
+    c = W.paged_inputs(w.B, w.H, w.d, lengths, w.seed, w.page_size, device="cuda", H_kv=8)
+    c = W.PagedCache(c.q, c.k_pages, c.v_pages, c.page_table.cuda(), c.seq_lens.cuda(),
+                     c.page_size, c.pages_per_seq)
+    o = _decode_gqa(c)
+    assert bool(torch.isfinite(o).all())
+    got, ref = [], []
+    for b in (0, 17, w.B - 1):
+        kp, vp, pt, sl = _mini(c, b)
+        o_ref, _ = oracle.decode_paged_gqa(c.q[b:b + 1].cpu(), kp, vp, pt, sl, PS)
+        got.append(to64(o[b:b + 1]))
+        ref.append(o_ref)
+    assert_o_close(np.concatenate(got), np.concatenate(ref), "gqa decode workload")

@@ -223,3 +223,67 @@ def test_bounded_wait_reports_timeout():
     o, lse = _fwd_gpu(q, k, v, True, 0.125)
     o_ref, lse_ref = oracle.attention(q, k, v, True, 0.125)
     assert_o_close(to64(o), o_ref, "after timeout")
+
+
+# -- grouped-query attention (fa_fwd_gqa) ----------------------------------------
+
+def _gqa_gpu(q, k, v, causal, scale):
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    B, H, N, d = q.shape
+    o = torch.full_like(qc, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda")
+    fa.fa_fwd_gqa(qc, kc, vc, causal, scale, o=o, lse=lse)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return o, lse
+
+
+# (B, H, H_kv, N, d): groups of 2, 3, 8, 1 (plain multi-head) and 4
+GQA_SHAPES = [(1, 4, 2, 129, 128), (2, 6, 3, 300, 64), (1, 3, 1, 255, 128), (1, 8, 1, 1000, 64),
+              (1, 2, 2, 127, 128), (2, 8, 4, 1, 64), (1, 16, 2, 2049, 128)]
+
+
+@pytest.mark.parametrize("shape", GQA_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_full_compare(shape, causal):
+    B, H, Hkv, N, d = shape
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=200 + N + H, device="cpu")
+    scale = 1 / math.sqrt(d)
+    o, lse = _gqa_gpu(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention_gqa(q, k, v, causal, scale)
+    assert_o_close(to64(o), o_ref, f"gqa {shape}")
+    assert_lse_close(to64(lse), lse_ref, f"gqa {shape}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_equals_fwd_on_repeated_heads(causal):
+    """A query head's rows are computed with the same tiles in the same order
+    whether its K/V head is shared or repeated (fa_fwd): the results are
+    bit-identical."""
+    B, H, Hkv, N, d = 2, 8, 2, 700, 128
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=17, device="cpu")
+    o, lse = _gqa_gpu(q, k, v, causal, 0.1)
+    g = H // Hkv
+    o2, l2 = _fwd_gpu(q, k.repeat_interleave(g, dim=1), v.repeat_interleave(g, dim=1), causal, 0.1)
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+def test_gqa_long_prefill_sampled():
+    """The long-prefill shape with 8 K/V heads for 32 query heads (groups of
+    4), sampled rows against the oracle."""
+    B, H, Hkv, N, d = 1, 32, 8, 16384, 128
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=21, device="cuda")
+    scale = 1 / math.sqrt(d)
+    o, lse = fa.fa_fwd_gqa(q, k, v, True, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    qc, kc, vc, oc, lc = q.cpu(), k.cpu(), v.cpu(), o.cpu(), lse.cpu()
+    got_o, ref_o, got_l, ref_l = [], [], [], []
+    for h in (0, 1, 5, 30, 31):
+        rows = sample_rows(N, 24, 500 + h)
+        o_ref, lse_ref = oracle.attention_gqa(qc[:, h:h + 1], kc[:, h // 4:h // 4 + 1],
+                                              vc[:, h // 4:h // 4 + 1], True, scale, rows=rows)
+        got_o.append(to64(oc[0, h, rows]))
+        ref_o.append(o_ref[0, 0, rows])
+        got_l.append(to64(lc[0, h, rows]))
+        ref_l.append(lse_ref[0, 0, rows])
+    assert_o_close(np.concatenate(got_o), np.concatenate(ref_o), "gqa long prefill")
+    assert_lse_close(np.concatenate(got_l), np.concatenate(ref_l), "gqa long prefill")
