@@ -48,6 +48,11 @@ def lib():
         L.oracle_attention_gqa.restype = ctypes.c_int
         L.oracle_decode_paged_gqa.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64]
         L.oracle_decode_paged_gqa.restype = ctypes.c_int
+        L.oracle_append_paged.argtypes = [P, P, P, P, P, I64, I64, I64, I64]
+        L.oracle_append_paged.restype = ctypes.c_int
+        L.oracle_prefill_paged.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64,
+                                           ctypes.c_int, ctypes.c_double]
+        L.oracle_prefill_paged.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         _LIB = L
@@ -193,4 +198,40 @@ def decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: int):
                                        _ptr(o), _ptr(lse), B, H, Hkv, d, page_size)
     if rc != 0:
         raise RuntimeError(f"oracle_decode_paged_gqa failed ({rc})")
+    return o, lse
+
+
+def append_paged(pages, page_table, seq_lens, new_rows, cu_new, page_size: int):
+    """Pages after writing each sequence's new rows [cu_new[B],Hkv,d] at its
+    last positions (seq_lens are the lengths after the append).  Returns a new
+    fp64 array; the input is not modified."""
+    out = _f64(pages).copy()
+    pt, sl, cu = _i64(page_table), _i64(seq_lens), _i64(cu_new)
+    rows = _f64(new_rows)
+    _, Hkv, ps, d = out.shape
+    assert ps == page_size and rows.shape[1:] == (Hkv, d)
+    rc = lib().oracle_append_paged(_ptr(out), _ptr(pt), _ptr(sl), _ptr(rows), _ptr(cu),
+                                   sl.size, Hkv, d, page_size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_append_paged failed ({rc})")
+    return out
+
+
+def prefill_paged(q, k_pages, v_pages, page_table, seq_lens, cu_q, page_size: int,
+                  causal: bool, scale: float):
+    """Queries [cu_q[B],H,d] that are the last positions of their cached
+    sequences, attending through the page table; returns (o [cu_q[B],H,d],
+    lse [H,cu_q[B]])."""
+    q = _f64(q)
+    kp, vp = _f64(k_pages), _f64(v_pages)
+    pt, sl, cu = _i64(page_table), _i64(seq_lens), _i64(cu_q)
+    total, H, d = q.shape
+    Hkv = kp.shape[1]
+    o = np.full((total, H, d), np.nan)
+    lse = np.full((H, total), np.nan)
+    rc = lib().oracle_prefill_paged(_ptr(q), _ptr(kp), _ptr(vp), _ptr(pt), _ptr(sl), _ptr(cu),
+                                    _ptr(o), _ptr(lse), sl.size, H, Hkv, d, page_size,
+                                    int(bool(causal)), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_prefill_paged failed ({rc})")
     return o, lse

@@ -385,6 +385,98 @@ int oracle_decode_paged_gqa(const double *q, const double *k_pages,
     return rc;
 }
 
+/* Appending new tokens to the paged cache, the step before decode in the
+ * serving loop of the page "“Flash”不是那个被时代淘汰的插件" (0539edu.com),
+ * section 2: a new token's K (or V) row is written into the page that holds
+ * its position.  Sequence b holds seq_lens[b] tokens AFTER the append; its
+ * n_b = cu_new[b+1] - cu_new[b] new tokens are its last n_b positions
+ * (pos = seq_lens[b] - n_b + i for new token i), and the packed page table
+ * already lists every page those positions need.  pages is [P, Hkv, page_size,
+ * d] and is updated in place; new_rows is [cu_new[B], Hkv, d]. */
+int oracle_append_paged(double *pages, const int64_t *page_table, const int64_t *seq_lens,
+                        const double *new_rows, const int64_t *cu_new, int64_t B,
+                        int64_t Hkv, int64_t d, int64_t page_size) {
+    if (page_size <= 0 || d <= 0 || Hkv <= 0 || B < 0) return -1;
+    int64_t off = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t len = seq_lens[b];
+        const int64_t n = cu_new[b + 1] - cu_new[b];
+        if (len < 0 || n < 0 || n > len) return -1;
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t pos = len - n + i;
+            const int64_t page = page_table[off + pos / page_size];
+            const int64_t slot = pos % page_size;
+            for (int64_t h = 0; h < Hkv; ++h) {
+                const double *src = new_rows + ((cu_new[b] + i) * Hkv + h) * d;
+                double *dst = pages + ((page * Hkv + h) * page_size + slot) * d;
+                for (int64_t c = 0; c < d; ++c) dst[c] = src[c];
+            }
+        }
+        off += (len + page_size - 1) / page_size;
+    }
+    return 0;
+}
+
+/* Prefill over the paged cache (decode with several query tokens): sequence
+ * b caches seq_lens[b] tokens, the last q_b = cu_q[b+1] - cu_q[b] of which are
+ * its new query tokens.  Query i of sequence b sits at position
+ * seq_lens[b] - q_b + i and, with causal set, sees the keys at positions up to
+ * its own (the mask aligned to the end of the sequence); without it, all
+ * seq_lens[b] keys.  q, o are [cu_q[B], H, d]; lse is [H, cu_q[B]]; the pages
+ * are [P, Hkv, page_size, d] with query head h reading K/V head h / (H/Hkv).
+ * The sequence's K/V are gathered first, then the definition applies. */
+int oracle_prefill_paged(const double *q, const double *k_pages, const double *v_pages,
+                         const int64_t *page_table, const int64_t *seq_lens,
+                         const int64_t *cu_q, double *o, double *lse, int64_t B, int64_t H,
+                         int64_t Hkv, int64_t d, int64_t page_size, int causal, double scale) {
+    if (page_size <= 0 || d <= 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || B < 0) return -1;
+    const int64_t group = H / Hkv;
+    const int64_t total_q = cu_q[B];
+    int64_t off = 0;
+    int rc = 0;
+    for (int64_t b = 0; b < B && rc == 0; ++b) {
+        const int64_t len = seq_lens[b];
+        const int64_t nq = cu_q[b + 1] - cu_q[b];
+        if (len < 0 || nq < 0 || nq > len) return -1;
+        double *kc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * Hkv * d));
+        double *vc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * Hkv * d));
+        if (!kc || !vc) {
+            free(kc);
+            free(vc);
+            return -2;
+        }
+        oracle_gather_paged(k_pages, page_table + off, &len, kc, 1, Hkv, d, page_size);
+        oracle_gather_paged(v_pages, page_table + off, &len, vc, 1, Hkv, d, page_size);
+        int failed = 0;
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+            if (!srow) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+#pragma omp for schedule(dynamic, 4)
+                for (int64_t t = 0; t < nq * H; ++t) {
+                    const int64_t i = t / H, h = t % H;
+                    const int64_t g = h / group;
+                    const int64_t row = cu_q[b] + i;
+                    const int64_t nk = causal ? (len - nq + i + 1) : len;
+                    double l;
+                    attention_row(q + (row * H + h) * d, kc + g * d, Hkv * d, vc + g * d,
+                                  Hkv * d, nk, d, d, scale, srow, o + (row * H + h) * d, &l);
+                    lse[h * total_q + row] = l;
+                }
+                free(srow);
+            }
+        }
+        if (failed) rc = -2;
+        free(kc);
+        free(vc);
+        off += (len + page_size - 1) / page_size;
+    }
+    return rc;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

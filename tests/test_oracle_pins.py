@@ -492,3 +492,92 @@ def test_decode_gqa_equals_brute_force():
                                    False, 1 / math.sqrt(d))
             np.testing.assert_allclose(o[b, h], ob[0], atol=TOL)
             assert abs(lse[b, h] - lb[0]) < TOL
+
+
+# -- appending to the paged cache and prefill through it (page
+#    "“Flash”不是那个被时代淘汰的插件", 0539edu.com, section 2) ------------------
+
+def _split_append(lens_before, n_new, Hkv, d, page_size, seed, table_seed=7):
+    """A cache built by the append simulation for the first lens_before[b]
+    tokens, with the pages for the n_new[b] further tokens already owned;
+    returns (pool, table, lens_after, full token arrays per sequence).  Pools
+    built with the same table_seed share their page table (K and V)."""
+    lens_after = [a + n for a, n in zip(lens_before, n_new)]
+    full = [_rand((L, Hkv, d), seed + i) for i, L in enumerate(lens_after)]
+    n_pool = sum((L + page_size - 1) // page_size for L in lens_after) + 2
+    pool, table, sl = _append_simulation(full, Hkv, d, page_size, n_pool, table_seed)
+    return pool, table, sl, full
+
+
+def test_append_then_gather_is_concatenation():
+    """Writing the new rows over their slots restores exactly the tokens a
+    one-at-a-time append produced: gather(append(...)) == concatenation."""
+    Hkv, d, ps = 2, 3, 4
+    lens_before, n_new = [0, 3, 4, 9, 5], [5, 1, 4, 0, 7]
+    pool, table, sl, full = _split_append(lens_before, n_new, Hkv, d, ps, 160)
+    # wipe the new tokens' slots, then append them back
+    wiped = pool.copy()
+    for b, (a, n) in enumerate(zip(lens_before, n_new)):
+        off = sum((L + ps - 1) // ps for L in sl[:b])
+        for pos in range(a, a + n):
+            wiped[table[off + pos // ps], :, pos % ps, :] = np.nan
+    new_rows = np.concatenate([full[b][a:] for b, a in enumerate(lens_before)], axis=0)
+    cu = np.concatenate([[0], np.cumsum(n_new)])
+    out = oracle.append_paged(wiped, table, sl, new_rows, cu, ps)
+    np.testing.assert_array_equal(oracle.gather_paged(out, table, sl, ps),
+                                  np.concatenate(full, axis=0))
+    # slots nobody owns (NaN before) stay NaN: nothing else was written
+    assert np.array_equal(np.isnan(out), np.isnan(pool))
+
+
+def test_prefill_paged_brute_force_bottom_right_mask():
+    """Queries are the LAST q_b positions: query i sees keys 0..L-q_b+i.  A
+    top-left mask (keys 0..i) is the plausible slip and fails here."""
+    H, Hkv, d, ps = 4, 2, 4, 4
+    lens, nq = [7, 10, 3], [3, 10, 1]
+    pool_k, table, sl, ks = _split_append([0, 0, 0], lens, Hkv, d, ps, 170)
+    pool_v, table_v, _, vs = _split_append([0, 0, 0], lens, Hkv, d, ps, 170 + 50)
+    assert np.array_equal(table, table_v)
+    cu = np.concatenate([[0], np.cumsum(nq)])
+    q = _rand((int(cu[-1]), H, d), 171)
+    for causal in (True, False):
+        o, lse = oracle.prefill_paged(q, pool_k, pool_v, table, sl, cu, ps, causal, 0.7)
+        g = H // Hkv
+        for b, (L, n) in enumerate(zip(lens, nq)):
+            for i in range(n):
+                keys = (L - n + i + 1) if causal else L
+                for h in range(H):
+                    ob, lb = _mp_attention(q[cu[b] + i, h][None], ks[b][:keys, h // g],
+                                           vs[b][:keys, h // g], False, 0.7)
+                    np.testing.assert_allclose(o[cu[b] + i, h], ob[0], atol=TOL)
+                    assert abs(lse[h, cu[b] + i] - lb[0]) < TOL
+
+
+def test_prefill_paged_one_query_is_decode():
+    H, d, ps = 3, 8, 4
+    lens = [1, 6, 13]
+    pool_k, table, sl, _ = _split_append([0, 0, 0], lens, H, d, ps, 180)
+    pool_v, table_v, _, _ = _split_append([0, 0, 0], lens, H, d, ps, 185)
+    assert np.array_equal(table, table_v)
+    q = _rand((3, H, d), 182)
+    o, lse = oracle.prefill_paged(q, pool_k, pool_v, table, sl, np.arange(4), ps, True,
+                                  1 / math.sqrt(d))
+    od, ld = oracle.decode_paged(q, pool_k, pool_v, table, sl, ps)
+    np.testing.assert_allclose(o, od, atol=1e-15)
+    np.testing.assert_allclose(lse.T, ld, atol=1e-15)
+
+
+def test_prefill_paged_whole_sequence_is_causal_varlen():
+    """When every cached token is a query, prefill is causal attention over
+    the (gathered) sequence."""
+    H, d, ps = 2, 8, 4
+    lens = [5, 12, 1]
+    pool_k, table, sl, ks = _split_append([0, 0, 0], lens, H, d, ps, 190)
+    pool_v, table_v, _, vs = _split_append([0, 0, 0], lens, H, d, ps, 195)
+    assert np.array_equal(table, table_v)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    q = _rand((int(cu[-1]), H, d), 192)
+    o, lse = oracle.prefill_paged(q, pool_k, pool_v, table, sl, cu, ps, True, 0.3)
+    o2, l2 = oracle.attention_varlen(q, np.concatenate(ks), np.concatenate(vs), cu, True, 0.3)
+    np.testing.assert_allclose(o, o2, atol=1e-15)
+    np.testing.assert_allclose(lse, l2, atol=1e-15)
