@@ -175,7 +175,7 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
-    return fa::launch_fwd(p, tq, tk, tv, d, false, reinterpret_cast<cudaStream_t>(stream));
+    return fa::launch_fwd(p, tq, tk, tv, d, fa::kFixed, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -227,7 +227,62 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
-    return fa::launch_fwd(p, tq, tk, tv, d, true, reinterpret_cast<cudaStream_t>(stream));
+    return fa::launch_fwd(p, tq, tk, tv, d, fa::kVarlen, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                     const int32_t* page_table, const int32_t* seq_lens, const int32_t* cu_q,
+                     void* o, float* lse, int B, int H, int H_kv, int total_q, int max_q,
+                     int num_pages, int d, int page_size, int causal, float scale,
+                     fa_stream_t stream) {
+    if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !cu_q || !o || !lse)
+        return FA_ERR_NULL;
+    if (B < 1 || H < 1 || H_kv < 1 || total_q < 1 || max_q < 1 || num_pages < 1)
+        return FA_ERR_SHAPE;
+    if (H % H_kv != 0) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (page_size != 256) return FA_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(num_pages) * H_kv > 0x7fffffff) return FA_ERR_SHAPE;
+    if (max_q > 0x7fffffff - 256) return FA_ERR_SHAPE;
+    if (!std::isfinite(scale)) return FA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
+        !aligned16(lse))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    CUtensorMap tq, tk, tv;
+    // queries: packed rows, as fa_fwd_varlen
+    const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                                 static_cast<cuuint64_t>(total_q)};
+    const cuuint64_t qstrides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                    static_cast<cuuint64_t>(H) * d * 2};
+    const cuuint32_t qbox[3] = {64, 1, 128};
+    // the page pool [P, H_kv, 256, d]: (d, slot, page * H_kv + head)
+    const cuuint64_t kdims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(page_size),
+                                 static_cast<cuuint64_t>(num_pages) * H_kv};
+    const cuuint64_t kstrides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                    static_cast<cuuint64_t>(page_size) * d * 2};
+    const cuuint32_t kbox[3] = {64, 128, 1};
+    if ((rc = make_map(&tq, q, qdims, qstrides, qbox)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k_pages, kdims, kstrides, kbox)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v_pages, kdims, kstrides, kbox)) != FA_OK) return rc;
+    fa::FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens = cu_q;
+    p.B = B;
+    p.H = H;
+    p.H_kv = H_kv;
+    p.page_table = page_table;
+    p.ctx_lens = seq_lens;
+    p.N = max_q;
+    p.total = total_q;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.err = s->err;
+    return fa::launch_fwd(p, tq, tk, tv, d, fa::kPaged, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -289,6 +344,30 @@ int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t*
         return rc;
     return fa::launch_gather(pages, page_table, seq_lens, out, B, H, d, page_size, ws, s->err,
                              s->num_sms, st);
+}
+
+int fa_append_paged(const void* k_new, const void* v_new, const int32_t* cu_new, void* k_pages,
+                    void* v_pages, const int32_t* page_table, const int32_t* seq_lens, int B,
+                    int H_kv, int total_new, int num_pages, int d, int page_size,
+                    fa_stream_t stream) {
+    if (!k_new || !v_new || !cu_new || !k_pages || !v_pages || !page_table || !seq_lens)
+        return FA_ERR_NULL;
+    if (B < 1 || H_kv < 1 || total_new < 0 || num_pages < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (page_size != 256) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pages) || !aligned16(v_pages))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    if (total_new == 0) return FA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H_kv, d, 1), st, &ws)) != FA_OK)
+        return rc;
+    return fa::launch_append(k_new, v_new, cu_new, k_pages, v_pages, page_table, seq_lens, B,
+                             H_kv, total_new, d, page_size, num_pages, ws, s->err, s->num_sms,
+                             st);
 }
 
 int fa_get_device_error(int* code, fa_stream_t stream) {

@@ -659,6 +659,49 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Appends the new K and V rows of every sequence to the paged cache: new row
+// g of sequence b (cu_new[b] <= g < cu_new[b+1]) is the sequence's token
+// pos = seq_lens[b] - n_b + (g - cu_new[b]) (seq_lens counts the tokens after
+// the append) and goes to slot pos % page_size of page
+// page_table[page_off[b] + pos / page_size].  Grid-stride over 16-byte words.
+// A sequence with more new rows than tokens, or a page index outside the
+// pool, is skipped and reported; no write leaves the pool.
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_append_kernel(const __nv_bfloat16* __restrict__ k_new,
+                     const __nv_bfloat16* __restrict__ v_new, const int32_t* __restrict__ cu_new,
+                     __nv_bfloat16* __restrict__ k_pages, __nv_bfloat16* __restrict__ v_pages,
+                     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens,
+                     const int32_t* __restrict__ page_off, int B, int Hk, int total_new,
+                     int page_size, int num_pages, unsigned int* err) {
+    constexpr int V = D / 8;  // 16-byte words per row
+    const int64_t words = static_cast<int64_t>(total_new) * Hk * V;
+    for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < words;
+         x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int vec = static_cast<int>(x % V);
+        const int hh = static_cast<int>((x / V) % Hk);
+        const int g = static_cast<int>(x / (static_cast<int64_t>(V) * Hk));
+        const int b = find_owner(cu_new, B, g);
+        const int n = __ldg(cu_new + b + 1) - __ldg(cu_new + b);
+        const int len = __ldg(seq_lens + b);
+        if (n > len || n < 0) {
+            if (vec == 0 && hh == 0) record_error(err, FA_DEVERR_BAD_INPUT);
+            continue;
+        }
+        const int pos = len - n + (g - __ldg(cu_new + b));
+        const int page = __ldg(page_table + __ldg(page_off + b) + pos / page_size);
+        if (page < 0 || page >= num_pages) {
+            record_error(err, FA_DEVERR_BAD_INPUT);
+            continue;
+        }
+        const int64_t src = (static_cast<int64_t>(g) * Hk + hh) * D + vec * 8;
+        const int64_t dst =
+            ((static_cast<int64_t>(page) * Hk + hh) * page_size + pos % page_size) * D + vec * 8;
+        *reinterpret_cast<uint4*>(k_pages + dst) = *reinterpret_cast<const uint4*>(k_new + src);
+        *reinterpret_cast<uint4*>(v_pages + dst) = *reinterpret_cast<const uint4*>(v_new + src);
+    }
+}
+
 template <int D, int GH>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
@@ -713,7 +756,39 @@ int launch_gather_impl(const void* pages, const int32_t* page_table, const int32
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <int D>
+int launch_append_impl(const void* k_new, const void* v_new, const int32_t* cu_new, void* k_pages,
+                       void* v_pages, const int32_t* page_table, const int32_t* seq_lens, int B,
+                       int Hk, int total_new, int page_size, int num_pages, void* workspace,
+                       unsigned int* err, int num_sms, cudaStream_t stream) {
+    int32_t* page_off = static_cast<int32_t*>(workspace);
+    int32_t* tok_off = page_off + (B + 1);
+    int32_t* unit_off = tok_off + (B + 1);
+    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, Hk, page_size, 1, page_off,
+                                                          tok_off, unit_off, err);
+    fa_append_kernel<D><<<num_sms * 8, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), cu_new,
+        static_cast<__nv_bfloat16*>(k_pages), static_cast<__nv_bfloat16*>(v_pages), page_table,
+        seq_lens, page_off, B, Hk, total_new, page_size, num_pages, err);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
+
+int launch_append(const void* k_new, const void* v_new, const int32_t* cu_new, void* k_pages,
+                  void* v_pages, const int32_t* page_table, const int32_t* seq_lens, int B,
+                  int Hk, int total_new, int d, int page_size, int num_pages, void* workspace,
+                  unsigned int* err, int num_sms, cudaStream_t stream) {
+    if (d == 128)
+        return launch_append_impl<128>(k_new, v_new, cu_new, k_pages, v_pages, page_table,
+                                       seq_lens, B, Hk, total_new, page_size, num_pages,
+                                       workspace, err, num_sms, stream);
+    if (d == 64)
+        return launch_append_impl<64>(k_new, v_new, cu_new, k_pages, v_pages, page_table,
+                                      seq_lens, B, Hk, total_new, page_size, num_pages,
+                                      workspace, err, num_sms, stream);
+    return FA_ERR_UNSUPPORTED;
+}
 
 size_t decode_workspace_bytes(int B, int H, int d, int max_splits) {
     return layout_of(B, H, d, max_splits).total;

@@ -24,14 +24,18 @@ struct FwdParams {
     const int32_t* cu_seqlens;  // varlen only
     int B, H, N;         // N: sequence length (fixed) or max_seqlen (varlen)
     int H_kv;            // K/V heads; query head h reads K/V head h / (H / H_kv)
+    const int32_t* page_table;  // paged prefill: packed page table
+    const int32_t* ctx_lens;    // paged prefill: cached tokens (keys) per sequence
     int total;           // varlen: packed rows
     int causal;
     float scale_log2;    // scale * log2(e)
     unsigned int* err;   // device error word
 };
 
+// forward modes
+constexpr int kFixed = 0, kVarlen = 1, kPaged = 2;
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, int d, bool varlen, cudaStream_t stream);
+               const CUtensorMap& tv, int d, int mode, cudaStream_t stream);
 
 // ---- paged decode ----------------------------------------------------------
 // Number of pages a split covers at least (a split is one CTA work unit) and
@@ -56,6 +60,11 @@ bool decode_group_supported(int H, int Hk);
 
 // The current device's error word and SM count (sm_100 devices only).
 int device_error_word(unsigned int** err, int* num_sms);
+
+int launch_append(const void* k_new, const void* v_new, const int32_t* cu_new, void* k_pages,
+                  void* v_pages, const int32_t* page_table, const int32_t* seq_lens, int B,
+                  int Hk, int total_new, int d, int page_size, int num_pages, void* workspace,
+                  unsigned int* err, int num_sms, cudaStream_t stream);
 
 int launch_gather(const void* pages, const int32_t* page_table, const int32_t* seq_lens,
                   void* out, int B, int H, int d, int page_size, void* workspace,

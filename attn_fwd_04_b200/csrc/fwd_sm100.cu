@@ -45,6 +45,7 @@ constexpr int BM = 128;       // query rows per tile (MMA M)
 constexpr int BN = 128;       // keys per K/V tile
 constexpr int kSlots = 4;     // K/V ring slots (each holds one K or one V tile)
 constexpr int kThreads = 512;
+constexpr int kHeadGroup = 4;  // (sequence, head) units scheduled together
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }  // O_t
@@ -70,6 +71,7 @@ struct alignas(1024) FwdSmem {
     uint64_t q_full[2];
     uint64_t kv_full[kSlots], kv_empty[kSlots];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
+    uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -168,22 +170,37 @@ __device__ __forceinline__ float exp_pairs(const uint32_t (&s)[BN], uint32_t (&p
     return f2_lo(a2) + f2_hi(a2);
 }
 
-template <int D, bool VARLEN>
+// MODE: kFixed ([B,H,N,d] tensors), kVarlen (packed [total,H,d] sequences),
+// kPaged (packed queries; keys and values read through the page table from a
+// pool of 256-token pages, the queries being the last positions of each
+// cached sequence).
+template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
+    constexpr bool VARLEN = MODE != kFixed;  // packed query rows
+    constexpr bool PAGED = MODE == kPaged;
     // ---- the work unit: (sequence/head, 256-row query block) --------------
-    // CTAs are numbered by rank first: rank r is the r-th 256-row block counted
-    // from the end of its sequence, so under a causal mask every head's (and
-    // sequence's) heaviest block is dispatched before any second-heaviest one
-    // and the last CTAs to start are the lightest.  With grouped K/V heads
-    // (H_kv < H) query head h reads K/V head h / (H / H_kv).
+    // CTAs walk the units in groups of kHeadGroup (sequence, head) pairs; in
+    // a group they are numbered by rank first, rank r being the r-th 256-row
+    // block counted from the end of its sequence.  Under a causal mask each
+    // group's heaviest blocks start before its lighter ones, and the CTAs in
+    // flight at any time read the K/V of a few heads only, which stay in L2
+    // (all heads at once would spill it and re-read K/V from DRAM).  With
+    // grouped K/V heads (H_kv < H) query head h reads K/V head h / (H / H_kv).
     const int units = p.B * p.H;
-    const int rank = static_cast<int>(blockIdx.x) / units;
-    const int unit = static_cast<int>(blockIdx.x) - rank * units;
-    int len, seq_start = 0, bh = 0, h = 0, bkv = 0;
+    const int nblk_all = (p.N + 2 * BM - 1) / (2 * BM);
+    const int gidx = static_cast<int>(blockIdx.x) / (kHeadGroup * nblk_all);
+    const int ug = min(kHeadGroup, units - gidx * kHeadGroup);
+    const int within = static_cast<int>(blockIdx.x) - gidx * kHeadGroup * nblk_all;
+    const int rank = within / ug;
+    const int unit = gidx * kHeadGroup + (within - rank * ug);
+    // len: query rows; klen: keys; a query row i may see keys up to
+    // kshift + i under the causal mask (kshift = klen - len for paged
+    // prefill, whose queries end the sequence; 0 otherwise)
+    int len, klen, kshift = 0, seq_start = 0, bh = 0, h = 0, bkv = 0, b = 0;
     if constexpr (VARLEN) {
-        const int b = unit / p.H;
+        b = unit / p.H;
         h = unit - b * p.H;
         const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
         // keep every access inside the [total, H, d] tensors whatever the offsets say
@@ -193,21 +210,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             record_error(p.err, FA_DEVERR_BAD_INPUT);
         seq_start = c0;
         len = c1m - c0;
+        klen = len;
+        if constexpr (PAGED) {
+            bkv = h / (p.H / p.H_kv);
+            const int ctx = p.ctx_lens[b];
+            if (ctx < len) {  // more queries than cached tokens: not computed
+                if (rank == 0 && threadIdx.x == 0) record_error(p.err, FA_DEVERR_BAD_INPUT);
+                return;
+            }
+            klen = ctx;
+            kshift = ctx - len;
+        }
     } else {
         bh = unit;
-        const int b = bh / p.H;
+        b = bh / p.H;
         bkv = b * p.H_kv + (bh - b * p.H) / (p.H / p.H_kv);
         len = p.N;
+        klen = len;
     }
     const int nblk = (len + 2 * BM - 1) / (2 * BM);
     const int blk = p.causal ? (nblk - 1 - rank) : rank;
     if (blk < 0 || blk >= nblk) return;
     const int row0 = blk * 2 * BM;
-    const int nkv_all = (len + BN - 1) / BN;
+    const int nkv_all = (klen + BN - 1) / BN;
     int n_t[2];
-    n_t[0] = p.causal ? min(2 * blk + 1, nkv_all) : nkv_all;
-    n_t[1] = (row0 + BM < len) ? (p.causal ? min(2 * blk + 2, nkv_all) : nkv_all) : 0;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int rf = row0 + t * BM;
+        n_t[t] = (rf < len) ? (p.causal ? min((kshift + rf + BM - 1) / BN + 1, nkv_all) : nkv_all)
+                            : 0;
+    }
     const int n = max(n_t[0], n_t[1]);
+    // paged: the last K/V tile runs past the sequence end into the rest of
+    // its page; those V rows are zeroed before P V (P is 0 there, but 0 * NaN
+    // would not be)
+    const bool zero_v_tail = PAGED && n == nkv_all && (klen % BN) != 0;
 
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
@@ -227,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
         }
+        mbar_init(&sm.vfix, 1);
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
@@ -246,8 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (wg == 3) {
         regs_dec<56>();
-        if (warp == 13 && lane == 0) {
+        if (warp == 13) {
             // ================= TMA producer =================
+            // paged: sequence b's pages start at entry sum_{b'<b} ceil(ctx_b'/256)
+            int page_base = 0;
+            if constexpr (PAGED) {
+                for (int i = lane; i < b; i += 32) page_base += (max(p.ctx_lens[i], 0) + 255) / 256;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) page_base += __shfl_xor_sync(0xffffffffu, page_base, o);
+            }
+            int issued = 0;  // ring uses issued so far
+            if (lane == 0) {
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
@@ -262,27 +309,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, row, head);
                 }
             };
+            // paged K/V: key tile j is the 128-slot half (j % 2) of page
+            // page_table[page_base + j / 2]; the pool map is (d, slot, page*H_kv + head)
+            auto load_kv = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int j) {
+                const int page = p.page_table[page_base + (j >> 1)];
+#pragma unroll
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, (j & 1) * BN,
+                                page * p.H_kv + bkv);
+            };
             for (int t = 0; t < 2; ++t) {
                 if (n_t[t] > 0) {
                     mbar_arrive_expect_tx(&sm.q_full[t], BM * D * 2);
                     load_tile(sm.q[t], &tq, &sm.q_full[t], row0 + t * BM, bh);
                 }
             }
-            int issued = 0;  // ring uses issued so far
             for (int u = 0; u < 2 * n; ++u) {
                 const int slot = u % kSlots;
                 const uint32_t ph = (u / kSlots) & 1;
                 if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
                 mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
-                load_tile(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], (u >> 1) * BN, bkv);
+                if constexpr (PAGED)
+                    load_kv(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], u >> 1);
+                else
+                    load_tile(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], (u >> 1) * BN,
+                              bkv);
                 issued = u + 1;
             }
+            }  // lane 0
+            issued = __shfl_sync(0xffffffffu, issued, 0);
+            if (zero_v_tail && issued == 2 * n) {
+                // the whole warp: once V_{n-1} has landed, clear its rows past
+                // the sequence end (whole 128-byte rows, so the swizzle does not
+                // matter), make the writes visible to the tensor core, release
+                const int vs = ring_slot(n - 1, 1);
+                if (warp_wait(&sm.kv_full[vs], ring_phase(n - 1, 1), err, abort)) {
+                    const int zr = klen - (n - 1) * BN;  // first row to clear
+                    uint4* base = reinterpret_cast<uint4*>(sm.kv[vs]);
+                    const int per_box = (BN - zr) * 8;   // 16-byte words per box
+#pragma unroll
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        for (int i = lane; i < per_box; i += 32)
+                            base[cb * (kBoxBytes / 16) + zr * 8 + i] = make_uint4(0, 0, 0, 0);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.vfix);
+                }
+            }
+            if (lane == 0) {
             // every copy this CTA started must land before it exits
             for (int t = 0; t < 2; ++t)
                 if (n_t[t] > 0) mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, nullptr);
             for (int u = max(0, issued - kSlots); u < issued; ++u)
                 mbar_wait(&sm.kv_full[u % kSlots], (u / kSlots) & 1, err, FA_DEVERR_TIMEOUT,
                           nullptr);
+            }  // lane 0
         } else if (warp == 12 && lane == 0) {
             // ================= MMA issuer =================
             // The tensor pipe runs this thread's MMAs in issue order, so
@@ -335,8 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(&sm.kv_empty[ring_slot(0, 0)]);
             }
             for (int j = 0; ok && j < n; ++j) {
-                if (!mbar_wait(&sm.kv_full[ring_slot(j, 1)], ring_phase(j, 1), err,
-                               FA_DEVERR_TIMEOUT, abort)) break;
+                if (zero_v_tail && j == n - 1) {
+                    if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort)) break;
+                } else if (!mbar_wait(&sm.kv_full[ring_slot(j, 1)], ring_phase(j, 1), err,
+                                      FA_DEVERR_TIMEOUT, abort)) {
+                    break;
+                }
                 const bool next_k = j + 1 < n;
                 if (next_k && !mbar_wait(&sm.kv_full[ring_slot(j + 1, 0)], ring_phase(j + 1, 0),
                                          err, FA_DEVERR_TIMEOUT, abort)) break;
@@ -383,11 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             // masked keys: past the sequence end, or after this row (causal)
             const int kbase = j * BN;
-            const bool need_mask = (kbase + BN > len) || (p.causal && kbase + BN - 1 > row_first);
+            const bool need_mask =
+                (kbase + BN > klen) || (p.causal && kbase + BN - 1 > kshift + row_first);
             int lim = BN;
             if (need_mask) {
-                lim = min(BN, len - kbase);
-                if (p.causal) lim = min(lim, qrow - kbase + 1);
+                lim = min(BN, klen - kbase);
+                if (p.causal) lim = min(lim, kshift + qrow - kbase + 1);
             }
             uint32_t s[BN];
             uint32_t pk[BN / 2];
@@ -513,18 +599,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 12) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, bool VARLEN>
+template <int D, int MODE>
 int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, cudaStream_t stream) {
     // Every CTA allocates all 512 TMEM columns, so one CTA per SM: ask for
     // enough shared memory that a second CTA cannot be co-resident.
     const size_t smem = sizeof(FwdSmem<D>) + 1024 > 120 * 1024 ? sizeof(FwdSmem<D>) + 1024
                                                                : 120 * 1024;
-    auto kern = fa_fwd_kernel<D, VARLEN>;
+    auto kern = fa_fwd_kernel<D, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
-    // one CTA per (rank, sequence/head); rank-major order, see the kernel
+    // one CTA per (sequence/head, 256-row block); see the kernel for the order
     const long long blocks = (p.N + 2 * BM - 1) / (2 * BM);
     const long long ctas = blocks * p.B * p.H;
     if (ctas > 0x7fffffffLL) return FA_ERR_SHAPE;
@@ -535,14 +621,20 @@ int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk
 }  // namespace
 
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, int d, bool varlen, cudaStream_t stream) {
-    if (d == 128)
-        return varlen ? launch_impl<128, true>(p, tq, tk, tv, stream)
-                      : launch_impl<128, false>(p, tq, tk, tv, stream);
-    if (d == 64)
-        return varlen ? launch_impl<64, true>(p, tq, tk, tv, stream)
-                      : launch_impl<64, false>(p, tq, tk, tv, stream);
-    return FA_ERR_UNSUPPORTED;
+               const CUtensorMap& tv, int d, int mode, cudaStream_t stream) {
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    switch (mode) {
+        case kFixed:
+            return d == 128 ? launch_impl<128, kFixed>(p, tq, tk, tv, stream)
+                            : launch_impl<64, kFixed>(p, tq, tk, tv, stream);
+        case kVarlen:
+            return d == 128 ? launch_impl<128, kVarlen>(p, tq, tk, tv, stream)
+                            : launch_impl<64, kVarlen>(p, tq, tk, tv, stream);
+        case kPaged:
+            return d == 128 ? launch_impl<128, kPaged>(p, tq, tk, tv, stream)
+                            : launch_impl<64, kPaged>(p, tq, tk, tv, stream);
+        default: return FA_ERR_UNSUPPORTED;
+    }
 }
 
 }  // namespace fa

@@ -25,7 +25,7 @@ FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
-           "fa_decode_paged_noalloc",
+           "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
            "fa_status_str", "fa_version")
@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_gather_paged.argtypes = [P, P, P, P, I, I, I, I, P]
+        L.fa_append_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+        L.fa_prefill_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P]
         L.fa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
         L.fa_selftest_bounded_wait.argtypes = [P]
         L.fa_release_workspace.argtypes = []
@@ -62,8 +64,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
         for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen", "fa_decode_paged",
-                     "fa_decode_paged_gqa", "fa_decode_paged_noalloc",
-                     "fa_gather_paged",
+                     "fa_decode_paged_gqa", "fa_decode_paged_noalloc", "fa_append_paged",
+                     "fa_prefill_paged", "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
                      "fa_version"):
             getattr(L, name).restype = I
@@ -220,6 +222,53 @@ def fa_decode_paged_noalloc(q, k_pages, v_pages, page_table, seq_lens, page_size
                                        B, H, d, int(page_size), _stream(stream))
     _raise_if(rc, "fa_decode_paged_noalloc")
     return o
+
+
+def fa_append_paged(k_new, v_new, cu_new, k_pages, v_pages, page_table, seq_lens,
+                    page_size: int = 256, stream=None):
+    """Write new rows [total_new,H_kv,d] into the [P,H_kv,page_size,d] pages
+    (in place) as the last tokens of their sequences; seq_lens are the
+    lengths after the append."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _check(t, n, torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(cu_new, "cu_new", torch.int32, 1)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    total_new, H_kv, d = k_new.shape
+    rc = lib().fa_append_paged(k_new.data_ptr(), v_new.data_ptr(), cu_new.data_ptr(),
+                               k_pages.data_ptr(), v_pages.data_ptr(), page_table.data_ptr(),
+                               seq_lens.data_ptr(), cu_new.numel() - 1, H_kv, total_new,
+                               k_pages.shape[0], d, int(page_size), _stream(stream))
+    _raise_if(rc, "fa_append_paged")
+
+
+def fa_prefill_paged(q, k_pages, v_pages, page_table, seq_lens, cu_q, max_q: int, causal: bool,
+                     scale: Optional[float] = None, page_size: int = 256, o=None, lse=None,
+                     stream=None):
+    """Queries [total_q,H,d] that end their cached sequences, attending
+    through the page table -> (o [total_q,H,d], lse [H,total_q] fp32)."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _check(cu_q, "cu_q", torch.int32, 1)
+    total_q, H, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    rc = lib().fa_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                page_table.data_ptr(), seq_lens.data_ptr(), cu_q.data_ptr(),
+                                o.data_ptr(), lse.data_ptr(), cu_q.numel() - 1, H,
+                                k_pages.shape[1], total_q, int(max_q), k_pages.shape[0], d,
+                                int(page_size), int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_prefill_paged")
+    return o, lse
 
 
 def fa_gather_paged(pages, page_table, seq_lens, total_tokens: int, page_size: int = 256,

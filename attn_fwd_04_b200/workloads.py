@@ -219,6 +219,47 @@ def paged_inputs(B: int, H: int, d: int, lengths: List[int], seed: int,
     return PagedCache(q, k_pages, v_pages, perm, seq_lens, page_size, pages_per_seq)
 
 
+@dataclass
+class PrefillWorkload:
+    """Chunked prefill over a paged cache: sequence b has ctx_lens[b] cached
+    tokens followed by q_len new ones (the queries)."""
+    name: str
+    B: int
+    H: int
+    H_kv: int
+    d: int
+    q_len: int
+    ctx_lo: int
+    ctx_hi: int
+    causal: bool
+    seed: int
+    page_size: int = PAGE_SIZE
+
+
+PAGED_PREFILL = PrefillWorkload("paged_prefill_b8_h32_d128_ctx1024to8192_q1024_page256",
+                                8, 32, 32, 128, 1024, 1024, 8192, True, 61)
+
+
+def prefill_inputs(B: int, H: int, H_kv: int, d: int, lens_after: List[int], q_lens: List[int],
+                   seed: int, page_size: int = PAGE_SIZE, device: Optional[str] = None):
+    """A paged cache holding lens_after[b] tokens per sequence (pages from a
+    shuffled pool, NaN past each sequence's end) and packed queries for the
+    last q_lens[b] positions: returns (cache, q [sum q_lens, H, d], cu_q)."""
+    cache = paged_inputs(B, H, d, lens_after, seed, page_size, device, H_kv=H_kv)
+    total_q = int(sum(q_lens))
+    dev = cache.k_pages.device.type
+    g = _gen(seed + 2, dev)
+    q = _randn_bf16((max(total_q, 1), H, d), g, 1.0, dev)[:total_q]
+    return cache, q, cu_seqlens_of(q_lens)
+
+
+def prefill_workload_inputs(w: PrefillWorkload, device: Optional[str] = None):
+    ctx = varlen_lengths(w.B, w.ctx_lo, w.ctx_hi, w.seed)
+    lens_after = [c + w.q_len for c in ctx]
+    return prefill_inputs(w.B, w.H, w.H_kv, w.d, lens_after, [w.q_len] * w.B, w.seed,
+                          w.page_size, device)
+
+
 def decode_workload_inputs(w: DecodeWorkload, device: Optional[str] = None) -> PagedCache:
     lengths = varlen_lengths(w.B, w.len_lo, w.len_hi, w.seed)
     return paged_inputs(w.B, w.H, w.d, lengths, w.seed, w.page_size, device)

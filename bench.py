@@ -313,15 +313,30 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
     out[name] = {"ms_per_launch": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
                  "bytes_per_launch": nbytes}
     del c, pt, sl, do
+    # paged prefill: 1024 new queries per sequence after 1024..8192 cached
+    # tokens, K/V read through the page table; FLOPs count every attended
+    # (query, key) pair (4*d per pair and head)
+    w = W.PAGED_PREFILL
+    cache, q, cu = W.prefill_workload_inputs(w, device="cuda")
+    pt, sl, cud = cache.page_table.cuda(), cache.seq_lens.cuda(), cu.cuda()
+    o = torch.empty_like(q)
+    lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=q.device)
+    pairs = sum(w.q_len * (int(L) - w.q_len) + w.q_len * (w.q_len + 1) // 2
+                for L in cache.seq_lens.tolist())
+    timed(lambda: fa.fa_prefill_paged(q, cache.k_pages, cache.v_pages, pt, sl, cud, w.q_len,
+                                      w.causal, 1 / math.sqrt(w.d), o=o, lse=lse, stream=stream),
+          4.0 * w.d * w.H * pairs, w.name, {"context_after": cache.seq_lens.tolist()})
+    del cache, q, cu, pt, sl, cud, o, lse
     torch.cuda.empty_cache()
     return out
 
 
-def decode_cache(batch: int) -> W.PagedCache:
-    if batch >= DEC.B:
+def decode_cache(batch: int, h_kv: int) -> W.PagedCache:
+    if batch >= DEC.B and h_kv == DEC.H:
         return W.decode_workload_inputs(DEC, device="cuda")
     lengths = W.varlen_lengths(DEC.B, DEC.len_lo, DEC.len_hi, DEC.seed)[:batch]
-    return W.paged_inputs(batch, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda")
+    return W.paged_inputs(len(lengths), DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size,
+                          device="cuda", H_kv=h_kv)
 
 
 def run_native(args, world, rank, local):
@@ -340,7 +355,8 @@ def run_native(args, world, rank, local):
         o = torch.empty_like(q)
         lse = torch.empty((FWD.B, FWD.H, FWD.N), dtype=torch.float32, device=dev)
     if do_dec:
-        cache = decode_cache(args.decode_batch)
+        cache = decode_cache(args.decode_batch, args.decode_hkv)
+        h_kv = int(cache.k_pages.shape[1])
         dpt, dsl = cache.page_table.to(dev), cache.seq_lens.to(dev)
         do = torch.empty_like(cache.q)
     torch.cuda.synchronize()
@@ -352,9 +368,12 @@ def run_native(args, world, rank, local):
             fa.fa_fwd(q, k, v, FWD.causal, scale, o=o, lse=lse, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        if do_dec:
+        if do_dec and h_kv == DEC.H:
             fa.fa_decode_paged(cache.q, cache.k_pages, cache.v_pages, dpt, dsl, DEC.page_size,
                                o=do, stream=stream)
+        elif do_dec:
+            fa.fa_decode_paged_gqa(cache.q, cache.k_pages, cache.v_pages, dpt, dsl,
+                                   DEC.page_size, o=do, stream=stream)
         if ev is not None:
             ev[2].record(stream)
 
@@ -391,7 +410,8 @@ def run_native(args, world, rank, local):
     fwd_tflops = world * flops * args.steps / (fwd_sum * 1e-3) / 1e12 if do_fwd else None
     per_launch_tf = flops / (fwd_sum / args.steps * 1e-3) / 1e12 if do_fwd else None
     if do_dec:
-        dbytes = decode_bytes(cache.seq_lens.tolist(), DEC.H, DEC.d, cache.q.shape[0])
+        dbytes = decode_bytes(cache.seq_lens.tolist(), DEC.H, DEC.d, cache.q.shape[0],
+                              H_kv=h_kv)
         dec_gbs = world * dbytes * args.steps / (dec_sum * 1e-3) / 1e9
         per_launch_gbs = dbytes / (dec_sum / args.steps * 1e-3) / 1e9
 
@@ -497,7 +517,8 @@ def run_native(args, world, rank, local):
                            "traffic": recorded_traffic("fa_fwd_kernel", fwd_sha),
                            "algorithmic_flops_per_launch": flops}
     if do_dec:
-        out["config"]["decode"] = {"B": int(cache.q.shape[0]), "H": DEC.H, "d": DEC.d,
+        out["config"]["decode"] = {"B": int(cache.q.shape[0]), "H": DEC.H, "H_kv": h_kv,
+                                   "d": DEC.d,
                                    "page_size": DEC.page_size,
                                    "len_range": [DEC.len_lo, DEC.len_hi], "seed": DEC.seed,
                                    "tokens": int(cache.seq_lens.sum())}
@@ -577,6 +598,9 @@ def main(argv=None):
     ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
                     help="profiling aid: run one entry point only (the JSON line then "
                          "reports that part alone)")
+    ap.add_argument("--decode-hkv", type=int, default=DEC.H,
+                    help="K/V heads of the decode cache (fewer than 32 runs the grouped-query "
+                         "decode)")
     ap.add_argument("--decode-batch", type=int, default=DEC.B,
                     help="profiling aid: decode over the first B sequences only")
     args = ap.parse_args(argv)

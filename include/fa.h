@@ -175,6 +175,64 @@ FA_API int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v
                     int B, int H, int H_kv, int d, int page_size, fa_stream_t stream);
 
 /*
+ * fa_append_paged -- write the K and V rows of new tokens into the paged
+ * cache: the step before attention in the serving loop of the page "“Flash”
+ * 不是那个被时代淘汰的插件" (0539edu.com), section 2 (a new token goes into a
+ * page taken from the fixed pool).
+ *   k_new, v_new : [total_new, H_kv, d] bf16, the new rows of all sequences
+ *                  packed back to back
+ *   cu_new       : DEVICE int32 [B+1], sequence b's new rows are
+ *                  cu_new[b] .. cu_new[b+1]-1
+ *   k_pages,
+ *   v_pages      : [num_pages, H_kv, page_size, d] bf16, updated in place
+ *   page_table   : packed as for fa_decode_paged, for the lengths AFTER the
+ *                  append; the caller has already taken the pages the new
+ *                  tokens need from its free list (page allocation is the
+ *                  caller's: the library holds no allocator)
+ *   seq_lens     : DEVICE int32 [B], tokens per sequence after the append
+ * Sequence b's n_b new rows become its last n_b tokens: new row i goes to
+ * position seq_lens[b] - n_b + i, i.e. slot (pos % page_size) of page
+ * page_table[off_b + pos / page_size].  page_size must be 256.  A sequence
+ * with n_b > seq_lens[b], or a page index outside [0, num_pages), is skipped
+ * and reported as FA_ERR_DEVICE_BAD_INPUT (no write leaves the pool).  Uses the
+ * library's per-GPU workspace for the page offsets.
+ */
+FA_API int fa_append_paged(const void* k_new, const void* v_new, const int32_t* cu_new,
+                    void* k_pages, void* v_pages, const int32_t* page_table,
+                    const int32_t* seq_lens, int B, int H_kv, int total_new, int num_pages,
+                    int d, int page_size, fa_stream_t stream);
+
+/*
+ * fa_prefill_paged -- attention of several new query tokens per sequence
+ * through the paged cache (decode with q_len > 1, or prefill of a chunk that
+ * continues cached context), with the forward kernel reading K and V tiles
+ * straight from the pages.
+ *   q, o       : [total_q, H, d] bf16, sequence b's queries are rows
+ *                cu_q[b] .. cu_q[b+1]-1 (cu_q: DEVICE int32 [B+1])
+ *   lse        : [H, total_q] fp32
+ *   k_pages,
+ *   v_pages    : [num_pages, H_kv, 256, d] bf16 (H a multiple of H_kv; query
+ *                head h reads K/V head h / (H / H_kv))
+ *   page_table,
+ *   seq_lens   : as fa_decode_paged; seq_lens[b] counts the cached tokens
+ *                INCLUDING the new ones (append them first with
+ *                fa_append_paged)
+ * Sequence b's q_b = cu_q[b+1] - cu_q[b] queries are its last q_b positions:
+ * query i sits at position seq_lens[b] - q_b + i and, with `causal`, attends
+ * to the keys at positions up to its own (the mask is aligned to the end of
+ * the sequence); without it, to all seq_lens[b] keys.  Softmax scale as
+ * fa_fwd.  max_q must be >= every q_b (it sizes the launch).  A sequence with
+ * q_b > seq_lens[b] is not computed and is reported as
+ * FA_ERR_DEVICE_BAD_INPUT.  Page indices outside [0, num_pages) read zeros.
+ * With q_b = 1 and `causal` this is fa_decode_paged for the same cache.
+ */
+FA_API int fa_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* seq_lens, const int32_t* cu_q,
+                    void* o, float* lse, int B, int H, int H_kv, int total_q, int max_q,
+                    int num_pages, int d, int page_size, int causal, float scale,
+                    fa_stream_t stream);
+
+/*
  * fa_gather_paged -- copy the cached tokens of every sequence out of the page
  * pool into contiguous rows (a checking aid for the decode path's address
  * arithmetic; same page_table / seq_lens conventions as fa_decode_paged).

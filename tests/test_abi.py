@@ -74,6 +74,33 @@ def decode_gqa(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=8, H_kv=2, d=128, ps=
     return L.fa_decode_paged_gqa(q, kp, vp, pt, sl, o, B, H, H_kv, d, ps, S)
 
 
+def append(L, kn=A, vn=A, cu=A, kp=A, vp=A, pt=A, sl=A, B=2, H_kv=2, total=10, P=8, d=128,
+           ps=256):
+    return L.fa_append_paged(kn, vn, cu, kp, vp, pt, sl, B, H_kv, total, P, d, ps, S)
+
+
+def prefill(L, q=A, kp=A, vp=A, pt=A, sl=A, cu=A, o=A, lse=A, B=2, H=8, H_kv=2, total=100,
+            maxq=60, P=8, d=128, ps=256, causal=1, scale=0.1):
+    return L.fa_prefill_paged(q, kp, vp, pt, sl, cu, o, lse, B, H, H_kv, total, maxq, P, d, ps,
+                              causal, scale, S)
+
+
+def test_append_and_prefill_argument_errors(L):
+    assert append(L, cu=None) == fa.FA_ERR_NULL
+    assert append(L, P=0) == fa.FA_ERR_SHAPE
+    assert append(L, total=-1) == fa.FA_ERR_SHAPE
+    assert append(L, ps=128) == fa.FA_ERR_UNSUPPORTED
+    assert append(L, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert append(L, kp=MIS) == fa.FA_ERR_ALIGN
+    assert prefill(L, cu=None) == fa.FA_ERR_NULL
+    assert prefill(L, H_kv=3) == fa.FA_ERR_SHAPE
+    assert prefill(L, maxq=0) == fa.FA_ERR_SHAPE
+    assert prefill(L, P=0) == fa.FA_ERR_SHAPE
+    assert prefill(L, ps=64) == fa.FA_ERR_UNSUPPORTED
+    assert prefill(L, scale=float("nan")) == fa.FA_ERR_SHAPE
+    assert prefill(L, lse=MIS) == fa.FA_ERR_ALIGN
+
+
 def gather(L, pages=A, pt=A, sl=A, out=A, B=4, H=2, d=128, ps=256):
     return L.fa_gather_paged(pages, pt, sl, out, B, H, d, ps, S)
 
@@ -137,6 +164,8 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
     assert fwd_gqa(L) == fa.FA_ERR_CUDA
     assert decode(L) == fa.FA_ERR_CUDA
     assert decode_gqa(L) == fa.FA_ERR_CUDA
+    assert append(L) == fa.FA_ERR_CUDA
+    assert prefill(L) == fa.FA_ERR_CUDA
     code = ctypes.c_int(7)
     assert L.fa_get_device_error(ctypes.byref(code), S) == fa.FA_ERR_CUDA
 
