@@ -136,6 +136,18 @@ def gqa_fwd_inputs(B, H, H_kv, N, d, seed, std=1.0, device=None):
     return q, k, v
 
 
+def rope_tables(max_pos: int, d: int, base: float = 10000.0, device: Optional[str] = None):
+    """The rotary-embedding lookup tables: cos and sin of p * base^(-2i/d) for
+    positions p < max_pos and i < d/2, evaluated in fp64 and stored as fp32
+    [max_pos, d/2] (the caller-side precomputation the attention calls take as
+    input)."""
+    i = torch.arange(d // 2, dtype=torch.float64)
+    inv = base ** (-2.0 * i / d)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * inv[None, :]
+    dev = device or "cpu"
+    return ang.cos().float().to(dev).contiguous(), ang.sin().float().to(dev).contiguous()
+
+
 def varlen_lengths(B: int, lo: int, hi: int, seed: int) -> List[int]:
     g = _gen(seed, "cpu")
     return [int(x) for x in torch.randint(lo, hi + 1, (B,), generator=g)]

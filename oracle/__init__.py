@@ -53,6 +53,10 @@ def lib():
         L.oracle_prefill_paged.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64,
                                            ctypes.c_int, ctypes.c_double]
         L.oracle_prefill_paged.restype = ctypes.c_int
+        L.oracle_rope_exact.argtypes = [P, P, P, I64, I64, I64]
+        L.oracle_rope_exact.restype = None
+        L.oracle_rope_bf16.argtypes = [P, P, P, I64, I64, I64]
+        L.oracle_rope_bf16.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         _LIB = L
@@ -235,3 +239,21 @@ def prefill_paged(q, k_pages, v_pages, page_table, seq_lens, cu_q, page_size: in
     if rc != 0:
         raise RuntimeError(f"oracle_prefill_paged failed ({rc})")
     return o, lse
+
+
+def rope(x, cos_t, sin_t, bf16_round: bool = True):
+    """Rotary embedding of x [..., N, d] (positions 0..N-1) with the fp32 tables
+    cos_t, sin_t [>=N, d/2]; returns a new fp64 array.  With bf16_round the
+    rotated values are computed in fp32 and rounded to bf16 as the GPU path
+    does before its tensor cores; without it, exactly in fp64."""
+    xs = _f64(x).copy()
+    N, d = xs.shape[-2], xs.shape[-1]
+    c = np.ascontiguousarray(np.asarray(cos_t.cpu() if hasattr(cos_t, "cpu") else cos_t,
+                                        dtype=np.float32)[:N])
+    s_ = np.ascontiguousarray(np.asarray(sin_t.cpu() if hasattr(sin_t, "cpu") else sin_t,
+                                         dtype=np.float32)[:N])
+    assert c.shape == (N, d // 2) and s_.shape == (N, d // 2)
+    rows = int(np.prod(xs.shape[:-2])) if xs.ndim > 2 else 1
+    fn = lib().oracle_rope_bf16 if bf16_round else lib().oracle_rope_exact
+    fn(_ptr(xs), c.ctypes.data_as(ctypes.c_void_p), s_.ctypes.data_as(ctypes.c_void_p), rows, N, d)
+    return xs

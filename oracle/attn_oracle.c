@@ -477,6 +477,66 @@ int oracle_prefill_paged(const double *q, const double *k_pages, const double *v
     return rc;
 }
 
+/* Rotary position embedding, applied to q and k before the scores (the page
+ * "“Flash”不是那个被时代淘汰的插件" (0539edu.com), section 2 -- the kernel
+ * fuses RoPE -- and section 3 -- from a precomputed sin/cos lookup table).
+ * Rotate-half pairing: for position p and i < d/2 the pair (x_i, x_{i+d/2})
+ * is rotated by the angle whose cosine and sine are cos_t[p*(d/2) + i],
+ * sin_t[p*(d/2) + i]:
+ *     x'_i       = x_i cos - x_{i+d/2} sin
+ *     x'_{i+d/2} = x_{i+d/2} cos + x_i sin
+ * x is [rows, N, d] (row r, position n at x + (r*N + n)*d), rotated in place.
+ * oracle_rope_exact computes in fp64.  oracle_rope_bf16 takes the decision
+ * the GPU path takes: the rotated values feed bf16 tensor cores, so they are
+ * computed in fp32 (sin term first, then one fused multiply-add with the cos
+ * term) and rounded to bf16, round-to-nearest-even. */
+void oracle_rope_exact(double *x, const float *cos_t, const float *sin_t, int64_t rows,
+                       int64_t N, int64_t d) {
+    const int64_t half = d / 2;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            double *v = x + (r * N + n) * d;
+            for (int64_t i = 0; i < half; ++i) {
+                const double c = cos_t[n * half + i], sn = sin_t[n * half + i];
+                const double a = v[i], b = v[i + half];
+                v[i] = a * c - b * sn;
+                v[i + half] = b * c + a * sn;
+            }
+        }
+}
+
+static double round_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) { /* inf or nan: keep, quiet the nan */
+        if (u & 0x007fffffu) u |= 0x00400000u;
+        u &= 0xffff0000u;
+    } else {
+        u += 0x7fffu + ((u >> 16) & 1u);
+        u &= 0xffff0000u;
+    }
+    float g;
+    memcpy(&g, &u, 4);
+    return (double)g;
+}
+
+void oracle_rope_bf16(double *x, const float *cos_t, const float *sin_t, int64_t rows,
+                      int64_t N, int64_t d) {
+    const int64_t half = d / 2;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            double *v = x + (r * N + n) * d;
+            for (int64_t i = 0; i < half; ++i) {
+                const float c = cos_t[n * half + i], sn = sin_t[n * half + i];
+                const float a = (float)v[i], b = (float)v[i + half];
+                const float ta = fmaf(a, c, -(b * sn));
+                const float tb = fmaf(b, c, a * sn);
+                v[i] = round_bf16(ta);
+                v[i + half] = round_bf16(tb);
+            }
+        }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -581,3 +581,80 @@ def test_prefill_paged_whole_sequence_is_causal_varlen():
     o2, l2 = oracle.attention_varlen(q, np.concatenate(ks), np.concatenate(vs), cu, True, 0.3)
     np.testing.assert_allclose(o, o2, atol=1e-15)
     np.testing.assert_allclose(lse, l2, atol=1e-15)
+
+
+# -- rotary position embedding (page "“Flash”不是那个被时代淘汰的插件",
+#    sections 2 and 3: RoPE fused into the kernel, sin/cos from a table) -----------
+
+def test_rope_table_closed_form():
+    from attn_fwd_04_b200 import workloads as W
+    c, s = W.rope_tables(300, 8, base=10000.0)
+    for p in (0, 1, 7, 299):
+        for i in range(4):
+            ang = p * 10000.0 ** (-2.0 * i / 8)
+            assert abs(float(c[p, i]) - math.cos(ang)) < 1e-7
+            assert abs(float(s[p, i]) - math.sin(ang)) < 1e-7
+    assert bool((c[0] == 1).all()) and bool((s[0] == 0).all())
+
+
+def test_rope_hand_worked_d2():
+    """d = 2: the single pair rotates by angle p (theta_0 = base^0 = 1):
+    (1, 0) -> (cos p, sin p) and (0, 1) -> (-sin p, cos p)."""
+    from attn_fwd_04_b200 import workloads as W
+    c, s = W.rope_tables(4, 2)
+    x = np.array([[[1.0, 0.0], [1.0, 0.0], [0.0, 1.0], [0.0, 1.0]]])
+    y = oracle.rope(x, c, s, bf16_round=False)
+    for p in range(4):
+        cp, sp = float(c[p, 0]), float(s[p, 0])
+        exp = (cp, sp) if p < 2 else (-sp, cp)
+        np.testing.assert_allclose(y[0, p], exp, atol=1e-15)
+    assert abs(float(c[3, 0]) - math.cos(3.0)) < 1e-7
+
+
+def test_rope_preserves_pair_norms_and_is_relative():
+    from attn_fwd_04_b200 import workloads as W
+    d, N = 16, 40
+    c, s = W.rope_tables(N, d)
+    q, k = _rand((1, N, d), 200), _rand((1, N, d), 201)
+    qr, kr = oracle.rope(q, c, s, False), oracle.rope(k, c, s, False)
+    h = d // 2
+    # norms are kept up to cos^2 + sin^2 = 1 of the fp32 table entries (~1e-7)
+    np.testing.assert_allclose(qr[..., :h] ** 2 + qr[..., h:] ** 2,
+                               q[..., :h] ** 2 + q[..., h:] ** 2, rtol=1e-6)
+    # the score of rotated q at p and k at p' depends on p - p' only (to the
+    # fp32 precision of the tables): shift both positions by 5
+    qs, ks = np.zeros_like(q), np.zeros_like(k)
+    qs[0, 5:], ks[0, 5:] = q[0, :-5], k[0, :-5]
+    qsr, ksr = oracle.rope(qs, c, s, False), oracle.rope(ks, c, s, False)
+    for p, pp in ((3, 1), (10, 0), (20, 20)):
+        a = qr[0, p] @ kr[0, pp]
+        b = qsr[0, p + 5] @ ksr[0, pp + 5]
+        assert abs(a - b) < 1e-5 * (1 + abs(a))
+
+
+def test_rope_bf16_is_the_rounded_rotation():
+    """The bf16 variant differs from the exact rotation by at most half a bf16
+    ulp (2^-9 relative) plus fp32 rounding, and its values are bf16 numbers."""
+    from attn_fwd_04_b200 import workloads as W
+    torch = pytest.importorskip("torch")
+    d, N = 64, 50
+    c, s = W.rope_tables(N, d)
+    x = torch.randn((2, N, d), generator=torch.Generator().manual_seed(202)).to(torch.bfloat16)
+    ex = oracle.rope(x, c, s, False)
+    rb = oracle.rope(x, c, s, True)
+    assert np.all(np.abs(rb - ex) <= np.abs(ex) * 2.0 ** -8 + 1e-30)
+    rt = torch.from_numpy(rb).float().to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(rt, rb)
+
+
+def test_rope_second_frequency_d4():
+    """d = 4: component 1 pairs with component 3 and turns at
+    theta_1 = base^(-1/2) = 0.01: e_1 at position p -> (0, cos, 0, sin)."""
+    from attn_fwd_04_b200 import workloads as W
+    c, s = W.rope_tables(60, 4)
+    x = np.zeros((1, 60, 4))
+    x[0, :, 1] = 1.0
+    y = oracle.rope(x, c, s, bf16_round=False)
+    for p in (0, 17, 59):
+        np.testing.assert_allclose(y[0, p], [0.0, math.cos(0.01 * p), 0.0, math.sin(0.01 * p)],
+                                   atol=1e-7)
