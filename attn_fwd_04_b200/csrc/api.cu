@@ -137,9 +137,15 @@ int device_error_word(unsigned int** err, int* num_sms) {
 
 namespace {
 
-// Fixed-length forward pass with H query heads and H_kv K/V heads.
+// Fixed-length forward pass with H query heads and H_kv K/V heads; with
+// rope_cos / rope_sin (tables of max_pos rows) Q and K are rotated first.
 int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-              int H_kv, int N, int d, int causal, float scale, fa_stream_t stream) {
+              int H_kv, int N, int d, int causal, float scale, fa_stream_t stream,
+              const float* rope_cos = nullptr, const float* rope_sin = nullptr,
+              int max_pos = 0) {
+    if ((rope_cos == nullptr) != (rope_sin == nullptr)) return FA_ERR_NULL;
+    if (rope_cos && (max_pos < N || !aligned16(rope_cos) || !aligned16(rope_sin)))
+        return max_pos < N ? FA_ERR_SHAPE : FA_ERR_ALIGN;
     if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
     if (B < 1 || H < 1 || H_kv < 1 || N < 1) return FA_ERR_SHAPE;
     if (H % H_kv != 0) return FA_ERR_SHAPE;
@@ -170,6 +176,8 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     p.B = B;
     p.H = H;
     p.H_kv = H_kv;
+    p.rope_cos = rope_cos;
+    p.rope_sin = rope_sin;
     p.N = N;
     p.total = 0;
     p.causal = causal ? 1 : 0;
@@ -190,6 +198,14 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int H_kv, int N, int d, int causal, float scale, fa_stream_t stream) {
     return fwd_fixed(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, stream);
+}
+
+int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse,
+                const float* rope_cos, const float* rope_sin, int max_pos, int B, int H,
+                int H_kv, int N, int d, int causal, float scale, fa_stream_t stream) {
+    if (!rope_cos || !rope_sin) return FA_ERR_NULL;
+    return fwd_fixed(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, stream, rope_cos,
+                     rope_sin, max_pos);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -26,6 +26,8 @@ struct FwdParams {
     int H_kv;            // K/V heads; query head h reads K/V head h / (H / H_kv)
     const int32_t* page_table;  // paged prefill: packed page table
     const int32_t* ctx_lens;    // paged prefill: cached tokens (keys) per sequence
+    const float* rope_cos;      // fixed-length RoPE: [>= N, d/2] tables, or null
+    const float* rope_sin;
     int total;           // varlen: packed rows
     int causal;
     float scale_log2;    // scale * log2(e)

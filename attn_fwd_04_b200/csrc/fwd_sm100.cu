@@ -72,6 +72,8 @@ struct alignas(1024) FwdSmem {
     uint64_t kv_full[kSlots], kv_empty[kSlots];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
+    uint64_t q_rot;      // RoPE: both Q tiles rotated
+    uint64_t k_rot[2];   // RoPE: K_j rotated (K tiles use ring slots 0 and 2: index j % 2)
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -170,11 +172,61 @@ __device__ __forceinline__ float exp_pairs(const uint32_t (&s)[BN], uint32_t (&p
     return f2_lo(a2) + f2_hi(a2);
 }
 
+// Rotary position embedding of row r of a tile in shared memory (one or two
+// 128-row x 64-column boxes, 128-byte swizzle) at position pos: the pairs
+// (i, i + D/2) are turned by the angle whose cosine and sine are
+// cos_t[pos*(D/2) + i], sin_t[...] -- the precomputed table of the page
+// "“Flash”不是那个被时代淘汰的插件" (0539edu.com), section 3.  Computed in fp32
+// (sin term first, then one fused multiply-add) and rounded to bf16.
+template <int D>
+__device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const float* cos_t,
+                                         const float* sin_t) {
+    constexpr int HALF = D / 2;
+    const float* ct = cos_t + static_cast<int64_t>(pos) * HALF;
+    const float* st = sin_t + static_cast<int64_t>(pos) * HALF;
+#pragma unroll 2
+    for (int c = 0; c < HALF / 8; ++c) {
+        const int i0 = 8 * c, i1 = 8 * c + HALF;  // first dims of the two chunks
+        uint4* pa = reinterpret_cast<uint4*>(tile + (i0 / 64) * kBoxBytes + r * 128 +
+                                             ((((i0 % 64) / 8) ^ (r & 7)) * 16));
+        uint4* pb = reinterpret_cast<uint4*>(tile + (i1 / 64) * kBoxBytes + r * 128 +
+                                             ((((i1 % 64) / 8) ^ (r & 7)) * 16));
+        const uint4 ua = *pa, ub = *pb;
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(ct + i0));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(ct + i0 + 4));
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(st + i0));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(st + i0 + 4));
+        const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float a[2] = {__uint_as_float(wa[e] << 16), __uint_as_float(wa[e] & 0xffff0000u)};
+            float b[2] = {__uint_as_float(wb[e] << 16), __uint_as_float(wb[e] & 0xffff0000u)};
+            float ra[2], rb[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const float cc = cs[2 * e + k], ss = sn[2 * e + k];
+                const float bs = b[k] * ss, as = a[k] * ss;
+                ra[k] = fmaf(a[k], cc, -bs);
+                rb[k] = fmaf(b[k], cc, as);
+            }
+            oa[e] = pack_bf16x2(ra[0], ra[1]);
+            ob[e] = pack_bf16x2(rb[0], rb[1]);
+        }
+        *pa = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *pb = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+}
+
 // MODE: kFixed ([B,H,N,d] tensors), kVarlen (packed [total,H,d] sequences),
 // kPaged (packed queries; keys and values read through the page table from a
 // pool of 256-token pages, the queries being the last positions of each
 // cached sequence).
-template <int D, int MODE>
+// ROPE (fixed-length only): Q and K are rotated in shared memory by the
+// epilogue warpgroup (idle until the last step) before their score products.
+template <int D, int MODE, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
@@ -265,6 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.stats_full[t], BM);
         }
         mbar_init(&sm.vfix, 1);
+        mbar_init(&sm.q_rot, BM);
+        mbar_init(&sm.k_rot[0], BM);
+        mbar_init(&sm.k_rot[1], BM);
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
@@ -401,10 +456,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                            idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
             };
             bool ok = true;
-            for (int t = 0; t < 2 && ok; ++t)
-                if (n_t[t] > 0) ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort);
-            ok = ok && mbar_wait(&sm.kv_full[ring_slot(0, 0)], ring_phase(0, 0), err,
-                                 FA_DEVERR_TIMEOUT, abort);
+            // K_j ready for its score products: landed, and rotated under ROPE
+            auto wait_k = [&](int j) {
+                if constexpr (ROPE)
+                    return mbar_wait(&sm.k_rot[j & 1], (j >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort);
+                else
+                    return mbar_wait(&sm.kv_full[ring_slot(j, 0)], ring_phase(j, 0), err,
+                                     FA_DEVERR_TIMEOUT, abort);
+            };
+            if constexpr (ROPE) {
+                ok = mbar_wait(&sm.q_rot, 0, err, FA_DEVERR_TIMEOUT, abort);
+            } else {
+                for (int t = 0; t < 2 && ok; ++t)
+                    if (n_t[t] > 0)
+                        ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort);
+            }
+            ok = ok && wait_k(0);
             if (ok) {
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t) {
@@ -423,8 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const bool next_k = j + 1 < n;
-                if (next_k && !mbar_wait(&sm.kv_full[ring_slot(j + 1, 0)], ring_phase(j + 1, 0),
-                                         err, FA_DEVERR_TIMEOUT, abort)) break;
+                if (next_k && !wait_k(j + 1)) break;
                 for (int t = 0; t < 2; ++t) {
                     if (j >= n_t[t]) continue;
                     if (!mbar_wait(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
@@ -542,6 +608,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = threadIdx.x - 2 * BM;
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
+        if constexpr (ROPE) {
+            // rotate both Q tiles, then every K tile as it lands; rows past
+            // the sequence end are TMA zero fill and stay zero
+            for (int t = 0; ok && t < 2; ++t) {
+                if (n_t[t] == 0) continue;
+                if (!warp_wait(&sm.q_full[t], 0, err, abort)) {
+                    ok = false;
+                    break;
+                }
+                const int pos = row0 + t * BM + r;
+                if (pos < len) rope_row<D>(sm.q[t], r, pos, p.rope_cos, p.rope_sin);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (ok) mbar_arrive(&sm.q_rot);
+            for (int j = 0; ok && j < n; ++j) {
+                if (!warp_wait(&sm.kv_full[ring_slot(j, 0)], ring_phase(j, 0), err, abort)) {
+                    ok = false;
+                    break;
+                }
+                const int pos = j * BN + r;
+                if (pos < len) rope_row<D>(sm.kv[ring_slot(j, 0)], r, pos, p.rope_cos, p.rope_sin);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(&sm.k_rot[j & 1]);
+            }
+        }
         // epilogue: O / l -> bf16, log-sum-exp
         for (int t = 0; ok && t < 2; ++t) {
             if (n_t[t] == 0) continue;
@@ -599,14 +690,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 12) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool ROPE = false>
 int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, cudaStream_t stream) {
     // Every CTA allocates all 512 TMEM columns, so one CTA per SM: ask for
     // enough shared memory that a second CTA cannot be co-resident.
     const size_t smem = sizeof(FwdSmem<D>) + 1024 > 120 * 1024 ? sizeof(FwdSmem<D>) + 1024
                                                                : 120 * 1024;
-    auto kern = fa_fwd_kernel<D, MODE>;
+    auto kern = fa_fwd_kernel<D, MODE, ROPE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -625,6 +716,9 @@ int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     switch (mode) {
         case kFixed:
+            if (p.rope_cos)
+                return d == 128 ? launch_impl<128, kFixed, true>(p, tq, tk, tv, stream)
+                                : launch_impl<64, kFixed, true>(p, tq, tk, tv, stream);
             return d == 128 ? launch_impl<128, kFixed>(p, tq, tk, tv, stream)
                             : launch_impl<64, kFixed>(p, tq, tk, tv, stream);
         case kVarlen:

@@ -24,7 +24,7 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+        L.fa_fwd_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
@@ -63,7 +64,7 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen", "fa_decode_paged",
+        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_fwd_varlen", "fa_decode_paged",
                      "fa_decode_paged_gqa", "fa_decode_paged_noalloc", "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
@@ -141,6 +142,34 @@ def fa_fwd_gqa(q, k, v, causal: bool, scale: Optional[float] = None, o=None, lse
     rc = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           B, H, H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
     _raise_if(rc, "fa_fwd_gqa")
+    return o, lse
+
+
+def fa_fwd_rope(q, k, v, rope_cos, rope_sin, causal: bool, scale: Optional[float] = None,
+                o=None, lse=None, stream=None):
+    """Forward with rotary embedding applied in the kernel: q [B,H,N,d],
+    k/v [B,H_kv,N,d] bf16 (unrotated), tables [max_pos,d/2] fp32 ->
+    (o [B,H,N,d], lse [B,H,N])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    _check(rope_cos, "rope_cos", torch.float32, 2)
+    _check(rope_sin, "rope_sin", torch.float32, 2)
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    if k.shape != (B, H_kv, N, d) or v.shape != k.shape:
+        raise ValueError("k, v must be [B,H_kv,N,d] with q's B, N, d")
+    if rope_cos.shape[1] != d // 2 or rope_sin.shape != rope_cos.shape:
+        raise ValueError("rope tables must be [max_pos, d/2]")
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = lib().fa_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           rope_cos.data_ptr(), rope_sin.data_ptr(), rope_cos.shape[0], B, H,
+                           H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_fwd_rope")
     return o, lse
 
 

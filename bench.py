@@ -299,6 +299,15 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
     timed(lambda: fa.fa_fwd_gqa(q, k, v, True, 1 / math.sqrt(w.d), o=o, lse=lse, stream=stream),
           fwd_flops(w), f"gqa_long_prefill_fwd_b1_h32_hkv{GQA_HKV}_n16384_d128_causal")
     del q, k, v, o, lse
+    # rotary embedding fused into the forward pass: the long-prefill workload
+    q, k, v = W.fwd_inputs(w, device="cuda")
+    rc, rs = W.rope_tables(w.N, w.d, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    timed(lambda: fa.fa_fwd_rope(q, k, v, rc, rs, True, 1 / math.sqrt(w.d), o=o, lse=lse,
+                                 stream=stream),
+          fwd_flops(w), f"rope_{w.name}")
+    del q, k, v, o, lse, rc, rs
     # grouped-query paged decode: the decode workload's lengths, 8 K/V heads
     lengths = W.varlen_lengths(DEC.B, DEC.len_lo, DEC.len_hi, DEC.seed)
     c = W.paged_inputs(DEC.B, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda",

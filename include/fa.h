@@ -107,6 +107,25 @@ FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, floa
            int B, int H, int H_kv, int N, int d, int causal, float scale, fa_stream_t stream);
 
 /*
+ * fa_fwd_rope -- fa_fwd_gqa with rotary position embedding fused into the
+ * kernel: the page "“Flash”不是那个被时代淘汰的插件" (0539edu.com) describes a
+ * kernel that fuses RoPE (section 2) from a precomputed sin/cos lookup table
+ * (section 3).  q and k are passed unrotated; each Q and K tile is rotated in
+ * on-chip memory after it is loaded and before its score product.
+ *   rope_cos, rope_sin : DEVICE fp32 [max_pos, d/2], row-major; entry (p, i)
+ *                        is cos / sin of the angle for position p and pair i
+ *                        (normally p * base^(-2i/d)); max_pos >= N
+ * Position of row n is n.  Rotate-half pairs: for i < d/2,
+ *   x'_i = x_i cos - x_{i+d/2} sin,  x'_{i+d/2} = x_{i+d/2} cos + x_i sin,
+ * evaluated in fp32 and rounded to bf16 (the tensor cores' input), then
+ * attention as fa_fwd_gqa on the rotated q, k.  Both tables NULL or unaligned:
+ * FA_ERR_NULL / FA_ERR_ALIGN; max_pos < N: FA_ERR_SHAPE.
+ */
+FA_API int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse,
+           const float* rope_cos, const float* rope_sin, int max_pos, int B, int H, int H_kv,
+           int N, int d, int causal, float scale, fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- the forward pass over B sequences of different lengths
  * packed back to back (the variable-length batches of the page "Flash
  * Attention 是什么", section 典型应用场景).

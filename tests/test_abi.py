@@ -129,6 +129,20 @@ def test_fwd_gqa_argument_errors(L):
     assert fwd_gqa(L, v=MIS) == fa.FA_ERR_ALIGN
 
 
+def rope_fwd(L, q=A, k=A, v=A, o=A, lse=A, c=A, sn=A, maxpos=256, B=1, H=4, H_kv=2, N=256,
+             d=128, causal=1, scale=0.1):
+    return L.fa_fwd_rope(q, k, v, o, lse, c, sn, maxpos, B, H, H_kv, N, d, causal, scale, S)
+
+
+def test_fwd_rope_argument_errors(L):
+    assert rope_fwd(L, c=None) == fa.FA_ERR_NULL
+    assert rope_fwd(L, sn=None) == fa.FA_ERR_NULL
+    assert rope_fwd(L, maxpos=100) == fa.FA_ERR_SHAPE      # table shorter than N
+    assert rope_fwd(L, c=MIS) == fa.FA_ERR_ALIGN
+    assert rope_fwd(L, H_kv=3) == fa.FA_ERR_SHAPE
+    assert rope_fwd(L, d=32) == fa.FA_ERR_UNSUPPORTED
+
+
 def test_varlen_argument_errors(L):
     assert varlen(L, cu=None) == fa.FA_ERR_NULL
     assert varlen(L, total=0) == fa.FA_ERR_SHAPE
@@ -162,6 +176,7 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
     # arguments pass validation; the device lookup then fails cleanly
     assert fwd(L) == fa.FA_ERR_CUDA
     assert fwd_gqa(L) == fa.FA_ERR_CUDA
+    assert rope_fwd(L) == fa.FA_ERR_CUDA
     assert decode(L) == fa.FA_ERR_CUDA
     assert decode_gqa(L) == fa.FA_ERR_CUDA
     assert append(L) == fa.FA_ERR_CUDA

@@ -287,3 +287,70 @@ def test_gqa_long_prefill_sampled():
         ref_l.append(lse_ref[0, 0, rows])
     assert_o_close(np.concatenate(got_o), np.concatenate(ref_o), "gqa long prefill")
     assert_lse_close(np.concatenate(got_l), np.concatenate(ref_l), "gqa long prefill")
+
+
+# -- rotary embedding fused into the forward pass (fa_fwd_rope) -------------------
+
+def _rope_ref(q, k, v, c, s, causal, scale):
+    """Oracle: rotate q and k (fp32 rotation rounded to bf16, the precision the
+    kernel feeds its tensor cores), then grouped-query attention in fp64."""
+    qr = oracle.rope(q, c, s, bf16_round=True)
+    kr = oracle.rope(k, c, s, bf16_round=True)
+    return oracle.attention_gqa(qr, kr, v, causal, scale), qr, kr
+
+
+ROPE_SHAPES = [(1, 2, 2, 300, 128), (2, 4, 2, 129, 64), (1, 2, 1, 1, 128), (1, 4, 4, 1000, 128),
+               (1, 2, 2, 2049, 64)]
+
+
+@pytest.mark.parametrize("shape", ROPE_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_rope_full_compare(shape, causal):
+    B, H, Hkv, N, d = shape
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=400 + N + d, device="cpu")
+    c, s = W.rope_tables(N + 17, d)
+    scale = 1 / math.sqrt(d)
+    o = torch.full_like(q.cuda(), float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda")
+    fa.fa_fwd_rope(q.cuda(), k.cuda(), v.cuda(), c.cuda(), s.cuda(), causal, scale, o=o, lse=lse)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    (o_ref, lse_ref), _, _ = _rope_ref(q, k, v, c, s, causal, scale)
+    assert_o_close(to64(o), o_ref, f"rope {shape}")
+    assert_lse_close(to64(lse), lse_ref, f"rope {shape}")
+
+
+def test_rope_equals_fwd_on_prerotated_inputs():
+    """The in-kernel rotation produces exactly the bf16 values of the oracle's
+    fp32 rotation, so fa_fwd_rope equals fa_fwd_gqa on pre-rotated q, k bit
+    for bit."""
+    B, H, Hkv, N, d = 1, 4, 2, 777, 128
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=410, device="cpu")
+    c, s = W.rope_tables(N, d)
+    o, lse = fa.fa_fwd_rope(q.cuda(), k.cuda(), v.cuda(), c.cuda(), s.cuda(), True, 0.1)
+    qr = torch.from_numpy(oracle.rope(q, c, s, True)).to(torch.bfloat16).cuda()
+    kr = torch.from_numpy(oracle.rope(k, c, s, True)).to(torch.bfloat16).cuda()
+    o2, l2 = fa.fa_fwd_gqa(qr, kr, v.cuda(), True, 0.1)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+def test_rope_long_prefill_sampled():
+    w = W.LONG_PREFILL
+    q, k, v = W.fwd_inputs(w, device="cuda")
+    c, s = W.rope_tables(w.N, w.d, device="cuda")
+    scale = 1 / math.sqrt(w.d)
+    o, lse = fa.fa_fwd_rope(q, k, v, c, s, True, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    cc, sc = c.cpu(), s.cpu()
+    got_o, ref_o, got_l, ref_l = [], [], [], []
+    for h in (0, 13, 31):
+        rows = sample_rows(w.N, 24, 600 + h)
+        qh, kh, vh = q[0, h].cpu()[None, None], k[0, h].cpu()[None, None], v[0, h].cpu()[None, None]
+        qr, kr = oracle.rope(qh, cc, sc, True), oracle.rope(kh, cc, sc, True)
+        o_ref, lse_ref = oracle.attention(qr, kr, vh, True, scale, rows=rows)
+        got_o.append(to64(o[0, h, rows]))
+        ref_o.append(o_ref[0, 0, rows])
+        got_l.append(to64(lse[0, h, rows]))
+        ref_l.append(lse_ref[0, 0, rows])
+    assert_o_close(np.concatenate(got_o), np.concatenate(ref_o), "rope long prefill")
+    assert_lse_close(np.concatenate(got_l), np.concatenate(ref_l), "rope long prefill")
