@@ -348,6 +348,54 @@ def decode_cache(batch: int, h_kv: int) -> W.PagedCache:
                           device="cuda", H_kv=h_kv)
 
 
+def run_single_path(args, local):
+    """Profiling aid (--only prefill / rope): the paged-prefill workload or the
+    RoPE forward pass on the long-prefill workload, alone, timed with CUDA
+    events; prints its own short JSON line."""
+    import attn_fwd_04_b200 as fa
+    torch.cuda.set_device(local)
+    stream = torch.cuda.current_stream()
+    if args.only == "prefill":
+        w = W.PAGED_PREFILL
+        cache, q, cu = W.prefill_workload_inputs(w, device="cuda")
+        pt, sl, cud = cache.page_table.cuda(), cache.seq_lens.cuda(), cu.cuda()
+        o = torch.empty_like(q)
+        lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=q.device)
+        pairs = sum(w.q_len * (int(L) - w.q_len) + w.q_len * (w.q_len + 1) // 2
+                    for L in cache.seq_lens.tolist())
+        flops = 4.0 * w.d * w.H * pairs
+        name = w.name
+
+        def fn():
+            fa.fa_prefill_paged(q, cache.k_pages, cache.v_pages, pt, sl, cud, w.q_len, w.causal,
+                                1 / math.sqrt(w.d), o=o, lse=lse, stream=stream)
+    else:
+        w = FWD
+        q, k, v = W.fwd_inputs(w, device="cuda")
+        rc, rs = W.rope_tables(w.N, w.d, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        flops = fwd_flops(w)
+        name = f"rope_{w.name}"
+
+        def fn():
+            fa.fa_fwd_rope(q, k, v, rc, rs, True, 1 / math.sqrt(w.d), o=o, lse=lse, stream=stream)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("device error")
+    ms = e0.elapsed_time(e1) / args.steps
+    return {"workload": name, "ms_per_launch": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+            "steps": args.steps, "warmup": args.warmup}
+
+
 def run_native(args, world, rank, local):
     import attn_fwd_04_b200 as fa
 
@@ -604,7 +652,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the forward pass on the other workloads")
-    ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "fwd", "decode", "prefill", "rope"], default="all",
                     help="profiling aid: run one entry point only (the JSON line then "
                          "reports that part alone)")
     ap.add_argument("--decode-hkv", type=int, default=DEC.H,
@@ -621,6 +669,10 @@ def main(argv=None):
         out = run_reference(args, world, int(os.environ.get("RANK", "0")))
         if out is not None:
             print(json.dumps(out), flush=True)
+        return
+    if args.only in ("prefill", "rope"):
+        print(json.dumps(run_single_path(args, int(os.environ.get("LOCAL_RANK", "0")))),
+              flush=True)
         return
     world, rank, local = dist_setup(args)
     try:
