@@ -57,6 +57,9 @@ def lib():
         L.oracle_rope_exact.restype = None
         L.oracle_rope_bf16.argtypes = [P, P, P, I64, I64, I64]
         L.oracle_rope_bf16.restype = None
+        L.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64,
+                                           ctypes.c_int, ctypes.c_double]
+        L.oracle_attention_bwd.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         _LIB = L
@@ -257,3 +260,17 @@ def rope(x, cos_t, sin_t, bf16_round: bool = True):
     fn = lib().oracle_rope_bf16 if bf16_round else lib().oracle_rope_exact
     fn(_ptr(xs), c.ctypes.data_as(ctypes.c_void_p), s_.ctypes.data_as(ctypes.c_void_p), rows, N, d)
     return xs
+
+
+def attention_bwd(q, k, v, dout, causal: bool, scale: float):
+    """Gradients (dq, dk, dv) of attention over q, k, v [B,H,N,d] for the
+    output gradient dout [B,H,N,d], in fp64."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    assert k.shape == v.shape == g.shape == (B, H, N, d)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    rc = lib().oracle_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), B, H, N, d, int(bool(causal)), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_bwd failed ({rc})")
+    return dq, dk, dv

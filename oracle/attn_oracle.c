@@ -537,6 +537,102 @@ void oracle_rope_bf16(double *x, const float *cos_t, const float *sin_t, int64_t
         }
 }
 
+/* Gradients of the attention of one problem with respect to q, k and v,
+ * given the output gradient do -- the backward pass the saved row statistics
+ * serve (page "Flash Attention 是什么", section 核心工作机制, recomputation
+ * paragraph: the max and sum kept from the forward pass let the backward pass
+ * rebuild the scores instead of storing them).  The oracle recomputes
+ * everything from q, k, v: for each (b, h) and row i,
+ *   p_ij  = exp(s_ij - lse_i),  s_ij = scale q_i.k_j  (j admissible)
+ *   dV_j += p_ij do_i
+ *   dp_ij = do_i . v_j
+ *   D_i   = sum_j p_ij dp_ij        (= do_i . o_i)
+ *   ds_ij = p_ij (dp_ij - D_i)
+ *   dQ_i  = scale sum_j ds_ij k_j
+ *   dK_j += scale ds_ij q_i
+ * q, k, v, do, dq, dk, dv are [B,H,N,d].  Rows are split over threads; each
+ * thread accumulates dK, dV of its rows privately and the partial sums are
+ * added in thread order, so the result does not depend on scheduling for a
+ * fixed thread count. */
+int oracle_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
+                         double *dq, double *dk, double *dv, int64_t B, int64_t H, int64_t N,
+                         int64_t d, int causal, double scale) {
+    if (B < 0 || H < 0 || N < 0 || d <= 0) return -1;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const double *qb = q + bh * N * d, *kb = k + bh * N * d, *vb = v + bh * N * d;
+        const double *gb = dout + bh * N * d;
+        double *dqb = dq + bh * N * d, *dkb = dk + bh * N * d, *dvb = dv + bh * N * d;
+        for (int64_t x = 0; x < N * d; ++x) dkb[x] = dvb[x] = 0.0;
+        int nthr = 1;
+#ifdef _OPENMP
+        nthr = omp_get_max_threads();
+#endif
+        double *acc = (double *)calloc((size_t)nthr * 2 * (size_t)(N * d), sizeof(double));
+        if (!acc) return -2;
+        int failed = 0;
+#pragma omp parallel
+        {
+            int tid = 0;
+#ifdef _OPENMP
+            tid = omp_get_thread_num();
+#endif
+            double *tdk = acc + (size_t)tid * 2 * (size_t)(N * d), *tdv = tdk + N * d;
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+            double *prow = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+            if (!srow || !prow) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+#pragma omp for schedule(static)
+                for (int64_t i = 0; i < N; ++i) {
+                    const int64_t nk = causal ? i + 1 : N;
+                    const double *qi = qb + i * d, *gi = gb + i * d;
+                    double m = -INFINITY;
+                    for (int64_t j = 0; j < nk; ++j) {
+                        double dot = 0.0;
+                        for (int64_t c = 0; c < d; ++c) dot += qi[c] * kb[j * d + c];
+                        srow[j] = scale * dot;
+                        if (srow[j] > m) m = srow[j];
+                    }
+                    double l = 0.0;
+                    for (int64_t j = 0; j < nk; ++j) l += exp(srow[j] - m);
+                    const double lse = m + log(l);
+                    double Di = 0.0;
+                    for (int64_t j = 0; j < nk; ++j) {
+                        prow[j] = exp(srow[j] - lse);
+                        double dp = 0.0;
+                        for (int64_t c = 0; c < d; ++c) dp += gi[c] * vb[j * d + c];
+                        srow[j] = dp; /* srow now holds dp_ij */
+                        Di += prow[j] * dp;
+                    }
+                    double *dqi = dqb + i * d;
+                    for (int64_t c = 0; c < d; ++c) dqi[c] = 0.0;
+                    for (int64_t j = 0; j < nk; ++j) {
+                        const double ds = prow[j] * (srow[j] - Di);
+                        for (int64_t c = 0; c < d; ++c) {
+                            dqi[c] += scale * ds * kb[j * d + c];
+                            tdk[j * d + c] += scale * ds * qi[c];
+                            tdv[j * d + c] += prow[j] * gi[c];
+                        }
+                    }
+                }
+            }
+            free(srow);
+            free(prow);
+        }
+        for (int t = 0; t < nthr; ++t) {
+            const double *tdk = acc + (size_t)t * 2 * (size_t)(N * d), *tdv = tdk + N * d;
+            for (int64_t x = 0; x < N * d; ++x) {
+                dkb[x] += tdk[x];
+                dvb[x] += tdv[x];
+            }
+        }
+        free(acc);
+        if (failed) return -2;
+    }
+    return 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -658,3 +658,60 @@ def test_rope_second_frequency_d4():
     for p in (0, 17, 59):
         np.testing.assert_allclose(y[0, p], [0.0, math.cos(0.01 * p), 0.0, math.sin(0.01 * p)],
                                    atol=1e-7)
+
+
+# -- backward pass (the saved statistics serve it: page "Flash Attention 是什么",
+#    section 核心工作机制, recomputation paragraph) -----------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_equals_finite_differences(causal):
+    """dq, dk, dv are the gradients of L = sum(O * G) for the forward
+    definition: central differences of L in every input entry."""
+    B, H, N, d = 1, 2, 5, 3
+    q, k, v = _rand((B, H, N, d), 210), _rand((B, H, N, d), 211), _rand((B, H, N, d), 212)
+    g = _rand((B, H, N, d), 213)
+    scale = 0.7
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, causal, scale)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.attention(q_, k_, v_, causal, scale)
+        return float(np.sum(o * g))
+
+    h = 1e-5
+    for x, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(grad, num, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_key_gradients_sum_to_zero(causal):
+    """Each row of dS sums to zero (the softmax Jacobian annihilates
+    constants), so sum_j dK_j = scale sum_i q_i sum_j dS_ij = 0; dropping the
+    row term D_i breaks it."""
+    q, k, v, g = (_rand((1, 1, 40, 8), s) for s in (214, 215, 216, 217))
+    _, dk, _ = oracle.attention_bwd(q, k, v, g, causal, 0.4)
+    assert np.all(np.abs(dk.sum(axis=2)) < 1e-12)
+
+
+def test_bwd_zero_query_closed_form():
+    """q = 0, non-causal: P is uniform, so dV_j = mean_i dO_i for every key j,
+    and dQ_i = scale sum_j (1/N)(dO_i.v_j - dO_i.mean(v)) k_j."""
+    N, d = 7, 4
+    k, v, g = _rand((1, 1, N, d), 218), _rand((1, 1, N, d), 219), _rand((1, 1, N, d), 220)
+    q = np.zeros((1, 1, N, d))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, False, 0.5)
+    for j in range(N):
+        np.testing.assert_allclose(dv[0, 0, j], g[0, 0].mean(axis=0), atol=1e-14)
+    vbar = v[0, 0].mean(axis=0)
+    for i in range(N):
+        exp = 0.5 * sum((g[0, 0, i] @ (v[0, 0, j] - vbar)) / N * k[0, 0, j] for j in range(N))
+        np.testing.assert_allclose(dq[0, 0, i], exp, atol=1e-14)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-15)  # q = 0 -> dK = scale dS^T q = 0
