@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfa.so")
-SOURCES = ["api.cu", "fwd_sm100.cu", "decode_sm100.cu", "decode_noalloc.cu"]
+SOURCES = ["api.cu", "fwd_sm100.cu", "bwd_sm100.cu", "decode_sm100.cu", "decode_noalloc.cu"]
 HEADERS = ["fa_ptx.cuh", "fa_internal.h"]
 
 NVCC_FLAGS = [

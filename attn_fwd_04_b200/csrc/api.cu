@@ -208,6 +208,39 @@ int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse
                      rope_sin, max_pos);
 }
 
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+           int causal, float scale, fa_stream_t stream) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * H > 65535) return FA_ERR_SHAPE;
+    if (N > 0x7fffffff - 128) return FA_ERR_SHAPE;
+    if (!std::isfinite(scale)) return FA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    CUtensorMap tq, tk, tv, tdo;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(N) * d * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tdo, dout, dims, strides, box)) != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if ((rc = ensure_workspace(s, fa::bwd_workspace_bytes(B, H, N, d), st, &ws)) != FA_OK)
+        return rc;
+    return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, B, H, N, d, causal ? 1 : 0,
+                          scale, ws, s->err, s->num_sms, st);
+}
+
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int32_t* cu_seqlens, int B, int H, int total, int max_seqlen, int d,
                   int causal, float scale, fa_stream_t stream) {

@@ -39,6 +39,13 @@ constexpr int kFixed = 0, kVarlen = 1, kPaged = 2;
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, int d, int mode, cudaStream_t stream);
 
+// ---- backward ------------------------------------------------------------
+size_t bwd_workspace_bytes(int B, int H, int N, int d);
+int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+               const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const CUtensorMap& tdo, int B, int H, int N, int d, int causal, float scale,
+               void* workspace, unsigned int* err, int num_sms, cudaStream_t stream);
+
 // ---- paged decode ----------------------------------------------------------
 // Number of pages a split covers at least (a split is one CTA work unit) and
 // the most splits one sequence is cut into.

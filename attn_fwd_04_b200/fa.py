@@ -24,7 +24,7 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_fwd_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
+        L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
@@ -64,7 +65,7 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_fwd_varlen", "fa_decode_paged",
+        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged",
                      "fa_decode_paged_gqa", "fa_decode_paged_noalloc", "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
@@ -171,6 +172,28 @@ def fa_fwd_rope(q, k, v, rope_cos, rope_sin, causal: bool, scale: Optional[float
                            H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
     _raise_if(rc, "fa_fwd_rope")
     return o, lse
+
+
+def fa_bwd(q, k, v, o, lse, dout, causal: bool, scale: Optional[float] = None, dq=None,
+           dk=None, dv=None, stream=None):
+    """Gradients of fa_fwd: (dq, dk, dv), each [B,H,N,d] bf16, from q, k, v, o,
+    dout [B,H,N,d] bf16 and lse [B,H,N] fp32 (as fa_fwd returned them)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, n, torch.bfloat16, 4)
+        if t.shape != q.shape:
+            raise ValueError(f"{n} must have q's shape")
+    _check(lse, "lse", torch.float32, 3)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                      int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_bwd")
+    return dq, dk, dv
 
 
 def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,

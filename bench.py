@@ -308,6 +308,17 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
                                  stream=stream),
           fwd_flops(w), f"rope_{w.name}")
     del q, k, v, o, lse, rc, rs
+    # backward pass on the long-prefill workload: five products per tile
+    # against the forward pass's two, so 2.5x its FLOPs
+    q, k, v = W.fwd_inputs(w, device="cuda")
+    o, lse = fa.fa_fwd(q, k, v, True, 1 / math.sqrt(w.d))
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(7),
+                    device="cuda").to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    timed(lambda: fa.fa_bwd(q, k, v, o, lse, g, True, 1 / math.sqrt(w.d), dq=dq, dk=dk, dv=dv,
+                            stream=stream),
+          2.5 * fwd_flops(w), f"bwd_{w.name}")
+    del q, k, v, o, lse, g, dq, dk, dv
     # grouped-query paged decode: the decode workload's lengths, 8 K/V heads
     lengths = W.varlen_lengths(DEC.B, DEC.len_lo, DEC.len_hi, DEC.seed)
     c = W.paged_inputs(DEC.B, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda",
@@ -349,13 +360,26 @@ def decode_cache(batch: int, h_kv: int) -> W.PagedCache:
 
 
 def run_single_path(args, local):
-    """Profiling aid (--only prefill / rope): the paged-prefill workload or the
-    RoPE forward pass on the long-prefill workload, alone, timed with CUDA
-    events; prints its own short JSON line."""
+    """Profiling aid (--only prefill / rope / bwd): the paged-prefill workload,
+    or the RoPE forward pass or the backward pass on the long-prefill workload,
+    alone, timed with CUDA events; prints its own short JSON line."""
     import attn_fwd_04_b200 as fa
     torch.cuda.set_device(local)
     stream = torch.cuda.current_stream()
-    if args.only == "prefill":
+    if args.only == "bwd":
+        w = FWD
+        q, k, v = W.fwd_inputs(w, device="cuda")
+        o, lse = fa.fa_fwd(q, k, v, True, 1 / math.sqrt(w.d), stream=stream)
+        g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(7),
+                        device="cuda").to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        flops = 2.5 * fwd_flops(w)
+        name = f"bwd_{w.name}"
+
+        def fn():
+            fa.fa_bwd(q, k, v, o, lse, g, True, 1 / math.sqrt(w.d), dq=dq, dk=dk, dv=dv,
+                      stream=stream)
+    elif args.only == "prefill":
         w = W.PAGED_PREFILL
         cache, q, cu = W.prefill_workload_inputs(w, device="cuda")
         pt, sl, cud = cache.page_table.cuda(), cache.seq_lens.cuda(), cu.cuda()
@@ -652,7 +676,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the forward pass on the other workloads")
-    ap.add_argument("--only", choices=["all", "fwd", "decode", "prefill", "rope"], default="all",
+    ap.add_argument("--only", choices=["all", "fwd", "decode", "prefill", "rope", "bwd"],
+                    default="all",
                     help="profiling aid: run one entry point only (the JSON line then "
                          "reports that part alone)")
     ap.add_argument("--decode-hkv", type=int, default=DEC.H,
@@ -670,7 +695,7 @@ def main(argv=None):
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    if args.only in ("prefill", "rope"):
+    if args.only in ("prefill", "rope", "bwd"):
         print(json.dumps(run_single_path(args, int(os.environ.get("LOCAL_RANK", "0")))),
               flush=True)
         return

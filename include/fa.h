@@ -126,6 +126,28 @@ FA_API int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, flo
            int N, int d, int causal, float scale, fa_stream_t stream);
 
 /*
+ * fa_bwd -- gradients of fa_fwd (multi-head, fixed length) with respect to
+ * q, k and v for an output gradient dout, rebuilding the probabilities from
+ * the saved log-sum-exp (the page "Flash Attention 是什么", section
+ * 核心工作机制, recomputation paragraph: the forward pass keeps the softmax
+ * statistics for the backward pass).
+ *   q, k, v, o, dout : [B, H, N, d] bf16 (o as returned by fa_fwd)
+ *   lse              : [B, H, N] fp32 as returned by fa_fwd (natural log)
+ *   dq, dk, dv       : [B, H, N, d] bf16 outputs
+ * With P = exp(scale q k^T - lse) (causal: keys after the query give 0),
+ * D_i = dout_i . o_i and dS = P o (dout v^T - D):
+ *   dv = P^T dout,   dq = scale dS k,   dk = scale dS^T q.
+ * Same `causal`, `scale` and limits as fa_fwd.  Uses the library's per-GPU
+ * workspace (B*H*N*(2 + d)*4 bytes: D, the statistics and an fp32 dq
+ * accumulator), grown on demand like the decode workspace.  Accumulation is in
+ * fp32; dq sums the contributions of the key blocks with fp32 atomics, so its
+ * last bits may differ between runs.
+ */
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+           int causal, float scale, fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- the forward pass over B sequences of different lengths
  * packed back to back (the variable-length batches of the page "Flash
  * Attention 是什么", section 典型应用场景).

@@ -1,0 +1,94 @@
+"""GPU parity of the backward pass (fa_bwd) against the fp64 oracle's
+gradients, through the C ABI.  The oracle's gradients are pinned by finite
+differences of the forward definition (test_oracle_pins.py)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import attn_fwd_04_b200 as fa
+import oracle
+from attn_fwd_04_b200 import workloads as W
+from helpers import assert_grad_close, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _bwd_gpu(q, k, v, g, causal, scale):
+    qc, kc, vc, gc = q.cuda(), k.cuda(), v.cuda(), g.cuda()
+    o, lse = fa.fa_fwd(qc, kc, vc, causal, scale)
+    dq = torch.full_like(qc, float("nan"))
+    dk = torch.full_like(qc, float("nan"))
+    dv = torch.full_like(qc, float("nan"))
+    fa.fa_bwd(qc, kc, vc, o, lse, gc, causal, scale, dq=dq, dk=dk, dv=dv)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return dq, dk, dv
+
+
+def _grad_out(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g).to(torch.bfloat16)
+
+
+SHAPES = [(1, 1, 128, 64), (1, 2, 127, 128), (2, 2, 300, 64), (1, 1, 1, 128), (1, 2, 1000, 128),
+          (1, 1, 129, 64)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_full_compare(shape, causal):
+    B, H, N, d = shape
+    q, k, v = W.custom_fwd_inputs(B, H, N, d, seed=700 + N + d)
+    g = _grad_out((B, H, N, d), 701 + N)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv = _bwd_gpu(q, k, v, g, causal, scale)
+    rq, rk, rv = oracle.attention_bwd(q, k, v, g, causal, scale)
+    assert_grad_close(to64(dv), rv, f"dv {shape}")
+    assert_grad_close(to64(dk), rk, f"dk {shape}")
+    assert_grad_close(to64(dq), rq, f"dq {shape}")
+
+
+def test_bwd_4k_two_heads():
+    """Several 128-key blocks per head and many query tiles per block."""
+    B, H, N, d = 1, 2, 4096, 128
+    q, k, v = W.custom_fwd_inputs(B, H, N, d, seed=710)
+    g = _grad_out((B, H, N, d), 711)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv = _bwd_gpu(q, k, v, g, True, scale)
+    rq, rk, rv = oracle.attention_bwd(q, k, v, g, True, scale)
+    assert_grad_close(to64(dv), rv, "dv 4k")
+    assert_grad_close(to64(dk), rk, "dk 4k")
+    assert_grad_close(to64(dq), rq, "dq 4k")
+
+
+def test_bwd_linear_in_dout():
+    """dk and dv are linear in the output gradient and scaling by 2 is exact
+    in every step, so bwd(2 g) = 2 bwd(g) bit for bit (dq is summed with
+    atomics in a varying order and is compared within the tolerance)."""
+    q, k, v = W.custom_fwd_inputs(1, 2, 513, 64, seed=712)
+    g = _grad_out((1, 2, 513, 64), 713)
+    a = _bwd_gpu(q, k, v, g, True, 0.2)
+    b = _bwd_gpu(q, k, v, (g.float() * 2).to(torch.bfloat16), True, 0.2)
+    for x, y in zip(a[1:], b[1:]):
+        assert torch.equal((x.float() * 2).to(torch.bfloat16), y)
+    assert_grad_close(to64(b[0]), 2 * to64(a[0]), "dq linearity")
+
+
+def test_bwd_long_prefill_runs_finite():
+    w = W.LONG_PREFILL
+    q, k, v = W.fwd_inputs(w, device="cuda")
+    scale = 1 / math.sqrt(w.d)
+    o, lse = fa.fa_fwd(q, k, v, True, scale)
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(714),
+                    device="cuda").to(torch.bfloat16)
+    dq, dk, dv = fa.fa_bwd(q, k, v, o, lse, g, True, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    # under the causal mask dq rows < 512 depend only on positions < 512, so
+    # they can be checked against the oracle on the first 512 positions of a
+    # head (dk, dv of those keys depend on every later row)
+    qh, kh, vh, gh = (t[0, 0, :512].cpu()[None, None] for t in (q, k, v, g))
+    rq, _, _ = oracle.attention_bwd(qh, kh, vh, gh, True, scale)
+    assert_grad_close(to64(dq[0, 0, :512].cpu())[None, None], rq, "dq rows < 512")
