@@ -101,6 +101,19 @@ int make_map(CUtensorMap* map, const void* base, const cuuint64_t dims[3],
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// fp32 tensor map over `dims` with 128-byte swizzle (box inner extent 32
+// floats = 128 bytes); used as the destination of bulk reduce-adds.
+int make_map_f32(CUtensorMap* map, const void* base, const cuuint64_t dims[3],
+                 const cuuint64_t strides[2], const cuuint32_t box[3]) {
+    if (get_encode_fn() != FA_OK) return FA_ERR_CUDA;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // Grow-only per-device workspace, allocated on the caller's stream.
 int ensure_workspace(DeviceState* s, size_t bytes, cudaStream_t stream, void** out) {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -237,8 +250,18 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     void* ws = nullptr;
     if ((rc = ensure_workspace(s, fa::bwd_workspace_bytes(B, H, N, d), st, &ws)) != FA_OK)
         return rc;
-    return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, B, H, N, d, causal ? 1 : 0,
-                          scale, ws, s->err, s->num_sms, st);
+    // the fp32 dQ accumulator [B*H, N, d] in the workspace, reduced into by TMA
+    CUtensorMap tdq;
+    const cuuint64_t adims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                 static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t astrides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                    static_cast<cuuint64_t>(N) * d * 4};
+    const cuuint32_t abox[3] = {32, 128, 1};
+    if ((rc = make_map_f32(&tdq, static_cast<uint8_t*>(ws) + fa::bwd_dq_acc_offset(B, H, N), adims,
+                           astrides, abox)) != FA_OK)
+        return rc;
+    return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, tdq, B, H, N, d,
+                          causal ? 1 : 0, scale, ws, s->err, s->num_sms, st);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

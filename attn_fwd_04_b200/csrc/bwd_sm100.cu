@@ -53,6 +53,9 @@ struct alignas(1024) BwdSmem {
     uint8_t q[2][kBT * D * 2];
     // dO_i (128 x D), then dS_i (128 x 128) once dO_i is consumed
     uint8_t dout[2][kBT * kBT * 2];
+    // one 128-row x 32-column fp32 slice of dQ_i on its way to the
+    // accumulator (128-byte swizzle, as the reduce's tensor map reads it)
+    float dq_stage[kBT * 32];
     float lse2[2][kBT];            // log2-domain statistics of the tile's rows
     float dsum[2][kBT];            // D of the tile's rows
     uint64_t kv_full;
@@ -147,7 +150,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tdq, const BwdParams p) {
     // ---- work unit: (sequence/head, 128-key block), longest first within
     // groups of kBwdHeadGroup heads (under a causal mask key block 0 meets
     // every query tile)
@@ -284,15 +287,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            kk > 0 ? 1u : 0u);
             };
             const uint32_t k_lo = lo(sm.k), v_lo = lo(sm.v);
-            bool ok = mbar_wait(&sm.kv_full, 0, err, FA_DEVERR_TIMEOUT, abort);
+            // S^T of the next tile is issued as soon as dP^T of this one is:
+            // the tensor pipe computes it while warpgroup 0 forms dS^T (the
+            // columns it overwrites held P^T, read by dV just before)
+            bool ok = mbar_wait(&sm.kv_full, 0, err, FA_DEVERR_TIMEOUT, abort) &&
+                      mbar_wait(&sm.in_full[0], 0, err, FA_DEVERR_TIMEOUT, abort);
+            if (ok) {
+                tc_fence_after();
+                issue_kk(kColS, k_lo, lo(sm.q[0]));  // S^T = K Q_0^T
+                tc_commit(&sm.s_full);
+            }
             for (int t = 0; ok && t < nt; ++t) {
                 const int s = t & 1;
                 const uint32_t ph = t & 1;
-                if (!mbar_wait(&sm.in_full[s], (t >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) break;
-                tc_fence_after();
                 const uint32_t q_lo = lo(sm.q[s]), do_lo = lo(sm.dout[s]);
-                issue_kk(kColS, k_lo, q_lo);  // S^T = K Q_i^T
-                tc_commit(&sm.s_full);
                 if (!mbar_wait(&sm.p_full, ph, err, FA_DEVERR_TIMEOUT, abort)) break;
                 tc_fence_after();
                 issue_tm(kColDV, kColS, do_lo, t > 0);  // dV += P^T dO_i
@@ -301,6 +309,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_fence_after();
                 issue_kk(kColDP, v_lo, do_lo);  // dP^T = V dO_i^T
                 tc_commit(&sm.dp_full);
+                if (t + 1 < nt) {
+                    const int s1 = (t + 1) & 1;
+                    if (!mbar_wait(&sm.in_full[s1], ((t + 1) >> 1) & 1, err, FA_DEVERR_TIMEOUT,
+                                   abort))
+                        break;
+                    tc_fence_after();
+                    issue_kk(kColS, k_lo, lo(sm.q[s1]));  // S^T of the next tile
+                    tc_commit(&sm.s_full);
+                }
                 if (!mbar_wait(&sm.ds_full, ph, err, FA_DEVERR_TIMEOUT, abort)) break;
                 tc_fence_after();
                 issue_tm(kColDK, kColDP, q_lo, t > 0);  // dK += dS^T Q_i
@@ -404,33 +421,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
         for (int t = 0; t < nt; ++t) {
-            if (!bwd_warp_wait(&sm.dq_full, t & 1, err, abort)) {
+            // the four warps leave together (they share named barriers below)
+            if (!bar_and_named(2, kBT, mbar_wait(&sm.dq_full, t & 1, err, FA_DEVERR_TIMEOUT,
+                                                 abort))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int qrow = (i_first + t) * kBT + r;  // TMEM lane == query row here
-            float* dst = p.dq_acc + (static_cast<int64_t>(bh) * p.N + qrow) * D;
+            // dQ_i (TMEM lane == query row) in slices of 32 columns: each row
+            // to the swizzled staging tile, then one TMA reduce-add of the
+            // 128 x 32 slice into the accumulator (rows past N are clipped)
+            const int q0 = (i_first + t) * kBT;
+            uint8_t* stage = reinterpret_cast<uint8_t*>(sm.dq_stage);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t z[32];
                 tmem_ld32(tmem + lane_off + kColDP + c * 32, z);
                 tmem_wait_ld();
-                if (qrow < p.N) {
+                if (c == D / 32 - 1) {  // the dQ columns are free for the next dP^T
+                    tc_fence_before();
+                    mbar_arrive(&sm.dq_free);
+                }
+                bar_sync_named(1, kBT);  // the previous slice's reduce has read the tile
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(
-                                         dst + c * 32 + e),
-                                     "f"(__uint_as_float(z[e]) * p.scale),
-                                     "f"(__uint_as_float(z[e + 1]) * p.scale),
-                                     "f"(__uint_as_float(z[e + 2]) * p.scale),
-                                     "f"(__uint_as_float(z[e + 3]) * p.scale)
-                                     : "memory");
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4*>(stage + r * 128 + ((j ^ (r & 7)) * 16)) =
+                        make_float4(__uint_as_float(z[4 * j]) * p.scale,
+                                    __uint_as_float(z[4 * j + 1]) * p.scale,
+                                    __uint_as_float(z[4 * j + 2]) * p.scale,
+                                    __uint_as_float(z[4 * j + 3]) * p.scale);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                bar_sync_named(1, kBT);  // every row is in the tile
+                if (r == 0) {
+                    tma_reduce_add_3d(&tdq, stage, c * 32, q0, bh);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&sm.dq_free);
         }
+        if (r == 0) bulk_wait_group0();  // the reductions have landed
         if (ok) {
             // every MMA has completed (the last dq_full follows the last one);
             // the whole warp loads (tcgen05.ld is warp-wide), rows past N are
@@ -476,8 +505,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 template <int D>
 int launch_bwd_impl(const void* o, const void* dout, const float* lse, float* lse2, float* dsum,
                     float* dq_acc, void* dq, const CUtensorMap& tq, const CUtensorMap& tk,
-                    const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int num_sms,
-                    cudaStream_t stream) {
+                    const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
+                    const BwdParams& p, int num_sms, cudaStream_t stream) {
     const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.N;
     fa_bwd_prep_kernel<D><<<num_sms * 8, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
@@ -489,7 +518,8 @@ int launch_bwd_impl(const void* o, const void* dout, const float* lse, float* ls
         return FA_ERR_CUDA;
     const long long ctas = static_cast<long long>((p.N + kBT - 1) / kBT) * p.B * p.H;
     if (ctas > 0x7fffffffLL) return FA_ERR_SHAPE;
-    kern<<<dim3(static_cast<unsigned>(ctas)), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+    kern<<<dim3(static_cast<unsigned>(ctas)), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq,
+                                                                           p);
     fa_bwd_dq_kernel<D><<<num_sms * 8, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
                                                           rows * D / 8);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -497,22 +527,25 @@ int launch_bwd_impl(const void* o, const void* dout, const float* lse, float* ls
 
 }  // namespace
 
-size_t bwd_workspace_bytes(int B, int H, int N, int d) {
+size_t bwd_dq_acc_offset(int B, int H, int N) {
     const size_t rows = static_cast<size_t>(B) * H * N;
-    const size_t stats = (2 * rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
-    return stats + rows * d * sizeof(float);
+    return (2 * rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+size_t bwd_workspace_bytes(int B, int H, int N, int d) {
+    return bwd_dq_acc_offset(B, H, N) + static_cast<size_t>(B) * H * N * d * sizeof(float);
 }
 
 int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& tdo, int B, int H, int N, int d, int causal, float scale,
-               void* workspace, unsigned int* err, int num_sms, cudaStream_t stream) {
+               const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int N, int d,
+               int causal, float scale, void* workspace, unsigned int* err, int num_sms,
+               cudaStream_t stream) {
     const size_t rows = static_cast<size_t>(B) * H * N;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* lse2 = reinterpret_cast<float*>(ws);
     float* dsum = lse2 + rows;
-    float* dq_acc = reinterpret_cast<float*>(
-        ws + ((2 * rows * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+    float* dq_acc = reinterpret_cast<float*>(ws + bwd_dq_acc_offset(B, H, N));
     BwdParams p{};
     p.lse2 = lse2;
     p.dsum = dsum;
@@ -527,11 +560,11 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = err;
     if (d == 128)
-        return launch_bwd_impl<128>(o, dout, lse, lse2, dsum, dq_acc, dq, tq, tk, tv, tdo, p,
-                                    num_sms, stream);
+        return launch_bwd_impl<128>(o, dout, lse, lse2, dsum, dq_acc, dq, tq, tk, tv, tdo, tdq,
+                                    p, num_sms, stream);
     if (d == 64)
-        return launch_bwd_impl<64>(o, dout, lse, lse2, dsum, dq_acc, dq, tq, tk, tv, tdo, p,
-                                   num_sms, stream);
+        return launch_bwd_impl<64>(o, dout, lse, lse2, dsum, dq_acc, dq, tq, tk, tv, tdo, tdq,
+                                   p, num_sms, stream);
     return FA_ERR_UNSUPPORTED;
 }
 

@@ -41,10 +41,12 @@ int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
 
 // ---- backward ------------------------------------------------------------
 size_t bwd_workspace_bytes(int B, int H, int N, int d);
+size_t bwd_dq_acc_offset(int B, int H, int N);  // fp32 dQ accumulator, in the workspace
 int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& tdo, int B, int H, int N, int d, int causal, float scale,
-               void* workspace, unsigned int* err, int num_sms, cudaStream_t stream);
+               const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int N, int d,
+               int causal, float scale, void* workspace, unsigned int* err, int num_sms,
+               cudaStream_t stream);
 
 // ---- paged decode ----------------------------------------------------------
 // Number of pages a split covers at least (a split is one CTA work unit) and
