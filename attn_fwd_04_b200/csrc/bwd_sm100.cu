@@ -433,23 +433,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // 128 x 32 slice into the accumulator (rows past N are clipped)
             const int q0 = (i_first + t) * kBT;
             uint8_t* stage = reinterpret_cast<uint8_t*>(sm.dq_stage);
+            // all of dQ_i into registers first, so that its TMEM columns are
+            // released to the next dP^T before the reductions
+            uint32_t z[D / 32][32];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + kColDP + c * 32, z[c]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.dq_free);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t z[32];
-                tmem_ld32(tmem + lane_off + kColDP + c * 32, z);
-                tmem_wait_ld();
-                if (c == D / 32 - 1) {  // the dQ columns are free for the next dP^T
-                    tc_fence_before();
-                    mbar_arrive(&sm.dq_free);
-                }
                 bar_sync_named(1, kBT);  // the previous slice's reduce has read the tile
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<float4*>(stage + r * 128 + ((j ^ (r & 7)) * 16)) =
-                        make_float4(__uint_as_float(z[4 * j]) * p.scale,
-                                    __uint_as_float(z[4 * j + 1]) * p.scale,
-                                    __uint_as_float(z[4 * j + 2]) * p.scale,
-                                    __uint_as_float(z[4 * j + 3]) * p.scale);
+                        make_float4(__uint_as_float(z[c][4 * j]) * p.scale,
+                                    __uint_as_float(z[c][4 * j + 1]) * p.scale,
+                                    __uint_as_float(z[c][4 * j + 2]) * p.scale,
+                                    __uint_as_float(z[c][4 * j + 3]) * p.scale);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 bar_sync_named(1, kBT);  // every row is in the tile
                 if (r == 0) {
