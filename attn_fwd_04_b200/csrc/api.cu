@@ -151,7 +151,8 @@ int device_error_word(unsigned int** err, int* num_sms) {
 namespace {
 
 // Fixed-length forward pass with H query heads and H_kv K/V heads; with
-// rope_cos / rope_sin (tables of max_pos rows) Q and K are rotated first.
+// rope_cos / rope_sin (tables of max_pos rows) Q and K are rotated first: K
+// once per position into the workspace, Q tile by tile inside the kernel.
 int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
               int H_kv, int N, int d, int causal, float scale, fa_stream_t stream,
               const float* rope_cos = nullptr, const float* rope_sin = nullptr,
@@ -171,6 +172,18 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     DeviceState* s = nullptr;
     int rc = lookup_device(&s);
     if (rc != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const void* k_use = k;
+    if (rope_cos) {
+        void* ws = nullptr;
+        const size_t kbytes = static_cast<size_t>(B) * H_kv * N * d * 2;
+        if ((rc = ensure_workspace(s, kbytes, st, &ws)) != FA_OK) return rc;
+        if ((rc = fa::launch_rope_rows(k, ws, rope_cos, rope_sin,
+                                       static_cast<int64_t>(B) * H_kv, N, d, s->num_sms, st)) !=
+            FA_OK)
+            return rc;
+        k_use = ws;
+    }
     CUtensorMap tq, tk, tv;
     const cuuint64_t dims_q[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                   static_cast<cuuint64_t>(B) * H};
@@ -180,7 +193,7 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
                                    static_cast<cuuint64_t>(N) * d * 2};
     const cuuint32_t box[3] = {64, 128, 1};
     if ((rc = make_map(&tq, q, dims_q, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tk, k, dims_kv, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k_use, dims_kv, strides, box)) != FA_OK) return rc;
     if ((rc = make_map(&tv, v, dims_kv, strides, box)) != FA_OK) return rc;
     fa::FwdParams p{};
     p.o = o;
@@ -196,7 +209,7 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
-    return fa::launch_fwd(p, tq, tk, tv, d, fa::kFixed, reinterpret_cast<cudaStream_t>(stream));
+    return fa::launch_fwd(p, tq, tk, tv, d, fa::kFixed, st);
 }
 
 }  // namespace

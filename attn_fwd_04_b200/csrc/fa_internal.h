@@ -34,6 +34,9 @@ struct FwdParams {
     unsigned int* err;   // device error word
 };
 
+// rotary embedding of x [rows, N, d] into y (positions 0..N-1)
+int launch_rope_rows(const void* x, void* y, const float* cos_t, const float* sin_t, int64_t rows,
+                     int N, int d, int num_sms, cudaStream_t stream);
 // forward modes
 constexpr int kFixed = 0, kVarlen = 1, kPaged = 2;
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,

@@ -73,7 +73,6 @@ struct alignas(1024) FwdSmem {
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
     uint64_t q_rot;      // RoPE: both Q tiles rotated
-    uint64_t k_rot[2];   // RoPE: K_j rotated (K tiles use ring slots 0 and 2: index j % 2)
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -224,8 +223,9 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const fl
 // kPaged (packed queries; keys and values read through the page table from a
 // pool of 256-token pages, the queries being the last positions of each
 // cached sequence).
-// ROPE (fixed-length only): Q and K are rotated in shared memory by the
-// epilogue warpgroup (idle until the last step) before their score products.
+// ROPE (fixed-length only): the Q tiles are rotated in shared memory by the
+// epilogue warpgroup (idle until the last step) before their first score
+// product; K arrives rotated (fa_rope_rows_kernel, once per position).
 template <int D, int MODE, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -318,8 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.vfix, 1);
         mbar_init(&sm.q_rot, BM);
-        mbar_init(&sm.k_rot[0], BM);
-        mbar_init(&sm.k_rot[1], BM);
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
@@ -456,13 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                            idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
             };
             bool ok = true;
-            // K_j ready for its score products: landed, and rotated under ROPE
             auto wait_k = [&](int j) {
-                if constexpr (ROPE)
-                    return mbar_wait(&sm.k_rot[j & 1], (j >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort);
-                else
-                    return mbar_wait(&sm.kv_full[ring_slot(j, 0)], ring_phase(j, 0), err,
-                                     FA_DEVERR_TIMEOUT, abort);
+                return mbar_wait(&sm.kv_full[ring_slot(j, 0)], ring_phase(j, 0), err,
+                                 FA_DEVERR_TIMEOUT, abort);
             };
             if constexpr (ROPE) {
                 ok = mbar_wait(&sm.q_rot, 0, err, FA_DEVERR_TIMEOUT, abort);
@@ -609,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
         if constexpr (ROPE) {
-            // rotate both Q tiles, then every K tile as it lands; rows past
-            // the sequence end are TMA zero fill and stay zero
+            // rotate both Q tiles; rows past the sequence end are TMA zero
+            // fill and stay zero
             for (int t = 0; ok && t < 2; ++t) {
                 if (n_t[t] == 0) continue;
                 if (!warp_wait(&sm.q_full[t], 0, err, abort)) {
@@ -622,16 +616,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             if (ok) mbar_arrive(&sm.q_rot);
-            for (int j = 0; ok && j < n; ++j) {
-                if (!warp_wait(&sm.kv_full[ring_slot(j, 0)], ring_phase(j, 0), err, abort)) {
-                    ok = false;
-                    break;
-                }
-                const int pos = j * BN + r;
-                if (pos < len) rope_row<D>(sm.kv[ring_slot(j, 0)], r, pos, p.rope_cos, p.rope_sin);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive(&sm.k_rot[j & 1]);
-            }
         }
         // epilogue: O / l -> bf16, log-sum-exp
         for (int t = 0; ok && t < 2; ++t) {
@@ -690,6 +674,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 12) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Rotary embedding of whole rows in device memory (used for K, whose tiles
+// every query block of a head would otherwise rotate again): x [rows, N, D]
+// -> y, row n at position n, the same fp32 formula and bf16 rounding as
+// rope_row.  One thread per (row, 8 pairs).
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_rope_rows_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                        const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+                        int64_t rows, int N) {
+    constexpr int HALF = D / 2, G = HALF / 8;  // 8-pair groups per row
+    const int64_t total = rows * N * G;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < total;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int g = static_cast<int>(w % G);
+        const int64_t rn = w / G;  // flat (row, position)
+        const int pos = static_cast<int>(rn % N);
+        const __nv_bfloat16* src = x + rn * D;
+        __nv_bfloat16* dst = y + rn * D;
+        const uint4 ua = *reinterpret_cast<const uint4*>(src + 8 * g);
+        const uint4 ub = *reinterpret_cast<const uint4*>(src + 8 * g + HALF);
+        const float* ct = cos_t + static_cast<int64_t>(pos) * HALF + 8 * g;
+        const float* st = sin_t + static_cast<int64_t>(pos) * HALF + 8 * g;
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(ct));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(ct + 4));
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(st));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(st + 4));
+        const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a[2] = {__uint_as_float(wa[e] << 16), __uint_as_float(wa[e] & 0xffff0000u)};
+            const float b[2] = {__uint_as_float(wb[e] << 16), __uint_as_float(wb[e] & 0xffff0000u)};
+            float ra[2], rb[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const float cc = cs[2 * e + k], ss = sn[2 * e + k];
+                const float bs = b[k] * ss, as = a[k] * ss;
+                ra[k] = fmaf(a[k], cc, -bs);
+                rb[k] = fmaf(b[k], cc, as);
+            }
+            oa[e] = pack_bf16x2(ra[0], ra[1]);
+            ob[e] = pack_bf16x2(rb[0], rb[1]);
+        }
+        *reinterpret_cast<uint4*>(dst + 8 * g) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *reinterpret_cast<uint4*>(dst + 8 * g + HALF) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+}
+
 template <int D, int MODE, bool ROPE = false>
 int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, cudaStream_t stream) {
@@ -710,6 +744,21 @@ int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk
 }
 
 }  // namespace
+
+int launch_rope_rows(const void* x, void* y, const float* cos_t, const float* sin_t, int64_t rows,
+                     int N, int d, int num_sms, cudaStream_t stream) {
+    if (d == 128)
+        fa_rope_rows_kernel<128><<<num_sms * 8, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), cos_t, sin_t,
+            rows, N);
+    else if (d == 64)
+        fa_rope_rows_kernel<64><<<num_sms * 8, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), cos_t, sin_t,
+            rows, N);
+    else
+        return FA_ERR_UNSUPPORTED;
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, int d, int mode, cudaStream_t stream) {

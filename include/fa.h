@@ -110,8 +110,12 @@ FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, floa
  * fa_fwd_rope -- fa_fwd_gqa with rotary position embedding fused into the
  * kernel: the page "“Flash”不是那个被时代淘汰的插件" (0539edu.com) describes a
  * kernel that fuses RoPE (section 2) from a precomputed sin/cos lookup table
- * (section 3).  q and k are passed unrotated; each Q and K tile is rotated in
- * on-chip memory after it is loaded and before its score product.
+ * (section 3).  q and k are passed unrotated.  The page applies RoPE with the
+ * QKV projection; here K, which every query block of a head reads, is rotated
+ * once per position into the library's per-GPU workspace (B*H_kv*N*d*2 bytes,
+ * grown on demand like the decode workspace; calls on different streams of
+ * one GPU must not overlap), and each Q tile is rotated in on-chip memory
+ * after it is loaded, before its first score product.
  *   rope_cos, rope_sin : DEVICE fp32 [max_pos, d/2], row-major; entry (p, i)
  *                        is cos / sin of the angle for position p and pair i
  *                        (normally p * base^(-2i/d)); max_pos >= N
