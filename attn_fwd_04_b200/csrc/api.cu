@@ -373,27 +373,44 @@ int fa_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
 }  // extern "C"
 
 namespace {
+// num_pages = 0x7fffffff: the pool size is unknown (fa_decode_paged's
+// signature has none), page indices are not bounded.
 int decode_impl(const void* q, const void* k_pages, const void* v_pages,
                 const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                int H_kv, int d, int page_size, fa_stream_t stream) {
+                int H_kv, int num_pages, int d, int page_size, fa_stream_t stream) {
     if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !o) return FA_ERR_NULL;
-    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0) return FA_ERR_SHAPE;
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || num_pages < 1) return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (page_size != 256) return FA_ERR_UNSUPPORTED;
     if (!fa::decode_group_supported(H, H_kv)) return FA_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(B) * H * fa::kDecodeMaxSplits > 0x7fffffff) return FA_ERR_SHAPE;
     if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
         return FA_ERR_ALIGN;
+    const bool grouped = H != H_kv;
+    if (grouped && static_cast<int64_t>(num_pages) * H_kv > 0x7fffffff) return FA_ERR_SHAPE;
     DeviceState* s = nullptr;
     int rc = lookup_device(&s);
     if (rc != FA_OK) return rc;
+    CUtensorMap tk, tv;
+    if (grouped) {
+        // the page pool [P, H_kv, 256, d] as (d, slot, page * H_kv + head)
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(page_size),
+                                    static_cast<cuuint64_t>(num_pages) * H_kv};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                       static_cast<cuuint64_t>(page_size) * d * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        if ((rc = make_map(&tk, k_pages, dims, strides, box)) != FA_OK) return rc;
+        if ((rc = make_map(&tv, v_pages, dims, strides, box)) != FA_OK) return rc;
+    }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     void* ws = nullptr;
     if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits), st,
                                &ws)) != FA_OK)
         return rc;
-    return fa::launch_decode(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H_kv, d,
-                             page_size, fa::kDecodeMaxSplits, ws, s->err, s->num_sms, st);
+    return fa::launch_decode(q, k_pages, v_pages, grouped ? &tk : nullptr,
+                             grouped ? &tv : nullptr, page_table, seq_lens, o, B, H, H_kv,
+                             num_pages, d, page_size, fa::kDecodeMaxSplits, ws, s->err,
+                             s->num_sms, st);
 }
 }  // namespace
 
@@ -402,15 +419,16 @@ extern "C" {
 int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                     const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
                     int d, int page_size, fa_stream_t stream) {
-    return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H, d, page_size,
-                       stream);
+    return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H, 0x7fffffff, d,
+                       page_size, stream);
 }
 
 int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v_pages,
                         const int32_t* page_table, const int32_t* seq_lens, void* o, int B,
-                        int H, int H_kv, int d, int page_size, fa_stream_t stream) {
-    return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H_kv, d, page_size,
-                       stream);
+                        int H, int H_kv, int num_pages, int d, int page_size,
+                        fa_stream_t stream) {
+    return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H_kv, num_pages, d,
+                       page_size, stream);
 }
 
 int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t* seq_lens,

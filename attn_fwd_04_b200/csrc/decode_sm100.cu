@@ -151,37 +151,21 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
     }
 }
 
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 constexpr int kDecTok = 64;           // tokens per ring stage (a quarter of a page)
 constexpr int kDecConsumerWarps = 8;
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;  // + one producer warp
 
-// GH: query heads served by each K/V head (1 = multi-head attention).  A
-// unit's K/V chunks are staged once in shared memory and every query head of
-// the group is evaluated against them: each consumer warp carries HW =
-// min(GH, 4) query heads, and the consumer warps form GH / HW teams, each
-// team covering all tokens of a chunk for its heads.
-template <int D, int GH>
+// Multi-head decode (one query head per K/V head): a token row is spread
+// over LPT lanes (16 bytes each), G token groups per CTA.
+template <int D>
 struct DecSmem {
     static constexpr int LPT = D / 8;                              // lanes per token
     static constexpr int G = kDecConsumerWarps * 32 / LPT;         // token groups
     static constexpr int STAGES = 6;                               // ring depth
-    static constexpr int HW = GH < 4 ? GH : 4;                     // query heads per warp
-    static constexpr int TEAM = kDecConsumerWarps / (GH / HW);     // warps per team
-    // combine slots per head: one per token group (GH = 1), or one per warp
-    // of the head's team once the groups of a warp are merged with shuffles
-    static constexpr int C = GH == 1 ? G : TEAM;
     alignas(128) uint8_t k[STAGES][kDecTok * D * 2];
     alignas(128) uint8_t v[STAGES][kDecTok * D * 2];
-    float cm[2][GH][C], cl[2][GH][C];  // per-slot partial state, by unit parity
-    float co[2][GH][C][D];
+    float cm[2][G], cl[2][G];  // per-group partial state, by unit parity
+    float co[2][G][D];
     uint64_t full[STAGES], empty[STAGES], cmb[2];
     int abort;
 };
@@ -226,19 +210,20 @@ __device__ __forceinline__ UnitShape unit_shape(int u, UnitCursor& cur,
     return us;
 }
 
-// H query heads, Hk = H / GH K/V heads.  Partial outputs are indexed by
-// (unit, query head within the group): u * GH + gi.
-template <int D, int GH>
+// One unit per (split, head); the partial output of unit u is row u.  A page
+// index outside [0, num_pages) is reported and page 0 is read in its place
+// (nothing outside the pool is touched; that sequence's output is garbage).
+template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_split_kernel(const __nv_bfloat16* __restrict__ q,
                            const __nv_bfloat16* __restrict__ k_pages,
                            const __nv_bfloat16* __restrict__ v_pages,
                            const int32_t* __restrict__ page_table,
-                           const int32_t* __restrict__ seq_lens, int B, int H, int Hk,
+                           const int32_t* __restrict__ seq_lens, int B, int H, int num_pages,
                            int page_size, int max_splits, const int32_t* __restrict__ page_off,
                            const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                            float* __restrict__ part_o, float scale_log2, unsigned int* err) {
-    using Sm = DecSmem<D, GH>;
+    using Sm = DecSmem<D>;
     constexpr int LPT = Sm::LPT, G = Sm::G;
     constexpr int kDecStages = Sm::STAGES;
     constexpr int GPW = 32 / LPT;  // token groups per warp
@@ -268,20 +253,26 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         int g = 0;  // ring uses so far
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
-            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk,
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
                                             page_size, max_splits);
             const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
             constexpr int per_page = 256 / kDecTok;  // page_size is 256
             int page = 0;
             for (int c = 0; c < nchunks; ++c, ++g) {
-                if (c % per_page == 0) page = __ldg(page_table + us.pt_base + c / per_page);
+                if (c % per_page == 0) {
+                    page = __ldg(page_table + us.pt_base + c / per_page);
+                    if (page < 0 || page >= num_pages) {
+                        if (lane == 0) record_error(err, FA_DEVERR_BAD_INPUT);
+                        page = 0;
+                    }
+                }
                 const int slot = g % kDecStages;
                 if (lane == 0) {
                     if (!mbar_wait(&sm.empty[slot], ((g / kDecStages) & 1) ^ 1, err,
                                    FA_DEVERR_TIMEOUT, abort)) {
                         ok = false;
                     } else {
-                        const int64_t row = (static_cast<int64_t>(page) * Hk + us.h) * page_size +
+                        const int64_t row = (static_cast<int64_t>(page) * H + us.h) * page_size +
                                             (c % per_page) * kDecTok;
                         mbar_arrive_expect_tx(&sm.full[slot], 2 * kChunkBytes);
                         bulk_load(sm.k[slot], k_pages + row * D, kChunkBytes, &sm.full[slot]);
@@ -306,9 +297,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const unsigned gmask = (LPT == 32) ? 0xffffffffu : (((1u << LPT) - 1u) << (sub * LPT));
         int g = 0, k = 0;  // ring uses, units done
         bool ok = true;
-        if constexpr (GH == 1) {
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
-            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk,
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
                                             page_size, max_splits);
             float qf[8];
             {
@@ -377,11 +367,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             // combine the G groups of this unit (buffers double-buffered by unit parity)
             const int par = k & 1;
             if (gl == 0) {
-                sm.cm[par][0][grp] = m;
-                sm.cl[par][0][grp] = l;
+                sm.cm[par][grp] = m;
+                sm.cl[par][grp] = l;
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sm.co[par][0][grp][gl * 8 + i] = acc[i];
+            for (int i = 0; i < 8; ++i) sm.co[par][grp][gl * 8 + i] = acc[i];
             mbar_arrive(&sm.cmb[par]);
             if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) {
                 ok = false;
@@ -390,200 +380,295 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             if (threadIdx.x < D) {
                 float M = -INFINITY;
 #pragma unroll
-                for (int gi = 0; gi < G; ++gi) M = fmaxf(M, sm.cm[par][0][gi]);
+                for (int gi = 0; gi < G; ++gi) M = fmaxf(M, sm.cm[par][gi]);
                 float L = 0.f, o = 0.f;
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
-                    const float w = (sm.cm[par][0][gi] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][0][gi] - M);
-                    L += w * sm.cl[par][0][gi];
-                    o += w * sm.co[par][0][gi][threadIdx.x];
+                    const float w = (sm.cm[par][gi] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][gi] - M);
+                    L += w * sm.cl[par][gi];
+                    o += w * sm.co[par][gi][threadIdx.x];
                 }
                 part_o[static_cast<int64_t>(u) * D + threadIdx.x] = o / L;
                 if (threadIdx.x == 0) part_lse[u] = M + __log2f(L);
             }
         }
-        } else {
-        // ---- grouped query heads: GH queries against each staged chunk ----
-        // Warp w serves query heads HW * (w / TEAM) + {0 .. HW-1} of the
-        // unit's group.  A token row is spread over LG lanes holding NP packed
-        // fp32 pairs (8 dims, one 16-byte shared-memory load) each, as in the
-        // single-head path; products use the paired fp32 FMA.
-        constexpr int HW = Sm::HW;                      // query heads per warp
-        constexpr int TEAM = Sm::TEAM;                  // warps per team
-        constexpr int LG = D / 8;                       // lanes per token
-        constexpr int NP = D / LG / 2;                  // fp32 pairs per lane
-        constexpr int GW = 32 / LG;                     // token groups per warp
-        constexpr int GG = TEAM * GW;                   // token groups per team
-        constexpr int TPG = kDecTok / GG;               // tokens per group per chunk
-        static_assert(GH % HW == 0 && TPG >= 1 && kDecTok % GG == 0, "chunk split");
-        const int team = warp / TEAM, wt = warp - team * TEAM;
-        const int gsub = lane / LG, glane = lane % LG;
-        const int ggrp = wt * GW + gsub;
-        const unsigned gm = (LG == 32) ? 0xffffffffu : (((1u << LG) - 1u) << (gsub * LG));
-        // bf16 pairs (low element in the low half) -> packed fp32 pairs
-        auto widen = [](const uint4* src, uint64_t (&dst)[NP]) {
-#pragma unroll
-            for (int v = 0; v < NP / 4; ++v) {
-                const uint4 u4 = src[v];
-                const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[v * 4 + i] = (static_cast<uint64_t>(w[i] & 0xffff0000u) << 32) | (w[i] << 16);
-            }
-        };
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
-            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk,
-                                            page_size, max_splits);
-            uint64_t q2[HW][NP];
-#pragma unroll
-            for (int hi = 0; hi < HW; ++hi) {
-                const uint4* src = reinterpret_cast<const uint4*>(
-                    q + (static_cast<int64_t>(us.b) * H + us.h * GH + team * HW + hi) * D +
-                    glane * 2 * NP);
-                widen(src, q2[hi]);
-                const uint64_t s2 = f2_pack(scale_log2, scale_log2);
-#pragma unroll
-                for (int i = 0; i < NP; ++i) q2[hi][i] = f2_mul(q2[hi][i], s2);
-            }
-            float m[HW], l[HW];
-            uint64_t acc[HW][NP];
-#pragma unroll
-            for (int hi = 0; hi < HW; ++hi) {
-                m[hi] = -INFINITY;
-                l[hi] = 0.f;
-#pragma unroll
-                for (int i = 0; i < NP; ++i) acc[hi][i] = 0;
-            }
-            const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
-            for (int c = 0; c < nchunks; ++c, ++g) {
-                const int slot = g % kDecStages;
-                if (!mbar_wait(&sm.full[slot], (g / kDecStages) & 1, err, FA_DEVERR_TIMEOUT,
-                               abort)) {
-                    ok = false;
-                    break;
-                }
-                float sc[HW][TPG];
-                const int base = c * kDecTok;
-#pragma unroll
-                for (int x = 0; x < TPG; ++x) {
-                    const int t = ggrp + x * GG;
-                    uint64_t k2[NP];
-                    widen(reinterpret_cast<const uint4*>(sm.k[slot] + t * D * 2 + glane * 4 * NP),
-                          k2);
-#pragma unroll
-                    for (int hi = 0; hi < HW; ++hi) {
-                        uint64_t d2 = f2_mul(q2[hi][0], k2[0]);
-#pragma unroll
-                        for (int i = 1; i < NP; ++i) d2 = f2_fma(q2[hi][i], k2[i], d2);
-                        float dot = f2_lo(d2) + f2_hi(d2);
-#pragma unroll
-                        for (int o = LG / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(gm, dot, o);
-                        sc[hi][x] = (base + t < us.ntok) ? dot : -INFINITY;
-                    }
-                }
-                float mn[HW];
-#pragma unroll
-                for (int hi = 0; hi < HW; ++hi) {
-                    float mb = sc[hi][0];
-#pragma unroll
-                    for (int x = 1; x < TPG; ++x) mb = fmaxf(mb, sc[hi][x]);
-                    mn[hi] = fmaxf(m[hi], mb);
-                    if (mn[hi] != -INFINITY && mn[hi] != m[hi]) {
-                        const float alpha = ex2_approx(m[hi] - mn[hi]);  // m = -inf -> 0
-                        l[hi] *= alpha;
-                        const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-                        for (int i = 0; i < NP; ++i) acc[hi][i] = f2_mul(acc[hi][i], a2);
-                    }
-                }
-#pragma unroll
-                for (int x = 0; x < TPG; ++x) {
-                    const int t = ggrp + x * GG;
-                    if (base + t < us.ntok) {
-                        uint64_t v2[NP];
-                        widen(reinterpret_cast<const uint4*>(sm.v[slot] + t * D * 2 +
-                                                             glane * 4 * NP),
-                              v2);
-#pragma unroll
-                        for (int hi = 0; hi < HW; ++hi) {
-                            const float pw = ex2_approx(sc[hi][x] - mn[hi]);
-                            l[hi] += pw;
-                            const uint64_t p2 = f2_pack(pw, pw);
-#pragma unroll
-                            for (int i = 0; i < NP; ++i) acc[hi][i] = f2_fma(p2, v2[i], acc[hi][i]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int hi = 0; hi < HW; ++hi)
-                    if (mn[hi] != -INFINITY) m[hi] = mn[hi];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.empty[slot]);
-            }
-            if (!ok) break;
-            // merge the token groups of this warp (their lanes glane hold the
-            // same columns) with shuffles, then the team's warps through
-            // shared memory
-            const int par = k & 1;
-#pragma unroll
-            for (int hi = 0; hi < HW; ++hi) {
-                const int hq = team * HW + hi;  // query head within the group
-                float mm = m[hi], ll = l[hi];
-#pragma unroll
-                for (int o = LG; o < 32; o <<= 1) {
-                    const float m2 = __shfl_xor_sync(0xffffffffu, mm, o);
-                    const float l2 = __shfl_xor_sync(0xffffffffu, ll, o);
-                    const float M = fmaxf(mm, m2);
-                    const float w1 = (mm == -INFINITY) ? 0.f : ex2_approx(mm - M);
-                    const float w2 = (m2 == -INFINITY) ? 0.f : ex2_approx(m2 - M);
-                    ll = ll * w1 + l2 * w2;
-                    const uint64_t w1p = f2_pack(w1, w1), w2p = f2_pack(w2, w2);
-#pragma unroll
-                    for (int i = 0; i < NP; ++i) {
-                        const float a_lo = __shfl_xor_sync(0xffffffffu, f2_lo(acc[hi][i]), o);
-                        const float a_hi = __shfl_xor_sync(0xffffffffu, f2_hi(acc[hi][i]), o);
-                        acc[hi][i] = f2_fma(acc[hi][i], w1p, f2_mul(f2_pack(a_lo, a_hi), w2p));
-                    }
-                    mm = M;
-                }
-                if (gsub == 0) {
-                    if (glane == 0) {
-                        sm.cm[par][hq][wt] = mm;
-                        sm.cl[par][hq][wt] = ll;
-                    }
-#pragma unroll
-                    for (int i = 0; i < NP; ++i) {
-                        sm.co[par][hq][wt][glane * 2 * NP + 2 * i] = f2_lo(acc[hi][i]);
-                        sm.co[par][hq][wt][glane * 2 * NP + 2 * i + 1] = f2_hi(acc[hi][i]);
-                    }
-                }
-            }
-            mbar_arrive(&sm.cmb[par]);
-            if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) {
-                ok = false;
-                break;
-            }
-            for (int idx = threadIdx.x; idx < GH * D; idx += kDecConsumerWarps * 32) {
-                const int hi = idx / D, x = idx - hi * D;
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < TEAM; ++w) M = fmaxf(M, sm.cm[par][hi][w]);
-                float L = 0.f, o = 0.f;
-#pragma unroll
-                for (int w = 0; w < TEAM; ++w) {
-                    const float wt = (sm.cm[par][hi][w] == -INFINITY) ? 0.f : ex2_approx(sm.cm[par][hi][w] - M);
-                    L += wt * sm.cl[par][hi][w];
-                    o += wt * sm.co[par][hi][w][x];
-                }
-                const int64_t pu = static_cast<int64_t>(u) * GH + hi;
-                part_o[pu * D + x] = o / L;
-                if (x == 0) part_lse[pu] = M + __log2f(L);
-            }
-        }
-        }
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Grouped query heads (GH = H / Hk in {2, 4, 8}).  A unit is (split, K/V
+// head); the GH query heads of its group are the rows of a 16-row MMA tile
+// (rows GH..15 are zero), so each staged K/V byte serves all of them and the
+// dot products run as two small matrix products per chunk on the tensor
+// cores (warp-level m16n8k16: a tcgen05 tile has at least 64 rows, 8x-32x
+// more than the group has).  K/V chunks of 64 tokens arrive by TMA in the
+// 128-byte-swizzled layout, so the ldmatrix reads of 8 token rows at one
+// column fall in 8 distinct bank groups.  Two teams of four warps take
+// alternate chunks; warp wt of a team owns tokens 16wt .. 16wt+15:
+//   S  = Q_g K^T   two 8-token n-tiles over D/16 k-steps (fp32)
+//   online softmax per query row (row = lane / 4; the 4 lanes of a quad
+//   share it), base 2 with scale * log2(e) applied to S
+//   O += P V       P from S's accumulators as the A operand, V through
+//                  ldmatrix.trans, D/8 n-tiles
+// and the 8 warps' (m, l, O) are merged per unit as in the multi-head path.
+// ---------------------------------------------------------------------------
+constexpr int kGqTok = 64;          // tokens per chunk
+constexpr int kGqWarps = 8;         // consumer warps (two teams of four)
+constexpr int kGqThreads = (kGqWarps + 1) * 32;
+constexpr int kGqSmemLimit = 232448;  // opt-in shared memory per block
+
+template <int D, int GH>
+struct GqSmem {
+    static constexpr int kTile = kGqTok * D * 2;   // one of K, V per stage
+    static constexpr int kCo = 2 * GH * kGqWarps * D * 4;
+    static constexpr int kFit = (kGqSmemLimit - 2048 - 1024 - kCo) / (2 * kTile);
+    // even: chunk g goes to team g % 2 and stage g % STAGES, so each stage
+    // belongs to one team, which then sees every phase of its barriers in
+    // order (with an odd count a team could wait on a stage two phases ahead
+    // of it, and a parity wait cannot tell those phases apart)
+    static constexpr int STAGES = (kFit < 6 ? kFit : 6) & ~1;
+    alignas(1024) uint8_t k[STAGES][kTile];
+    alignas(1024) uint8_t v[STAGES][kTile];
+    float co[2][GH][kGqWarps][D];  // per-warp partial state, by unit parity
+    float cm[2][GH][kGqWarps], cl[2][GH][kGqWarps];
+    uint64_t full[STAGES], empty[STAGES], cmb[2];
+    int abort;
+};
+
+// Byte offset of (token t, 16-byte column chunk c) in a staged tile: D/64
+// TMA boxes of 64 rows x 128 bytes, chunk index XOR (row % 8) inside a box.
+__device__ __forceinline__ uint32_t gq_swz(int t, int c) {
+    return static_cast<uint32_t>((c >> 3) * (kGqTok * 128) + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
+template <int D, int GH>
+__global__ void __launch_bounds__(kGqThreads, 1)
+    fa_decode_gqa_kernel(const __grid_constant__ CUtensorMap tk,
+                         const __grid_constant__ CUtensorMap tv,
+                         const __nv_bfloat16* __restrict__ q,
+                         const int32_t* __restrict__ page_table,
+                         const int32_t* __restrict__ seq_lens, int B, int H, int Hk,
+                         int num_pages, int max_splits, const int32_t* __restrict__ page_off,
+                         const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
+                         float* __restrict__ part_o, float scale_log2, unsigned int* err) {
+    using Sm = GqSmem<D, GH>;
+    constexpr int STAGES = Sm::STAGES;
+    constexpr int KS = D / 16;  // k-steps of S
+    constexpr int NT = D / 8;   // n-tiles of O
+    constexpr int kPage = 256;
+    static_assert(STAGES >= 2 && STAGES % 2 == 0, "ring: an even number of stages");
+    static_assert(sizeof(Sm) + 1024 <= kGqSmemLimit, "shared memory");
+    extern __shared__ uint8_t gq_smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(gq_smem_raw) + 1023) &
+                                    ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort = &sm.abort;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kGqWarps / 2);  // the four warps of the chunk's team
+        }
+        mbar_init(&sm.cmb[0], kGqWarps * 32);
+        mbar_init(&sm.cmb[1], kGqWarps * 32);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int total_units = __ldg(unit_off + B);
+    UnitCursor cur;
+    cur.next_off = (B > 1) ? __ldg(unit_off + 1) : 0x7fffffff;
+
+    if (warp == kGqWarps) {
+        // ================= producer: TMA boxes of (page, K/V head) slices =================
+        if (lane == 0) {
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+        }
+        int g = 0;  // ring uses so far
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+            const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk, kPage,
+                                            max_splits);
+            const int nchunks = (us.ntok + kGqTok - 1) / kGqTok;
+            constexpr int per_page = kPage / kGqTok;
+            int z = 0;  // (page, head) slice; -1 reads zeros
+            for (int c = 0; c < nchunks; ++c, ++g) {
+                if (c % per_page == 0) {
+                    const int page = __ldg(page_table + us.pt_base + c / per_page);
+                    if (page < 0 || page >= num_pages) {
+                        if (lane == 0) record_error(err, FA_DEVERR_BAD_INPUT);
+                        z = -1;
+                    } else {
+                        z = page * Hk + us.h;
+                    }
+                }
+                const int slot = g % STAGES;
+                if (lane == 0) {
+                    if (!mbar_wait(&sm.empty[slot], ((g / STAGES) & 1) ^ 1, err, FA_DEVERR_TIMEOUT,
+                                   abort)) {
+                        ok = false;
+                    } else {
+                        const int y = (c % per_page) * kGqTok;
+                        mbar_arrive_expect_tx(&sm.full[slot], 2 * Sm::kTile);
+#pragma unroll
+                        for (int cb = 0; cb < D / 64; ++cb) {
+                            tma_load_3d(sm.k[slot] + cb * kGqTok * 128, &tk, &sm.full[slot],
+                                        cb * 64, y, z);
+                            tma_load_3d(sm.v[slot] + cb * kGqTok * 128, &tv, &sm.full[slot],
+                                        cb * 64, y, z);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
+        }
+        // every copy this CTA started must land before it exits
+        if (lane == 0)
+            for (int i = max(0, g - STAGES); i < g; ++i)
+                mbar_wait(&sm.full[i % STAGES], (i / STAGES) & 1, err, FA_DEVERR_TIMEOUT, nullptr);
+        __syncwarp();
+        return;
+    }
+
+    // ================= consumers =================
+    const int team = warp >> 2, wt = warp & 3;
+    const int grp = lane >> 2, tig = lane & 3;    // fragment row, column pair
+    const int lrow = lane & 7, lmat = lane >> 3;  // ldmatrix row and matrix
+    int g = 0, k = 0;                             // ring uses, units done
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
+        const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk, kPage,
+                                        max_splits);
+        // the group's query rows as A fragments: a0 = cols 16ks + 2tig..+1,
+        // a2 = cols +8, of row grp (zero past GH); rows 8..15 are zero
+        uint32_t qa[KS][2];
+        {
+            const bool row_in = grp < GH;
+            const __nv_bfloat16* qr =
+                q + (static_cast<int64_t>(us.b) * H + us.h * GH + (row_in ? grp : 0)) * D;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                qa[ks][0] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tig)) : 0u;
+                qa[ks][1] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tig)) : 0u;
+            }
+        }
+        float m = -INFINITY, l = 0.f;
+        float acc[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+        const int nchunks = (us.ntok + kGqTok - 1) / kGqTok;
+        for (int c = 0; c < nchunks; ++c, ++g) {
+            if ((g & 1) != team) continue;
+            const int slot = g % STAGES;
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (g / STAGES) & 1, err,
+                                                   FA_DEVERR_TIMEOUT, abort));
+            if (!ok) break;
+            const uint32_t kb = smem_u32(sm.k[slot]), vb = smem_u32(sm.v[slot]);
+            const int t0 = c * kGqTok + 16 * wt;  // the warp's first token in the unit
+            // ---- S = Q K^T: n-tile j holds tokens t0 + 8j .. +7
+            float s[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < KS / 2; ++kp) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    // matrices: column chunks 4kp .. 4kp+3 of token rows 16wt + 8j ..
+                    uint32_t b[4];
+                    ldsm_x4(b, kb + gq_swz(16 * wt + 8 * j + lrow, 4 * kp + lmat));
+                    mma_bf16_16816(s[j], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b[0], b[1]);
+                    mma_bf16_16816(s[j], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b[2], b[3]);
+                }
+            }
+            // ---- online softmax of row grp over this warp's 16 tokens
+            const bool partial = t0 + 16 > us.ntok;
+            float sv[4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float x = s[j][e] * scale_log2;
+                    sv[2 * j + e] = (partial && t0 + 8 * j + 2 * tig + e >= us.ntok) ? -INFINITY : x;
+                }
+            float mb = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+            const float mn = fmaxf(m, mb);
+            const float mu = (mn == -INFINITY) ? 0.f : mn;  // no finite score yet
+            const float alpha = ex2_approx(m - mu);          // m = -inf -> 0
+            l *= alpha;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                acc[n][0] *= alpha;
+                acc[n][1] *= alpha;
+            }
+            float pv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pv[i] = ex2_approx(sv[i] - mu);  // -inf -> 0
+            l += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+            m = mn;
+            // P as the A operand: tokens 2tig..+1 of n-tile 0 (a0) and 1 (a2)
+            const uint32_t pa0 = pack_bf16x2(pv[0], pv[1]);
+            const uint32_t pa2 = pack_bf16x2(pv[2], pv[3]);
+            // V rows past the unit's tokens may hold anything (0 * NaN): zero
+            // their halves of the B fragments
+            uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+            if (partial) {
+                const int tt = t0 + 2 * tig;
+                mlo = (tt < us.ntok ? 0x0000ffffu : 0u) | (tt + 1 < us.ntok ? 0xffff0000u : 0u);
+                mhi = (tt + 8 < us.ntok ? 0x0000ffffu : 0u) | (tt + 9 < us.ntok ? 0xffff0000u : 0u);
+            }
+            // ---- O += P V: matrices (tokens 0-7 | 8-15) x (column chunk 2np | 2np+1)
+#pragma unroll
+            for (int np = 0; np < NT / 2; ++np) {
+                uint32_t b[4];
+                ldsm_x4_trans(b, vb + gq_swz(16 * wt + 8 * (lmat & 1) + lrow, 2 * np + (lmat >> 1)));
+                mma_bf16_16816(acc[2 * np], pa0, 0u, pa2, 0u, b[0] & mlo, b[1] & mhi);
+                mma_bf16_16816(acc[2 * np + 1], pa0, 0u, pa2, 0u, b[2] & mlo, b[3] & mhi);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[slot]);
+        }
+        if (!ok) break;
+        // ---- merge the 8 warps' states of this unit (buffers by unit parity)
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        const int par = k & 1;
+        if (grp < GH) {
+            if (tig == 0) {
+                sm.cm[par][grp][warp] = m;
+                sm.cl[par][grp][warp] = l;
+            }
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+                *reinterpret_cast<float2*>(&sm.co[par][grp][warp][n * 8 + 2 * tig]) =
+                    make_float2(acc[n][0], acc[n][1]);
+        }
+        mbar_arrive(&sm.cmb[par]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT,
+                                               abort));
+        if (!ok) break;
+        for (int idx = threadIdx.x; idx < GH * D; idx += kGqWarps * 32) {
+            const int hi = idx / D, x = idx - hi * D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kGqWarps; ++w) M = fmaxf(M, sm.cm[par][hi][w]);
+            float L = 0.f, o = 0.f;
+#pragma unroll
+            for (int w = 0; w < kGqWarps; ++w) {
+                const float mw = sm.cm[par][hi][w];
+                const float wgt = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+                L += wgt * sm.cl[par][hi][w];
+                o += wgt * sm.co[par][hi][w][x];
+            }
+            const int64_t pu = static_cast<int64_t>(u) * GH + hi;
+            part_o[pu * D + x] = o / L;
+            if (x == 0) part_lse[pu] = M + __log2f(L);
+        }
+    }
+}
 
 // One warp per (sequence, query head).  Sequence b's partials start at
 // unit_off[b] * GH and are split-major with H per split.
@@ -704,7 +789,8 @@ __global__ void __launch_bounds__(256)
 
 template <int D, int GH>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
-                       const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                       const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
+                       const int32_t* seq_lens, void* o, int B, int H, int num_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
                        int num_sms, cudaStream_t stream) {
     const int Hk = H / GH;
@@ -719,21 +805,38 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
     fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, Hk, page_size, max_splits,
                                                           page_off, tok_off, unit_off, err);
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-    auto split = fa_decode_split_kernel<D, GH>;
-    const size_t smem = sizeof(DecSmem<D, GH>) + 128;
-    if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return FA_ERR_CUDA;
-    // a persistent grid of the CTAs that are resident at once
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, split, kDecThreads, smem) !=
-            cudaSuccess ||
-        occ < 1)
-        return FA_ERR_CUDA;
-    split<<<num_sms * occ, kDecThreads, smem, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pages),
-        static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, Hk, page_size,
-        max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
+    if constexpr (GH == 1) {
+        auto split = fa_decode_split_kernel<D>;
+        const size_t smem = sizeof(DecSmem<D>) + 128;
+        if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return FA_ERR_CUDA;
+        // a persistent grid of the CTAs that are resident at once
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, split, kDecThreads, smem) !=
+                cudaSuccess ||
+            occ < 1)
+            return FA_ERR_CUDA;
+        split<<<num_sms * occ, kDecThreads, smem, stream>>>(
+            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pages),
+            static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, num_pages,
+            page_size, max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
+    } else {
+        if (!tk || !tv) return FA_ERR_NULL;
+        auto split = fa_decode_gqa_kernel<D, GH>;
+        const size_t smem = sizeof(GqSmem<D, GH>) + 1024;
+        if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return FA_ERR_CUDA;
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, split, kGqThreads, smem) !=
+                cudaSuccess ||
+            occ < 1)
+            return FA_ERR_CUDA;
+        split<<<num_sms * occ, kGqThreads, smem, stream>>>(
+            *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk,
+            num_pages, max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
+    }
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
         seq_lens, B, H, GH, page_size, max_splits, unit_off, part_lse, part_o,
@@ -797,14 +900,16 @@ size_t decode_workspace_bytes(int B, int H, int d, int max_splits) {
 namespace {
 template <int D>
 int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
-                    const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                    int Hk, int page_size, int max_splits, void* workspace, unsigned int* err,
+                    const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
+                    const int32_t* seq_lens, void* o, int B, int H, int Hk, int num_pages,
+                    int page_size, int max_splits, void* workspace, unsigned int* err,
                     int num_sms, cudaStream_t stream) {
     switch (H / Hk) {
 #define FA_DECODE_GH(GH)                                                                        \
     case GH:                                                                                    \
-        return launch_decode_impl<D, GH>(q, k_pages, v_pages, page_table, seq_lens, o, B, H,   \
-                                         page_size, max_splits, workspace, err, num_sms, stream);
+        return launch_decode_impl<D, GH>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, \
+                                         B, H, num_pages, page_size, max_splits, workspace,    \
+                                         err, num_sms, stream);
         FA_DECODE_GH(1)
         FA_DECODE_GH(2)
         FA_DECODE_GH(4)
@@ -822,16 +927,19 @@ bool decode_group_supported(int H, int Hk) {
 }
 
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,
-                  const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                  int Hk, int d, int page_size, int max_splits, void* workspace,
-                  unsigned int* err, int num_sms, cudaStream_t stream) {
+                  const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
+                  const int32_t* seq_lens, void* o, int B, int H, int Hk, int num_pages, int d,
+                  int page_size, int max_splits, void* workspace, unsigned int* err, int num_sms,
+                  cudaStream_t stream) {
     if (!decode_group_supported(H, Hk)) return FA_ERR_UNSUPPORTED;
     if (d == 128)
-        return launch_decode_d<128>(q, k_pages, v_pages, page_table, seq_lens, o, B, H, Hk,
-                                    page_size, max_splits, workspace, err, num_sms, stream);
+        return launch_decode_d<128>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, B, H,
+                                    Hk, num_pages, page_size, max_splits, workspace, err, num_sms,
+                                    stream);
     if (d == 64)
-        return launch_decode_d<64>(q, k_pages, v_pages, page_table, seq_lens, o, B, H, Hk,
-                                   page_size, max_splits, workspace, err, num_sms, stream);
+        return launch_decode_d<64>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, B, H, Hk,
+                                   num_pages, page_size, max_splits, workspace, err, num_sms,
+                                   stream);
     return FA_ERR_UNSUPPORTED;
 }
 

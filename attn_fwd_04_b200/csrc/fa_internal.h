@@ -65,11 +65,16 @@ struct DecodePlan {
 
 size_t decode_workspace_bytes(int B, int H, int d, int max_splits);
 
-// H query heads over Hk K/V heads (H / Hk in {1, 2, 4, 8}).
+// H query heads over Hk K/V heads (H / Hk in {1, 2, 4, 8}).  The grouped
+// kernels (H > Hk) read the pool through tk, tv: (d, 256, num_pages * Hk)
+// maps with 64 x 64 x 1 boxes and 128-byte swizzle; H == Hk reads it with
+// bulk copies and takes no maps (may be null).  Page indices outside
+// [0, num_pages) are reported.
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,
-                  const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                  int Hk, int d, int page_size, int max_splits, void* workspace,
-                  unsigned int* err, int num_sms, cudaStream_t stream);
+                  const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
+                  const int32_t* seq_lens, void* o, int B, int H, int Hk, int num_pages, int d,
+                  int page_size, int max_splits, void* workspace, unsigned int* err, int num_sms,
+                  cudaStream_t stream);
 bool decode_group_supported(int H, int Hk);
 
 // The current device's error word and SM count (sm_100 devices only).

@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
-        L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+        L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_gather_paged.argtypes = [P, P, P, P, I, I, I, I, P]
         L.fa_append_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
@@ -239,7 +239,7 @@ def fa_decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 
 def fa_decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 256, o=None,
                         stream=None):
     """Decode with grouped K/V heads: q [B,H,d], pages [P,H_kv,page_size,d]
-    -> o [B,H,d] bf16."""
+    -> o [B,H,d] bf16.  The pool size P bounds the page indices read."""
     _check(q, "q", torch.bfloat16, 3)
     _check(k_pages, "k_pages", torch.bfloat16, 4)
     _check(v_pages, "v_pages", torch.bfloat16, 4)
@@ -251,7 +251,8 @@ def fa_decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: in
         o = torch.empty_like(q)
     rc = lib().fa_decode_paged_gqa(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                    page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
-                                   B, H, H_kv, d, int(page_size), _stream(stream))
+                                   B, H, H_kv, k_pages.shape[0], d, int(page_size),
+                                   _stream(stream))
     _raise_if(rc, "fa_decode_paged_gqa")
     return o
 

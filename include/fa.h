@@ -207,17 +207,22 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
  * 是什么", section 进阶学习路径, item 4).
  *   q, o       : [B, H, d] bf16
  *   k_pages,
- *   v_pages    : [P, H_kv, page_size, d] bf16 -- the cache holds H_kv heads
+ *   v_pages    : [num_pages, H_kv, page_size, d] bf16 -- the cache holds
+ *                H_kv heads
  * Query head h attends to K/V head h / (H / H_kv) of its sequence's cached
  * tokens; everything else (page table, lengths, scale 1/sqrt(d), no mask,
  * workspace) as fa_decode_paged.  H / H_kv must be 1, 2, 4 or 8
  * (FA_ERR_UNSUPPORTED otherwise; FA_ERR_SHAPE if H is not a multiple of
- * H_kv).  Each (page, K/V head) slice is read from device memory once and
- * serves all H / H_kv query heads of its group.
+ * H_kv, or num_pages < 1).  Each (page, K/V head) slice is read from device
+ * memory once and serves all H / H_kv query heads of its group.  A page
+ * index outside [0, num_pages) is reported as FA_ERR_DEVICE_BAD_INPUT (see
+ * fa_get_device_error); nothing outside the pool is read, and the output of
+ * that sequence is unspecified.
  */
 FA_API int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v_pages,
                     const int32_t* page_table, const int32_t* seq_lens, void* o,
-                    int B, int H, int H_kv, int d, int page_size, fa_stream_t stream);
+                    int B, int H, int H_kv, int num_pages, int d, int page_size,
+                    fa_stream_t stream);
 
 /*
  * fa_append_paged -- write the K and V rows of new tokens into the paged

@@ -70,8 +70,8 @@ def decode(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=2, d=128, ps=256):
     return L.fa_decode_paged(q, kp, vp, pt, sl, o, B, H, d, ps, S)
 
 
-def decode_gqa(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=8, H_kv=2, d=128, ps=256):
-    return L.fa_decode_paged_gqa(q, kp, vp, pt, sl, o, B, H, H_kv, d, ps, S)
+def decode_gqa(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=8, H_kv=2, P=64, d=128, ps=256):
+    return L.fa_decode_paged_gqa(q, kp, vp, pt, sl, o, B, H, H_kv, P, d, ps, S)
 
 
 def append(L, kn=A, vn=A, cu=A, kp=A, vp=A, pt=A, sl=A, B=2, H_kv=2, total=10, P=8, d=128,
@@ -162,6 +162,7 @@ def test_decode_argument_errors(L):
     assert decode_gqa(L, vp=None) == fa.FA_ERR_NULL
     assert decode_gqa(L, H_kv=0) == fa.FA_ERR_SHAPE
     assert decode_gqa(L, H_kv=3) == fa.FA_ERR_SHAPE       # 8 is not a multiple of 3
+    assert decode_gqa(L, P=0) == fa.FA_ERR_SHAPE          # empty pool
     assert decode_gqa(L, H=24, H_kv=8) == fa.FA_ERR_UNSUPPORTED  # group of 3
     assert decode_gqa(L, H=32, H_kv=2) == fa.FA_ERR_UNSUPPORTED  # group of 16
     assert decode_gqa(L, ps=128) == fa.FA_ERR_UNSUPPORTED

@@ -201,11 +201,13 @@ def test_decode_gqa_group1_equals_decode():
     assert torch.equal(_decode_gqa(g), _decode(g))
 
 
-def test_decode_gqa_workload_sampled():
-    """The paged-decode workload's lengths with 8 K/V heads for 32 query heads."""
+@pytest.mark.parametrize("H_kv", [16, 8, 4])
+def test_decode_gqa_workload_sampled(H_kv):
+    """The paged-decode workload's lengths with 16, 8 or 4 K/V heads for 32
+    query heads (every CTA of the persistent grid runs many units)."""
     w = W.PAGED_DECODE
     lengths = W.varlen_lengths(w.B, w.len_lo, w.len_hi, w.seed)
-    c = W.paged_inputs(w.B, w.H, w.d, lengths, w.seed, w.page_size, device="cuda", H_kv=8)
+    c = W.paged_inputs(w.B, w.H, w.d, lengths, w.seed, w.page_size, device="cuda", H_kv=H_kv)
     c = W.PagedCache(c.q, c.k_pages, c.v_pages, c.page_table.cuda(), c.seq_lens.cuda(),
                      c.page_size, c.pages_per_seq)
     o = _decode_gqa(c)
@@ -216,4 +218,33 @@ def test_decode_gqa_workload_sampled():
         o_ref, _ = oracle.decode_paged_gqa(c.q[b:b + 1].cpu(), kp, vp, pt, sl, PS)
         got.append(to64(o[b:b + 1]))
         ref.append(o_ref)
-    assert_o_close(np.concatenate(got), np.concatenate(ref), "gqa decode workload")
+    assert_o_close(np.concatenate(got), np.concatenate(ref), f"gqa decode workload H_kv={H_kv}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,H_kv", [(8, 4), (8, 2), (16, 2)])
+def test_decode_gqa_chunk_and_warp_edges(d, H, H_kv):
+    """Lengths that end inside, and right at, the 16-token slices the warps own
+    and the 64-token chunks the two warp teams alternate on; the poisoned
+    (NaN) slots past each length must not reach the output."""
+    lens = [15, 16, 17, 48, 49, 64, 65, 127, 128, 129, 191, 320, 513, 767]
+    c = W.paged_inputs(len(lens), H, d, lens, seed=90 + H + H_kv + d, device="cpu", H_kv=H_kv)
+    o = _decode_gqa(_on_gpu(c))
+    o_ref, _ = oracle.decode_paged_gqa(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
+    assert_o_close(to64(o), o_ref, f"decode gqa edges d={d} H={H} H_kv={H_kv}")
+
+
+@pytest.mark.parametrize("H,H_kv", [(8, 2), (4, 4)])
+def test_decode_gqa_page_outside_pool_reported(H, H_kv):
+    """A page index past the pool is reported through the device error word and
+    nothing outside the pool is read; the other sequences are unaffected."""
+    lens = [300, 700, 40]
+    c = _on_gpu(W.paged_inputs(len(lens), H, 128, lens, seed=77, device="cpu", H_kv=H_kv))
+    P = c.k_pages.shape[0]
+    good = _decode_gqa(c)
+    pt = c.page_table.clone()
+    pt[c.pages_per_seq[0]] = P + 5  # the first page of sequence 1
+    o = torch.zeros_like(c.q)
+    fa.fa_decode_paged_gqa(c.q, c.k_pages, c.v_pages, pt, c.seq_lens, c.page_size, o=o)
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_BAD_INPUT
+    assert torch.equal(o[0], good[0]) and torch.equal(o[2], good[2])
