@@ -607,11 +607,12 @@ def run_native(args, world, rank, local):
                          "bytes_per_launch": dbytes,
                          "pct_of_hbm": {"datasheet_8000": 100 * per_launch_gbs / 8000.0,
                                         "measured": 100 * per_launch_gbs / peaks["hbm_gbs"]}}
+        dec_kernel = "fa_decode_split_kernel" if h_kv == DEC.H else "fa_decode_gqa_kernel"
         out["roofline_decode"] = {
-            "bound": "hbm", "kernel": "fa_decode_split_kernel (+plan, merge)",
+            "bound": "hbm", "kernel": f"{dec_kernel} (+plan, merge)",
             "achieved": per_launch_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": per_launch_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy",
-            "traffic": recorded_traffic("fa_decode_split_kernel", dec_sha),
+            "traffic": recorded_traffic(dec_kernel, dec_sha),
             "algorithmic_bytes_per_launch": dbytes}
     return out
 
