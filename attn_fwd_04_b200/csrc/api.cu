@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "fa_ptx.cuh"
@@ -39,6 +40,10 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+// fixed-length forward with d = 128 and no RoPE on CTA pairs (fa_fwd_set_cta_pairs);
+// off by default: on B200 at the 1000 W cap the pair kernel measured ~4% below
+// the single-CTA kernel on the long-prefill workload
+std::atomic<int> g_fwd_pairs{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -184,6 +189,8 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
             return rc;
         k_use = ws;
     }
+    // CTA pairs (2-SM products) load K in halves of 64 keys
+    const bool pair = d == 128 && rope_cos == nullptr && g_fwd_pairs.load() != 0;
     CUtensorMap tq, tk, tv;
     const cuuint64_t dims_q[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                   static_cast<cuuint64_t>(B) * H};
@@ -192,8 +199,9 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                    static_cast<cuuint64_t>(N) * d * 2};
     const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t box_k[3] = {64, pair ? 64u : 128u, 1};
     if ((rc = make_map(&tq, q, dims_q, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tk, k_use, dims_kv, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k_use, dims_kv, strides, box_k)) != FA_OK) return rc;
     if ((rc = make_map(&tv, v, dims_kv, strides, box)) != FA_OK) return rc;
     fa::FwdParams p{};
     p.o = o;
@@ -209,7 +217,7 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
-    return fa::launch_fwd(p, tq, tk, tv, d, fa::kFixed, st);
+    return fa::launch_fwd(p, tq, tk, tv, d, pair ? fa::kFixedPair : fa::kFixed, st);
 }
 
 }  // namespace
@@ -534,5 +542,7 @@ const char* fa_status_str(int status) {
 }
 
 int fa_version(void) { return 100; }
+
+int fa_fwd_set_cta_pairs(int enable) { return g_fwd_pairs.exchange(enable ? 1 : 0); }
 
 }  // extern "C"

@@ -37,8 +37,9 @@ struct FwdParams {
 // rotary embedding of x [rows, N, d] into y (positions 0..N-1)
 int launch_rope_rows(const void* x, void* y, const float* cos_t, const float* sin_t, int64_t rows,
                      int N, int d, int num_sms, cudaStream_t stream);
-// forward modes
-constexpr int kFixed = 0, kVarlen = 1, kPaged = 2;
+// forward modes; kFixedPair: fixed length on CTA pairs (2-SM products; d = 128,
+// no RoPE), its K map with 64 x 64 boxes (tq, tv: 64 x 128 as for kFixed)
+constexpr int kFixed = 0, kVarlen = 1, kPaged = 2, kFixedPair = 3;
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, int d, int mode, cudaStream_t stream);
 

@@ -28,6 +28,10 @@
 //     switched off because it measured slower here); O is rescaled only when
 //     the running max has grown by more than 2^8 (the stale max is used for
 //     both the numerator and l, so the result is unchanged up to rounding).
+//   * opt-in (fa_fwd_set_cta_pairs, d = 128, fixed length): CTA pairs whose
+//     products span both SMs (tcgen05 cta_group::2, M = 256), each CTA loading
+//     half of every K/V tile; it moves half the K/V bytes per query row but
+//     couples both CTAs' softmax to every product, and measured slower.
 //
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
 // P_t (bf16 pairs) overwrites the first 64 columns of S_t; the next S_t is
@@ -62,14 +66,22 @@ constexpr int kPolyPairs = 0;
 constexpr float kExp2P0 = 0.9999280571937561f, kExp2P1 = 0.6932609677314758f,
                 kExp2P2 = 0.2426111251115799f, kExp2P3 = 0.0551716685295105f;
 
-template <int D>
+// PAIR: the CTA is one of a pair whose products run on both SMs' tensor cores
+// (M = 256: each CTA's query tile is half of the A operand); a ring slot then
+// holds this CTA's half of a K tile (64 keys) or of a V tile (64 of the 128
+// dimensions), so the ring has twice the slots in the same space.
+template <bool PAIR> constexpr int ring_slots() { return PAIR ? 2 * kSlots : kSlots; }
+
+template <int D, bool PAIR>
 struct alignas(1024) FwdSmem {
+    static constexpr int kRing = ring_slots<PAIR>();
+    static constexpr int kSlotBytes = PAIR ? BN * D : BN * D * 2;
     uint8_t q[2][BM * D * 2];
-    uint8_t kv[kSlots][BN * D * 2];
+    uint8_t kv[kRing][kSlotBytes];
     float row_m[2][BM];   // final running max (log2 domain) per row
     float row_l[2][BM];   // final normaliser per row
     uint64_t q_full[2];
-    uint64_t kv_full[kSlots], kv_empty[kSlots];
+    uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
     uint64_t q_rot;      // RoPE: both Q tiles rotated
@@ -84,9 +96,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsign
     return __all_sync(0xffffffffu, ok);
 }
 
-// K/V ring position of tile j's K (v = 0) or V (v = 1)
-__device__ __forceinline__ int ring_slot(int j, int v) { return (2 * j + v) % kSlots; }
-__device__ __forceinline__ uint32_t ring_phase(int j, int v) { return ((2 * j + v) / kSlots) & 1; }
+// K/V ring position of tile j's K (v = 0) or V (v = 1) in a ring of R slots
+template <int R = kSlots>
+__device__ __forceinline__ int ring_slot(int j, int v) { return (2 * j + v) % R; }
+template <int R = kSlots>
+__device__ __forceinline__ uint32_t ring_phase(int j, int v) { return ((2 * j + v) / R) & 1; }
 
 // Max (or, for a negative scale, min) of the 128 raw scores of a row.
 __device__ __forceinline__ float row_extreme(const uint32_t (&s)[BN], bool neg) {
@@ -226,25 +240,38 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const fl
 // ROPE (fixed-length only): the Q tiles are rotated in shared memory by the
 // epilogue warpgroup (idle until the last step) before their first score
 // product; K arrives rotated (fa_rope_rows_kernel, once per position).
-template <int D, int MODE, bool ROPE>
+// PAIR (fixed-length, d = 128, no RoPE): CTAs run in clusters of two and a
+// pair shares one 512-row query block: CTA c of the pair holds 128-row tiles
+// 2t + c (t = 0, 1), and tile pair t (rows 256t .. 256t + 255 of the block) is
+// one M = 256 product on both SMs.  Each CTA loads half of every K tile (64
+// keys) and half of every V tile (64 dimensions), so each K/V byte crosses
+// from L2 once per 512 query rows instead of once per 256, and the B operand
+// is read from shared memory once for both SMs.  The even CTA issues every
+// MMA; both CTAs run the softmax and epilogue of their own tiles.
+template <int D, int MODE, bool ROPE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
     constexpr bool VARLEN = MODE != kFixed;  // packed query rows
     constexpr bool PAGED = MODE == kPaged;
-    // ---- the work unit: (sequence/head, 256-row query block) --------------
-    // CTAs walk the units in groups of kHeadGroup (sequence, head) pairs; in
-    // a group they are numbered by rank first, rank r being the r-th 256-row
+    static_assert(!PAIR || (D == 128 && MODE == kFixed && !ROPE), "pair mode: fixed length, d=128");
+    constexpr int R = ring_slots<PAIR>();          // K/V ring slots
+    constexpr int kRows = PAIR ? 4 * BM : 2 * BM;  // query rows per work unit
+    // ---- the work unit: (sequence/head, query block of kRows rows) ---------
+    // CTAs (CTA pairs) walk the units in groups of kHeadGroup (sequence, head)
+    // pairs; in a group they are numbered by rank first, rank r being the r-th
     // block counted from the end of its sequence.  Under a causal mask each
     // group's heaviest blocks start before its lighter ones, and the CTAs in
     // flight at any time read the K/V of a few heads only, which stay in L2
     // (all heads at once would spill it and re-read K/V from DRAM).  With
     // grouped K/V heads (H_kv < H) query head h reads K/V head h / (H / H_kv).
+    const int wu = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const uint32_t crank = PAIR ? cluster_ctarank() : 0u;  // 0: issues the pair's MMAs
     const int units = p.B * p.H;
-    const int nblk_all = (p.N + 2 * BM - 1) / (2 * BM);
-    const int gidx = static_cast<int>(blockIdx.x) / (kHeadGroup * nblk_all);
+    const int nblk_all = (p.N + kRows - 1) / kRows;
+    const int gidx = wu / (kHeadGroup * nblk_all);
     const int ug = min(kHeadGroup, units - gidx * kHeadGroup);
-    const int within = static_cast<int>(blockIdx.x) - gidx * kHeadGroup * nblk_all;
+    const int within = wu - gidx * kHeadGroup * nblk_all;
     const int rank = within / ug;
     const int unit = gidx * kHeadGroup + (within - rank * ug);
     // len: query rows; klen: keys; a query row i may see keys up to
@@ -280,16 +307,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         len = p.N;
         klen = len;
     }
-    const int nblk = (len + 2 * BM - 1) / (2 * BM);
+    const int nblk = (len + kRows - 1) / kRows;
     const int blk = p.causal ? (nblk - 1 - rank) : rank;
-    if (blk < 0 || blk >= nblk) return;
-    const int row0 = blk * 2 * BM;
+    if (blk < 0 || blk >= nblk) return;  // (both CTAs of a pair return together)
+    const int row0 = blk * kRows;
+    // first query row of this CTA's tile t
+    auto tile_row = [&](int t) { return PAIR ? row0 + (2 * t + static_cast<int>(crank)) * BM
+                                             : row0 + t * BM; };
     const int nkv_all = (klen + BN - 1) / BN;
+    // n_t[t]: K/V tiles tile t takes part in; a pair's two tiles share one
+    // count, that of its later tile (the earlier tile's last step is then
+    // fully masked under a causal mask and contributes P = 0)
     int n_t[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        const int rf = row0 + t * BM;
-        n_t[t] = (rf < len) ? (p.causal ? min((kshift + rf + BM - 1) / BN + 1, nkv_all) : nkv_all)
+        const int rf = PAIR ? row0 + 2 * t * BM : row0 + t * BM;   // first row that must be computed
+        const int rl = PAIR ? rf + BM : rf;                         // first row of the last tile
+        n_t[t] = (rf < len) ? (p.causal ? min((kshift + rl + BM - 1) / BN + 1, nkv_all) : nkv_all)
                             : 0;
     }
     const int n = max(n_t[0], n_t[1]);
@@ -299,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool zero_v_tail = PAGED && n == nkv_all && (klen % BN) != 0;
 
     extern __shared__ uint8_t smem_raw[];
-    FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
+    FwdSmem<D, PAIR>& sm = *reinterpret_cast<FwdSmem<D, PAIR>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
     const uint32_t warp = warp_id_uniform();
@@ -312,13 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm.q_full[t], 1);
             mbar_init(&sm.s_full[t], 1);
-            mbar_init(&sm.p_full[t], BM);
+            mbar_init(&sm.p_full[t], PAIR ? 8 : BM);  // pair: one arrival per softmax warp
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
         }
         mbar_init(&sm.vfix, 1);
         mbar_init(&sm.q_rot, BM);
-        for (int s = 0; s < kSlots; ++s) {
+        for (int s = 0; s < R; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
@@ -327,11 +361,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
     }
     if (warp == 12) {
-        tmem_alloc(&sm.tmem_base, kTmemCols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(&sm.tmem_base, kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&sm.tmem_base, kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    // a pair: the other CTA's barriers must be initialised before any copy,
+    // commit or arrival reaches them
+    if constexpr (PAIR) cluster_sync_all();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
@@ -371,15 +413,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, (j & 1) * BN,
                                 page * p.H_kv + bkv);
             };
+            if constexpr (PAIR) {
+                // Both CTAs copy into their own shared memory and complete the
+                // bytes on the even CTA's barriers, whose single arrival (with
+                // the byte count of both halves) the even CTA makes.
+                for (int t = 0; t < 2; ++t) {
+                    if (n_t[t] == 0) continue;
+                    if (crank == 0) mbar_arrive_expect_tx(&sm.q_full[t], 2 * BM * D * 2);
+                    const uint32_t bar = mapa_rank(smem_u32(&sm.q_full[t]), 0);
+#pragma unroll
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_load_3d_pair(sm.q[t] + cb * kBoxBytes, &tq, bar, cb * 64, tile_row(t),
+                                         bh);
+                }
+                for (int u = 0; u < 2 * n; ++u) {
+                    const int slot = u % R;
+                    const uint32_t ph = (u / R) & 1;
+                    if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
+                    if (crank == 0) mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
+                    const uint32_t bar = mapa_rank(smem_u32(&sm.kv_full[slot]), 0);
+                    const int j = u >> 1;
+                    if ((u & 1) == 0) {
+                        // K: keys [j*BN + crank*BN/2, +BN/2), every dimension
+                        // (D/64 boxes of BN/2 rows x 64 columns)
+#pragma unroll
+                        for (int cb = 0; cb < D / 64; ++cb)
+                            tma_load_3d_pair(sm.kv[slot] + cb * (kBoxBytes / 2), &tk, bar, cb * 64,
+                                             j * BN + static_cast<int>(crank) * (BN / 2), bkv);
+                    } else {
+                        // V: every key of the tile, dimensions [crank*64, +64)
+                        tma_load_3d_pair(sm.kv[slot], &tv, bar, static_cast<int>(crank) * 64,
+                                         j * BN, bkv);
+                    }
+                    issued = u + 1;
+                }
+            } else {
             for (int t = 0; t < 2; ++t) {
                 if (n_t[t] > 0) {
                     mbar_arrive_expect_tx(&sm.q_full[t], BM * D * 2);
-                    load_tile(sm.q[t], &tq, &sm.q_full[t], row0 + t * BM, bh);
+                    load_tile(sm.q[t], &tq, &sm.q_full[t], tile_row(t), bh);
                 }
             }
             for (int u = 0; u < 2 * n; ++u) {
-                const int slot = u % kSlots;
-                const uint32_t ph = (u / kSlots) & 1;
+                const int slot = u % R;
+                const uint32_t ph = (u / R) & 1;
                 if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
                 mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
                 if constexpr (PAGED)
@@ -389,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                               bkv);
                 issued = u + 1;
             }
+            }  // PAIR
             }  // lane 0
             issued = __shfl_sync(0xffffffffu, issued, 0);
             if (zero_v_tail && issued == 2 * n) {
@@ -411,51 +489,81 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (lane == 0) {
             // every copy this CTA started must land before it exits
-            for (int t = 0; t < 2; ++t)
-                if (n_t[t] > 0) mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, nullptr);
-            for (int u = max(0, issued - kSlots); u < issued; ++u)
-                mbar_wait(&sm.kv_full[u % kSlots], (u / kSlots) & 1, err, FA_DEVERR_TIMEOUT,
-                          nullptr);
+            if (crank == 0) {
+                for (int t = 0; t < 2; ++t)
+                    if (n_t[t] > 0) mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, nullptr);
+                for (int u = max(0, issued - R); u < issued; ++u)
+                    mbar_wait(&sm.kv_full[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, nullptr);
+            } else {
+                // the odd CTA of a pair cannot wait on the even CTA's barriers:
+                // a slot released by the MMAs has landed (and so has Q, read
+                // by earlier products)
+                for (int u = max(0, issued - R); u < issued; ++u)
+                    mbar_wait(&sm.kv_empty[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, abort);
+            }
             }  // lane 0
-        } else if (warp == 12 && lane == 0) {
+        } else if (warp == 12 && lane == 0 && crank == 0) {
             // ================= MMA issuer =================
             // The tensor pipe runs this thread's MMAs in issue order, so
             // S_t(j+1), which overwrites the TMEM columns holding P_t(j), is
             // issued right behind P_t(j) V_j without waiting: P_t is read first.
-            constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
+            // A pair's products have M = 256 (this CTA's tile, then the odd
+            // CTA's) and take half of B's columns from each CTA.
+            constexpr uint32_t kM = PAIR ? 2 * BM : BM;
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kM, BN, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, D, 0, 1);
             // descriptor words: high = SBO 1024 B | version 1 | 128-byte swizzle;
             // low = LBO (16 B for K-major, the 64-column block stride for V) | addr>>4
             constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
             constexpr uint32_t kLboK = (16u >> 4) << 16;
             constexpr uint32_t kLboV = (static_cast<uint32_t>(kBoxBytes) >> 4) << 16;
-            constexpr uint32_t kTile16 = (BN * D * 2) >> 4;  // one ring slot, in 16-byte units
+            constexpr uint32_t kSlot16 = FwdSmem<D, PAIR>::kSlotBytes >> 4;  // ring slot, 16-B units
+            // K in a slot: D/64 boxes of (PAIR ? 64 : 128) keys x 128 bytes
+            constexpr uint32_t kKBox16 = (PAIR ? kBoxBytes / 2 : kBoxBytes) >> 4;
             const uint32_t q_lo0 = smem_u32(sm.q[0]) >> 4;
             const uint32_t q_lo1 = smem_u32(sm.q[1]) >> 4;
             const uint32_t kv_lo = smem_u32(sm.kv[0]) >> 4;
             auto issue_s = [&](int t, int j) {
                 const uint32_t qa = t ? q_lo1 : q_lo0;
-                const uint32_t kb = kv_lo + ring_slot(j, 0) * kTile16;
+                const uint32_t kb = kv_lo + ring_slot<R>(j, 0) * kSlot16;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t o = (kk >> 2) * (kBoxBytes >> 4) + (kk & 3) * 2;
-                    mma_ss(tmem + col_s(t),
-                           (static_cast<uint64_t>(kDescHi) << 32) | (kLboK | (qa + o)),
-                           (static_cast<uint64_t>(kDescHi) << 32) | (kLboK | (kb + o)), idesc_s,
-                           kk > 0 ? 1u : 0u);
+                    const uint32_t oa = (kk >> 2) * (kBoxBytes >> 4) + (kk & 3) * 2;
+                    const uint32_t ob = (kk >> 2) * kKBox16 + (kk & 3) * 2;
+                    const uint64_t da = (static_cast<uint64_t>(kDescHi) << 32) | (kLboK | (qa + oa));
+                    const uint64_t db = (static_cast<uint64_t>(kDescHi) << 32) | (kLboK | (kb + ob));
+                    if constexpr (PAIR)
+                        mma_ss_pair(tmem + col_s(t), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss(tmem + col_s(t), da, db, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int t, int j) {
-                const uint32_t vb = kv_lo + ring_slot(j, 1) * kTile16;
+                const uint32_t vb = kv_lo + ring_slot<R>(j, 1) * kSlot16;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 16 rows of 128 bytes
-                    mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                           (static_cast<uint64_t>(kDescHi) << 32) | (kLboV | (vb + kk * 128)),
-                           idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < BN / 16; ++kk) {  // 16 keys = 16 rows of 128 bytes
+                    const uint64_t db =
+                        (static_cast<uint64_t>(kDescHi) << 32) | (kLboV | (vb + kk * 128));
+                    if constexpr (PAIR)
+                        mma_ts_pair(tmem + col_o(t), tmem + col_s(t) + kk * 8, db, idesc_pv,
+                                    (j > 0 || kk > 0) ? 1u : 0u);
+                    else
+                        mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, db, idesc_pv,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
+            };
+            // completion of everything issued so far, signalled to this CTA's
+            // barrier and, for a pair, to the same barrier of the odd CTA
+            auto commit = [&](uint64_t* bar) {
+                if constexpr (PAIR) {
+                    tc_commit_pair_both(smem_u32(bar));
+                } else {
+                    tc_commit(bar);
+                }
             };
             bool ok = true;
             auto wait_k = [&](int j) {
-                return mbar_wait(&sm.kv_full[ring_slot(j, 0)], ring_phase(j, 0), err,
+                return mbar_wait(&sm.kv_full[ring_slot<R>(j, 0)], ring_phase<R>(j, 0), err,
                                  FA_DEVERR_TIMEOUT, abort);
             };
             if constexpr (ROPE) {
@@ -471,15 +579,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < 2; ++t) {
                     if (n_t[t] > 0) {
                         issue_s(t, 0);
-                        tc_commit(&sm.s_full[t]);
+                        commit(&sm.s_full[t]);
                     }
                 }
-                tc_commit(&sm.kv_empty[ring_slot(0, 0)]);
+                commit(&sm.kv_empty[ring_slot<R>(0, 0)]);
             }
             for (int j = 0; ok && j < n; ++j) {
                 if (zero_v_tail && j == n - 1) {
                     if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort)) break;
-                } else if (!mbar_wait(&sm.kv_full[ring_slot(j, 1)], ring_phase(j, 1), err,
+                } else if (!mbar_wait(&sm.kv_full[ring_slot<R>(j, 1)], ring_phase<R>(j, 1), err,
                                       FA_DEVERR_TIMEOUT, abort)) {
                     break;
                 }
@@ -487,24 +595,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (next_k && !wait_k(j + 1)) break;
                 for (int t = 0; t < 2; ++t) {
                     if (j >= n_t[t]) continue;
-                    if (!mbar_wait(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+                    // a pair's P comes from both CTAs' softmax warps
+                    if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     issue_pv(t, j);
-                    tc_commit(&sm.pv_done[t]);
+                    if (j + 1 == n_t[t]) commit(&sm.pv_done[t]);  // O_t final
                     if (j + 1 < n_t[t]) {
                         issue_s(t, j + 1);
-                        tc_commit(&sm.s_full[t]);
+                        commit(&sm.s_full[t]);
                     }
                 }
                 if (!ok) break;
-                tc_commit(&sm.kv_empty[ring_slot(j, 1)]);
-                if (next_k) tc_commit(&sm.kv_empty[ring_slot(j + 1, 0)]);
+                commit(&sm.kv_empty[ring_slot<R>(j, 1)]);
+                if (next_k) commit(&sm.kv_empty[ring_slot<R>(j + 1, 0)]);
             }
             // every MMA this thread issued must be complete before TMEM is freed
-            tc_commit(&sm.drain);
+            if constexpr (PAIR) tc_commit_pair(smem_u32(&sm.drain));
+            else tc_commit(&sm.drain);
             mbar_wait(&sm.drain, 0, err, FA_DEVERR_TIMEOUT, nullptr);
         }
         __syncwarp();
@@ -516,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         const uint32_t s_addr = tmem + lane_off + col_s(t);
         const uint32_t o_addr = tmem + lane_off + col_o(t);
-        const int row_first = row0 + t * BM;
+        const int row_first = tile_row(t);
         const int qrow = row_first + r;
         const float sl = p.scale_log2;
         const bool neg = sl < 0.f;
@@ -589,7 +699,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.p_full[t]);
+            if constexpr (PAIR) {
+                // one arrival per warp on the even CTA's barrier
+                __syncwarp();
+                if (lane == 0) {
+                    if (crank == 0) mbar_arrive(&sm.p_full[t]);
+                    else mbar_arrive_cluster(mapa_rank(smem_u32(&sm.p_full[t]), 0));
+                }
+            } else {
+                mbar_arrive(&sm.p_full[t]);
+            }
         }
         if (ok && n_t[t] > 0) {
             sm.row_m[t][r] = m_used;
@@ -611,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const int pos = row0 + t * BM + r;
+                const int pos = tile_row(t) + r;
                 if (pos < len) rope_row<D>(sm.q[t], r, pos, p.rope_cos, p.rope_sin);
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -621,10 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; ok && t < 2; ++t) {
             if (n_t[t] == 0) continue;
             if (!warp_wait(&sm.stats_full[t], 0, err, abort) ||
-                !warp_wait(&sm.pv_done[t], (n_t[t] - 1) & 1, err, abort))
+                !warp_wait(&sm.pv_done[t], 0, err, abort))
                 break;
             tc_fence_after();
-            const int qrow = row0 + t * BM + r;
+            const int qrow = tile_row(t) + r;
             const bool store = qrow < len;
             const float m = sm.row_m[t][r], l = sm.row_l[t][r];
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -669,9 +788,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    // a pair: neither CTA may free its TMEM or leave (its shared memory still
+    // read by the pair's products, its barriers still arrived on) before both
+    // are done
+    if constexpr (PAIR) cluster_sync_all();
+    else __syncthreads();
     tc_fence_after();
-    if (warp == 12) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 12) {
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, kTmemCols);
+        else tmem_dealloc(tmem, kTmemCols);
+    }
 }
 
 // Rotary embedding of whole rows in device memory (used for K, whose tiles
@@ -724,23 +850,44 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <int D, int MODE, bool ROPE = false>
+template <int D, int MODE, bool ROPE = false, bool PAIR = false>
 int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, cudaStream_t stream) {
     // Every CTA allocates all 512 TMEM columns, so one CTA per SM: ask for
     // enough shared memory that a second CTA cannot be co-resident.
-    const size_t smem = sizeof(FwdSmem<D>) + 1024 > 120 * 1024 ? sizeof(FwdSmem<D>) + 1024
-                                                               : 120 * 1024;
-    auto kern = fa_fwd_kernel<D, MODE, ROPE>;
+    constexpr size_t kSmemUse = sizeof(FwdSmem<D, PAIR>) + 1024;
+    const size_t smem = kSmemUse > 120 * 1024 ? kSmemUse : 120 * 1024;
+    auto kern = fa_fwd_kernel<D, MODE, ROPE, PAIR>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
-    // one CTA per (sequence/head, 256-row block); see the kernel for the order
-    const long long blocks = (p.N + 2 * BM - 1) / (2 * BM);
-    const long long ctas = blocks * p.B * p.H;
+    // one CTA (pair) per (sequence/head, query block); see the kernel for the order
+    constexpr int kRows = PAIR ? 4 * BM : 2 * BM;
+    const long long blocks = (p.N + kRows - 1) / kRows;
+    const long long ctas = blocks * p.B * p.H * (PAIR ? 2 : 1);
     if (ctas > 0x7fffffffLL) return FA_ERR_SHAPE;
-    kern<<<dim3(static_cast<unsigned>(ctas)), kThreads, smem, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    if constexpr (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_CUDA;
+        }
+        return FA_OK;
+    } else {
+        kern<<<dim3(static_cast<unsigned>(ctas)), kThreads, smem, stream>>>(tq, tk, tv, p);
+        return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
 }
 
 }  // namespace
@@ -764,6 +911,9 @@ int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, int d, int mode, cudaStream_t stream) {
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     switch (mode) {
+        case kFixedPair:
+            if (d != 128 || p.rope_cos) return FA_ERR_UNSUPPORTED;
+            return launch_impl<128, kFixed, false, true>(p, tq, tk, tv, stream);
         case kFixed:
             if (p.rope_cos)
                 return d == 128 ? launch_impl<128, kFixed, true>(p, tq, tk, tv, stream)

@@ -28,7 +28,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
-           "fa_status_str", "fa_version")
+           "fa_status_str", "fa_version", "fa_fwd_set_cta_pairs")
 
 _lib = None
 
@@ -65,11 +65,12 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
+        L.fa_fwd_set_cta_pairs.argtypes = [I]
         for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged",
                      "fa_decode_paged_gqa", "fa_decode_paged_noalloc", "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
-                     "fa_version"):
+                     "fa_version", "fa_fwd_set_cta_pairs"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -359,3 +360,9 @@ def fa_release_workspace() -> None:
 
 def fa_version() -> int:
     return lib().fa_version()
+
+
+def fa_fwd_set_cta_pairs(enable: bool) -> bool:
+    """Select the CTA-pair (True) or single-CTA (False, default) forward kernel
+    for d = 128; returns the previous setting."""
+    return bool(lib().fa_fwd_set_cta_pairs(int(bool(enable))))

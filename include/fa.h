@@ -354,6 +354,19 @@ FA_API const char* fa_status_str(int status);
 /* Library ABI version: 100 * major + minor. */
 FA_API int fa_version(void);
 
+/*
+ * fa_fwd_set_cta_pairs -- choose the kernel that fa_fwd and fa_fwd_gqa run for
+ * d = 128 (process-wide; the results agree within the stated tolerances, not
+ * bit for bit).  Zero (the default): one CTA per 256 query rows.  Non-zero:
+ * CTA pairs on two SMs share each K/V tile and each product (M = 256 rows
+ * across the pair), so every K/V byte leaves L2 once per 512 query rows; it
+ * draws less power but waits longer per step (both CTAs' softmax gates each
+ * product) and measured slower on B200.  Calls already enqueued are not
+ * affected.  Returns the previous setting.  (A tuning control with no
+ * counterpart on the pages.)
+ */
+FA_API int fa_fwd_set_cta_pairs(int enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -45,6 +45,16 @@ def test_status_strings(L):
     assert fa.fa_version() == 100
 
 
+def test_cta_pair_setting_round_trips(L):
+    prev = fa.fa_fwd_set_cta_pairs(True)
+    try:
+        assert fa.fa_fwd_set_cta_pairs(False) is True
+        assert fa.fa_fwd_set_cta_pairs(False) is False
+    finally:
+        fa.fa_fwd_set_cta_pairs(prev)
+    assert prev is False  # the default
+
+
 # Fake, never-dereferenced device addresses: validation rejects the calls
 # before any CUDA call is made.
 A = 1 << 20          # 16-byte aligned

@@ -57,6 +57,51 @@ def test_shapes_full_compare(shape, causal):
     assert_lse_close(to64(lse), lse_ref, str(shape))
 
 
+@pytest.fixture(params=[True, False], ids=["pairs", "single"])
+def cta_pairs(request):
+    """Run a d = 128 test on the CTA-pair kernel and on the single-CTA kernel."""
+    prev = fa.fa_fwd_set_cta_pairs(request.param)
+    yield request.param
+    fa.fa_fwd_set_cta_pairs(prev)
+
+
+# d = 128 lengths around the pair kernel's 512-row blocks: a pair whose odd
+# CTA's tile starts past the end (1, 127, 257), whose second tile pair is
+# empty (255, 256), partial blocks (384, 511, 513, 1000) and several heads,
+# batches and grouped K/V heads
+PAIR_SHAPES = [(1, 1, 1, 1), (1, 2, 2, 127), (1, 2, 2, 256), (2, 2, 1, 257), (1, 3, 3, 384),
+               (1, 2, 2, 511), (1, 1, 1, 513), (1, 4, 2, 1000), (2, 2, 2, 1536)]
+
+
+@pytest.mark.parametrize("shape", PAIR_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_d128_both_kernels_full_compare(shape, causal, cta_pairs):
+    B, H, Hkv, N = shape
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, 128, seed=900 + N + H, device="cpu")
+    scale = 1 / math.sqrt(128)
+    o, lse = _gqa_gpu(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention_gqa(q, k, v, causal, scale)
+    assert_o_close(to64(o), o_ref, f"{shape} pairs={cta_pairs}")
+    assert_lse_close(to64(lse), lse_ref, f"{shape} pairs={cta_pairs}")
+
+
+def test_pair_kernel_matches_single_kernel():
+    """Both kernels take the same steps per query row (the pair kernel's extra
+    fully masked step adds exact zeros), so they agree to the tolerance; the
+    comparison also reports whether they agree bit for bit."""
+    q, k, v = W.custom_fwd_inputs(1, 4, 1500, 128, seed=910)
+    got = {}
+    for pairs in (True, False):
+        prev = fa.fa_fwd_set_cta_pairs(pairs)
+        try:
+            got[pairs] = _fwd_gpu(q, k, v, True, 0.09)
+        finally:
+            fa.fa_fwd_set_cta_pairs(prev)
+    (o1, l1), (o2, l2) = got[True], got[False]
+    assert_o_close(to64(o1), to64(o2), "pairs vs single")
+    assert_lse_close(to64(l1), to64(l2), "pairs vs single")
+
+
 @pytest.mark.parametrize("scale", [0.0, 0.02, 0.3, -0.1])
 def test_other_scales(scale):
     q, k, v = W.custom_fwd_inputs(1, 2, 300, 128, seed=7)
@@ -329,7 +374,11 @@ def test_rope_equals_fwd_on_prerotated_inputs():
     o, lse = fa.fa_fwd_rope(q.cuda(), k.cuda(), v.cuda(), c.cuda(), s.cuda(), True, 0.1)
     qr = torch.from_numpy(oracle.rope(q, c, s, True)).to(torch.bfloat16).cuda()
     kr = torch.from_numpy(oracle.rope(k, c, s, True)).to(torch.bfloat16).cuda()
-    o2, l2 = fa.fa_fwd_gqa(qr, kr, v.cuda(), True, 0.1)
+    prev = fa.fa_fwd_set_cta_pairs(False)  # the kernel fa_fwd_rope runs on (the default)
+    try:
+        o2, l2 = fa.fa_fwd_gqa(qr, kr, v.cuda(), True, 0.1)
+    finally:
+        fa.fa_fwd_set_cta_pairs(prev)
     assert fa.fa_get_device_error() == fa.FA_OK
     assert torch.equal(o, o2) and torch.equal(lse, l2)
 
