@@ -20,19 +20,23 @@
 //   S^T  = K Q_i^T          (TMEM, lanes = keys)
 //   dV  += P^T dO_i         (P^T from TMEM as bf16)
 //   dP^T = V dO_i^T         (TMEM)
-//   dK  += dS^T Q_i         (dS^T from TMEM as bf16)
 //   dQ_i = dS K             (dS from shared memory, written over the dO_i
 //                            tile once its last reader has completed)
+//   dK  += dS^T Q_i         (the same shared-memory tile, read K-major)
 // Warpgroup 0 (one thread per key) turns S^T into P^T and dP^T into dS^T;
 // warpgroup 1 adds each dQ_i into an fp32 accumulator in device memory (the
 // key blocks of a head all contribute to every dQ row) and writes dK, dV at
-// the end; warp 8 issues the MMAs, warp 9 the TMA loads.  A prep kernel forms
-// D and the log2-domain statistics and clears the dQ accumulator; a final
-// kernel rounds dQ to bf16.
+// the end; warp 8 issues the MMAs, warp 9 the TMA loads (warps 10, 11 only
+// complete warpgroup 2, whose registers setmaxnreg moves to warpgroup 0).
+// dP^T of a tile needs no P^T, so it is issued as soon as the previous dQ_i
+// has left TMEM: warpgroup 0 finds it ready right after P^T, and the tensor
+// pipe runs dV and the next S^T while warpgroup 0 forms dS.  A prep
+// kernel forms D and the log2-domain statistics and clears the dQ
+// accumulator; a final kernel rounds dQ to bf16.
 //
 // TMEM columns: S^T [0,128) (P^T as bf16 pairs in [0,64)), dP^T [128,256)
-// (dS^T in [128,192); dQ_i reuses [128,128+D) once dK has read dS^T),
-// dV [256,256+D), dK [384,384+D).
+// (dQ_i reuses [128,128+D) once warpgroup 0 has read dP^T), dV [256,256+D),
+// dK [384,384+D).
 #include <cuda_bf16.h>
 
 #include "fa_ptx.cuh"
@@ -41,7 +45,12 @@ namespace fa {
 namespace {
 
 constexpr int kBT = 128;            // keys per CTA, queries per tile
-constexpr int kBwdThreads = 320;    // 10 warps
+constexpr int kBwdThreads = 384;    // 12 warps: 3 warpgroups
+// setmaxnreg split of the 168 registers per thread the block launches with
+// (65536 / 384, rounded down to 8): warpgroup 0 holds a whole S^T or dP^T row
+// (128 values) next to its P^T row, warpgroup 1 a whole dQ_i row
+constexpr uint32_t kRegsWg0 = 216, kRegsWg1 = 184, kRegsWg2 = 104;
+static_assert(kRegsWg0 + kRegsWg1 + kRegsWg2 <= 3 * 168, "register split exceeds the launch share");
 constexpr int kBwdHeadGroup = 4;    // (sequence, head) units scheduled together
 constexpr int kBoxB = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
@@ -56,11 +65,11 @@ struct alignas(1024) BwdSmem {
     // one 128-row x 32-column fp32 slice of dQ_i on its way to the
     // accumulator (128-byte swizzle, as the reduce's tensor map reads it)
     float dq_stage[kBT * 32];
-    float lse2[2][kBT];            // log2-domain statistics of the tile's rows
-    float dsum[2][kBT];            // D of the tile's rows
+    float nlse2[2][kBT];           // -(log2-domain statistics) of the tile's rows
+    float ndsum[2][kBT];           // -D of the tile's rows
     uint64_t kv_full;
     uint64_t in_full[2], in_free[2];  // Q/dO/statistics slot loaded / released
-    uint64_t s_full, p_full, dp_full, ds_full, dq_full, dq_free;
+    uint64_t s_full, p_full, dp_full, dv_done, ds_full, dq_full, dq_free;
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -183,6 +192,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.p_full, kBT);
         mbar_init(&sm.dp_full, 1);
+        mbar_init(&sm.dv_done, 1);
         mbar_init(&sm.ds_full, kBT);
         mbar_init(&sm.dq_full, 1);
         mbar_init(&sm.dq_free, kBT);
@@ -199,6 +209,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
+    if (warp >= 8) regs_dec<kRegsWg2>();
     if (warp == 9) {
         // ================= TMA producer (+ per-tile statistics) =================
         auto load2 = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row) {
@@ -234,8 +245,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int r = lane * 4 + e, qr = q0 + r;
                 const bool in = qr < p.N;
                 const int64_t gi = static_cast<int64_t>(bh) * p.N + qr;
-                sm.lse2[s][r] = in ? p.lse2[gi] : INFINITY;  // rows past N: P = 0
-                sm.dsum[s][r] = in ? p.dsum[gi] : 0.f;
+                sm.nlse2[s][r] = in ? -p.lse2[gi] : -INFINITY;  // rows past N: P = 0
+                sm.ndsum[s][r] = in ? -p.dsum[gi] : 0.f;
             }
             mbar_arrive(&sm.in_full[s]);
             issued = t + 1;
@@ -279,6 +290,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     mma_ts(tmem + col, tmem + acol + kk * 8, dmn(b_lo, kk * 128), idesc_tm,
                            (acc || kk > 0) ? 1u : 0u);
             };
+            // D[col] (+)= A (K-major rows of a) * B (MN-major rows) over 128
+            auto issue_sm = [&](uint32_t col, uint32_t a_lo, uint32_t b_lo, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < kBT / 16; ++kk)
+                    mma_ss(tmem + col, dk_(a_lo, (kk >> 2) * (kBoxB >> 4) + (kk & 3) * 2),
+                           dmn(b_lo, kk * 128), idesc_tm, (acc || kk > 0) ? 1u : 0u);
+            };
             // D[col] = A (MN-major) * B (MN-major) over 128
             auto issue_mm = [&](uint32_t col, uint32_t a_lo, uint32_t b_lo) {
 #pragma unroll
@@ -287,15 +305,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            kk > 0 ? 1u : 0u);
             };
             const uint32_t k_lo = lo(sm.k), v_lo = lo(sm.v);
-            // S^T of the next tile is issued as soon as dP^T of this one is:
-            // the tensor pipe computes it while warpgroup 0 forms dS^T (the
-            // columns it overwrites held P^T, read by dV just before)
+            // Per tile: dV once P^T is in TMEM, then the next tile's S^T, dQ_i
+            // and dK once dS is in shared memory, then the next tile's dP^T
+            // once dQ_i has been read out of the columns it shares;
+            // warpgroup 0 forms dS while dV and the next S^T run
             bool ok = mbar_wait(&sm.kv_full, 0, err, FA_DEVERR_TIMEOUT, abort) &&
                       mbar_wait(&sm.in_full[0], 0, err, FA_DEVERR_TIMEOUT, abort);
             if (ok) {
                 tc_fence_after();
                 issue_kk(kColS, k_lo, lo(sm.q[0]));  // S^T = K Q_0^T
                 tc_commit(&sm.s_full);
+                issue_kk(kColDP, v_lo, lo(sm.dout[0]));  // dP^T = V dO_0^T
+                tc_commit(&sm.dp_full);
             }
             for (int t = 0; ok && t < nt; ++t) {
                 const int s = t & 1;
@@ -304,26 +325,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!mbar_wait(&sm.p_full, ph, err, FA_DEVERR_TIMEOUT, abort)) break;
                 tc_fence_after();
                 issue_tm(kColDV, kColS, do_lo, t > 0);  // dV += P^T dO_i
-                if (t > 0 && !mbar_wait(&sm.dq_free, (t - 1) & 1, err, FA_DEVERR_TIMEOUT, abort))
-                    break;
-                tc_fence_after();
-                issue_kk(kColDP, v_lo, do_lo);  // dP^T = V dO_i^T
-                tc_commit(&sm.dp_full);
+                tc_commit(&sm.dv_done);                 // dO_i's last reader before dS
+                const int s1 = (t + 1) & 1;
                 if (t + 1 < nt) {
-                    const int s1 = (t + 1) & 1;
+                    // S^T of the next tile (its columns held P^T, read by dV above)
                     if (!mbar_wait(&sm.in_full[s1], ((t + 1) >> 1) & 1, err, FA_DEVERR_TIMEOUT,
                                    abort))
                         break;
                     tc_fence_after();
-                    issue_kk(kColS, k_lo, lo(sm.q[s1]));  // S^T of the next tile
+                    issue_kk(kColS, k_lo, lo(sm.q[s1]));
                     tc_commit(&sm.s_full);
                 }
                 if (!mbar_wait(&sm.ds_full, ph, err, FA_DEVERR_TIMEOUT, abort)) break;
                 tc_fence_after();
-                issue_tm(kColDK, kColDP, q_lo, t > 0);  // dK += dS^T Q_i
-                issue_mm(kColDP, do_lo, k_lo);          // dQ_i = dS K (dS in the dO_i slot)
+                issue_mm(kColDP, do_lo, k_lo);  // dQ_i = dS K (dS in the dO_i slot)
                 tc_commit(&sm.dq_full);
+                issue_sm(kColDK, do_lo, q_lo, t > 0);  // dK += dS^T Q_i, same tile K-major
                 tc_commit(&sm.in_free[s]);
+                if (t + 1 < nt) {
+                    // dP^T of the next tile, once dQ_i has left its columns
+                    if (!mbar_wait(&sm.dq_free, ph, err, FA_DEVERR_TIMEOUT, abort)) break;
+                    tc_fence_after();
+                    issue_kk(kColDP, v_lo, lo(sm.dout[s1]));
+                    tc_commit(&sm.dp_full);
+                }
             }
             // every MMA issued must be complete before TMEM is freed
             tc_commit(&sm.drain);
@@ -332,6 +357,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncwarp();
     } else if (warp < 4) {
         // ================= warpgroup 0: P^T and dS^T, one thread per key =================
+        regs_inc<kRegsWg0>();
         const int r = threadIdx.x;  // TMEM lane == key row of the block
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         const int key = key0 + r;
@@ -347,76 +373,108 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // P^T = 2^(scale log2e S^T - lse2); keys past N, queries past N
             // (lse2 = +inf) and, on the diagonal, keys after the query give 0
             uint32_t pk[kBT / 2];
+            {
+                uint32_t x[kBT];  // the whole S^T row, one wait for all four loads
 #pragma unroll
-            for (int c = 0; c < kBT / 32; ++c) {
-                uint32_t x[32];
-                tmem_ld32(tmem + lane_off + kColS + c * 32, x);
+                for (int c = 0; c < kBT / 32; ++c)
+                    tmem_ld32(tmem + lane_off + kColS + c * 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
                 tmem_wait_ld();
-                const float4* l4 = reinterpret_cast<const float4*>(&sm.lse2[s][c * 32]);
+                const float4* l4 = reinterpret_cast<const float4*>(sm.nlse2[s]);
+                const uint64_t sl2 = f2_pack(sl, sl);
+                if (key_in && !diag) {
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 lv = l4[e4];
-                    const float ls[4] = {lv.x, lv.y, lv.z, lv.w};
-                    float pv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = e4 * 4 + u;
-                        float v = ex2_approx(fmaf(__uint_as_float(x[e]), sl, -ls[u]));
-                        if (!key_in || (diag && key > q0 + c * 32 + e)) v = 0.f;
-                        pv[u] = v;
+                    for (int e4 = 0; e4 < kBT / 4; ++e4) {
+                        const float4 lv = l4[e4];
+                        const uint64_t a = f2_fma(f2_pack(__uint_as_float(x[4 * e4]),
+                                                          __uint_as_float(x[4 * e4 + 1])),
+                                                  sl2, f2_pack(lv.x, lv.y));
+                        const uint64_t b = f2_fma(f2_pack(__uint_as_float(x[4 * e4 + 2]),
+                                                          __uint_as_float(x[4 * e4 + 3])),
+                                                  sl2, f2_pack(lv.z, lv.w));
+                        pk[e4 * 2] = pack_bf16x2(ex2_approx(f2_lo(a)), ex2_approx(f2_hi(a)));
+                        pk[e4 * 2 + 1] = pack_bf16x2(ex2_approx(f2_lo(b)), ex2_approx(f2_hi(b)));
                     }
-                    pk[c * 16 + e4 * 2] = pack_bf16x2(pv[0], pv[1]);
-                    pk[c * 16 + e4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                } else {
+#pragma unroll
+                    for (int e4 = 0; e4 < kBT / 4; ++e4) {
+                        const float4 lv = l4[e4];
+                        const float ls[4] = {lv.x, lv.y, lv.z, lv.w};
+                        float pv[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = e4 * 4 + u;
+                            float v = ex2_approx(fmaf(__uint_as_float(x[e]), sl, ls[u]));
+                            if (!key_in || (diag && key > q0 + e)) v = 0.f;
+                            pv[u] = v;
+                        }
+                        pk[e4 * 2] = pack_bf16x2(pv[0], pv[1]);
+                        pk[e4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                    }
                 }
-                // columns [16c, 16c+16) were read by this or the previous chunk
-                tmem_st16(tmem + lane_off + kColS + c * 16, &pk[c * 16]);
             }
+            tmem_st32(tmem + lane_off + kColS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(tmem + lane_off + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full);
-            // dS^T = P^T o (dP^T - D); to TMEM for dK and, transposed, to the
-            // dO_i slot for dQ (dV and dP^T, its readers, have completed)
+            // dS^T = P^T o (dP^T - D), packed over pk; written transposed
+            // (row = key) into the dO_i slot once dV, the slot's last reader
+            // (dP^T has completed), is done: dQ_i reads it as dS (MN-major),
+            // dK as dS^T (K-major)
             if (!bwd_warp_wait(&sm.dp_full, ph, err, abort)) break;
             tc_fence_after();
+            {
+                uint32_t y[kBT];
+#pragma unroll
+                for (int c = 0; c < kBT / 32; ++c)
+                    tmem_ld32(tmem + lane_off + kColDP + c * 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(&y[c * 32]));
+                tmem_wait_ld();
+                const float4* d4 = reinterpret_cast<const float4*>(sm.ndsum[s]);
+#pragma unroll
+                for (int e4 = 0; e4 < kBT / 4; ++e4) {
+                    const float4 dv4 = d4[e4];
+                    const int e = e4 * 4;
+                    const uint32_t w0 = pk[e4 * 2], w1 = pk[e4 * 2 + 1];
+                    const uint64_t a = f2_mul(f2_add(f2_pack(__uint_as_float(y[e]),
+                                                             __uint_as_float(y[e + 1])),
+                                                     f2_pack(dv4.x, dv4.y)),
+                                              f2_pack(__uint_as_float(w0 << 16),
+                                                      __uint_as_float(w0 & 0xffff0000u)));
+                    const uint64_t b = f2_mul(f2_add(f2_pack(__uint_as_float(y[e + 2]),
+                                                             __uint_as_float(y[e + 3])),
+                                                     f2_pack(dv4.z, dv4.w)),
+                                              f2_pack(__uint_as_float(w1 << 16),
+                                                      __uint_as_float(w1 & 0xffff0000u)));
+                    pk[e4 * 2] = pack_bf16x2(f2_lo(a), f2_hi(a));
+                    pk[e4 * 2 + 1] = pack_bf16x2(f2_lo(b), f2_hi(b));
+                }
+            }
+            // every thread has read its dP^T row: dQ_i may overwrite it once
+            // ds_full completes
+            if (!bwd_warp_wait(&sm.dv_done, ph, err, abort)) break;
+            // row r of the dS tile: queries [32c, 32c+32) are box c/2, 16-byte
+            // chunks (c%2)*4 .. +3 of the 128-byte row, 128-byte swizzle
             uint8_t* ds_tile = sm.dout[s];
 #pragma unroll
             for (int c = 0; c < kBT / 32; ++c) {
-                uint32_t y[32];
-                tmem_ld32(tmem + lane_off + kColDP + c * 32, y);
-                tmem_wait_ld();
-                const float4* d4 = reinterpret_cast<const float4*>(&sm.dsum[s][c * 32]);
-                uint32_t dk2[16];
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 dv4 = d4[e4];
-                    const float dd[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-                    float p0, p1, p2, p3;
-                    unpack_bf16x2(pk[c * 16 + e4 * 2], p0, p1);
-                    unpack_bf16x2(pk[c * 16 + e4 * 2 + 1], p2, p3);
-                    const int e = e4 * 4;
-                    dk2[e4 * 2] = pack_bf16x2(p0 * (__uint_as_float(y[e]) - dd[0]),
-                                              p1 * (__uint_as_float(y[e + 1]) - dd[1]));
-                    dk2[e4 * 2 + 1] = pack_bf16x2(p2 * (__uint_as_float(y[e + 2]) - dd[2]),
-                                                  p3 * (__uint_as_float(y[e + 3]) - dd[3]));
-                }
-                tmem_st16(tmem + lane_off + kColDP + c * 16, dk2);
-                // row r of the dS tile, queries [32c, 32c+32): box c/2, chunks
-                // (c%2)*4 .. +3 of the 128-byte row, 128-byte swizzle
                 uint8_t* row = ds_tile + (c >> 1) * kBoxB + r * 128;
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int chunk = (c & 1) * 4 + h;
+                    const uint32_t* w = &pk[c * 16 + h * 4];
                     *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) * 16)) =
-                        make_uint4(dk2[h * 4], dk2[h * 4 + 1], dk2[h * 4 + 2], dk2[h * 4 + 3]);
+                        make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            tmem_wait_st();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             mbar_arrive(&sm.ds_full);
         }
-    } else {
+    } else if (warp < 8) {
         // ================= warpgroup 1: dQ_i accumulation, then dK and dV =================
+        regs_inc<kRegsWg1>();
         const int r = threadIdx.x - 128;
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
