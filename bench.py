@@ -253,24 +253,35 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
     reported beside the headline number, not part of the timed step."""
     out = {}
 
-    def timed(fn, flops, name, extra=None):
+    def timed(fn, flops, name, extra=None, n=steps):
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(steps):
+        for _ in range(n):
             fn()
         e1.record(stream)
         torch.cuda.synchronize()
         if fa.fa_get_device_error() != fa.FA_OK:
             raise RuntimeError(f"device error on {name}")
-        ms = e0.elapsed_time(e1) / steps
+        ms = e0.elapsed_time(e1) / n
         d = {"ms_per_launch": ms, "tflops": flops / (ms * 1e-3) / 1e12,
              "pct_of_2250": 100 * flops / (ms * 1e-3) / 1e12 / DATASHEET_BF16_TFLOPS}
         d.update(extra or {})
         out[name] = d
 
+    # the headline forward alone in a short burst after an idle pause: the
+    # power controller has not yet brought the clock down (the headline value
+    # is the sustained rate of the long timed region)
+    q, k, v = W.fwd_inputs(FWD, device="cuda")[:3]
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    time.sleep(0.5)
+    timed(lambda: fa.fa_fwd(q, k, v, FWD.causal, 1 / math.sqrt(FWD.d), o=o, lse=lse,
+                            stream=stream),
+          fwd_flops(FWD), FWD.name + "_burst20", {"what": "20 launches after 0.5 s idle"}, n=20)
+    del q, k, v, o, lse
     for w in (W.TINY_CAUSAL, W.BATCHED, W.CTX128K):
         q, k, v = W.fwd_inputs(w, device="cuda")[:3]
         o = torch.empty_like(q)
@@ -497,40 +508,73 @@ def run_native(args, world, rank, local):
         per_launch_gbs = dbytes / (dec_sum / args.steps * 1e-3) / 1e9
 
     # ---- end to end through the public API, host buffers ------------------
+    # Every step copies its q, k, v from pinned host memory, runs fa_fwd and
+    # copies o and lse back.  Two sets of device buffers and three streams let
+    # step i+1's host-to-device copies run while step i computes and its
+    # results travel back (PCIe is full duplex); events order each buffer's
+    # reuse.
     e2e = None
     if do_fwd and not args.no_e2e:
-        e2e_steps = max(1, min(args.steps, 5))
+        e2e_steps = max(1, min(args.steps, 8))
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
+        hl = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+        dbuf = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(o),
+                 torch.empty_like(lse)) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        used = [False, False]
 
-        def e2e_step():
-            dq2.copy_(hq, non_blocking=True)
-            dk2.copy_(hk, non_blocking=True)
-            dv2.copy_(hv, non_blocking=True)
-            fa.fa_fwd(dq2, dk2, dv2, FWD.causal, scale, o=o, lse=lse, stream=stream)
-            ho.copy_(o, non_blocking=True)
-            hl.copy_(lse, non_blocking=True)
+        def e2e_step(i):
+            b = i & 1
+            dq2, dk2, dv2, do2, dl2 = dbuf[b]
+            if used[b]:
+                s_in.wait_event(comp_done[b])      # step i-2 has read this buffer's inputs
+                stream.wait_event(out_done[b])     # and its outputs have gone back
+            with torch.cuda.stream(s_in):
+                dq2.copy_(hq, non_blocking=True)
+                dk2.copy_(hk, non_blocking=True)
+                dv2.copy_(hv, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            fa.fa_fwd(dq2, dk2, dv2, FWD.causal, scale, o=do2, lse=dl2, stream=stream)
+            comp_done[b].record(stream)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                ho[b].copy_(do2, non_blocking=True)
+                hl[b].copy_(dl2, non_blocking=True)
+                out_done[b].record(s_out)
+            used[b] = True
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        s_in.wait_event(e0)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        s_out.wait_event(out_done[0])
+        s_out.wait_event(out_done[1])
+        e1.record(s_out)
         torch.cuda.synchronize()
         barrier(world)
         (e2e_ms,) = reduce_max([e0.elapsed_time(e1)], world)
+        # the results that came back are the device pass's, bit for bit
+        last = (e2e_steps - 1) & 1
+        if not (torch.equal(ho[last], o.cpu()) and torch.equal(hl[last], lse.cpu())):
+            raise RuntimeError("end-to-end outputs differ from the device-resident pass")
         e2e = {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
-               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
+               "d2h_bytes_per_step": ho[0].numel() * ho[0].element_size() +
+                                     hl[0].numel() * hl[0].element_size(),
                "steps": e2e_steps,
-               "what": "fa_fwd through the Python binding, q/k/v copied from pinned host "
-                       "memory and o/lse copied back inside the timed region"}
+               "what": "fa_fwd through the Python binding; every step copies q/k/v from pinned "
+                       "host memory and o/lse back inside the timed region, two steps in "
+                       "flight (copies in, compute and copies out on three streams)"}
 
     secondary = None
     if do_fwd and not args.no_secondary:
