@@ -177,6 +177,12 @@ def reduce_max(values, world):
     return t.cpu().tolist()
 
 
+def job_rate(world: int, work_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the work every rank did (ranks are replicas of
+    the same step) over the slowest rank's time, in work units per second."""
+    return world * work_per_rank_step * steps / (max_ms * 1e-3)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -499,12 +505,12 @@ def run_native(args, world, rank, local):
     fwd_sum, dec_sum, total_ms = reduce_max([sum(fwd_ms), sum(dec_ms), total_ms], world)
 
     flops = fwd_flops()
-    fwd_tflops = world * flops * args.steps / (fwd_sum * 1e-3) / 1e12 if do_fwd else None
+    fwd_tflops = job_rate(world, flops, args.steps, fwd_sum) / 1e12 if do_fwd else None
     per_launch_tf = flops / (fwd_sum / args.steps * 1e-3) / 1e12 if do_fwd else None
     if do_dec:
         dbytes = decode_bytes(cache.seq_lens.tolist(), DEC.H, DEC.d, cache.q.shape[0],
                               H_kv=h_kv)
-        dec_gbs = world * dbytes * args.steps / (dec_sum * 1e-3) / 1e9
+        dec_gbs = job_rate(world, dbytes, args.steps, dec_sum) / 1e9
         per_launch_gbs = dbytes / (dec_sum / args.steps * 1e-3) / 1e9
 
     # ---- end to end through the public API, host buffers ------------------
@@ -567,7 +573,7 @@ def run_native(args, world, rank, local):
         last = (e2e_steps - 1) & 1
         if not (torch.equal(ho[last], o.cpu()) and torch.equal(hl[last], lse.cpu())):
             raise RuntimeError("end-to-end outputs differ from the device-resident pass")
-        e2e = {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_rate(world, flops, e2e_steps, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
                "d2h_bytes_per_step": ho[0].numel() * ho[0].element_size() +
                                      hl[0].numel() * hl[0].element_size(),
