@@ -280,14 +280,6 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
         : "memory");
 }
 
-// ... and on the mbarrier at the same offset in both CTAs of the pair
-__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(bar), "h"(static_cast<uint16_t>(3))
-        : "memory");
-}
-
 // D[tmem] (+)= A[smem desc] * B[smem desc]
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {

@@ -556,7 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // barrier and, for a pair, to the same barrier of the odd CTA
             auto commit = [&](uint64_t* bar) {
                 if constexpr (PAIR) {
-                    tc_commit_pair_both(smem_u32(bar));
+                    tc_commit_pair(smem_u32(bar));
+                    tc_commit_pair(mapa_rank(smem_u32(bar), 1));
                 } else {
                     tc_commit(bar);
                 }
