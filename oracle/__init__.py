@@ -48,6 +48,9 @@ def lib():
         L.oracle_attention_gqa.restype = ctypes.c_int
         L.oracle_decode_paged_gqa.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64]
         L.oracle_decode_paged_gqa.restype = ctypes.c_int
+        L.oracle_decode_paged_strided.argtypes = [P, P, P, P, I64, P, P, P, I64, I64, I64,
+                                                  I64, I64]
+        L.oracle_decode_paged_strided.restype = ctypes.c_int
         L.oracle_append_paged.argtypes = [P, P, P, P, P, I64, I64, I64, I64]
         L.oracle_append_paged.restype = ctypes.c_int
         L.oracle_prefill_paged.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64,
@@ -205,6 +208,26 @@ def decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: int):
                                        _ptr(o), _ptr(lse), B, H, Hkv, d, page_size)
     if rc != 0:
         raise RuntimeError(f"oracle_decode_paged_gqa failed ({rc})")
+    return o, lse
+
+
+def decode_paged_strided(q, k_pages, v_pages, block_table, seq_lens, page_size: int):
+    """Single-token decode through a block table [B, max_pages] (sequence b's
+    k-th page at block_table[b, k]; entries past its pages unused): q [B,H,d],
+    pages [P,Hkv,page_size,d]; returns (o [B,H,d], lse [B,H]).  Scale 1/sqrt(d)."""
+    q = _f64(q)
+    kp, vp = _f64(k_pages), _f64(v_pages)
+    bt, sl = _i64(block_table), _i64(seq_lens)
+    B, H, d = q.shape
+    Hkv = kp.shape[1]
+    assert bt.ndim == 2 and bt.shape[0] == B and H % Hkv == 0
+    o = np.zeros((B, H, d))
+    lse = np.zeros((B, H))
+    rc = lib().oracle_decode_paged_strided(_ptr(q), _ptr(kp), _ptr(vp), _ptr(bt), bt.shape[1],
+                                           _ptr(sl), _ptr(o), _ptr(lse), B, H, Hkv, d,
+                                           page_size)
+    if rc != 0:
+        raise RuntimeError(f"oracle_decode_paged_strided failed ({rc})")
     return o, lse
 
 

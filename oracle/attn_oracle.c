@@ -37,7 +37,9 @@
  * (256 tokens by default), each page a contiguous K (or V) slice, and a
  * sequence owns a list of pages.  The oracle first gathers a sequence's
  * pages back into a contiguous [len, d] array per head, then applies the
- * definition above with a single query row and no mask.
+ * definition above with a single query row and no mask.  A sequence's page
+ * list is read either from a packed table (sequences' lists back to back) or
+ * from its own fixed-width row of a block table.
  *
  * Parallelism: OpenMP over independent output rows.  Each row is computed by
  * one thread in a fixed order, so results do not depend on the thread count.
@@ -381,6 +383,65 @@ int oracle_decode_paged_gqa(const double *q, const double *k_pages,
         free(kc);
         free(vc);
         off += np;
+    }
+    return rc;
+}
+
+/* Single-token decode through a block table: one row of max_pages entries
+ * per sequence, sequence b's k-th page being block_table[b * max_pages + k]
+ * (the "page table per sequence" of the paged cache on the page
+ * "“Flash”不是那个被时代淘汰的插件", 0539edu.com, section 2, kept as a
+ * fixed-width row; entries past a sequence's pages are not read).  q, o are
+ * [B,H,d], the pages [P_pool, Hkv, page_size, d]; query head h of sequence b
+ * attends to K/V head h / (H / Hkv) of its seq_lens[b] cached tokens, which
+ * must fit its row (seq_lens[b] <= max_pages * page_size).  lse (optional)
+ * is [B,H]. */
+int oracle_decode_paged_strided(const double *q, const double *k_pages,
+                                const double *v_pages, const int64_t *block_table,
+                                int64_t max_pages, const int64_t *seq_lens, double *o,
+                                double *lse, int64_t B, int64_t H, int64_t Hkv, int64_t d,
+                                int64_t page_size) {
+    if (page_size <= 0 || d <= 0 || H < 0 || B < 0 || Hkv <= 0 || H % Hkv != 0 ||
+        max_pages < 0)
+        return -1;
+    const int64_t group = H / Hkv;
+    int rc = 0;
+    for (int64_t b = 0; b < B && rc == 0; ++b) {
+        const int64_t len = seq_lens[b];
+        if (len < 0 || len > max_pages * page_size) return -1;
+        double *kc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * Hkv * d));
+        double *vc = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * Hkv * d));
+        if (!kc || !vc) {
+            free(kc);
+            free(vc);
+            return -2;
+        }
+        /* the sequence's row is a one-sequence packed table */
+        oracle_gather_paged(k_pages, block_table + b * max_pages, &len, kc, 1, Hkv, d, page_size);
+        oracle_gather_paged(v_pages, block_table + b * max_pages, &len, vc, 1, Hkv, d, page_size);
+        int failed = 0;
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+            if (!srow) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+#pragma omp for schedule(static)
+                for (int64_t h = 0; h < H; ++h) {
+                    const int64_t g = h / group;
+                    double l;
+                    attention_row(q + (b * H + h) * d, kc + g * d, Hkv * d, vc + g * d,
+                                  Hkv * d, len, d, d, 1.0 / sqrt((double)d), srow,
+                                  o + (b * H + h) * d, &l);
+                    if (lse) lse[b * H + h] = l;
+                }
+                free(srow);
+            }
+        }
+        if (failed) rc = -2;
+        free(kc);
+        free(vc);
     }
     return rc;
 }

@@ -494,6 +494,74 @@ def test_decode_gqa_equals_brute_force():
             assert abs(lse[b, h] - lb[0]) < TOL
 
 
+def _block_table(table, lens, page_size, max_pages, pad):
+    """The packed table's pages laid out one row of max_pages per sequence,
+    unused entries set to `pad`."""
+    bt = np.full((len(lens), max_pages), pad, dtype=np.int64)
+    off = 0
+    for b, L in enumerate(lens):
+        n = (L + page_size - 1) // page_size
+        bt[b, :n] = table[off:off + n]
+        off += n
+    return bt
+
+
+def test_decode_strided_equals_brute_force():
+    """Decode through a block table: each sequence reads its own row; the
+    padding entries point at a NaN-filled page and are never read."""
+    H, Hkv, d, page_size = 4, 2, 8, 4
+    lens = [1, 7, 12, 0, 4]
+    kseqs = [_rand((L, Hkv, d), 160 + i) for i, L in enumerate(lens)]
+    vseqs = [_rand((L, Hkv, d), 170 + i) for i, L in enumerate(lens)]
+    n_pool = sum((L + page_size - 1) // page_size for L in lens) + 1  # last page: spare
+    kpool, table, sl = _append_simulation(kseqs, Hkv, d, page_size, n_pool, 161)
+    vpool, _, _ = _append_simulation(vseqs, Hkv, d, page_size, n_pool, 161)
+    spare = sorted(set(range(n_pool)) - set(table.tolist()))[0]
+    assert np.all(np.isnan(kpool[spare]))
+    bt = _block_table(table, lens, page_size, 5, spare)
+    q = _rand((len(lens), H, d), 162)
+    o, lse = oracle.decode_paged_strided(q, kpool, vpool, bt, sl, page_size)
+    g = H // Hkv
+    for b, L in enumerate(lens):
+        for h in range(H):
+            if L == 0:
+                assert np.all(o[b, h] == 0) and np.isneginf(lse[b, h])
+                continue
+            ob, lb = _mp_attention(q[b, h][None], kseqs[b][:, h // g], vseqs[b][:, h // g],
+                                   False, 1 / math.sqrt(d))
+            np.testing.assert_allclose(o[b, h], ob[0], atol=TOL)
+            assert abs(lse[b, h] - lb[0]) < TOL
+
+
+def test_decode_strided_equals_packed_decode():
+    """The same pages listed one row per sequence or back to back give the same
+    decode; a row index slip (reading row b+1) would not."""
+    H, d, page_size = 3, 8, 4
+    lens = [9, 3, 16]
+    kseqs = [_rand((L, H, d), 180 + i) for i, L in enumerate(lens)]
+    vseqs = [_rand((L, H, d), 190 + i) for i, L in enumerate(lens)]
+    n_pool = sum((L + page_size - 1) // page_size for L in lens)
+    kpool, table, sl = _append_simulation(kseqs, H, d, page_size, n_pool, 181)
+    vpool, _, _ = _append_simulation(vseqs, H, d, page_size, n_pool, 181)
+    bt = _block_table(table, lens, page_size, 6, 0)
+    q = _rand((len(lens), H, d), 182)
+    o1, l1 = oracle.decode_paged_strided(q, kpool, vpool, bt, sl, page_size)
+    o2, l2 = oracle.decode_paged(q, kpool, vpool, table, sl, page_size)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, atol=1e-13)
+    shifted = np.roll(bt, 1, axis=0)  # each sequence reading its neighbour's row
+    o3, _ = oracle.decode_paged_strided(q, kpool, vpool, shifted, [3, 9, 3], page_size)
+    assert np.abs(o3 - o1).max() > 1e-3
+
+
+def test_decode_strided_rejects_a_row_overflow():
+    H, d, page_size = 1, 4, 4
+    pool = _rand((2, H, page_size, d), 195)
+    with pytest.raises(RuntimeError):
+        oracle.decode_paged_strided(_rand((1, H, d), 196), pool, pool, np.array([[0, 1]]),
+                                    [9], page_size)
+
+
 # -- appending to the paged cache and prefill through it (page
 #    "“Flash”不是那个被时代淘汰的插件", 0539edu.com, section 2) ------------------
 
