@@ -382,12 +382,17 @@ int fa_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
 
 namespace {
 // num_pages = 0x7fffffff: the pool size is unknown (fa_decode_paged's
-// signature has none), page indices are not bounded.
+// signature has none), page indices are not bounded.  max_pages > 0: the
+// table is a block table [B, max_pages], packed into the workspace first.
 int decode_impl(const void* q, const void* k_pages, const void* v_pages,
                 const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
-                int H_kv, int num_pages, int d, int page_size, fa_stream_t stream) {
+                int H_kv, int num_pages, int d, int page_size, fa_stream_t stream,
+                int max_pages = 0) {
     if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !o) return FA_ERR_NULL;
     if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || num_pages < 1) return FA_ERR_SHAPE;
+    if (max_pages < 0 || static_cast<int64_t>(B) * max_pages > 0x7fffffff ||
+        static_cast<int64_t>(max_pages) * page_size > 0x7fffffff)
+        return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (page_size != 256) return FA_ERR_UNSUPPORTED;
     if (!fa::decode_group_supported(H, H_kv)) return FA_ERR_UNSUPPORTED;
@@ -411,14 +416,27 @@ int decode_impl(const void* q, const void* k_pages, const void* v_pages,
         if ((rc = make_map(&tv, v_pages, dims, strides, box)) != FA_OK) return rc;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t dec_bytes =
+        (fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits) + 255) & ~static_cast<size_t>(255);
+    // block table: the packed table and the cut lengths follow the decode's own workspace
+    const size_t pack_bytes =
+        max_pages > 0 ? (static_cast<size_t>(B) * max_pages + B) * sizeof(int32_t) : 0;
     void* ws = nullptr;
-    if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits), st,
-                               &ws)) != FA_OK)
-        return rc;
+    if ((rc = ensure_workspace(s, dec_bytes + pack_bytes, st, &ws)) != FA_OK) return rc;
+    const int32_t* table = page_table;
+    const int32_t* lens = seq_lens;
+    if (max_pages > 0) {
+        int32_t* packed = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + dec_bytes);
+        int32_t* cut = packed + static_cast<size_t>(B) * max_pages;
+        if ((rc = fa::launch_decode_pack(page_table, max_pages, seq_lens, B, page_size, packed,
+                                         cut, s->err, st)) != FA_OK)
+            return rc;
+        table = packed;
+        lens = cut;
+    }
     return fa::launch_decode(q, k_pages, v_pages, grouped ? &tk : nullptr,
-                             grouped ? &tv : nullptr, page_table, seq_lens, o, B, H, H_kv,
-                             num_pages, d, page_size, fa::kDecodeMaxSplits, ws, s->err,
-                             s->num_sms, st);
+                             grouped ? &tv : nullptr, table, lens, o, B, H, H_kv, num_pages, d,
+                             page_size, fa::kDecodeMaxSplits, ws, s->err, s->num_sms, st);
 }
 }  // namespace
 
@@ -437,6 +455,15 @@ int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v_pages,
                         fa_stream_t stream) {
     return decode_impl(q, k_pages, v_pages, page_table, seq_lens, o, B, H, H_kv, num_pages, d,
                        page_size, stream);
+}
+
+int fa_decode_paged_strided(const void* q, const void* k_pages, const void* v_pages,
+                            const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                            void* o, int B, int H, int H_kv, int num_pages, int d, int page_size,
+                            fa_stream_t stream) {
+    if (max_pages < 1) return block_table ? FA_ERR_SHAPE : FA_ERR_NULL;
+    return decode_impl(q, k_pages, v_pages, block_table, seq_lens, o, B, H, H_kv, num_pages, d,
+                       page_size, stream, max_pages);
 }
 
 int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t* seq_lens,

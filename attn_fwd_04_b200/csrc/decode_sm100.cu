@@ -129,6 +129,46 @@ __global__ void __launch_bounds__(kPlanThreads)
     }
 }
 
+// A block table [B, max_pages] (sequence b's k-th page at row b, entry k)
+// turned into what the decode kernels read: the used entries of every row,
+// back to back (the packed table), and the lengths.  A negative length is
+// reported and taken as 0; a length beyond its row (max_pages * page_size
+// tokens) is reported and cut to the row, so no entry outside the table is
+// read.  One CTA.
+__global__ void __launch_bounds__(kPlanThreads)
+    fa_decode_pack_kernel(const int32_t* __restrict__ block_table, int max_pages,
+                          const int32_t* __restrict__ seq_lens, int B, int page_size,
+                          int32_t* __restrict__ packed, int32_t* __restrict__ lens,
+                          unsigned int* err) {
+    __shared__ int sh[32];
+    const int64_t cap = static_cast<int64_t>(max_pages) * page_size;
+    int carry = 0;
+    for (int base = 0; base < B; base += kPlanThreads) {
+        const int i = base + threadIdx.x;
+        int len = 0;
+        if (i < B) {
+            len = seq_lens[i];
+            if (len < 0) {
+                record_error(err, FA_DEVERR_BAD_INPUT);
+                len = 0;
+            } else if (len > cap) {
+                record_error(err, FA_DEVERR_BAD_INPUT);
+                len = static_cast<int>(cap);
+            }
+        }
+        const int np = (len + page_size - 1) / page_size;
+        int tot;
+        const int inc = block_incl_scan(np, sh, tot);
+        if (i < B) {
+            lens[i] = len;
+            const int32_t* row = block_table + static_cast<int64_t>(i) * max_pages;
+            int32_t* dst = packed + carry + inc - np;
+            for (int k = 0; k < np; ++k) dst[k] = __ldg(row + k);
+        }
+        carry += tot;
+    }
+}
+
 // Largest b in [0, B) with off[b] <= x (off non-decreasing, off[0] = 0).
 __device__ __forceinline__ int find_owner(const int32_t* off, int B, int x) {
     int lo = 0, hi = B - 1;
@@ -895,6 +935,14 @@ int launch_append(const void* k_new, const void* v_new, const int32_t* cu_new, v
 
 size_t decode_workspace_bytes(int B, int H, int d, int max_splits) {
     return layout_of(B, H, d, max_splits).total;
+}
+
+int launch_decode_pack(const int32_t* block_table, int max_pages, const int32_t* seq_lens, int B,
+                       int page_size, int32_t* packed, int32_t* lens, unsigned int* err,
+                       cudaStream_t stream) {
+    fa_decode_pack_kernel<<<1, kPlanThreads, 0, stream>>>(block_table, max_pages, seq_lens, B,
+                                                          page_size, packed, lens, err);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 namespace {

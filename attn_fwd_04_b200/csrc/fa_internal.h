@@ -78,6 +78,12 @@ int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   cudaStream_t stream);
 bool decode_group_supported(int H, int Hk);
 
+// Block table [B, max_pages] -> packed table `packed` (at most B * max_pages
+// entries) and lengths `lens` [B] cut to each row, for launch_decode.
+int launch_decode_pack(const int32_t* block_table, int max_pages, const int32_t* seq_lens, int B,
+                       int page_size, int32_t* packed, int32_t* lens, unsigned int* err,
+                       cudaStream_t stream);
+
 // The current device's error word and SM count (sm_100 devices only).
 int device_error_word(unsigned int** err, int* num_sms);
 

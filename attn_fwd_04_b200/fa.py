@@ -24,7 +24,8 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged", "fa_decode_paged_gqa",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged",
+           "fa_decode_paged_gqa", "fa_decode_paged_strided",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
@@ -56,6 +57,7 @@ def lib() -> ctypes.CDLL:
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        L.fa_decode_paged_strided.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, I, P]
         L.fa_gather_paged.argtypes = [P, P, P, P, I, I, I, I, P]
         L.fa_append_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_prefill_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P]
@@ -67,7 +69,8 @@ def lib() -> ctypes.CDLL:
         L.fa_version.argtypes = []
         L.fa_fwd_set_cta_pairs.argtypes = [I]
         for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged",
-                     "fa_decode_paged_gqa", "fa_decode_paged_noalloc", "fa_append_paged",
+                     "fa_decode_paged_gqa", "fa_decode_paged_strided", "fa_decode_paged_noalloc",
+                     "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
                      "fa_version", "fa_fwd_set_cta_pairs"):
@@ -255,6 +258,29 @@ def fa_decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: in
                                    B, H, H_kv, k_pages.shape[0], d, int(page_size),
                                    _stream(stream))
     _raise_if(rc, "fa_decode_paged_gqa")
+    return o
+
+
+def fa_decode_paged_strided(q, k_pages, v_pages, block_table, seq_lens, page_size: int = 256,
+                            o=None, stream=None):
+    """Decode through a block table [B, max_pages] int32 (row b lists sequence
+    b's pages): q [B,H,d], pages [P,H_kv,page_size,d] -> o [B,H,d] bf16."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, H, d = q.shape
+    H_kv = k_pages.shape[1]
+    if block_table.shape[0] != B:
+        raise ValueError("block_table must have one row per sequence")
+    if o is None:
+        o = torch.empty_like(q)
+    rc = lib().fa_decode_paged_strided(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                       block_table.data_ptr(), block_table.shape[1],
+                                       seq_lens.data_ptr(), o.data_ptr(), B, H, H_kv,
+                                       k_pages.shape[0], d, int(page_size), _stream(stream))
+    _raise_if(rc, "fa_decode_paged_strided")
     return o
 
 

@@ -225,6 +225,33 @@ FA_API int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v
                     fa_stream_t stream);
 
 /*
+ * fa_decode_paged_strided -- fa_decode_paged_gqa with the page table given
+ * as a block table: one fixed-width row of page indices per sequence (the
+ * page list each sequence owns in the cache of the page "“Flash”不是那个被
+ * 时代淘汰的插件" (0539edu.com), section 2, kept as a [B, max_pages] array,
+ * the layout serving engines usually hold).
+ *   block_table : [B, max_pages] int32, row-major; sequence b's k-th page is
+ *                 block_table[b * max_pages + k]; entries past a sequence's
+ *                 ceil(seq_lens[b] / page_size) pages are not read
+ *   max_pages   : the row width (>= 1; B * max_pages and
+ *                 max_pages * page_size must fit in int32, FA_ERR_SHAPE
+ *                 otherwise)
+ *   q, k_pages, v_pages, seq_lens, o, B, H, H_kv, num_pages, d, page_size:
+ *                 as fa_decode_paged_gqa (H_kv = H for plain multi-head)
+ * A length beyond its row (seq_lens[b] > max_pages * page_size) is reported
+ * as FA_ERR_DEVICE_BAD_INPUT and decoded over the row's tokens only; no
+ * entry outside the table is read.  A first kernel copies the used entries
+ * of every row, back to back, into the library's per-GPU workspace (B *
+ * max_pages + B int32 beyond the decode's own part), then the decode of
+ * fa_decode_paged_gqa runs on that packed table, so results equal
+ * fa_decode_paged_gqa's on the same pages bit for bit.
+ */
+FA_API int fa_decode_paged_strided(const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* block_table, int max_pages,
+                                   const int32_t* seq_lens, void* o, int B, int H, int H_kv,
+                                   int num_pages, int d, int page_size, fa_stream_t stream);
+
+/*
  * fa_append_paged -- write the K and V rows of new tokens into the paged
  * cache: the step before attention in the serving loop of the page "“Flash”
  * 不是那个被时代淘汰的插件" (0539edu.com), section 2 (a new token goes into a

@@ -84,6 +84,11 @@ def decode_gqa(L, q=A, kp=A, vp=A, pt=A, sl=A, o=A, B=4, H=8, H_kv=2, P=64, d=12
     return L.fa_decode_paged_gqa(q, kp, vp, pt, sl, o, B, H, H_kv, P, d, ps, S)
 
 
+def decode_strided(L, q=A, kp=A, vp=A, bt=A, mp=70, sl=A, o=A, B=4, H=8, H_kv=2, P=64, d=128,
+                   ps=256):
+    return L.fa_decode_paged_strided(q, kp, vp, bt, mp, sl, o, B, H, H_kv, P, d, ps, S)
+
+
 def append(L, kn=A, vn=A, cu=A, kp=A, vp=A, pt=A, sl=A, B=2, H_kv=2, total=10, P=8, d=128,
            ps=256):
     return L.fa_append_paged(kn, vn, cu, kp, vp, pt, sl, B, H_kv, total, P, d, ps, S)
@@ -177,6 +182,13 @@ def test_decode_argument_errors(L):
     assert decode_gqa(L, H=32, H_kv=2) == fa.FA_ERR_UNSUPPORTED  # group of 16
     assert decode_gqa(L, ps=128) == fa.FA_ERR_UNSUPPORTED
     assert decode_gqa(L, o=MIS) == fa.FA_ERR_ALIGN
+    assert decode_strided(L, bt=None) == fa.FA_ERR_NULL
+    assert decode_strided(L, mp=0) == fa.FA_ERR_SHAPE
+    assert decode_strided(L, mp=1 << 24) == fa.FA_ERR_SHAPE  # row of 2^32 tokens
+    assert decode_strided(L, B=1 << 10, mp=1 << 22) == fa.FA_ERR_SHAPE  # 2^32 entries
+    assert decode_strided(L, H=24, H_kv=8) == fa.FA_ERR_UNSUPPORTED
+    assert decode_strided(L, ps=128) == fa.FA_ERR_UNSUPPORTED
+    assert decode_strided(L, q=MIS) == fa.FA_ERR_ALIGN
     assert gather(L, out=None) == fa.FA_ERR_NULL
     assert gather(L, ps=255) == fa.FA_ERR_UNSUPPORTED
     assert gather(L, pages=MIS) == fa.FA_ERR_ALIGN
@@ -190,6 +202,7 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
     assert rope_fwd(L) == fa.FA_ERR_CUDA
     assert decode(L) == fa.FA_ERR_CUDA
     assert decode_gqa(L) == fa.FA_ERR_CUDA
+    assert decode_strided(L) == fa.FA_ERR_CUDA
     assert append(L) == fa.FA_ERR_CUDA
     assert prefill(L) == fa.FA_ERR_CUDA
     code = ctypes.c_int(7)

@@ -248,3 +248,74 @@ def test_decode_gqa_page_outside_pool_reported(H, H_kv):
     fa.fa_decode_paged_gqa(c.q, c.k_pages, c.v_pages, pt, c.seq_lens, c.page_size, o=o)
     assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_BAD_INPUT
     assert torch.equal(o[0], good[0]) and torch.equal(o[2], good[2])
+
+
+# -- decode through a block table (fa_decode_paged_strided) -----------------------
+
+def _block_table(c: W.PagedCache, max_pages: int, pad: int = -1) -> torch.Tensor:
+    """The packed table's pages, one row of max_pages per sequence; unused
+    entries hold `pad` (an index outside the pool: reading one is reported)."""
+    bt = torch.full((len(c.pages_per_seq), max_pages), pad, dtype=torch.int32)
+    pt = c.page_table.cpu()
+    off = 0
+    for b, n in enumerate(c.pages_per_seq):
+        bt[b, :n] = pt[off:off + n]
+        off += n
+    return bt
+
+
+def _decode_strided(c: W.PagedCache, bt: torch.Tensor, lens=None):
+    o = torch.full_like(c.q, float("nan"))
+    fa.fa_decode_paged_strided(c.q, c.k_pages, c.v_pages, bt.cuda(),
+                               c.seq_lens if lens is None else lens, c.page_size, o=o)
+    return o
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,H_kv", [(4, 4), (8, 2)])
+def test_decode_strided_small_full_compare(d, H, H_kv):
+    lens = [1, 255, 257, 1000, 0, 4103]
+    c = W.paged_inputs(len(lens), H, d, lens, seed=120 + H + d, device="cpu", H_kv=H_kv)
+    bt = _block_table(c, 20)
+    o = _decode_strided(_on_gpu(c), bt)
+    assert fa.fa_get_device_error() == fa.FA_OK  # no padding entry was read
+    o_ref, _ = oracle.decode_paged_strided(c.q, c.k_pages, c.v_pages, bt, c.seq_lens, PS)
+    assert torch.all(o[4] == 0)
+    assert_o_close(to64(o), o_ref, f"decode strided d={d} H={H} H_kv={H_kv}")
+
+
+@pytest.mark.parametrize("H,H_kv", [(4, 4), (8, 2)])
+def test_decode_strided_equals_packed_bitwise(H, H_kv):
+    """The block table is packed on the device, then the same decode runs."""
+    lens = [700, 3, 2049, 256]
+    c = _on_gpu(W.paged_inputs(len(lens), H, 128, lens, seed=130 + H, device="cpu", H_kv=H_kv))
+    o1 = _decode_strided(c, _block_table(c, 9))
+    assert fa.fa_get_device_error() == fa.FA_OK
+    assert torch.equal(o1, _decode_gqa(c))
+
+
+def test_decode_strided_row_overflow_reported_and_cut():
+    """A length past its row is reported; the sequence is decoded over the
+    row's pages only (entries of the next row are not read)."""
+    lens = [600, 1024]  # 3 pages, 4 full pages
+    c = _on_gpu(W.paged_inputs(len(lens), 4, 128, lens, seed=140, device="cpu"))
+    bt = _block_table(c, 4)
+    too_long = torch.tensor([600, 1500], dtype=torch.int32, device="cuda")
+    o = _decode_strided(c, bt, too_long)
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_BAD_INPUT
+    assert torch.equal(o, _decode_gqa(c))  # row 1 cut to its 4 pages = 1024 tokens
+    neg = torch.tensor([600, -5], dtype=torch.int32, device="cuda")
+    o = _decode_strided(c, bt, neg)
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_BAD_INPUT
+    assert torch.all(o[1] == 0)
+
+
+def test_decode_strided_workload_bitwise():
+    """The paged-decode workload (64 sequences of 1K-32K tokens) through a
+    block table of 128 pages per row equals the packed-table decode."""
+    c = W.decode_workload_inputs(W.PAGED_DECODE, device="cuda")
+    c = W.PagedCache(c.q, c.k_pages, c.v_pages, c.page_table.cuda(), c.seq_lens.cuda(),
+                     c.page_size, c.pages_per_seq)
+    o1 = _decode_strided(c, _block_table(c, 128))
+    assert fa.fa_get_device_error() == fa.FA_OK
+    assert torch.equal(o1, _decode(c))
