@@ -437,9 +437,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 
 // ---------------------------------------------------------------------------
-// Grouped query heads (GH = H / Hk in {2, 4, 8}).  A unit is (split, K/V
-// head); the GH query heads of its group are the rows of a 16-row MMA tile
-// (rows GH..15 are zero), so each staged K/V byte serves all of them and the
+// Grouped query heads (GH = H / Hk in {2, 4, 8, 16}).  A unit is (split,
+// K/V head); the GH query heads of its group are the rows of a 16-row MMA
+// tile (rows GH..15 are zero), so each staged K/V byte serves all of them and the
 // dot products run as two small matrix products per chunk on the tensor
 // cores (warp-level m16n8k16: a tcgen05 tile has at least 64 rows, 8x-32x
 // more than the group has).  K/V chunks of 64 tokens arrive by TMA in the
@@ -447,11 +447,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // column fall in 8 distinct bank groups.  Two teams of four warps take
 // alternate chunks; warp wt of a team owns tokens 16wt .. 16wt+15:
 //   S  = Q_g K^T   two 8-token n-tiles over D/16 k-steps (fp32)
-//   online softmax per query row (row = lane / 4; the 4 lanes of a quad
-//   share it), base 2 with scale * log2(e) applied to S
+//   online softmax per query row (rows lane / 4 and, for groups of 16,
+//   lane / 4 + 8; the 4 lanes of a quad share them), base 2 with
+//   scale * log2(e) applied to S
 //   O += P V       P from S's accumulators as the A operand, V through
 //                  ldmatrix.trans, D/8 n-tiles
-// and the 8 warps' (m, l, O) are merged per unit as in the multi-head path.
+// and the 8 warps' (m, l, O) are merged per unit through one shared buffer
+// (a second barrier tells the writers of the next unit that every reader of
+// this one is done), which leaves room for more ring stages.
 // ---------------------------------------------------------------------------
 constexpr int kGqTok = 64;          // tokens per chunk
 constexpr int kGqWarps = 8;         // consumer warps (two teams of four)
@@ -461,7 +464,7 @@ constexpr int kGqSmemLimit = 232448;  // opt-in shared memory per block
 template <int D, int GH>
 struct GqSmem {
     static constexpr int kTile = kGqTok * D * 2;   // one of K, V per stage
-    static constexpr int kCo = 2 * GH * kGqWarps * D * 4;
+    static constexpr int kCo = GH * kGqWarps * D * 4;
     static constexpr int kFit = (kGqSmemLimit - 2048 - 1024 - kCo) / (2 * kTile);
     // even: chunk g goes to team g % 2 and stage g % STAGES, so each stage
     // belongs to one team, which then sees every phase of its barriers in
@@ -470,9 +473,11 @@ struct GqSmem {
     static constexpr int STAGES = (kFit < 6 ? kFit : 6) & ~1;
     alignas(1024) uint8_t k[STAGES][kTile];
     alignas(1024) uint8_t v[STAGES][kTile];
-    float co[2][GH][kGqWarps][D];  // per-warp partial state, by unit parity
-    float cm[2][GH][kGqWarps], cl[2][GH][kGqWarps];
-    uint64_t full[STAGES], empty[STAGES], cmb[2];
+    // per-warp partial state of the unit being merged; cmb: every consumer
+    // has written its state, cfree: every consumer has read the merged unit
+    float co[GH][kGqWarps][D];
+    float cm[GH][kGqWarps], cl[GH][kGqWarps];
+    uint64_t full[STAGES], empty[STAGES], cmb, cfree;
     int abort;
 };
 
@@ -497,6 +502,8 @@ __global__ void __launch_bounds__(kGqThreads, 1)
     constexpr int KS = D / 16;  // k-steps of S
     constexpr int NT = D / 8;   // n-tiles of O
     constexpr int kPage = 256;
+    constexpr bool kTwoRows = GH > 8;  // the group fills rows 8..15 of the MMA tile too
+    static_assert(GH <= 16, "a group is at most the 16 rows of one MMA tile");
     static_assert(STAGES >= 2 && STAGES % 2 == 0, "ring: an even number of stages");
     static_assert(sizeof(Sm) + 1024 <= kGqSmemLimit, "shared memory");
     extern __shared__ uint8_t gq_smem_raw[];
@@ -509,8 +516,8 @@ __global__ void __launch_bounds__(kGqThreads, 1)
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], kGqWarps / 2);  // the four warps of the chunk's team
         }
-        mbar_init(&sm.cmb[0], kGqWarps * 32);
-        mbar_init(&sm.cmb[1], kGqWarps * 32);
+        mbar_init(&sm.cmb, kGqWarps * 32);
+        mbar_init(&sm.cfree, kGqWarps * 32);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -581,20 +588,25 @@ __global__ void __launch_bounds__(kGqThreads, 1)
     for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
         const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk, kPage,
                                         max_splits);
-        // the group's query rows as A fragments: a0 = cols 16ks + 2tig..+1,
-        // a2 = cols +8, of row grp (zero past GH); rows 8..15 are zero
-        uint32_t qa[KS][2];
-        {
-            const bool row_in = grp < GH;
+        // the group's query rows as A fragments: a0 / a2 = row grp, columns
+        // 16ks + 2tig..+1 / +8; a1 / a3 = the same of row grp + 8 (groups of
+        // 16); rows GH..15 are zero
+        uint32_t qa[KS][4];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int row = grp + 8 * rr;
+            const bool row_in = row < GH;
             const __nv_bfloat16* qr =
-                q + (static_cast<int64_t>(us.b) * H + us.h * GH + (row_in ? grp : 0)) * D;
+                q + (static_cast<int64_t>(us.b) * H + us.h * GH + (row_in ? row : 0)) * D;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-                qa[ks][0] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tig)) : 0u;
-                qa[ks][1] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tig)) : 0u;
+                qa[ks][rr] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tig)) : 0u;
+                qa[ks][rr + 2] =
+                    row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tig)) : 0u;
             }
         }
-        float m = -INFINITY, l = 0.f;
+        // rows grp (index 0) and grp + 8 (index 1, groups of 16 only)
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
         float acc[NT][4];
 #pragma unroll
         for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -618,40 +630,48 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                     // matrices: column chunks 4kp .. 4kp+3 of token rows 16wt + 8j ..
                     uint32_t b[4];
                     ldsm_x4(b, kb + gq_swz(16 * wt + 8 * j + lrow, 4 * kp + lmat));
-                    mma_bf16_16816(s[j], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b[0], b[1]);
-                    mma_bf16_16816(s[j], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b[2], b[3]);
+                    mma_bf16_16816(s[j], qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2],
+                                   qa[2 * kp][3], b[0], b[1]);
+                    mma_bf16_16816(s[j], qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2],
+                                   qa[2 * kp + 1][3], b[2], b[3]);
                 }
             }
-            // ---- online softmax of row grp over this warp's 16 tokens
+            // ---- online softmax of rows grp (and grp + 8) over this warp's 16 tokens
             const bool partial = t0 + 16 > us.ntok;
-            float sv[4];
+            uint32_t pa[4];  // P as the A operand, as qa
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int rr = 0; rr < (kTwoRows ? 2 : 1); ++rr) {
+                float sv[4];
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float x = s[j][e] * scale_log2;
-                    sv[2 * j + e] = (partial && t0 + 8 * j + 2 * tig + e >= us.ntok) ? -INFINITY : x;
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float x = s[j][2 * rr + e] * scale_log2;
+                        sv[2 * j + e] =
+                            (partial && t0 + 8 * j + 2 * tig + e >= us.ntok) ? -INFINITY : x;
+                    }
+                float mb = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+                const float mn = fmaxf(m[rr], mb);
+                const float mu = (mn == -INFINITY) ? 0.f : mn;  // no finite score yet
+                const float alpha = ex2_approx(m[rr] - mu);      // m = -inf -> 0
+                l[rr] *= alpha;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    acc[n][2 * rr] *= alpha;
+                    acc[n][2 * rr + 1] *= alpha;
                 }
-            float mb = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
-            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-            const float mn = fmaxf(m, mb);
-            const float mu = (mn == -INFINITY) ? 0.f : mn;  // no finite score yet
-            const float alpha = ex2_approx(m - mu);          // m = -inf -> 0
-            l *= alpha;
+                float pv[4];
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                acc[n][0] *= alpha;
-                acc[n][1] *= alpha;
+                for (int i = 0; i < 4; ++i) pv[i] = ex2_approx(sv[i] - mu);  // -inf -> 0
+                l[rr] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+                m[rr] = mn;
+                // tokens 2tig..+1 of n-tile 0 (k columns 0-7) and n-tile 1 (8-15)
+                pa[rr] = pack_bf16x2(pv[0], pv[1]);
+                pa[rr + 2] = pack_bf16x2(pv[2], pv[3]);
             }
-            float pv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) pv[i] = ex2_approx(sv[i] - mu);  // -inf -> 0
-            l += (pv[0] + pv[1]) + (pv[2] + pv[3]);
-            m = mn;
-            // P as the A operand: tokens 2tig..+1 of n-tile 0 (a0) and 1 (a2)
-            const uint32_t pa0 = pack_bf16x2(pv[0], pv[1]);
-            const uint32_t pa2 = pack_bf16x2(pv[2], pv[3]);
+            if constexpr (!kTwoRows) pa[1] = pa[3] = 0u;
             // V rows past the unit's tokens may hold anything (0 * NaN): zero
             // their halves of the B fragments
             uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
@@ -665,48 +685,61 @@ __global__ void __launch_bounds__(kGqThreads, 1)
             for (int np = 0; np < NT / 2; ++np) {
                 uint32_t b[4];
                 ldsm_x4_trans(b, vb + gq_swz(16 * wt + 8 * (lmat & 1) + lrow, 2 * np + (lmat >> 1)));
-                mma_bf16_16816(acc[2 * np], pa0, 0u, pa2, 0u, b[0] & mlo, b[1] & mhi);
-                mma_bf16_16816(acc[2 * np + 1], pa0, 0u, pa2, 0u, b[2] & mlo, b[3] & mhi);
+                mma_bf16_16816(acc[2 * np], pa[0], pa[1], pa[2], pa[3], b[0] & mlo, b[1] & mhi);
+                mma_bf16_16816(acc[2 * np + 1], pa[0], pa[1], pa[2], pa[3], b[2] & mlo,
+                               b[3] & mhi);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[slot]);
         }
         if (!ok) break;
-        // ---- merge the 8 warps' states of this unit (buffers by unit parity)
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        const int par = k & 1;
-        if (grp < GH) {
-            if (tig == 0) {
-                sm.cm[par][grp][warp] = m;
-                sm.cl[par][grp][warp] = l;
-            }
+        // ---- merge the 8 warps' states of this unit through the one buffer,
+        // once every consumer has read the previous unit's merge out of it
 #pragma unroll
-            for (int n = 0; n < NT; ++n)
-                *reinterpret_cast<float2*>(&sm.co[par][grp][warp][n * 8 + 2 * tig]) =
-                    make_float2(acc[n][0], acc[n][1]);
+        for (int rr = 0; rr < 2; ++rr) {
+            l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
+            l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 2);
         }
-        mbar_arrive(&sm.cmb[par]);
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT,
-                                               abort));
+        if (k > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.cfree, (k - 1) & 1, err, FA_DEVERR_TIMEOUT,
+                                                   abort));
+            if (!ok) break;
+        }
+#pragma unroll
+        for (int rr = 0; rr < (kTwoRows ? 2 : 1); ++rr) {
+            const int row = grp + 8 * rr;
+            if (row < GH) {
+                if (tig == 0) {
+                    sm.cm[row][warp] = m[rr];
+                    sm.cl[row][warp] = l[rr];
+                }
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+                    *reinterpret_cast<float2*>(&sm.co[row][warp][n * 8 + 2 * tig]) =
+                        make_float2(acc[n][2 * rr], acc[n][2 * rr + 1]);
+            }
+        }
+        mbar_arrive(&sm.cmb);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.cmb, k & 1, err, FA_DEVERR_TIMEOUT, abort));
         if (!ok) break;
         for (int idx = threadIdx.x; idx < GH * D; idx += kGqWarps * 32) {
             const int hi = idx / D, x = idx - hi * D;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kGqWarps; ++w) M = fmaxf(M, sm.cm[par][hi][w]);
+            for (int w = 0; w < kGqWarps; ++w) M = fmaxf(M, sm.cm[hi][w]);
             float L = 0.f, o = 0.f;
 #pragma unroll
             for (int w = 0; w < kGqWarps; ++w) {
-                const float mw = sm.cm[par][hi][w];
+                const float mw = sm.cm[hi][w];
                 const float wgt = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-                L += wgt * sm.cl[par][hi][w];
-                o += wgt * sm.co[par][hi][w][x];
+                L += wgt * sm.cl[hi][w];
+                o += wgt * sm.co[hi][w][x];
             }
             const int64_t pu = static_cast<int64_t>(u) * GH + hi;
             part_o[pu * D + x] = o / L;
             if (x == 0) part_lse[pu] = M + __log2f(L);
         }
+        mbar_arrive(&sm.cfree);
     }
 }
 
@@ -962,6 +995,7 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
         FA_DECODE_GH(2)
         FA_DECODE_GH(4)
         FA_DECODE_GH(8)
+        FA_DECODE_GH(16)
 #undef FA_DECODE_GH
         default: return FA_ERR_UNSUPPORTED;
     }
@@ -971,7 +1005,7 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
 bool decode_group_supported(int H, int Hk) {
     if (Hk < 1 || H % Hk != 0) return false;
     const int g = H / Hk;
-    return g == 1 || g == 2 || g == 4 || g == 8;
+    return g == 1 || g == 2 || g == 4 || g == 8 || g == 16;
 }
 
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,

@@ -183,7 +183,7 @@ def _decode_gqa(c: W.PagedCache):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (8, 1), (16, 2), (3, 3)])
+@pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (8, 1), (16, 2), (3, 3), (16, 1), (32, 2)])
 def test_decode_gqa_small_full_compare(d, H, H_kv):
     lens = [1, 255, 257, 1000, 4103, 0]
     c = W.paged_inputs(len(lens), H, d, lens, seed=40 + H + H_kv, device="cpu", H_kv=H_kv)
@@ -201,9 +201,9 @@ def test_decode_gqa_group1_equals_decode():
     assert torch.equal(_decode_gqa(g), _decode(g))
 
 
-@pytest.mark.parametrize("H_kv", [16, 8, 4])
+@pytest.mark.parametrize("H_kv", [16, 8, 4, 2])
 def test_decode_gqa_workload_sampled(H_kv):
-    """The paged-decode workload's lengths with 16, 8 or 4 K/V heads for 32
+    """The paged-decode workload's lengths with 16, 8, 4 or 2 K/V heads for 32
     query heads (every CTA of the persistent grid runs many units)."""
     w = W.PAGED_DECODE
     lengths = W.varlen_lengths(w.B, w.len_lo, w.len_hi, w.seed)
@@ -222,7 +222,7 @@ def test_decode_gqa_workload_sampled(H_kv):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("H,H_kv", [(8, 4), (8, 2), (16, 2)])
+@pytest.mark.parametrize("H,H_kv", [(8, 4), (8, 2), (16, 2), (16, 1)])
 def test_decode_gqa_chunk_and_warp_edges(d, H, H_kv):
     """Lengths that end inside, and right at, the 16-token slices the warps own
     and the 64-token chunks the two warp teams alternate on; the poisoned
