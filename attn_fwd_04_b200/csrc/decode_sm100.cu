@@ -437,7 +437,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 
 // ---------------------------------------------------------------------------
-// Grouped query heads (GH = H / Hk in {2, 4, 8, 16}).  A unit is (split,
+// Grouped query heads (GH = H / Hk in {2, 4, 8, 16}; see below for larger
+// groups).  A unit is (split,
 // K/V head); the GH query heads of its group are the rows of a 16-row MMA
 // tile (rows GH..15 are zero), so each staged K/V byte serves all of them and the
 // dot products run as two small matrix products per chunk on the tensor
@@ -455,6 +456,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // and the 8 warps' (m, l, O) are merged per unit through one shared buffer
 // (a second barrier tells the writers of the next unit that every reader of
 // this one is done), which leaves room for more ring stages.
+// Groups larger than 16 (sub = group / 16 > 1, multi-query attention with
+// many heads) are cut into sub-groups of 16 query heads, each a unit of its
+// own with the K/V head's pages: Hk counts those sub-groups (H / 16) and K/V
+// head h / sub is read, once per sub-group.
 // ---------------------------------------------------------------------------
 constexpr int kGqTok = 64;          // tokens per chunk
 constexpr int kGqWarps = 8;         // consumer warps (two teams of four)
@@ -493,7 +498,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                          const __grid_constant__ CUtensorMap tv,
                          const __nv_bfloat16* __restrict__ q,
                          const int32_t* __restrict__ page_table,
-                         const int32_t* __restrict__ seq_lens, int B, int H, int Hk,
+                         const int32_t* __restrict__ seq_lens, int B, int H, int Hk, int sub,
                          int num_pages, int max_splits, const int32_t* __restrict__ page_off,
                          const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                          float* __restrict__ part_o, float scale_log2, unsigned int* err) {
@@ -547,7 +552,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                         if (lane == 0) record_error(err, FA_DEVERR_BAD_INPUT);
                         z = -1;
                     } else {
-                        z = page * Hk + us.h;
+                        z = page * (Hk / sub) + us.h / sub;
                     }
                 }
                 const int slot = g % STAGES;
@@ -860,13 +865,14 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// GH query heads per unit; sub units per K/V head (groups of 16 * sub)
 template <int D, int GH>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
                        const int32_t* seq_lens, void* o, int B, int H, int num_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
-                       int num_sms, cudaStream_t stream) {
-    const int Hk = H / GH;
+                       int num_sms, cudaStream_t stream, int sub = 1) {
+    const int Hk = H / GH;  // units per split
     const WorkspaceLayout L = layout_of(B, H, D, max_splits);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* page_off = reinterpret_cast<int32_t*>(ws);
@@ -907,7 +913,7 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
             occ < 1)
             return FA_ERR_CUDA;
         split<<<num_sms * occ, kGqThreads, smem, stream>>>(
-            *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk,
+            *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk, sub,
             num_pages, max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
     }
     const int warps = B * H;
@@ -997,7 +1003,11 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
         FA_DECODE_GH(8)
         FA_DECODE_GH(16)
 #undef FA_DECODE_GH
-        default: return FA_ERR_UNSUPPORTED;
+        default:
+            if ((H / Hk) % 16 != 0) return FA_ERR_UNSUPPORTED;
+            return launch_decode_impl<D, 16>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o,
+                                             B, H, num_pages, page_size, max_splits, workspace,
+                                             err, num_sms, stream, H / Hk / 16);
     }
 }
 }  // namespace
@@ -1005,7 +1015,7 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
 bool decode_group_supported(int H, int Hk) {
     if (Hk < 1 || H % Hk != 0) return false;
     const int g = H / Hk;
-    return g == 1 || g == 2 || g == 4 || g == 8 || g == 16;
+    return g == 1 || g == 2 || g == 4 || g == 8 || g % 16 == 0;
 }
 
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,

@@ -179,7 +179,7 @@ def test_decode_argument_errors(L):
     assert decode_gqa(L, H_kv=3) == fa.FA_ERR_SHAPE       # 8 is not a multiple of 3
     assert decode_gqa(L, P=0) == fa.FA_ERR_SHAPE          # empty pool
     assert decode_gqa(L, H=24, H_kv=8) == fa.FA_ERR_UNSUPPORTED  # group of 3
-    assert decode_gqa(L, H=32, H_kv=1) == fa.FA_ERR_UNSUPPORTED  # group of 32
+    assert decode_gqa(L, H=24, H_kv=1) == fa.FA_ERR_UNSUPPORTED  # group of 24
     assert decode_gqa(L, ps=128) == fa.FA_ERR_UNSUPPORTED
     assert decode_gqa(L, o=MIS) == fa.FA_ERR_ALIGN
     assert decode_strided(L, bt=None) == fa.FA_ERR_NULL

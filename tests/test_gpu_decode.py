@@ -183,7 +183,8 @@ def _decode_gqa(c: W.PagedCache):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (8, 1), (16, 2), (3, 3), (16, 1), (32, 2)])
+@pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (8, 1), (16, 2), (3, 3), (16, 1), (32, 2),
+                                    (32, 1), (64, 2), (48, 1)])
 def test_decode_gqa_small_full_compare(d, H, H_kv):
     lens = [1, 255, 257, 1000, 4103, 0]
     c = W.paged_inputs(len(lens), H, d, lens, seed=40 + H + H_kv, device="cpu", H_kv=H_kv)
@@ -201,10 +202,10 @@ def test_decode_gqa_group1_equals_decode():
     assert torch.equal(_decode_gqa(g), _decode(g))
 
 
-@pytest.mark.parametrize("H_kv", [16, 8, 4, 2])
+@pytest.mark.parametrize("H_kv", [16, 8, 4, 2, 1])
 def test_decode_gqa_workload_sampled(H_kv):
-    """The paged-decode workload's lengths with 16, 8, 4 or 2 K/V heads for 32
-    query heads (every CTA of the persistent grid runs many units)."""
+    """The paged-decode workload's lengths with 16, 8, 4, 2 or 1 K/V heads for
+    32 query heads (every CTA of the persistent grid runs many units)."""
     w = W.PAGED_DECODE
     lengths = W.varlen_lengths(w.B, w.len_lo, w.len_hi, w.seed)
     c = W.paged_inputs(w.B, w.H, w.d, lengths, w.seed, w.page_size, device="cuda", H_kv=H_kv)
