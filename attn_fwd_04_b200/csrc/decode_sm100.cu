@@ -437,8 +437,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 
 // ---------------------------------------------------------------------------
-// Grouped query heads (GH = H / Hk in {2, 4, 8, 16}; see below for larger
-// groups).  A unit is (split,
+// Grouped query heads (groups of 2 or more; see below for the sizes).  A
+// unit is (split,
 // K/V head); the GH query heads of its group are the rows of a 16-row MMA
 // tile (rows GH..15 are zero), so each staged K/V byte serves all of them and the
 // dot products run as two small matrix products per chunk on the tensor
@@ -456,10 +456,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // and the 8 warps' (m, l, O) are merged per unit through one shared buffer
 // (a second barrier tells the writers of the next unit that every reader of
 // this one is done), which leaves room for more ring stages.
-// Groups larger than 16 (sub = group / 16 > 1, multi-query attention with
-// many heads) are cut into sub-groups of 16 query heads, each a unit of its
-// own with the K/V head's pages: Hk counts those sub-groups (H / 16) and K/V
-// head h / sub is read, once per sub-group.
+// A unit holds gr <= GH query heads (GH, the template, is the capacity of
+// its registers and merge buffer).  Groups larger than 16 (multi-query
+// attention with many heads) are cut into sub equal sub-groups of gr <= 16
+// query heads, each a unit of its own with its K/V head's pages: Hk counts
+// the units per split (H / gr) and K/V head h / sub is read, once per
+// sub-group.
 // ---------------------------------------------------------------------------
 constexpr int kGqTok = 64;          // tokens per chunk
 constexpr int kGqWarps = 8;         // consumer warps (two teams of four)
@@ -498,7 +500,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                          const __grid_constant__ CUtensorMap tv,
                          const __nv_bfloat16* __restrict__ q,
                          const int32_t* __restrict__ page_table,
-                         const int32_t* __restrict__ seq_lens, int B, int H, int Hk, int sub,
+                         const int32_t* __restrict__ seq_lens, int B, int H, int Hk, int gr, int sub,
                          int num_pages, int max_splits, const int32_t* __restrict__ page_off,
                          const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                          float* __restrict__ part_o, float scale_log2, unsigned int* err) {
@@ -595,14 +597,14 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                                         max_splits);
         // the group's query rows as A fragments: a0 / a2 = row grp, columns
         // 16ks + 2tig..+1 / +8; a1 / a3 = the same of row grp + 8 (groups of
-        // 16); rows GH..15 are zero
+        // 16); rows gr..15 are zero
         uint32_t qa[KS][4];
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
             const int row = grp + 8 * rr;
-            const bool row_in = row < GH;
+            const bool row_in = row < gr;
             const __nv_bfloat16* qr =
-                q + (static_cast<int64_t>(us.b) * H + us.h * GH + (row_in ? row : 0)) * D;
+                q + (static_cast<int64_t>(us.b) * H + us.h * gr + (row_in ? row : 0)) * D;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 qa[ks][rr] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tig)) : 0u;
@@ -713,7 +715,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < (kTwoRows ? 2 : 1); ++rr) {
             const int row = grp + 8 * rr;
-            if (row < GH) {
+            if (row < gr) {
                 if (tig == 0) {
                     sm.cm[row][warp] = m[rr];
                     sm.cl[row][warp] = l[rr];
@@ -727,7 +729,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
         mbar_arrive(&sm.cmb);
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.cmb, k & 1, err, FA_DEVERR_TIMEOUT, abort));
         if (!ok) break;
-        for (int idx = threadIdx.x; idx < GH * D; idx += kGqWarps * 32) {
+        for (int idx = threadIdx.x; idx < gr * D; idx += kGqWarps * 32) {
             const int hi = idx / D, x = idx - hi * D;
             float M = -INFINITY;
 #pragma unroll
@@ -740,7 +742,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                 L += wgt * sm.cl[hi][w];
                 o += wgt * sm.co[hi][w][x];
             }
-            const int64_t pu = static_cast<int64_t>(u) * GH + hi;
+            const int64_t pu = static_cast<int64_t>(u) * gr + hi;
             part_o[pu * D + x] = o / L;
             if (x == 0) part_lse[pu] = M + __log2f(L);
         }
@@ -865,14 +867,15 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// GH query heads per unit; sub units per K/V head (groups of 16 * sub)
+// gr query heads per unit (gr <= GH, the kernel's capacity; GH == 1 is the
+// multi-head kernel), sub units per K/V head (a group of gr * sub)
 template <int D, int GH>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
                        const int32_t* seq_lens, void* o, int B, int H, int num_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
-                       int num_sms, cudaStream_t stream, int sub = 1) {
-    const int Hk = H / GH;  // units per split
+                       int num_sms, cudaStream_t stream, int gr, int sub) {
+    const int Hk = H / gr;  // units per split
     const WorkspaceLayout L = layout_of(B, H, D, max_splits);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* page_off = reinterpret_cast<int32_t*>(ws);
@@ -913,12 +916,12 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
             occ < 1)
             return FA_ERR_CUDA;
         split<<<num_sms * occ, kGqThreads, smem, stream>>>(
-            *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk, sub,
+            *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk, gr, sub,
             num_pages, max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
     }
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
-        seq_lens, B, H, GH, page_size, max_splits, unit_off, part_lse, part_o,
+        seq_lens, B, H, gr, page_size, max_splits, unit_off, part_lse, part_o,
         static_cast<__nv_bfloat16*>(o));
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -991,32 +994,31 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
                     const int32_t* seq_lens, void* o, int B, int H, int Hk, int num_pages,
                     int page_size, int max_splits, void* workspace, unsigned int* err,
                     int num_sms, cudaStream_t stream) {
-    switch (H / Hk) {
+    // a group of G query heads per K/V head runs as sub units of gr = G / sub
+    // heads, sub the fewest that leaves gr <= 16
+    const int G = H / Hk;
+    int sub = (G + 15) / 16;
+    while (G % sub != 0) ++sub;
+    const int gr = G / sub;
+    if (G == 1)
+        return launch_decode_impl<D, 1>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, B,
+                                        H, num_pages, page_size, max_splits, workspace, err,
+                                        num_sms, stream, 1, 1);
 #define FA_DECODE_GH(GH)                                                                        \
-    case GH:                                                                                    \
+    if (gr <= GH)                                                                               \
         return launch_decode_impl<D, GH>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, \
                                          B, H, num_pages, page_size, max_splits, workspace,    \
-                                         err, num_sms, stream);
-        FA_DECODE_GH(1)
-        FA_DECODE_GH(2)
-        FA_DECODE_GH(4)
-        FA_DECODE_GH(8)
-        FA_DECODE_GH(16)
+                                         err, num_sms, stream, gr, sub);
+    FA_DECODE_GH(2)
+    FA_DECODE_GH(4)
+    FA_DECODE_GH(8)
+    FA_DECODE_GH(16)
 #undef FA_DECODE_GH
-        default:
-            if ((H / Hk) % 16 != 0) return FA_ERR_UNSUPPORTED;
-            return launch_decode_impl<D, 16>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o,
-                                             B, H, num_pages, page_size, max_splits, workspace,
-                                             err, num_sms, stream, H / Hk / 16);
-    }
+    return FA_ERR_UNSUPPORTED;
 }
 }  // namespace
 
-bool decode_group_supported(int H, int Hk) {
-    if (Hk < 1 || H % Hk != 0) return false;
-    const int g = H / Hk;
-    return g == 1 || g == 2 || g == 4 || g == 8 || g % 16 == 0;
-}
+bool decode_group_supported(int H, int Hk) { return Hk >= 1 && H % Hk == 0; }
 
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,

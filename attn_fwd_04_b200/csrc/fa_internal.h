@@ -66,7 +66,7 @@ struct DecodePlan {
 
 size_t decode_workspace_bytes(int B, int H, int d, int max_splits);
 
-// H query heads over Hk K/V heads (H / Hk in {1, 2, 4, 8} or a multiple of 16).  The grouped
+// H query heads over Hk K/V heads (any H % Hk == 0).  The grouped
 // kernels (H > Hk) read the pool through tk, tv: (d, 256, num_pages * Hk)
 // maps with 64 x 64 x 1 boxes and 128-byte swizzle; H == Hk reads it with
 // bulk copies and takes no maps (may be null).  Page indices outside

@@ -211,9 +211,10 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
  *                H_kv heads
  * Query head h attends to K/V head h / (H / H_kv) of its sequence's cached
  * tokens; everything else (page table, lengths, scale 1/sqrt(d), no mask,
- * workspace) as fa_decode_paged.  H / H_kv must be 1, 2, 4, 8 or a multiple
- * of 16 (multi-query attention with many heads; groups beyond 16 read each
- * K/V slice once per 16 query heads)
+ * workspace) as fa_decode_paged.  Any H that is a multiple of H_kv works;
+ * a group of more than 16 query heads (multi-query attention with many
+ * heads) runs as equal sub-groups of at most 16, each reading the K/V
+ * slices once
  * (FA_ERR_UNSUPPORTED otherwise; FA_ERR_SHAPE if H is not a multiple of
  * H_kv, or num_pages < 1).  Each (page, K/V head) slice is read from device
  * memory once and serves all H / H_kv query heads of its group.  A page

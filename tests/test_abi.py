@@ -178,15 +178,14 @@ def test_decode_argument_errors(L):
     assert decode_gqa(L, H_kv=0) == fa.FA_ERR_SHAPE
     assert decode_gqa(L, H_kv=3) == fa.FA_ERR_SHAPE       # 8 is not a multiple of 3
     assert decode_gqa(L, P=0) == fa.FA_ERR_SHAPE          # empty pool
-    assert decode_gqa(L, H=24, H_kv=8) == fa.FA_ERR_UNSUPPORTED  # group of 3
-    assert decode_gqa(L, H=24, H_kv=1) == fa.FA_ERR_UNSUPPORTED  # group of 24
+    assert decode_gqa(L, H=24, H_kv=5) == fa.FA_ERR_SHAPE  # 24 is not a multiple of 5
     assert decode_gqa(L, ps=128) == fa.FA_ERR_UNSUPPORTED
     assert decode_gqa(L, o=MIS) == fa.FA_ERR_ALIGN
     assert decode_strided(L, bt=None) == fa.FA_ERR_NULL
     assert decode_strided(L, mp=0) == fa.FA_ERR_SHAPE
     assert decode_strided(L, mp=1 << 24) == fa.FA_ERR_SHAPE  # row of 2^32 tokens
     assert decode_strided(L, B=1 << 10, mp=1 << 22) == fa.FA_ERR_SHAPE  # 2^32 entries
-    assert decode_strided(L, H=24, H_kv=8) == fa.FA_ERR_UNSUPPORTED
+    assert decode_strided(L, H=24, H_kv=7) == fa.FA_ERR_SHAPE
     assert decode_strided(L, ps=128) == fa.FA_ERR_UNSUPPORTED
     assert decode_strided(L, q=MIS) == fa.FA_ERR_ALIGN
     assert gather(L, out=None) == fa.FA_ERR_NULL

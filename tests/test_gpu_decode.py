@@ -184,7 +184,7 @@ def _decode_gqa(c: W.PagedCache):
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (8, 1), (16, 2), (3, 3), (16, 1), (32, 2),
-                                    (32, 1), (64, 2), (48, 1)])
+                                    (32, 1), (64, 2), (48, 1), (6, 2), (12, 1), (40, 2), (17, 1)])
 def test_decode_gqa_small_full_compare(d, H, H_kv):
     lens = [1, 255, 257, 1000, 4103, 0]
     c = W.paged_inputs(len(lens), H, d, lens, seed=40 + H + H_kv, device="cpu", H_kv=H_kv)
