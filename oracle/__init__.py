@@ -60,7 +60,7 @@ def lib():
         L.oracle_rope_exact.restype = None
         L.oracle_rope_bf16.argtypes = [P, P, P, I64, I64, I64]
         L.oracle_rope_bf16.restype = None
-        L.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64,
+        L.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64,
                                            ctypes.c_int, ctypes.c_double]
         L.oracle_attention_bwd.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
@@ -286,14 +286,16 @@ def rope(x, cos_t, sin_t, bf16_round: bool = True):
 
 
 def attention_bwd(q, k, v, dout, causal: bool, scale: float):
-    """Gradients (dq, dk, dv) of attention over q, k, v [B,H,N,d] for the
-    output gradient dout [B,H,N,d], in fp64."""
+    """Gradients (dq, dk, dv) of attention over q [B,H,N,d] and k, v
+    [B,Hkv,N,d] (query head h uses K/V head h // (H/Hkv); Hkv = H is plain
+    multi-head) for the output gradient dout [B,H,N,d], in fp64."""
     q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, H, N, d = q.shape
-    assert k.shape == v.shape == g.shape == (B, H, N, d)
-    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    Hkv = k.shape[1]
+    assert k.shape == v.shape == (B, Hkv, N, d) and g.shape == q.shape and H % Hkv == 0
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     rc = lib().oracle_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dq), _ptr(dk),
-                                    _ptr(dv), B, H, N, d, int(bool(causal)), float(scale))
+                                    _ptr(dv), B, H, Hkv, N, d, int(bool(causal)), float(scale))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_bwd failed ({rc})")
     return dq, dk, dv

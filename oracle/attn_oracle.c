@@ -611,19 +611,24 @@ void oracle_rope_bf16(double *x, const float *cos_t, const float *sin_t, int64_t
  *   ds_ij = p_ij (dp_ij - D_i)
  *   dQ_i  = scale sum_j ds_ij k_j
  *   dK_j += scale ds_ij q_i
- * q, k, v, do, dq, dk, dv are [B,H,N,d].  Rows are split over threads; each
- * thread accumulates dK, dV of its rows privately and the partial sums are
- * added in thread order, so the result does not depend on scheduling for a
- * fixed thread count. */
+ * q, do, dq are [B,H,N,d]; k, v, dk, dv are [B,Hkv,N,d] and query head h
+ * uses K/V head h / (H / Hkv) (grouped-query attention; Hkv = H is plain
+ * multi-head), so a K/V head's dK and dV are the sums of the contributions of
+ * every query head of its group.  Rows are split over threads; each thread
+ * accumulates dK, dV of its rows privately and the partial sums are added in
+ * thread order (query heads in order), so the result does not depend on
+ * scheduling for a fixed thread count. */
 int oracle_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
-                         double *dq, double *dk, double *dv, int64_t B, int64_t H, int64_t N,
-                         int64_t d, int causal, double scale) {
-    if (B < 0 || H < 0 || N < 0 || d <= 0) return -1;
+                         double *dq, double *dk, double *dv, int64_t B, int64_t H, int64_t Hkv,
+                         int64_t N, int64_t d, int causal, double scale) {
+    if (B < 0 || H < 0 || N < 0 || d <= 0 || Hkv <= 0 || H % Hkv != 0) return -1;
+    const int64_t group = H / Hkv;
+    for (int64_t x = 0; x < B * Hkv * N * d; ++x) dk[x] = dv[x] = 0.0;
     for (int64_t bh = 0; bh < B * H; ++bh) {
-        const double *qb = q + bh * N * d, *kb = k + bh * N * d, *vb = v + bh * N * d;
+        const int64_t bkv = (bh / H) * Hkv + (bh % H) / group;
+        const double *qb = q + bh * N * d, *kb = k + bkv * N * d, *vb = v + bkv * N * d;
         const double *gb = dout + bh * N * d;
-        double *dqb = dq + bh * N * d, *dkb = dk + bh * N * d, *dvb = dv + bh * N * d;
-        for (int64_t x = 0; x < N * d; ++x) dkb[x] = dvb[x] = 0.0;
+        double *dqb = dq + bh * N * d, *dkb = dk + bkv * N * d, *dvb = dv + bkv * N * d;
         int nthr = 1;
 #ifdef _OPENMP
         nthr = omp_get_max_threads();

@@ -760,6 +760,51 @@ def test_bwd_equals_finite_differences(causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+def test_bwd_gqa_equals_finite_differences(causal):
+    """Grouped K/V heads: a K/V entry feeds every query head of its group, so
+    its gradient is the central difference of the loss summed over them (a
+    gradient written to only the first query head's share would fail)."""
+    B, H, Hkv, N, d = 1, 4, 2, 4, 3
+    q, g = _rand((B, H, N, d), 230), _rand((B, H, N, d), 231)
+    k, v = _rand((B, Hkv, N, d), 232), _rand((B, Hkv, N, d), 233)
+    scale = 0.6
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, causal, scale)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.attention_gqa(q_, k_, v_, causal, scale)
+        return float(np.sum(o * g))
+
+    h = 1e-5
+    for x, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(grad, num, atol=1e-8)
+
+
+def test_bwd_gqa_equals_repeated_heads_summed():
+    """Attention with grouped heads is attention with each K/V head repeated
+    for its query heads; dK, dV of a K/V head are then the sums of the
+    repeated copies' gradients."""
+    B, H, Hkv, N, d = 2, 6, 2, 9, 4
+    q, g = _rand((B, H, N, d), 234), _rand((B, H, N, d), 235)
+    k, v = _rand((B, Hkv, N, d), 236), _rand((B, Hkv, N, d), 237)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, True, 0.5)
+    r = H // Hkv
+    dq2, dk2, dv2 = oracle.attention_bwd(q, np.repeat(k, r, axis=1), np.repeat(v, r, axis=1), g,
+                                         True, 0.5)
+    np.testing.assert_allclose(dq, dq2, atol=1e-13)
+    np.testing.assert_allclose(dk, dk2.reshape(B, Hkv, r, N, d).sum(axis=2), atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, r, N, d).sum(axis=2), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
 def test_bwd_key_gradients_sum_to_zero(causal):
     """Each row of dS sums to zero (the softmax Jacobian annihilates
     constants), so sum_j dK_j = scale sum_i q_i sum_j dS_ij = 0; dropping the
