@@ -242,11 +242,11 @@ int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse
                      rope_sin, max_pos);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-           const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-           int causal, float scale, fa_stream_t stream) {
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+               int d, int causal, float scale, fa_stream_t stream) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
-    if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+    if (B < 1 || H < 1 || N < 1 || H_kv < 1 || H % H_kv != 0) return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(B) * H > 65535) return FA_ERR_SHAPE;
     if (N > 0x7fffffff - 128) return FA_ERR_SHAPE;
@@ -260,12 +260,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     CUtensorMap tq, tk, tv, tdo;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                 static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t dims_kv[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                   static_cast<cuuint64_t>(B) * H_kv};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                    static_cast<cuuint64_t>(N) * d * 2};
     const cuuint32_t box[3] = {64, 128, 1};
     if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tk, k, dims, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tv, v, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims_kv, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims_kv, strides, box)) != FA_OK) return rc;
     if ((rc = make_map(&tdo, dout, dims, strides, box)) != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     void* ws = nullptr;
@@ -281,8 +283,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     if ((rc = make_map_f32(&tdq, static_cast<uint8_t*>(ws) + fa::bwd_dq_acc_offset(B, H, N), adims,
                            astrides, abox)) != FA_OK)
         return rc;
-    return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, tdq, B, H, N, d,
+    return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, tdq, B, H, H_kv, N, d,
                           causal ? 1 : 0, scale, ws, s->err, s->num_sms, st);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+           int causal, float scale, fa_stream_t stream) {
+    return fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, causal, scale, stream);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

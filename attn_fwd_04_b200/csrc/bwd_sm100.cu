@@ -81,7 +81,7 @@ struct BwdParams {
     float* dq_acc;       // [B*H*N*D] fp32, cleared by the prep kernel
     void* dk;
     void* dv;
-    int B, H, N, causal;
+    int B, H, H_kv, N, causal;  // query head h uses K/V head h / (H / H_kv)
     float scale, scale_log2;
     unsigned int* err;
 };
@@ -163,17 +163,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ---- work unit: (sequence/head, 128-key block), longest first within
     // groups of kBwdHeadGroup heads (under a causal mask key block 0 meets
     // every query tile)
-    const int units = p.B * p.H;
+    const int units = p.B * p.H_kv;  // (sequence, K/V head)
     const int nkb = (p.N + kBT - 1) / kBT;
     const int gidx = static_cast<int>(blockIdx.x) / (kBwdHeadGroup * nkb);
     const int ug = min(kBwdHeadGroup, units - gidx * kBwdHeadGroup);
     const int within = static_cast<int>(blockIdx.x) - gidx * kBwdHeadGroup * nkb;
     const int jb = within / ug;
-    const int bh = gidx * kBwdHeadGroup + (within - jb * ug);
+    const int bh = gidx * kBwdHeadGroup + (within - jb * ug);  // flat (sequence, K/V head)
     if (jb >= nkb || bh >= units) return;
     const int key0 = jb * kBT;
     const int i_first = p.causal ? jb : 0;
-    const int nt = nkb - i_first;  // query tiles that see this key block
+    const int nt = nkb - i_first;  // query tiles of one query head that see this key block
+    // the CTA walks the query tiles of every query head of its K/V head's
+    // group (dK, dV sum over all of them): tile t is query tile
+    // i_first + t % nt of query head t / nt of the group
+    const int G = p.H / p.H_kv;
+    const int ntt = G * nt;
+    const int qh0 = (bh / p.H_kv) * p.H + (bh % p.H_kv) * G;  // flat first query head
+    auto tile_q0 = [&](int t) { return (i_first + t % nt) * kBT; };
+    auto tile_qh = [&](int t) { return qh0 + t / nt; };
 
     extern __shared__ uint8_t bwd_smem_raw[];
     BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(
@@ -212,10 +220,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp >= 8) regs_dec<kRegsWg2>();
     if (warp == 9) {
         // ================= TMA producer (+ per-tile statistics) =================
-        auto load2 = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row) {
+        auto load2 = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row, int head) {
 #pragma unroll
             for (int cb = 0; cb < D / 64; ++cb)
-                tma_load_3d(dst + cb * kBoxB, map, bar, cb * 64, row, bh);
+                tma_load_3d(dst + cb * kBoxB, map, bar, cb * 64, row, head);
         };
         bool ok = true;
         if (lane == 0) {
@@ -224,27 +232,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_prefetch_desc(&tv);
             tma_prefetch_desc(&tdo);
             mbar_arrive_expect_tx(&sm.kv_full, 2 * kBT * D * 2);
-            load2(sm.k, &tk, &sm.kv_full, key0);
-            load2(sm.v, &tv, &sm.kv_full, key0);
+            load2(sm.k, &tk, &sm.kv_full, key0, bh);
+            load2(sm.v, &tv, &sm.kv_full, key0, bh);
         }
         int issued = 0;
-        for (int t = 0; t < nt; ++t) {
+        for (int t = 0; t < ntt; ++t) {
             const int s = t & 1;
             if (t >= 2 && !bwd_warp_wait(&sm.in_free[s], ((t - 2) >> 1) & 1, err, abort)) {
                 ok = false;
                 break;
             }
-            const int q0 = (i_first + t) * kBT;
+            const int q0 = tile_q0(t), qh = tile_qh(t);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.in_full[s], 2 * kBT * D * 2);
-                load2(sm.q[s], &tq, &sm.in_full[s], q0);
-                load2(sm.dout[s], &tdo, &sm.in_full[s], q0);
+                load2(sm.q[s], &tq, &sm.in_full[s], q0, qh);
+                load2(sm.dout[s], &tdo, &sm.in_full[s], q0, qh);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = lane * 4 + e, qr = q0 + r;
                 const bool in = qr < p.N;
-                const int64_t gi = static_cast<int64_t>(bh) * p.N + qr;
+                const int64_t gi = static_cast<int64_t>(qh) * p.N + qr;
                 sm.nlse2[s][r] = in ? -p.lse2[gi] : -INFINITY;  // rows past N: P = 0
                 sm.ndsum[s][r] = in ? -p.dsum[gi] : 0.f;
             }
@@ -318,7 +326,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 issue_kk(kColDP, v_lo, lo(sm.dout[0]));  // dP^T = V dO_0^T
                 tc_commit(&sm.dp_full);
             }
-            for (int t = 0; ok && t < nt; ++t) {
+            for (int t = 0; ok && t < ntt; ++t) {
                 const int s = t & 1;
                 const uint32_t ph = t & 1;
                 const uint32_t q_lo = lo(sm.q[s]), do_lo = lo(sm.dout[s]);
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 issue_tm(kColDV, kColS, do_lo, t > 0);  // dV += P^T dO_i
                 tc_commit(&sm.dv_done);                 // dO_i's last reader before dS
                 const int s1 = (t + 1) & 1;
-                if (t + 1 < nt) {
+                if (t + 1 < ntt) {
                     // S^T of the next tile (its columns held P^T, read by dV above)
                     if (!mbar_wait(&sm.in_full[s1], ((t + 1) >> 1) & 1, err, FA_DEVERR_TIMEOUT,
                                    abort))
@@ -342,7 +350,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_commit(&sm.dq_full);
                 issue_sm(kColDK, do_lo, q_lo, t > 0);  // dK += dS^T Q_i, same tile K-major
                 tc_commit(&sm.in_free[s]);
-                if (t + 1 < nt) {
+                if (t + 1 < ntt) {
                     // dP^T of the next tile, once dQ_i has left its columns
                     if (!mbar_wait(&sm.dq_free, ph, err, FA_DEVERR_TIMEOUT, abort)) break;
                     tc_fence_after();
@@ -363,11 +371,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int key = key0 + r;
         const bool key_in = key < p.N;
         const float sl = p.scale_log2;
-        for (int t = 0; t < nt; ++t) {
+        for (int t = 0; t < ntt; ++t) {
             const int s = t & 1;
             const uint32_t ph = t & 1;
-            const int q0 = (i_first + t) * kBT;
-            const bool diag = p.causal && (i_first + t == jb);
+            const int q0 = tile_q0(t);
+            const bool diag = p.causal && (i_first + t % nt == jb);
             if (!bwd_warp_wait(&sm.s_full, ph, err, abort)) break;
             tc_fence_after();
             // P^T = 2^(scale log2e S^T - lse2); keys past N, queries past N
@@ -478,7 +486,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int r = threadIdx.x - 128;
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
-        for (int t = 0; t < nt; ++t) {
+        for (int t = 0; t < ntt; ++t) {
             // the four warps leave together (they share named barriers below)
             if (!bar_and_named(2, kBT, mbar_wait(&sm.dq_full, t & 1, err, FA_DEVERR_TIMEOUT,
                                                  abort))) {
@@ -489,7 +497,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // dQ_i (TMEM lane == query row) in slices of 32 columns: each row
             // to the swizzled staging tile, then one TMA reduce-add of the
             // 128 x 32 slice into the accumulator (rows past N are clipped)
-            const int q0 = (i_first + t) * kBT;
+            const int q0 = tile_q0(t), qh = tile_qh(t);
             uint8_t* stage = reinterpret_cast<uint8_t*>(sm.dq_stage);
             // all of dQ_i into registers first, so that its TMEM columns are
             // released to the next dP^T before the reductions
@@ -512,7 +520,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 bar_sync_named(1, kBT);  // every row is in the tile
                 if (r == 0) {
-                    tma_reduce_add_3d(&tdq, stage, c * 32, q0, bh);
+                    tma_reduce_add_3d(&tdq, stage, c * 32, q0, qh);
                     bulk_commit_group();
                     bulk_wait_group_read0();
                 }
@@ -575,7 +583,7 @@ int launch_bwd_impl(const void* o, const void* dout, const float* lse, float* ls
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
-    const long long ctas = static_cast<long long>((p.N + kBT - 1) / kBT) * p.B * p.H;
+    const long long ctas = static_cast<long long>((p.N + kBT - 1) / kBT) * p.B * p.H_kv;
     if (ctas > 0x7fffffffLL) return FA_ERR_SHAPE;
     kern<<<dim3(static_cast<unsigned>(ctas)), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq,
                                                                            p);
@@ -597,7 +605,7 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d) {
 
 int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int N, int d,
+               const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int H_kv, int N, int d,
                int causal, float scale, void* workspace, unsigned int* err, int num_sms,
                cudaStream_t stream) {
     const size_t rows = static_cast<size_t>(B) * H * N;
@@ -613,6 +621,7 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
     p.dv = dv;
     p.B = B;
     p.H = H;
+    p.H_kv = H_kv;
     p.N = N;
     p.causal = causal;
     p.scale = scale;

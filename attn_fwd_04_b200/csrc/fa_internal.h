@@ -48,7 +48,7 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d);
 size_t bwd_dq_acc_offset(int B, int H, int N);  // fp32 dQ accumulator, in the workspace
 int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int N, int d,
+               const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int H_kv, int N, int d,
                int causal, float scale, void* workspace, unsigned int* err, int num_sms,
                cudaStream_t stream);
 

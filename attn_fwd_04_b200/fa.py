@@ -24,7 +24,8 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_fwd_varlen",
+           "fa_decode_paged",
            "fa_decode_paged_gqa", "fa_decode_paged_strided",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
@@ -54,6 +55,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_fwd_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
+        L.fa_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
@@ -68,7 +70,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
         L.fa_fwd_set_cta_pairs.argtypes = [I]
-        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_fwd_varlen", "fa_decode_paged",
+        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_fwd_varlen",
+                     "fa_decode_paged",
                      "fa_decode_paged_gqa", "fa_decode_paged_strided", "fa_decode_paged_noalloc",
                      "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
@@ -197,6 +200,30 @@ def fa_bwd(q, k, v, o, lse, dout, causal: bool, scale: Optional[float] = None, d
                       dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
                       int(bool(causal)), float(scale), _stream(stream))
     _raise_if(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_bwd_gqa(q, k, v, o, lse, dout, causal: bool, scale: Optional[float] = None, dq=None,
+               dk=None, dv=None, stream=None):
+    """Gradients of fa_fwd_gqa: dq [B,H,N,d] and dk, dv [B,H_kv,N,d] bf16, from
+    q, o, dout [B,H,N,d], k, v [B,H_kv,N,d] bf16 and lse [B,H,N] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    if o.shape != q.shape or dout.shape != q.shape or k.shape != (B, H_kv, N, d) or \
+            v.shape != k.shape:
+        raise ValueError("q, o, dout must be [B,H,N,d] and k, v [B,H_kv,N,d]")
+    _check(lse, "lse", torch.float32, 3)
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = lib().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H,
+                          H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_bwd_gqa")
     return dq, dk, dv
 
 

@@ -152,6 +152,22 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, co
            int causal, float scale, fa_stream_t stream);
 
 /*
+ * fa_bwd_gqa -- fa_bwd for fa_fwd_gqa: grouped K/V heads (grouped- or
+ * multi-query attention, the variants named by the page "Flash Attention
+ * 是什么", section 进阶学习路径, item 4).
+ *   q, o, dout, dq : [B, H, N, d] bf16;  lse : [B, H, N] fp32
+ *   k, v, dk, dv   : [B, H_kv, N, d] bf16 (H a multiple of H_kv, FA_ERR_SHAPE
+ *                    otherwise)
+ * Query head h uses K/V head h / (H / H_kv); the gradient of a K/V head sums
+ * the contributions of every query head of its group (one CTA per K/V head
+ * and 128-key block walks the query tiles of all of them).  Everything else
+ * as fa_bwd, which is this call with H_kv = H.
+ */
+FA_API int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                      int H, int H_kv, int N, int d, int causal, float scale, fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- the forward pass over B sequences of different lengths
  * packed back to back (the variable-length batches of the page "Flash
  * Attention 是什么", section 典型应用场景).

@@ -92,3 +92,46 @@ def test_bwd_long_prefill_runs_finite():
     qh, kh, vh, gh = (t[0, 0, :512].cpu()[None, None] for t in (q, k, v, g))
     rq, _, _ = oracle.attention_bwd(qh, kh, vh, gh, True, scale)
     assert_grad_close(to64(dq[0, 0, :512].cpu())[None, None], rq, "dq rows < 512")
+
+
+# -- grouped K/V heads (fa_bwd_gqa) -----------------------------------------------
+
+def _bwd_gqa_gpu(q, k, v, g, causal, scale):
+    qc, kc, vc, gc = q.cuda(), k.cuda(), v.cuda(), g.cuda()
+    o, lse = fa.fa_fwd_gqa(qc, kc, vc, causal, scale)
+    dq = torch.full_like(qc, float("nan"))
+    dk = torch.full_like(kc, float("nan"))
+    dv = torch.full_like(vc, float("nan"))
+    fa.fa_bwd_gqa(qc, kc, vc, o, lse, gc, causal, scale, dq=dq, dk=dk, dv=dv)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return dq, dk, dv
+
+
+# (B, H, H_kv, N, d): groups of 2, 4, 3 and multi-query
+GQA_SHAPES = [(1, 4, 2, 300, 128), (2, 8, 2, 129, 64), (1, 6, 2, 1000, 128), (1, 4, 1, 257, 128)]
+
+
+@pytest.mark.parametrize("shape", GQA_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_gqa_full_compare(shape, causal):
+    B, H, Hkv, N, d = shape
+    q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=800 + N + H, device="cpu")
+    g = _grad_out((B, H, N, d), 801 + N)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv = _bwd_gqa_gpu(q, k, v, g, causal, scale)
+    rq, rk, rv = oracle.attention_bwd(q, k, v, g, causal, scale)
+    assert_grad_close(to64(dv), rv, f"dv {shape}")
+    assert_grad_close(to64(dk), rk, f"dk {shape}")
+    assert_grad_close(to64(dq), rq, f"dq {shape}")
+
+
+def test_bwd_gqa_group1_equals_bwd():
+    """With one query head per K/V head the grouped entry point is fa_bwd: dk
+    and dv bit for bit (dq sums key blocks with atomics, so only closely)."""
+    q, k, v = W.custom_fwd_inputs(1, 3, 700, 128, seed=810)
+    g = _grad_out((1, 3, 700, 128), 811)
+    a = _bwd_gpu(q, k, v, g, True, 0.1)
+    b = _bwd_gqa_gpu(q, k, v, g, True, 0.1)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert_grad_close(to64(b[0]), to64(a[0]), "dq group 1")
+
