@@ -267,6 +267,26 @@ def prefill_paged(q, k_pages, v_pages, page_table, seq_lens, cu_q, page_size: in
     return o, lse
 
 
+def attention_bwd_varlen(q, k, v, dout, cu_seqlens, causal: bool, scale: float):
+    """Gradients over packed sequences: q, dout [total,H,d], k, v [total,Hkv,d]
+    (query head h uses K/V head h // (H/Hkv)); sequence b owns rows
+    cu_seqlens[b] .. cu_seqlens[b+1]-1 and attends within itself only (the
+    variable-length batches of the page "Flash Attention 是什么", section
+    典型应用场景).  Each sequence's gradients are those of attention_bwd on
+    its own rows.  Returns (dq [total,H,d], dk, dv [total,Hkv,d])."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+    cu = _i64(cu_seqlens)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(cu.size - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        if s1 <= s0:
+            continue
+        per = [x[s0:s1].transpose(1, 0, 2)[None] for x in (q, k, v, g)]  # [1, heads, len, d]
+        gq, gk, gv = attention_bwd(*per, causal, scale)
+        dq[s0:s1], dk[s0:s1], dv[s0:s1] = (x[0].transpose(1, 0, 2) for x in (gq, gk, gv))
+    return dq, dk, dv
+
+
 def rope(x, cos_t, sin_t, bf16_round: bool = True):
     """Rotary embedding of x [..., N, d] (positions 0..N-1) with the fp32 tables
     cos_t, sin_t [>=N, d/2]; returns a new fp64 array.  With bf16_round the

@@ -805,6 +805,54 @@ def test_bwd_gqa_equals_repeated_heads_summed():
 
 
 @pytest.mark.parametrize("causal", [False, True])
+def test_bwd_varlen_equals_finite_differences(causal):
+    """Packed sequences: central differences of L = sum(O * G) with O from the
+    varlen forward definition; a gradient leaking across a sequence boundary
+    (or a boundary read off by one row) would fail."""
+    lens = [3, 1, 4]
+    H, Hkv, d = 2, 1, 3
+    total = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    q, g = _rand((total, H, d), 240), _rand((total, H, d), 241)
+    k, v = _rand((total, Hkv, d), 242), _rand((total, Hkv, d), 243)
+    scale = 0.8
+    dq, dk, dv = oracle.attention_bwd_varlen(q, k, v, g, cu, causal, scale)
+
+    def loss(q_, k_, v_):
+        o = np.zeros_like(q_)
+        for b in range(len(lens)):
+            s0, s1 = cu[b], cu[b + 1]
+            ob, _ = oracle.attention_gqa(q_[s0:s1].transpose(1, 0, 2)[None],
+                                         k_[s0:s1].transpose(1, 0, 2)[None],
+                                         v_[s0:s1].transpose(1, 0, 2)[None], causal, scale)
+            o[s0:s1] = ob[0].transpose(1, 0, 2)
+        return float(np.sum(o * g))
+
+    h = 1e-5
+    for x, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(grad, num, atol=1e-8)
+
+
+def test_bwd_varlen_single_sequence_is_fixed_length():
+    N, H, d = 11, 2, 4
+    q, k, v, g = (_rand((N, H, d), s) for s in (244, 245, 246, 247))
+    dq, dk, dv = oracle.attention_bwd_varlen(q, k, v, g, [0, N], True, 0.5)
+    t = lambda x: x.transpose(1, 0, 2)[None]
+    rq, rk, rv = oracle.attention_bwd(t(q), t(k), t(v), t(g), True, 0.5)
+    for a, b in ((dq, rq), (dk, rk), (dv, rv)):
+        np.testing.assert_allclose(t(a), b, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
 def test_bwd_key_gradients_sum_to_zero(causal):
     """Each row of dS sums to zero (the softmax Jacobian annihilates
     constants), so sum_j dK_j = scale sum_i q_i sum_j dS_ij = 0; dropping the
