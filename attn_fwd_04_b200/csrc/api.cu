@@ -293,6 +293,58 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     return fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, causal, scale, stream);
 }
 
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, const int32_t* cu_seqlens,
+                  int B, int H, int H_kv, int total, int max_seqlen, int d, int causal,
+                  float scale, fa_stream_t stream) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !cu_seqlens)
+        return FA_ERR_NULL;
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || total < 1 || max_seqlen < 1)
+        return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (max_seqlen > 0x7fffffff - 128 || static_cast<int64_t>(total) * H > 0x7fffffff / 128)
+        return FA_ERR_SHAPE;
+    if (static_cast<int64_t>((max_seqlen + 127) / 128) * B * H_kv > 0x7fffffff)
+        return FA_ERR_SHAPE;
+    if (!std::isfinite(scale)) return FA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    // packed [total, heads, d] as (d, heads, total), a box of 128 rows of one head
+    CUtensorMap tq, tk, tv, tdo;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(total)};
+    const cuuint64_t dims_kv[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_kv),
+                                   static_cast<cuuint64_t>(total)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(H) * d * 2};
+    const cuuint64_t strides_kv[2] = {static_cast<cuuint64_t>(d) * 2,
+                                      static_cast<cuuint64_t>(H_kv) * d * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims_kv, strides_kv, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims_kv, strides_kv, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tdo, dout, dims, strides, box)) != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if ((rc = ensure_workspace(s, fa::bwd_workspace_bytes(1, H, total, d), st, &ws)) != FA_OK)
+        return rc;
+    // the fp32 dQ accumulator [total, H, d] in the workspace, reduced into by TMA
+    CUtensorMap tdq;
+    const cuuint64_t astrides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                    static_cast<cuuint64_t>(H) * d * 4};
+    const cuuint32_t abox[3] = {32, 1, 128};
+    if ((rc = make_map_f32(&tdq, static_cast<uint8_t*>(ws) + fa::bwd_dq_acc_offset(1, H, total),
+                           dims, astrides, abox)) != FA_OK)
+        return rc;
+    return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, tdq, B, H, H_kv, max_seqlen,
+                          d, causal ? 1 : 0, scale, ws, s->err, s->num_sms, st, cu_seqlens,
+                          total);
+}
+
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int32_t* cu_seqlens, int B, int H, int total, int max_seqlen, int d,
                   int causal, float scale, fa_stream_t stream) {

@@ -76,12 +76,14 @@ struct alignas(1024) BwdSmem {
 };
 
 struct BwdParams {
-    const float* lse2;   // [B*H*N] lse * log2(e)
-    const float* dsum;   // [B*H*N] D
+    const float* lse2;   // per row of O: lse * log2(e)
+    const float* dsum;   // per row of O: D
     float* dq_acc;       // [B*H*N*D] fp32, cleared by the prep kernel
     void* dk;
     void* dv;
     int B, H, H_kv, N, causal;  // query head h uses K/V head h / (H / H_kv)
+    const int32_t* cu_seqlens;  // packed sequences: offsets [B+1]; N is the longest length
+    int total;                  // packed sequences: rows of q, k, v
     float scale, scale_log2;
     unsigned int* err;
 };
@@ -100,13 +102,16 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) 
 
 // ---------------------------------------------------------------------------
 // prep: D_i = dO_i . O_i, lse2_i = lse_i * log2(e), dQ accumulator rows = 0.
-// One warp per row.
+// One warp per row r of O.  lse_total = 0: lse is indexed like the rows of O;
+// otherwise O is packed [total, H, d] (row r = token r / H, head r % H) and
+// lse is [H, total].
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                        const float* __restrict__ lse, float* __restrict__ lse2,
-                       float* __restrict__ dsum, float* __restrict__ dq_acc, int64_t rows) {
+                       float* __restrict__ dsum, float* __restrict__ dq_acc, int64_t rows, int H,
+                       int64_t lse_total) {
     constexpr int PER = D / 32;  // elements per lane
     const int lane = threadIdx.x & 31;
     for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
@@ -127,7 +132,8 @@ __global__ void __launch_bounds__(256)
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) {
             dsum[r] = acc;
-            lse2[r] = lse[r] * 1.4426950408889634f;
+            const int64_t li = lse_total ? (r % H) * lse_total + r / H : r;
+            lse2[r] = lse[li] * 1.4426950408889634f;
         }
         float4* dq = reinterpret_cast<float4*>(dq_acc + r * D);
         for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -155,7 +161,13 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // main kernel
 // ---------------------------------------------------------------------------
-template <int D>
+// VARLEN: q, k, v, o, dout packed [total, heads, d] (maps over (d, heads,
+// total), 64 x 1 x 128 boxes); sequence b owns rows cu_seqlens[b] ..
+// cu_seqlens[b+1]-1 and attends within itself.  Rows of a tile past its
+// sequence belong to the next one (or lie past the tensor): their P is 0
+// (statistics lse = +inf), so their dQ rows add exact zeros and their keys
+// contribute nothing; dK, dV rows past the sequence are not stored.
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -171,9 +183,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int jb = within / ug;
     const int bh = gidx * kBwdHeadGroup + (within - jb * ug);  // flat (sequence, K/V head)
     if (jb >= nkb || bh >= units) return;
+    // the sequence: its first packed row and length (fixed length: N rows)
+    int seq0 = 0, len = p.N;
+    if constexpr (VARLEN) {
+        const int b = bh / p.H_kv;
+        const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
+        // keep every access inside the packed tensors whatever the offsets say
+        const int c0 = min(max(s0, 0), p.total), c1 = min(max(s1, c0), p.total);
+        const int c1m = min(c1, c0 + p.N);
+        if ((c0 != s0 || c1m != s1) && jb == 0 && bh % p.H_kv == 0 && threadIdx.x == 0)
+            record_error(p.err, FA_DEVERR_BAD_INPUT);
+        seq0 = c0;
+        len = c1m - c0;
+    }
+    const int nkb_seq = (len + kBT - 1) / kBT;
+    if (jb >= nkb_seq) return;
     const int key0 = jb * kBT;
     const int i_first = p.causal ? jb : 0;
-    const int nt = nkb - i_first;  // query tiles of one query head that see this key block
+    const int nt = nkb_seq - i_first;  // query tiles of one query head that see this key block
     // the CTA walks the query tiles of every query head of its K/V head's
     // group (dK, dV sum over all of them): tile t is query tile
     // i_first + t % nt of query head t / nt of the group
@@ -182,6 +209,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int qh0 = (bh / p.H_kv) * p.H + (bh % p.H_kv) * G;  // flat first query head
     auto tile_q0 = [&](int t) { return (i_first + t % nt) * kBT; };
     auto tile_qh = [&](int t) { return qh0 + t / nt; };
+    // row `row` of the sequence for (flat) head `head` as tensor-map
+    // coordinates, and the index of that row of O (statistics)
+    auto map_row = [&](int row) { return VARLEN ? seq0 + row : row; };
+    auto map_head = [&](int head, int heads) { return VARLEN ? head % heads : head; };
+    auto stat_index = [&](int head, int row) -> int64_t {
+        return VARLEN ? static_cast<int64_t>(seq0 + row) * p.H + head % p.H
+                      : static_cast<int64_t>(head) * p.N + row;
+    };
 
     extern __shared__ uint8_t bwd_smem_raw[];
     BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(
@@ -220,10 +255,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp >= 8) regs_dec<kRegsWg2>();
     if (warp == 9) {
         // ================= TMA producer (+ per-tile statistics) =================
-        auto load2 = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row, int head) {
+        // fixed length: maps over (d, N, sequences * heads); packed: (d, heads, total)
+        auto load2 = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row, int head,
+                         int heads) {
 #pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb)
-                tma_load_3d(dst + cb * kBoxB, map, bar, cb * 64, row, head);
+            for (int cb = 0; cb < D / 64; ++cb) {
+                if constexpr (VARLEN)
+                    tma_load_3d(dst + cb * kBoxB, map, bar, cb * 64, map_head(head, heads),
+                                map_row(row));
+                else
+                    tma_load_3d(dst + cb * kBoxB, map, bar, cb * 64, row, head);
+            }
         };
         bool ok = true;
         if (lane == 0) {
@@ -232,8 +274,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_prefetch_desc(&tv);
             tma_prefetch_desc(&tdo);
             mbar_arrive_expect_tx(&sm.kv_full, 2 * kBT * D * 2);
-            load2(sm.k, &tk, &sm.kv_full, key0, bh);
-            load2(sm.v, &tv, &sm.kv_full, key0, bh);
+            load2(sm.k, &tk, &sm.kv_full, key0, bh, p.H_kv);
+            load2(sm.v, &tv, &sm.kv_full, key0, bh, p.H_kv);
         }
         int issued = 0;
         for (int t = 0; t < ntt; ++t) {
@@ -245,14 +287,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int q0 = tile_q0(t), qh = tile_qh(t);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.in_full[s], 2 * kBT * D * 2);
-                load2(sm.q[s], &tq, &sm.in_full[s], q0, qh);
-                load2(sm.dout[s], &tdo, &sm.in_full[s], q0, qh);
+                load2(sm.q[s], &tq, &sm.in_full[s], q0, qh, p.H);
+                load2(sm.dout[s], &tdo, &sm.in_full[s], q0, qh, p.H);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = lane * 4 + e, qr = q0 + r;
-                const bool in = qr < p.N;
-                const int64_t gi = static_cast<int64_t>(qh) * p.N + qr;
+                const bool in = qr < len;
+                const int64_t gi = in ? stat_index(qh, qr) : 0;
                 sm.nlse2[s][r] = in ? -p.lse2[gi] : -INFINITY;  // rows past N: P = 0
                 sm.ndsum[s][r] = in ? -p.dsum[gi] : 0.f;
             }
@@ -369,7 +411,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int r = threadIdx.x;  // TMEM lane == key row of the block
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         const int key = key0 + r;
-        const bool key_in = key < p.N;
+        const bool key_in = key < len;
         const float sl = p.scale_log2;
         for (int t = 0; t < ntt; ++t) {
             const int s = t & 1;
@@ -520,7 +562,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 bar_sync_named(1, kBT);  // every row is in the tile
                 if (r == 0) {
-                    tma_reduce_add_3d(&tdq, stage, c * 32, q0, qh);
+                    if constexpr (VARLEN)
+                        tma_reduce_add_3d(&tdq, stage, c * 32, qh % p.H, seq0 + q0);
+                    else
+                        tma_reduce_add_3d(&tdq, stage, c * 32, q0, qh);
                     bulk_commit_group();
                     bulk_wait_group_read0();
                 }
@@ -529,14 +574,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (r == 0) bulk_wait_group0();  // the reductions have landed
         if (ok) {
             // every MMA has completed (the last dq_full follows the last one);
-            // the whole warp loads (tcgen05.ld is warp-wide), rows past N are
-            // not stored
+            // the whole warp loads (tcgen05.ld is warp-wide), rows past the
+            // sequence are not stored
             const int key = key0 + r;
-            const bool store = key < p.N;
-            __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(p.dv) +
-                                 (static_cast<int64_t>(bh) * p.N + key) * D;
-            __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(p.dk) +
-                                 (static_cast<int64_t>(bh) * p.N + key) * D;
+            const bool store = key < len;
+            const int64_t krow = VARLEN ? static_cast<int64_t>(seq0 + key) * p.H_kv + bh % p.H_kv
+                                        : static_cast<int64_t>(bh) * p.N + key;
+            __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(p.dv) + krow * D;
+            __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(p.dk) + krow * D;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const uint32_t col = which ? kColDK : kColDV;
@@ -574,12 +619,14 @@ int launch_bwd_impl(const void* o, const void* dout, const float* lse, float* ls
                     float* dq_acc, void* dq, const CUtensorMap& tq, const CUtensorMap& tk,
                     const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
                     const BwdParams& p, int num_sms, cudaStream_t stream) {
-    const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.N;
+    const bool varlen = p.cu_seqlens != nullptr;
+    const int64_t rows = varlen ? static_cast<int64_t>(p.total) * p.H
+                                : static_cast<int64_t>(p.B) * p.H * p.N;
     fa_bwd_prep_kernel<D><<<num_sms * 8, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
-        dsum, dq_acc, rows);
+        dsum, dq_acc, rows, p.H, varlen ? p.total : 0);
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
-    auto kern = fa_bwd_kernel<D>;
+    auto kern = varlen ? fa_bwd_kernel<D, true> : fa_bwd_kernel<D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -607,12 +654,14 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int H_kv, int N, int d,
                int causal, float scale, void* workspace, unsigned int* err, int num_sms,
-               cudaStream_t stream) {
-    const size_t rows = static_cast<size_t>(B) * H * N;
+               cudaStream_t stream, const int32_t* cu_seqlens, int total) {
+    // statistics and the dQ accumulator: one entry per row of O
+    const int Bw = cu_seqlens ? 1 : B, Nw = cu_seqlens ? total : N;
+    const size_t rows = static_cast<size_t>(Bw) * H * Nw;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* lse2 = reinterpret_cast<float*>(ws);
     float* dsum = lse2 + rows;
-    float* dq_acc = reinterpret_cast<float*>(ws + bwd_dq_acc_offset(B, H, N));
+    float* dq_acc = reinterpret_cast<float*>(ws + bwd_dq_acc_offset(Bw, H, Nw));
     BwdParams p{};
     p.lse2 = lse2;
     p.dsum = dsum;
@@ -624,6 +673,8 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
     p.H_kv = H_kv;
     p.N = N;
     p.causal = causal;
+    p.cu_seqlens = cu_seqlens;
+    p.total = total;
     p.scale = scale;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = err;

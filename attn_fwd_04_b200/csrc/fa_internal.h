@@ -50,7 +50,7 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& tdo, const CUtensorMap& tdq, int B, int H, int H_kv, int N, int d,
                int causal, float scale, void* workspace, unsigned int* err, int num_sms,
-               cudaStream_t stream);
+               cudaStream_t stream, const int32_t* cu_seqlens = nullptr, int total = 0);
 
 // ---- paged decode ----------------------------------------------------------
 // Number of pages a split covers at least (a split is one CTA work unit) and

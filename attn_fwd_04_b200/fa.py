@@ -24,7 +24,8 @@ FA_ERR_NOMEM = -7
 FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
-EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_fwd_varlen",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_bwd_varlen",
+           "fa_fwd_varlen",
            "fa_decode_paged",
            "fa_decode_paged_gqa", "fa_decode_paged_strided",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
@@ -56,6 +57,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+        L.fa_bwd_varlen.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.fa_decode_paged_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_decode_paged_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
@@ -70,7 +72,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
         L.fa_fwd_set_cta_pairs.argtypes = [I]
-        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_fwd_varlen",
+        for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_bwd_varlen",
+                     "fa_fwd_varlen",
                      "fa_decode_paged",
                      "fa_decode_paged_gqa", "fa_decode_paged_strided", "fa_decode_paged_noalloc",
                      "fa_append_paged",
@@ -224,6 +227,34 @@ def fa_bwd_gqa(q, k, v, o, lse, dout, causal: bool, scale: Optional[float] = Non
                           dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H,
                           H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
     _raise_if(rc, "fa_bwd_gqa")
+    return dq, dk, dv
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen: int, causal: bool,
+                  scale: Optional[float] = None, dq=None, dk=None, dv=None, stream=None):
+    """Gradients of fa_fwd_varlen over packed sequences: dq [total,H,d] and dk, dv
+    [total,H_kv,d] bf16, from q, o, dout [total,H,d], k, v [total,H_kv,d] bf16 and
+    lse [H,total] fp32 (as fa_fwd_varlen returned it)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, n, torch.bfloat16, 3)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    _check(lse, "lse", torch.float32, 2)
+    total, H, d = q.shape
+    H_kv = k.shape[1]
+    if o.shape != q.shape or dout.shape != q.shape or k.shape != (total, H_kv, d) or \
+            v.shape != k.shape:
+        raise ValueError("q, o, dout must be [total,H,d] and k, v [total,H_kv,d]")
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), cu_seqlens.data_ptr(), B, H, H_kv, total,
+                             int(max_seqlen), d, int(bool(causal)), float(scale), _stream(stream))
+    _raise_if(rc, "fa_bwd_varlen")
     return dq, dk, dv
 
 

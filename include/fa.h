@@ -168,6 +168,25 @@ FA_API int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o
                       int H, int H_kv, int N, int d, int causal, float scale, fa_stream_t stream);
 
 /*
+ * fa_bwd_varlen -- gradients of fa_fwd_varlen (with grouped K/V heads) over
+ * B packed sequences of different lengths.
+ *   q, o, dout, dq : [total, H, d] bf16;  lse : [H, total] fp32 as returned
+ *                    by fa_fwd_varlen
+ *   k, v, dk, dv   : [total, H_kv, d] bf16 (H_kv = H for plain multi-head;
+ *                    query head h uses K/V head h / (H / H_kv))
+ *   cu_seqlens     : DEVICE int32 [B+1], as for fa_fwd_varlen; max_seqlen
+ *                    bounds every length (a longer sequence is cut to it and
+ *                    reported, like out-of-range offsets)
+ * Each sequence's gradients are those of fa_bwd on its own rows.  Workspace:
+ * total*H*(2 + d)*4 bytes, as fa_bwd.  Same `causal`, `scale`, d and alignment
+ * rules as fa_fwd_varlen.
+ */
+FA_API int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                         const int32_t* cu_seqlens, int B, int H, int H_kv, int total,
+                         int max_seqlen, int d, int causal, float scale, fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- the forward pass over B sequences of different lengths
  * packed back to back (the variable-length batches of the page "Flash
  * Attention 是什么", section 典型应用场景).

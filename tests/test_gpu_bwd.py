@@ -135,3 +135,76 @@ def test_bwd_gqa_group1_equals_bwd():
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     assert_grad_close(to64(b[0]), to64(a[0]), "dq group 1")
 
+
+
+# -- packed variable-length sequences (fa_bwd_varlen) --------------------------------
+
+def _varlen(lengths, H, Hkv, d, seed):
+    total = sum(lengths)
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    q, k, v = W.gqa_fwd_inputs(1, H, Hkv, total, d, seed=seed, device="cpu")
+    # [1, heads, total, d] -> packed [total, heads, d]
+    q, k, v = (x[0].transpose(0, 1).contiguous() for x in (q, k, v))
+    g = _grad_out((total, H, d), seed + 1)
+    return q, k, v, g, cu
+
+
+def _bwd_varlen_gpu(q, k, v, g, cu, o, lse, causal, scale):
+    dq = torch.full_like(q.cuda(), float("nan"))
+    dk = torch.full_like(k.cuda(), float("nan"))
+    dv = torch.full_like(v.cuda(), float("nan"))
+    maxlen = int((cu[1:] - cu[:-1]).max())
+    fa.fa_bwd_varlen(q.cuda(), k.cuda(), v.cuda(), o, lse, g.cuda(), cu.cuda(), maxlen, causal,
+                     scale, dq=dq, dk=dk, dv=dv)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_varlen_full_compare(d, causal):
+    lengths = [300, 1, 129, 0, 513, 128]
+    q, k, v, g, cu = _varlen(lengths, 2, 2, d, 820 + d)
+    scale = 1 / math.sqrt(d)
+    o, lse = fa.fa_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lengths), causal,
+                              scale)
+    dq, dk, dv = _bwd_varlen_gpu(q, k, v, g, cu, o, lse, causal, scale)
+    rq, rk, rv = oracle.attention_bwd_varlen(q, k, v, g, cu, causal, scale)
+    assert_grad_close(to64(dv), rv, "dv varlen")
+    assert_grad_close(to64(dk), rk, "dk varlen")
+    assert_grad_close(to64(dq), rq, "dq varlen")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_varlen_gqa_full_compare(causal):
+    """Grouped K/V heads over packed sequences; o and lse come from the oracle's
+    forward pass (rounded as the GPU forward rounds them)."""
+    lengths = [257, 40, 700]
+    H, Hkv, d = 4, 2, 128
+    q, k, v, g, cu = _varlen(lengths, H, Hkv, d, 830)
+    scale = 1 / math.sqrt(d)
+    o = torch.zeros(q.shape, dtype=torch.bfloat16)
+    lse = torch.zeros((H, q.shape[0]), dtype=torch.float32)
+    for b in range(len(lengths)):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        ob, lb = oracle.attention_gqa(q[s0:s1].transpose(0, 1)[None], k[s0:s1].transpose(0, 1)[None],
+                                      v[s0:s1].transpose(0, 1)[None], causal, scale)
+        o[s0:s1] = torch.from_numpy(ob[0]).transpose(0, 1).to(torch.bfloat16)
+        lse[:, s0:s1] = torch.from_numpy(lb[0]).float()
+    dq, dk, dv = _bwd_varlen_gpu(q, k, v, g, cu, o.cuda(), lse.cuda(), causal, scale)
+    rq, rk, rv = oracle.attention_bwd_varlen(q, k, v, g, cu, causal, scale)
+    assert_grad_close(to64(dv), rv, "dv varlen gqa")
+    assert_grad_close(to64(dk), rk, "dk varlen gqa")
+    assert_grad_close(to64(dq), rq, "dq varlen gqa")
+
+
+def test_bwd_varlen_one_sequence_equals_fixed():
+    """A single packed sequence gives fa_bwd's dk, dv bit for bit."""
+    N, H, d = 700, 2, 128
+    q, k, v, g, cu = _varlen([N], H, H, d, 840)
+    o, lse = fa.fa_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), N, True, 0.1)
+    a = _bwd_varlen_gpu(q, k, v, g, cu, o, lse, True, 0.1)
+    t = lambda x: x.transpose(0, 1)[None].contiguous()
+    b = _bwd_gpu(t(q), t(k), t(v), t(g), True, 0.1)
+    assert torch.equal(t(a[1]), b[1]) and torch.equal(t(a[2]), b[2])
+    assert_grad_close(to64(t(a[0])), to64(b[0]), "dq one sequence")
