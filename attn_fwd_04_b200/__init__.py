@@ -9,7 +9,7 @@ from .fa import (EXPORTS, FA_ERR_ALIGN, FA_ERR_CUDA, FA_ERR_DEVICE_BAD_INPUT,  #
                  fa_decode_paged_strided,
                  fa_decode_paged_noalloc, fa_append_paged, fa_prefill_paged,
                  fa_bwd, fa_bwd_gqa, fa_bwd_varlen, fa_fwd, fa_fwd_gqa, fa_fwd_rope,
-                 fa_fwd_set_cta_pairs,
+                 fa_fwd_set_cta_pairs, fa_fwd_varlen_gqa,
                  fa_fwd_varlen,
                  fa_gather_paged, fa_get_device_error, fa_release_workspace, fa_selftest_bounded_wait,
                  fa_status_str,

@@ -345,11 +345,12 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                           total);
 }
 
-int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
-                  const int32_t* cu_seqlens, int B, int H, int total, int max_seqlen, int d,
-                  int causal, float scale, fa_stream_t stream) {
+int fa_fwd_varlen_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int32_t* cu_seqlens, int B, int H, int H_kv, int total,
+                      int max_seqlen, int d, int causal, float scale, fa_stream_t stream) {
     if (!q || !k || !v || !o || !lse || !cu_seqlens) return FA_ERR_NULL;
-    if (B < 1 || H < 1 || total < 1 || max_seqlen < 1) return FA_ERR_SHAPE;
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || total < 1 || max_seqlen < 1)
+        return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (B > 65535 || H > 65535) return FA_ERR_SHAPE;
     if (max_seqlen > 0x7fffffff - 128) return FA_ERR_SHAPE;
@@ -362,25 +363,36 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
     CUtensorMap tq, tk, tv;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(total)};
+    const cuuint64_t dims_kv[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_kv),
+                                   static_cast<cuuint64_t>(total)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                    static_cast<cuuint64_t>(H) * d * 2};
+    const cuuint64_t strides_kv[2] = {static_cast<cuuint64_t>(d) * 2,
+                                      static_cast<cuuint64_t>(H_kv) * d * 2};
     const cuuint32_t box[3] = {64, 1, 128};
     if ((rc = make_map(&tq, q, dims, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tk, k, dims, strides, box)) != FA_OK) return rc;
-    if ((rc = make_map(&tv, v, dims, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, dims_kv, strides_kv, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, dims_kv, strides_kv, box)) != FA_OK) return rc;
     fa::FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.cu_seqlens = cu_seqlens;
     p.B = B;
     p.H = H;
-    p.H_kv = H;
+    p.H_kv = H_kv;
     p.N = max_seqlen;
     p.total = total;
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
     return fa::launch_fwd(p, tq, tk, tv, d, fa::kVarlen, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens, int B, int H, int total, int max_seqlen, int d,
+                  int causal, float scale, fa_stream_t stream) {
+    return fa_fwd_varlen_gqa(q, k, v, o, lse, cu_seqlens, B, H, H, total, max_seqlen, d, causal,
+                             scale, stream);
 }
 
 int fa_prefill_paged(const void* q, const void* k_pages, const void* v_pages,

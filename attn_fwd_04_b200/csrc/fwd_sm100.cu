@@ -290,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         seq_start = c0;
         len = c1m - c0;
         klen = len;
+        bkv = h / (p.H / p.H_kv);  // packed K/V: the head coordinate of the token rows
         if constexpr (PAGED) {
-            bkv = h / (p.H / p.H_kv);
             const int ctx = p.ctx_lens[b];
             if (ctx < len) {  // more queries than cached tokens: not computed
                 if (rank == 0 && threadIdx.x == 0) record_error(p.err, FA_DEVERR_BAD_INPUT);
@@ -393,13 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            // head: the fixed-length maps' outer coordinate (flat sequence/head)
+            // head: the fixed-length maps' outer coordinate (flat sequence/head),
+            // or the packed maps' head coordinate
             auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row,
                                  int head) {
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb) {
                     if constexpr (VARLEN)
-                        tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, h, seq_start + row);
+                        tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, head, seq_start + row);
                     else
                         tma_load_3d(dst + cb * kBoxBytes, map, bar, cb * 64, row, head);
                 }
@@ -451,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = 0; t < 2; ++t) {
                 if (n_t[t] > 0) {
                     mbar_arrive_expect_tx(&sm.q_full[t], BM * D * 2);
-                    load_tile(sm.q[t], &tq, &sm.q_full[t], tile_row(t), bh);
+                    load_tile(sm.q[t], &tq, &sm.q_full[t], tile_row(t), VARLEN ? h : bh);
                 }
             }
             for (int u = 0; u < 2 * n; ++u) {

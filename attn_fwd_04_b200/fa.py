@@ -25,7 +25,7 @@ FA_ERR_DEVICE_BAD_INPUT = -8
 
 # every symbol include/fa.h declares
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_bwd_varlen",
-           "fa_fwd_varlen",
+           "fa_fwd_varlen", "fa_fwd_varlen_gqa",
            "fa_decode_paged",
            "fa_decode_paged_gqa", "fa_decode_paged_strided",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+        L.fa_fwd_varlen_gqa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_fwd_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
         L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
         L.fa_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
@@ -73,7 +74,7 @@ def lib() -> ctypes.CDLL:
         L.fa_version.argtypes = []
         L.fa_fwd_set_cta_pairs.argtypes = [I]
         for name in ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_bwd_varlen",
-                     "fa_fwd_varlen",
+                     "fa_fwd_varlen", "fa_fwd_varlen_gqa",
                      "fa_decode_paged",
                      "fa_decode_paged_gqa", "fa_decode_paged_strided", "fa_decode_paged_noalloc",
                      "fa_append_paged",
@@ -277,6 +278,32 @@ def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
                              int(max_seqlen), d, int(bool(causal)), float(scale),
                              _stream(stream))
     _raise_if(rc, "fa_fwd_varlen")
+    return o, lse
+
+
+def fa_fwd_varlen_gqa(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
+                      scale: Optional[float] = None, o=None, lse=None, stream=None):
+    """Forward over packed sequences with grouped K/V heads: q [total,H,d], k, v
+    [total,H_kv,d] -> (o [total,H,d], lse [H,total] fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 3)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    total, H, d = q.shape
+    H_kv = k.shape[1]
+    if k.shape != (total, H_kv, d) or v.shape != k.shape:
+        raise ValueError("k, v must be [total,H_kv,d]")
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    rc = lib().fa_fwd_varlen_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), cu_seqlens.data_ptr(), B, H, H_kv, total,
+                                 int(max_seqlen), d, int(bool(causal)), float(scale),
+                                 _stream(stream))
+    _raise_if(rc, "fa_fwd_varlen_gqa")
     return o, lse
 
 

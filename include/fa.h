@@ -208,6 +208,16 @@ FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, f
                   int causal, float scale, fa_stream_t stream);
 
 /*
+ * fa_fwd_varlen_gqa -- fa_fwd_varlen with grouped K/V heads: q, o
+ * [total, H, d], k, v [total, H_kv, d] bf16 (H a multiple of H_kv,
+ * FA_ERR_SHAPE otherwise); query head h attends with K/V head h / (H / H_kv)
+ * of its own sequence.  fa_fwd_varlen is this call with H_kv = H.
+ */
+FA_API int fa_fwd_varlen_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const int32_t* cu_seqlens, int B, int H, int H_kv, int total,
+                             int max_seqlen, int d, int causal, float scale, fa_stream_t stream);
+
+/*
  * fa_decode_paged -- single-token decode over a paged KV cache, split over
  * the cache pages and merged by log-sum-exp.
  *

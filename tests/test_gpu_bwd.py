@@ -10,7 +10,7 @@ import torch
 import attn_fwd_04_b200 as fa
 import oracle
 from attn_fwd_04_b200 import workloads as W
-from helpers import assert_grad_close, to64
+from helpers import assert_grad_close, assert_lse_close, assert_o_close, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -176,22 +176,23 @@ def test_bwd_varlen_full_compare(d, causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_bwd_varlen_gqa_full_compare(causal):
-    """Grouped K/V heads over packed sequences; o and lse come from the oracle's
-    forward pass (rounded as the GPU forward rounds them)."""
+def test_varlen_gqa_forward_and_backward(causal):
+    """Grouped K/V heads over packed sequences: the forward pass against the
+    oracle, then the backward pass from its o and lse."""
     lengths = [257, 40, 700]
     H, Hkv, d = 4, 2, 128
     q, k, v, g, cu = _varlen(lengths, H, Hkv, d, 830)
     scale = 1 / math.sqrt(d)
-    o = torch.zeros(q.shape, dtype=torch.bfloat16)
-    lse = torch.zeros((H, q.shape[0]), dtype=torch.float32)
+    o, lse = fa.fa_fwd_varlen_gqa(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lengths), causal,
+                                  scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
     for b in range(len(lengths)):
         s0, s1 = int(cu[b]), int(cu[b + 1])
         ob, lb = oracle.attention_gqa(q[s0:s1].transpose(0, 1)[None], k[s0:s1].transpose(0, 1)[None],
                                       v[s0:s1].transpose(0, 1)[None], causal, scale)
-        o[s0:s1] = torch.from_numpy(ob[0]).transpose(0, 1).to(torch.bfloat16)
-        lse[:, s0:s1] = torch.from_numpy(lb[0]).float()
-    dq, dk, dv = _bwd_varlen_gpu(q, k, v, g, cu, o.cuda(), lse.cuda(), causal, scale)
+        assert_o_close(to64(o[s0:s1].transpose(0, 1)), ob[0], f"fwd varlen gqa seq {b}")
+        assert_lse_close(to64(lse[:, s0:s1]), lb[0], f"fwd varlen gqa seq {b}")
+    dq, dk, dv = _bwd_varlen_gpu(q, k, v, g, cu, o, lse, causal, scale)
     rq, rk, rv = oracle.attention_bwd_varlen(q, k, v, g, cu, causal, scale)
     assert_grad_close(to64(dv), rv, "dv varlen gqa")
     assert_grad_close(to64(dk), rk, "dk varlen gqa")
