@@ -332,13 +332,16 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
     void* ws = nullptr;
     if ((rc = ensure_workspace(s, fa::bwd_workspace_bytes(1, H, total, d), st, &ws)) != FA_OK)
         return rc;
-    // the fp32 dQ accumulator [total, H, d] in the workspace, reduced into by TMA
+    // the fp32 dQ accumulator, head-major [H, total, d] in the workspace (a
+    // tile's rows contiguous), reduced into by TMA
     CUtensorMap tdq;
+    const cuuint64_t adims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(total),
+                                 static_cast<cuuint64_t>(H)};
     const cuuint64_t astrides[2] = {static_cast<cuuint64_t>(d) * 4,
-                                    static_cast<cuuint64_t>(H) * d * 4};
-    const cuuint32_t abox[3] = {32, 1, 128};
+                                    static_cast<cuuint64_t>(total) * d * 4};
+    const cuuint32_t abox[3] = {32, 128, 1};
     if ((rc = make_map_f32(&tdq, static_cast<uint8_t*>(ws) + fa::bwd_dq_acc_offset(1, H, total),
-                           dims, astrides, abox)) != FA_OK)
+                           adims, astrides, abox)) != FA_OK)
         return rc;
     return fa::launch_bwd(o, dout, lse, dq, dk, dv, tq, tk, tv, tdo, tdq, B, H, H_kv, max_seqlen,
                           d, causal ? 1 : 0, scale, ws, s->err, s->num_sms, st, cu_seqlens,

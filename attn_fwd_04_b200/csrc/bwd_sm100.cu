@@ -102,9 +102,11 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) 
 
 // ---------------------------------------------------------------------------
 // prep: D_i = dO_i . O_i, lse2_i = lse_i * log2(e), dQ accumulator rows = 0.
-// One warp per row r of O.  lse_total = 0: lse is indexed like the rows of O;
-// otherwise O is packed [total, H, d] (row r = token r / H, head r % H) and
-// lse is [H, total].
+// One warp per row r of O.  lse_total = 0: lse, the statistics and the
+// accumulator are indexed like the rows of O; otherwise O is packed
+// [total, H, d] (row r = token r / H, head r % H) and lse, the statistics and
+// the accumulator rows are head-major ([H, total], [H, total, d]), so that a
+// tile's rows are contiguous in them.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
@@ -130,25 +132,31 @@ __global__ void __launch_bounds__(256)
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        const int64_t li = lse_total ? (r % H) * lse_total + r / H : r;
         if (lane == 0) {
-            dsum[r] = acc;
-            const int64_t li = lse_total ? (r % H) * lse_total + r / H : r;
-            lse2[r] = lse[li] * 1.4426950408889634f;
+            dsum[li] = acc;
+            lse2[li] = lse[li] * 1.4426950408889634f;
         }
-        float4* dq = reinterpret_cast<float4*>(dq_acc + r * D);
+        float4* dq = reinterpret_cast<float4*>(dq_acc + li * D);
         for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
-// dq (bf16) <- dQ accumulator (fp32), 8 values per thread
+// dq (bf16) <- dQ accumulator (fp32), 8 values per thread; with lse_total
+// the accumulator is head-major [H, total, D] and dq packed [total, H, D]
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_dq_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq,
-                     int64_t n8) {
+                     int64_t n8, int H, int64_t lse_total) {
     for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < n8;
          x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * x];
-        const float4 b = reinterpret_cast<const float4*>(dq_acc)[2 * x + 1];
+        int64_t src = x;  // in units of 8 values
+        if (lse_total) {
+            const int64_t r = x / (D / 8), c = x - r * (D / 8);  // row of dq, 8-column chunk
+            src = ((r % H) * lse_total + r / H) * (D / 8) + c;
+        }
+        const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * src];
+        const float4 b = reinterpret_cast<const float4*>(dq_acc)[2 * src + 1];
         uint4 w;
         w.x = pack_bf16x2(a.x, a.y);
         w.y = pack_bf16x2(a.z, a.w);
@@ -162,7 +170,8 @@ __global__ void __launch_bounds__(256)
 // main kernel
 // ---------------------------------------------------------------------------
 // VARLEN: q, k, v, o, dout packed [total, heads, d] (maps over (d, heads,
-// total), 64 x 1 x 128 boxes); sequence b owns rows cu_seqlens[b] ..
+// total), 64 x 1 x 128 boxes; the statistics and the fp32 dQ accumulator are
+// head-major, [H, total] and [H, total, d]); sequence b owns rows cu_seqlens[b] ..
 // cu_seqlens[b+1]-1 and attends within itself.  Rows of a tile past its
 // sequence belong to the next one (or lie past the tensor): their P is 0
 // (statistics lse = +inf), so their dQ rows add exact zeros and their keys
@@ -214,7 +223,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto map_row = [&](int row) { return VARLEN ? seq0 + row : row; };
     auto map_head = [&](int head, int heads) { return VARLEN ? head % heads : head; };
     auto stat_index = [&](int head, int row) -> int64_t {
-        return VARLEN ? static_cast<int64_t>(seq0 + row) * p.H + head % p.H
+        return VARLEN ? static_cast<int64_t>(head % p.H) * p.total + seq0 + row
                       : static_cast<int64_t>(head) * p.N + row;
     };
 
@@ -562,8 +571,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 bar_sync_named(1, kBT);  // every row is in the tile
                 if (r == 0) {
-                    if constexpr (VARLEN)
-                        tma_reduce_add_3d(&tdq, stage, c * 32, qh % p.H, seq0 + q0);
+                    if constexpr (VARLEN)  // head-major accumulator (d, total, H)
+                        tma_reduce_add_3d(&tdq, stage, c * 32, seq0 + q0, qh % p.H);
                     else
                         tma_reduce_add_3d(&tdq, stage, c * 32, q0, qh);
                     bulk_commit_group();
@@ -635,7 +644,8 @@ int launch_bwd_impl(const void* o, const void* dout, const float* lse, float* ls
     kern<<<dim3(static_cast<unsigned>(ctas)), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq,
                                                                            p);
     fa_bwd_dq_kernel<D><<<num_sms * 8, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
-                                                          rows * D / 8);
+                                                          rows * D / 8, p.H,
+                                                          varlen ? p.total : 0);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

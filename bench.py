@@ -336,6 +336,30 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
                             stream=stream),
           2.5 * fwd_flops(w), f"bwd_{w.name}")
     del q, k, v, o, lse, g, dq, dk, dv
+    # backward pass with 8 K/V heads (each CTA walks the tiles of 4 query heads)
+    q, k, v = W.gqa_fwd_inputs(w.B, w.H, GQA_HKV, w.N, w.d, seed=21, device="cuda")
+    o, lse = fa.fa_fwd_gqa(q, k, v, True, 1 / math.sqrt(w.d))
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(7),
+                    device="cuda").to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    timed(lambda: fa.fa_bwd_gqa(q, k, v, o, lse, g, True, 1 / math.sqrt(w.d), dq=dq, dk=dk,
+                                dv=dv, stream=stream),
+          2.5 * fwd_flops(w), f"bwd_gqa_long_prefill_b1_h32_hkv{GQA_HKV}_n16384_d128_causal")
+    del q, k, v, o, lse, g, dq, dk, dv
+    # backward pass over the variable-length workload's packed sequences
+    wv = W.BATCHED_VARLEN
+    q, k, v, cu = W.varlen_workload_inputs(wv, device="cuda")
+    lens = (cu[1:] - cu[:-1]).tolist()
+    cud = cu.cuda()
+    o, lse = fa.fa_fwd_varlen(q, k, v, cud, max(lens), wv.causal, 1 / math.sqrt(wv.d))
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(8),
+                    device="cuda").to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    vflops = sum(4.0 * wv.H * L * L * wv.d / (2 if wv.causal else 1) for L in lens)
+    timed(lambda: fa.fa_bwd_varlen(q, k, v, o, lse, g, cud, max(lens), wv.causal,
+                                   1 / math.sqrt(wv.d), dq=dq, dk=dk, dv=dv, stream=stream),
+          2.5 * vflops, f"bwd_{wv.name}")
+    del q, k, v, cu, cud, o, lse, g, dq, dk, dv
     # grouped-query paged decode: the decode workload's lengths, 8 K/V heads
     lengths = W.varlen_lengths(DEC.B, DEC.len_lo, DEC.len_hi, DEC.seed)
     c = W.paged_inputs(DEC.B, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda",
