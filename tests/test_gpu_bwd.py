@@ -75,23 +75,78 @@ def test_bwd_linear_in_dout():
     assert_grad_close(to64(b[0]), 2 * to64(a[0]), "dq linearity")
 
 
-def test_bwd_long_prefill_runs_finite():
+def _cpu_head(x, h):
+    """Head h of a [B, heads, N, d] CUDA tensor as a [1, 1, N, d] CPU tensor."""
+    return x[:, h:h + 1].cpu()
+
+
+def test_bwd_long_prefill_one_head_full():
+    """The long-prefill workload's backward pass (B=1 H=32 N=16384 d=128,
+    causal) in the launch configuration the benchmark times: every gradient
+    finite, and query head 13 (dq) with its K/V head (dk, dv) compared whole
+    against the oracle (a head's gradients depend on that head alone)."""
     w = W.LONG_PREFILL
     q, k, v = W.fwd_inputs(w, device="cuda")
     scale = 1 / math.sqrt(w.d)
     o, lse = fa.fa_fwd(q, k, v, True, scale)
-    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(714),
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(7),
                     device="cuda").to(torch.bfloat16)
     dq, dk, dv = fa.fa_bwd(q, k, v, o, lse, g, True, scale)
     assert fa.fa_get_device_error() == fa.FA_OK
     for t in (dq, dk, dv):
         assert bool(torch.isfinite(t).all())
-    # under the causal mask dq rows < 512 depend only on positions < 512, so
-    # they can be checked against the oracle on the first 512 positions of a
-    # head (dk, dv of those keys depend on every later row)
-    qh, kh, vh, gh = (t[0, 0, :512].cpu()[None, None] for t in (q, k, v, g))
-    rq, _, _ = oracle.attention_bwd(qh, kh, vh, gh, True, scale)
-    assert_grad_close(to64(dq[0, 0, :512].cpu())[None, None], rq, "dq rows < 512")
+    h = 13
+    rq, rk, rv = oracle.attention_bwd(*(_cpu_head(t, h) for t in (q, k, v, g)), True, scale)
+    assert_grad_close(to64(_cpu_head(dv, h)), rv, "dv head 13")
+    assert_grad_close(to64(_cpu_head(dk, h)), rk, "dk head 13")
+    assert_grad_close(to64(_cpu_head(dq, h)), rq, "dq head 13")
+
+
+def test_bwd_gqa_long_prefill_one_group_full():
+    """The grouped backward on the long-prefill shape with 8 K/V heads, as the
+    benchmark runs it: K/V head 5 and its four query heads 20..23 compared
+    whole against the oracle (dk, dv sum the group's four query heads)."""
+    w = W.LONG_PREFILL
+    H_kv, kv = 8, 5
+    q, k, v = W.gqa_fwd_inputs(w.B, w.H, H_kv, w.N, w.d, seed=21, device="cuda")
+    scale = 1 / math.sqrt(w.d)
+    o, lse = fa.fa_fwd_gqa(q, k, v, True, scale)
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(7),
+                    device="cuda").to(torch.bfloat16)
+    dq, dk, dv = fa.fa_bwd_gqa(q, k, v, o, lse, g, True, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    G = w.H // H_kv
+    hs = slice(kv * G, (kv + 1) * G)
+    rq, rk, rv = oracle.attention_bwd(q[:, hs].cpu(), _cpu_head(k, kv), _cpu_head(v, kv),
+                                      g[:, hs].cpu(), True, scale)
+    assert_grad_close(to64(_cpu_head(dv, kv)), rv, "dv K/V head 5")
+    assert_grad_close(to64(_cpu_head(dk, kv)), rk, "dk K/V head 5")
+    assert_grad_close(to64(dq[:, hs].cpu()), rq, "dq query heads 20..23")
+
+
+def test_bwd_varlen_workload_one_head_full():
+    """The packed backward on the variable-length prefill workload (8
+    sequences of 1024..8192 tokens, H=32, d=128, causal), as the benchmark
+    runs it: head 30 of every sequence compared whole against the oracle."""
+    wv = W.BATCHED_VARLEN
+    q, k, v, cu = W.varlen_workload_inputs(wv, device="cuda")
+    lens = (cu[1:] - cu[:-1]).tolist()
+    scale = 1 / math.sqrt(wv.d)
+    cud = cu.cuda()
+    o, lse = fa.fa_fwd_varlen(q, k, v, cud, max(lens), wv.causal, scale)
+    g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(8),
+                    device="cuda").to(torch.bfloat16)
+    dq, dk, dv = fa.fa_bwd_varlen(q, k, v, o, lse, g, cud, max(lens), wv.causal, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    h = 30
+    sl = lambda x: x[:, h:h + 1].cpu()  # packed [total, heads, d] -> [total, 1, d]
+    rq, rk, rv = oracle.attention_bwd_varlen(sl(q), sl(k), sl(v), sl(g), cu.cpu(), wv.causal,
+                                             scale)
+    assert_grad_close(to64(sl(dv)), rv, "dv head 30")
+    assert_grad_close(to64(sl(dk)), rk, "dk head 30")
+    assert_grad_close(to64(sl(dq)), rq, "dq head 30")
 
 
 # -- grouped K/V heads (fa_bwd_gqa) -----------------------------------------------
