@@ -688,6 +688,15 @@ def run_native(args, world, rank, local):
             "frac": per_launch_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy",
             "traffic": recorded_traffic(dec_kernel, dec_sha),
             "algorithmic_bytes_per_launch": dbytes}
+    # each kernel's share of the step's device time (CUDA events); the one with
+    # the larger share is the step's dominant kernel
+    if do_fwd and do_dec and fwd_sum + dec_sum > 0:
+        shares = {"roofline": fwd_sum / (fwd_sum + dec_sum),
+                  "roofline_decode": dec_sum / (fwd_sum + dec_sum)}
+        top = max(shares, key=shares.get)
+        for key, share in shares.items():
+            out[key]["share_of_step"] = share
+            out[key]["dominant"] = key == top
     return out
 
 
