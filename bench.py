@@ -627,8 +627,8 @@ def run_native(args, world, rank, local):
 
     if rank != 0:
         return None
-    fwd_sha = kernel_source_sha(["fwd_sm100.cu", "fa_ptx.cuh"])
-    dec_sha = kernel_source_sha(["decode_sm100.cu", "fa_ptx.cuh"])
+    fwd_sha = kernel_source_sha(["fwd_sm100.cu", "fa_ptx.cuh", "fa_internal.h"])
+    dec_sha = kernel_source_sha(["decode_sm100.cu", "fa_ptx.cuh", "fa_internal.h"])
     # The timed region is a seconds-long loop that runs the GPU at its power
     # cap, like the sustained GEMM measurement; the burst figure is reported
     # beside it in pct_of_bf16_peak.

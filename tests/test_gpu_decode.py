@@ -69,8 +69,8 @@ def test_decode_small_full_compare(d):
 
 
 def test_decode_long_sequence_bigger_splits():
-    # more pages than splits x chunk: each split covers more than the minimum
-    lens = [256 * 130 + 17, 300]
+    # more pages than splits x chunk (64 x 4): each split covers more than the minimum
+    lens = [256 * 260 + 17, 300]
     c = W.paged_inputs(2, 2, 128, lens, seed=23, device="cpu")
     o = _decode(_on_gpu(c))
     o_ref, _ = oracle.decode_paged(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
