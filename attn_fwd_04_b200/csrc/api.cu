@@ -1,5 +1,5 @@
 // api.cu -- the extern "C" boundary of libfa.so (declared in include/fa.h):
-// argument checks, TMA tensor maps, the per-GPU decode workspace and the
+// argument checks, TMA tensor maps, the per-GPU library workspace and the
 // device error word.  No kernel arithmetic lives here.
 #include <cmath>
 #include <cstdint>
@@ -34,7 +34,7 @@ struct DeviceState {
     int num_sms = 0;
     int cc_major = 0;
     unsigned int* err = nullptr;  // device address of g_device_error
-    void* ws = nullptr;           // decode workspace
+    void* ws = nullptr;           // library workspace (decode partials, rotated K, bwd scratch)
     size_t ws_bytes = 0;
 };
 

@@ -30,11 +30,15 @@
  *  - Faults found on the device (a bounded wait that ran out, a negative
  *    sequence length) do not trap: the kernel records a code in the library's
  *    device error word and returns; fa_get_device_error reads it.
- *  - The library holds one device workspace per GPU for the decode split
- *    partials (grown on demand with cudaMallocAsync on the caller's stream,
- *    freed by fa_release_workspace).  Calls that use it (fa_decode_paged,
- *    fa_gather_paged) on different streams of the same GPU must not overlap:
- *    order them on one stream or with events.
+ *  - The library holds one device workspace per GPU (grown on demand with
+ *    cudaMallocAsync on the caller's stream, freed by fa_release_workspace):
+ *    the decode split partials, the rotated K of fa_fwd_rope, the backward
+ *    pass's statistics and fp32 dq accumulator, the page offsets of the paged
+ *    prefill, append and gather.  Calls that use it (fa_fwd_rope, fa_bwd,
+ *    fa_bwd_gqa, fa_bwd_varlen, the fa_decode_paged calls except the _noalloc
+ *    one, fa_prefill_paged, fa_append_paged, fa_gather_paged) on different
+ *    streams of the same GPU must not overlap: order them on one stream or
+ *    with events.
  *  - Thread safety: the host entry points may be called from several host
  *    threads; the workspace bookkeeping is guarded by a mutex.
  */
@@ -65,7 +69,7 @@ enum fa_status {
     FA_ERR_ALIGN = -4,          /* a tensor base pointer is not 16-byte aligned */
     FA_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
     FA_ERR_DEVICE_TIMEOUT = -6, /* reported through fa_get_device_error: a bounded device wait ran out */
-    FA_ERR_NOMEM = -7,          /* the decode workspace could not be allocated */
+    FA_ERR_NOMEM = -7,          /* the library workspace could not be allocated */
     FA_ERR_DEVICE_BAD_INPUT = -8 /* reported through fa_get_device_error: e.g. a negative seq_lens entry */
 };
 
@@ -113,7 +117,7 @@ FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, floa
  * (section 3).  q and k are passed unrotated.  The page applies RoPE with the
  * QKV projection; here K, which every query block of a head reads, is rotated
  * once per position into the library's per-GPU workspace (B*H_kv*N*d*2 bytes,
- * grown on demand like the decode workspace; calls on different streams of
+ * grown on demand like the rest of the workspace; calls on different streams of
  * one GPU must not overlap), and each Q tile is rotated in on-chip memory
  * after it is loaded, before its first score product.
  *   rope_cos, rope_sin : DEVICE fp32 [max_pos, d/2], row-major; entry (p, i)
@@ -143,7 +147,7 @@ FA_API int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, flo
  *   dv = P^T dout,   dq = scale dS k,   dk = scale dS^T q.
  * Same `causal`, `scale` and limits as fa_fwd.  Uses the library's per-GPU
  * workspace (B*H*N*(2 + d)*4 bytes: D, the statistics and an fp32 dq
- * accumulator), grown on demand like the decode workspace.  Accumulation is in
+ * accumulator), grown on demand like the rest of the workspace.  Accumulation is in
  * fp32; dq sums the contributions of the key blocks with fp32 atomics, so its
  * last bits may differ between runs.
  */
@@ -419,7 +423,7 @@ FA_API int fa_get_device_error(int* code, fa_stream_t stream);
  */
 FA_API int fa_selftest_bounded_wait(fa_stream_t stream);
 
-/* Free the current GPU's decode workspace (synchronises the device first).
+/* Free the current GPU's library workspace (synchronises the device first).
  * Returns FA_OK or FA_ERR_CUDA. */
 FA_API int fa_release_workspace(void);
 
