@@ -6,6 +6,7 @@
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "fa_ptx.cuh"
 
@@ -29,13 +30,20 @@ __device__ unsigned int g_device_error = 0;
 
 constexpr int kMaxDevices = 64;
 
+// One grow-only workspace per stream (decode partials, rotated K, backward
+// scratch, page offsets): calls on different streams never share scratch.
+struct StreamWorkspace {
+    cudaStream_t stream = nullptr;
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+
 struct DeviceState {
     bool init = false;
     int num_sms = 0;
     int cc_major = 0;
     unsigned int* err = nullptr;  // device address of g_device_error
-    void* ws = nullptr;           // library workspace (decode partials, rotated K, bwd scratch)
-    size_t ws_bytes = 0;
+    std::vector<StreamWorkspace> ws;
 };
 
 std::mutex g_mu;
@@ -119,24 +127,32 @@ int make_map_f32(CUtensorMap* map, const void* base, const cuuint64_t dims[3],
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// Grow-only per-device workspace, allocated on the caller's stream.
+// The stream's grow-only workspace on this device, allocated (and, when it
+// grows, freed) in the stream's own order.
 int ensure_workspace(DeviceState* s, size_t bytes, cudaStream_t stream, void** out) {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (s->ws_bytes < bytes) {
-        if (s->ws) {
-            if (cudaFreeAsync(s->ws, stream) != cudaSuccess) return FA_ERR_CUDA;
-            s->ws = nullptr;
-            s->ws_bytes = 0;
+    StreamWorkspace* w = nullptr;
+    for (StreamWorkspace& e : s->ws)
+        if (e.stream == stream) w = &e;
+    if (!w) {
+        s->ws.push_back(StreamWorkspace{stream, nullptr, 0});
+        w = &s->ws.back();
+    }
+    if (w->bytes < bytes) {
+        if (w->ptr) {
+            if (cudaFreeAsync(w->ptr, stream) != cudaSuccess) return FA_ERR_CUDA;
+            w->ptr = nullptr;
+            w->bytes = 0;
         }
         void* p = nullptr;
         if (cudaMallocAsync(&p, bytes, stream) != cudaSuccess) {
             cudaGetLastError();
             return FA_ERR_NOMEM;
         }
-        s->ws = p;
-        s->ws_bytes = bytes;
+        w->ptr = p;
+        w->bytes = bytes;
     }
-    *out = s->ws;
+    *out = w->ptr;
     return FA_OK;
 }
 
@@ -619,11 +635,11 @@ int fa_release_workspace(void) {
     if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return FA_OK;
     DeviceState& s = g_dev[dev];
-    if (s.ws) {
+    if (!s.ws.empty()) {
         if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
-        if (cudaFree(s.ws) != cudaSuccess) return FA_ERR_CUDA;
-        s.ws = nullptr;
-        s.ws_bytes = 0;
+        for (StreamWorkspace& w : s.ws)
+            if (w.ptr && cudaFree(w.ptr) != cudaSuccess) return FA_ERR_CUDA;
+        s.ws.clear();
     }
     return FA_OK;
 }

@@ -30,15 +30,17 @@
  *  - Faults found on the device (a bounded wait that ran out, a negative
  *    sequence length) do not trap: the kernel records a code in the library's
  *    device error word and returns; fa_get_device_error reads it.
- *  - The library holds one device workspace per GPU (grown on demand with
- *    cudaMallocAsync on the caller's stream, freed by fa_release_workspace):
- *    the decode split partials, the rotated K of fa_fwd_rope, the backward
- *    pass's statistics and fp32 dq accumulator, the page offsets of the paged
- *    prefill, append and gather.  Calls that use it (fa_fwd_rope, fa_bwd,
- *    fa_bwd_gqa, fa_bwd_varlen, the fa_decode_paged calls except the _noalloc
- *    one, fa_prefill_paged, fa_append_paged, fa_gather_paged) on different
- *    streams of the same GPU must not overlap: order them on one stream or
- *    with events.
+ *  - The library holds one device workspace per (GPU, stream): the decode
+ *    split partials, the rotated K of fa_fwd_rope, the backward pass's
+ *    statistics and fp32 dq accumulator, the page offsets of the paged
+ *    prefill, append and gather.  It is allocated with cudaMallocAsync on that
+ *    stream, grown (freed and reallocated) in the stream's order, and freed by
+ *    fa_release_workspace.  So calls on different streams may overlap on the
+ *    GPU (e.g. a prefill on one stream and a decode on another); calls on one
+ *    stream are ordered by the stream.  The key is the stream handle: destroy
+ *    a stream only after its calls have completed (a new stream may get the
+ *    same handle), and call fa_release_workspace to return the memory of
+ *    streams no longer used.
  *  - Thread safety: the host entry points may be called from several host
  *    threads; the workspace bookkeeping is guarded by a mutex.
  */
@@ -116,9 +118,8 @@ FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, floa
  * kernel that fuses RoPE (section 2) from a precomputed sin/cos lookup table
  * (section 3).  q and k are passed unrotated.  The page applies RoPE with the
  * QKV projection; here K, which every query block of a head reads, is rotated
- * once per position into the library's per-GPU workspace (B*H_kv*N*d*2 bytes,
- * grown on demand like the rest of the workspace; calls on different streams of
- * one GPU must not overlap), and each Q tile is rotated in on-chip memory
+ * once per position into the library workspace of the call's stream
+ * (B*H_kv*N*d*2 bytes, grown on demand), and each Q tile is rotated in on-chip memory
  * after it is loaded, before its first score product.
  *   rope_cos, rope_sin : DEVICE fp32 [max_pos, d/2], row-major; entry (p, i)
  *                        is cos / sin of the angle for position p and pair i
@@ -145,11 +146,11 @@ FA_API int fa_fwd_rope(const void* q, const void* k, const void* v, void* o, flo
  * With P = exp(scale q k^T - lse) (causal: keys after the query give 0),
  * D_i = dout_i . o_i and dS = P o (dout v^T - D):
  *   dv = P^T dout,   dq = scale dS k,   dk = scale dS^T q.
- * Same `causal`, `scale` and limits as fa_fwd.  Uses the library's per-GPU
- * workspace (B*H*N*(2 + d)*4 bytes: D, the statistics and an fp32 dq
- * accumulator), grown on demand like the rest of the workspace.  Accumulation is in
- * fp32; dq sums the contributions of the key blocks with fp32 atomics, so its
- * last bits may differ between runs.
+ * Same `causal`, `scale` and limits as fa_fwd.  Uses the library workspace
+ * of the call's stream (B*H*N*(2 + d)*4 bytes: D, the statistics and an fp32
+ * dq accumulator), grown on demand.  Accumulation is in fp32; dq sums the
+ * contributions of the key blocks with fp32 bulk reduce-adds, so its last
+ * bits may differ between runs.
  */
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
@@ -244,7 +245,7 @@ FA_API int fa_fwd_varlen_gqa(const void* q, const void* k, const void* v, void* 
  * The query attends, without a mask, to all seq_lens[b] cached tokens, with
  * softmax scale 1/sqrt(d) (the default of the lqnn.cn page, section 3.3; the
  * call has no scale argument).  page_size must be 256.
- * Uses the library's per-GPU workspace (see the conventions above).
+ * Uses the library workspace of the call's stream (see the conventions above).
  */
 FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                     const int32_t* page_table, const int32_t* seq_lens, void* o,
@@ -293,8 +294,8 @@ FA_API int fa_decode_paged_gqa(const void* q, const void* k_pages, const void* v
  * A length beyond its row (seq_lens[b] > max_pages * page_size) is reported
  * as FA_ERR_DEVICE_BAD_INPUT and decoded over the row's tokens only; no
  * entry outside the table is read.  A first kernel copies the used entries
- * of every row, back to back, into the library's per-GPU workspace (B *
- * max_pages + B int32 beyond the decode's own part), then the decode of
+ * of every row, back to back, into the library workspace of the call's
+ * stream (B * max_pages + B int32 beyond the decode's own part), then the decode of
  * fa_decode_paged_gqa runs on that packed table, so results equal
  * fa_decode_paged_gqa's on the same pages bit for bit.
  */
@@ -324,7 +325,7 @@ FA_API int fa_decode_paged_strided(const void* q, const void* k_pages, const voi
  * page_table[off_b + pos / page_size].  page_size must be 256.  A sequence
  * with n_b > seq_lens[b], or a page index outside [0, num_pages), is skipped
  * and reported as FA_ERR_DEVICE_BAD_INPUT (no write leaves the pool).  Uses the
- * library's per-GPU workspace for the page offsets.
+ * library workspace of the call's stream for the page offsets.
  */
 FA_API int fa_append_paged(const void* k_new, const void* v_new, const int32_t* cu_new,
                     void* k_pages, void* v_pages, const int32_t* page_table,
@@ -368,7 +369,7 @@ FA_API int fa_prefill_paged(const void* q, const void* k_pages, const void* v_pa
  *   pages : [P, H, page_size, d] bf16
  *   out   : [sum_b seq_lens[b], H, d] bf16, sequence b starting at row
  *           sum_{b' < b} seq_lens[b']
- * page_size must be 256.  Uses the library's per-GPU workspace.
+ * page_size must be 256.  Uses the library workspace of the call's stream.
  */
 FA_API int fa_gather_paged(const void* pages, const int32_t* page_table, const int32_t* seq_lens,
                     void* out, int B, int H, int d, int page_size, fa_stream_t stream);
@@ -423,8 +424,8 @@ FA_API int fa_get_device_error(int* code, fa_stream_t stream);
  */
 FA_API int fa_selftest_bounded_wait(fa_stream_t stream);
 
-/* Free the current GPU's library workspace (synchronises the device first).
- * Returns FA_OK or FA_ERR_CUDA. */
+/* Free the library workspaces of every stream on the current GPU
+ * (synchronises the device first).  Returns FA_OK or FA_ERR_CUDA. */
 FA_API int fa_release_workspace(void);
 
 /* A static, human-readable name for a status code. */
