@@ -50,15 +50,16 @@ __host__ __device__ inline WorkspaceLayout layout_of(int B, int H, int d, int ma
     return L;
 }
 
-// Splits of a sequence with np pages: at least kDecodeChunkPages pages each,
-// at most max_splits of them, none empty.
-__device__ __forceinline__ void split_shape(int np, int max_splits, int& ns, int& cp) {
+// Splits of a sequence with np pages: at least min_pages pages each, at most
+// max_splits of them, none empty.
+__device__ __forceinline__ void split_shape(int np, int max_splits, int min_pages, int& ns,
+                                            int& cp) {
     if (np <= 0) {
         ns = 0;
         cp = 1;
         return;
     }
-    int want = (np + kDecodeChunkPages - 1) / kDecodeChunkPages;
+    int want = (np + min_pages - 1) / min_pages;
     if (want > max_splits) want = max_splits;
     cp = (np + want - 1) / want;
     ns = (np + cp - 1) / cp;
@@ -92,8 +93,8 @@ __device__ __forceinline__ int block_incl_scan(int v, int* sh /*[32]*/, int& tot
 
 __global__ void __launch_bounds__(kPlanThreads)
     fa_decode_plan_kernel(const int32_t* __restrict__ seq_lens, int B, int H, int page_size,
-                          int max_splits, int32_t* page_off, int32_t* tok_off, int32_t* unit_off,
-                          unsigned int* err) {
+                          int max_splits, int min_pages, int32_t* page_off, int32_t* tok_off,
+                          int32_t* unit_off, unsigned int* err) {
     __shared__ int sh[3][32];
     int carry_p = 0, carry_t = 0, carry_u = 0;
     if (threadIdx.x == 0) {
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(kPlanThreads)
         }
         const int np = (len + page_size - 1) / page_size;
         int ns, cp;
-        split_shape(np, max_splits, ns, cp);
+        split_shape(np, max_splits, min_pages, ns, cp);
         int tp, tt, tu;
         const int ip = block_incl_scan(np, sh[0], tp);
         const int it = block_incl_scan(len, sh[1], tt);
@@ -232,7 +233,8 @@ __device__ __forceinline__ UnitShape unit_shape(int u, UnitCursor& cur,
                                                 const int32_t* __restrict__ unit_off,
                                                 const int32_t* __restrict__ page_off,
                                                 const int32_t* __restrict__ seq_lens, int B,
-                                                int Hk, int page_size, int max_splits) {
+                                                int Hk, int page_size, int max_splits,
+                                                int min_pages) {
     cur.seek(unit_off, B, u);
     UnitShape us;
     us.b = cur.b;
@@ -243,7 +245,7 @@ __device__ __forceinline__ UnitShape unit_shape(int u, UnitCursor& cur,
     if (len < 0) len = 0;
     const int np = (len + page_size - 1) / page_size;
     int ns;
-    split_shape(np, max_splits, ns, us.cp);
+    split_shape(np, max_splits, min_pages, ns, us.cp);
     us.tok0 = us.s * us.cp * page_size;
     us.ntok = min(len, us.tok0 + us.cp * page_size) - us.tok0;
     us.pt_base = __ldg(page_off + us.b) + us.s * us.cp;
@@ -260,7 +262,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                            const __nv_bfloat16* __restrict__ v_pages,
                            const int32_t* __restrict__ page_table,
                            const int32_t* __restrict__ seq_lens, int B, int H, int num_pages,
-                           int page_size, int max_splits, const int32_t* __restrict__ page_off,
+                           int page_size, int max_splits, int min_pages,
+                           const int32_t* __restrict__ page_off,
                            const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                            float* __restrict__ part_o, float scale_log2, unsigned int* err) {
     using Sm = DecSmem<D>;
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
             const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
-                                            page_size, max_splits);
+                                            page_size, max_splits, min_pages);
             const int nchunks = (us.ntok + kDecTok - 1) / kDecTok;
             constexpr int per_page = 256 / kDecTok;  // page_size is 256
             int page = 0;
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
             const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, H,
-                                            page_size, max_splits);
+                                            page_size, max_splits, min_pages);
             float qf[8];
             {
                 const uint4 qu = *reinterpret_cast<const uint4*>(
@@ -501,7 +504,8 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                          const __nv_bfloat16* __restrict__ q,
                          const int32_t* __restrict__ page_table,
                          const int32_t* __restrict__ seq_lens, int B, int H, int Hk, int gr, int sub,
-                         int num_pages, int max_splits, const int32_t* __restrict__ page_off,
+                         int num_pages, int max_splits, int min_pages,
+                         const int32_t* __restrict__ page_off,
                          const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                          float* __restrict__ part_o, float scale_log2, unsigned int* err) {
     using Sm = GqSmem<D, GH>;
@@ -543,7 +547,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
             const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk, kPage,
-                                            max_splits);
+                                            max_splits, min_pages);
             const int nchunks = (us.ntok + kGqTok - 1) / kGqTok;
             constexpr int per_page = kPage / kGqTok;
             int z = 0;  // (page, head) slice; -1 reads zeros
@@ -594,7 +598,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++k) {
         const UnitShape us = unit_shape(u, cur, unit_off, page_off, seq_lens, B, Hk, kPage,
-                                        max_splits);
+                                        max_splits, min_pages);
         // the group's query rows as A fragments: a0 / a2 = row grp, columns
         // 16ks + 2tig..+1 / +8; a1 / a3 = the same of row grp + 8 (groups of
         // 16); rows gr..15 are zero
@@ -755,7 +759,8 @@ __global__ void __launch_bounds__(kGqThreads, 1)
 template <int D>
 __global__ void __launch_bounds__(128)
     fa_decode_merge_kernel(const int32_t* __restrict__ seq_lens, int B, int H, int GH,
-                           int page_size, int max_splits, const int32_t* __restrict__ unit_off,
+                           int page_size, int max_splits, int min_pages,
+                           const int32_t* __restrict__ unit_off,
                            const float* __restrict__ part_lse, const float* __restrict__ part_o,
                            __nv_bfloat16* __restrict__ o) {
     constexpr int PER = D / 32;
@@ -767,7 +772,7 @@ __global__ void __launch_bounds__(128)
     if (len < 0) len = 0;
     const int np = (len + page_size - 1) / page_size;
     int ns, cp;
-    split_shape(np, max_splits, ns, cp);
+    split_shape(np, max_splits, min_pages, ns, cp);
     const int base = __ldg(unit_off + b) * GH;
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32) M = fmaxf(M, part_lse[base + s * H + h]);
@@ -876,6 +881,9 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
                        int num_sms, cudaStream_t stream, int gr, int sub) {
     const int Hk = H / gr;  // units per split
+    // pages a split covers at least: with few units per split (few K/V heads),
+    // larger splits keep the partials and per-unit merges down
+    const int min_pages = Hk >= kDecodeManyUnits ? kDecodeChunkPages : kDecodeChunkPagesFew;
     const WorkspaceLayout L = layout_of(B, H, D, max_splits);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* page_off = reinterpret_cast<int32_t*>(ws);
@@ -885,7 +893,8 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
     float* part_o = reinterpret_cast<float*>(ws + L.o_off);
     // units are (split, K/V head) pairs
     fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, Hk, page_size, max_splits,
-                                                          page_off, tok_off, unit_off, err);
+                                                          min_pages, page_off, tok_off, unit_off,
+                                                          err);
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
     if constexpr (GH == 1) {
         auto split = fa_decode_split_kernel<D>;
@@ -902,7 +911,8 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
         split<<<num_sms * occ, kDecThreads, smem, stream>>>(
             static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pages),
             static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, num_pages,
-            page_size, max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
+            page_size, max_splits, min_pages, page_off, unit_off, part_lse, part_o, scale_log2,
+            err);
     } else {
         if (!tk || !tv) return FA_ERR_NULL;
         auto split = fa_decode_gqa_kernel<D, GH>;
@@ -917,11 +927,12 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
             return FA_ERR_CUDA;
         split<<<num_sms * occ, kGqThreads, smem, stream>>>(
             *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk, gr, sub,
-            num_pages, max_splits, page_off, unit_off, part_lse, part_o, scale_log2, err);
+            num_pages, max_splits, min_pages, page_off, unit_off, part_lse, part_o, scale_log2,
+            err);
     }
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
-        seq_lens, B, H, gr, page_size, max_splits, unit_off, part_lse, part_o,
+        seq_lens, B, H, gr, page_size, max_splits, min_pages, unit_off, part_lse, part_o,
         static_cast<__nv_bfloat16*>(o));
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -933,7 +944,7 @@ int launch_gather_impl(const void* pages, const int32_t* page_table, const int32
     int32_t* page_off = static_cast<int32_t*>(workspace);
     int32_t* tok_off = page_off + (B + 1);
     int32_t* unit_off = tok_off + (B + 1);
-    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, H, page_size, 1, page_off,
+    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, H, page_size, 1, 1, page_off,
                                                           tok_off, unit_off, err);
     fa_gather_kernel<D><<<num_sms * 8, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(pages), page_table, seq_lens, B, H, page_size,
@@ -949,7 +960,7 @@ int launch_append_impl(const void* k_new, const void* v_new, const int32_t* cu_n
     int32_t* page_off = static_cast<int32_t*>(workspace);
     int32_t* tok_off = page_off + (B + 1);
     int32_t* unit_off = tok_off + (B + 1);
-    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, Hk, page_size, 1, page_off,
+    fa_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(seq_lens, B, Hk, page_size, 1, 1, page_off,
                                                           tok_off, unit_off, err);
     fa_append_kernel<D><<<num_sms * 8, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), cu_new,

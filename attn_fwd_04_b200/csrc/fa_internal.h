@@ -54,10 +54,15 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
 
 // ---- paged decode ----------------------------------------------------------
 // Number of pages a split covers at least (a split is one CTA work unit) and
-// the most splits one sequence is cut into.  4 pages measured fastest on the
-// paged-decode workload for 32, 8 and 4 K/V heads (2: 2-9 % slower, more
-// partials and more per-unit combines; 8: a longer tail with few K/V heads).
+// the most splits one sequence is cut into.  With at least kDecodeManyUnits
+// units per split (K/V heads, or sub-groups of large groups), 4 pages measured
+// fastest on the paged-decode workload for 32 and 8 K/V heads (2: 2-3 %
+// slower, more partials and per-unit combines; 8: a longer tail).  With fewer
+// units per split the launch is short and 6 pages measured faster (4 K/V
+// heads: 6486-6518 GB/s against 6253-6296 with 4 pages).
 constexpr int kDecodeChunkPages = 4;
+constexpr int kDecodeChunkPagesFew = 6;
+constexpr int kDecodeManyUnits = 8;
 constexpr int kDecodeMaxSplits = 64;
 
 struct DecodePlan {
