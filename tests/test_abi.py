@@ -35,6 +35,45 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def _prototypes():
+    """name -> parameter kinds ('p' pointer or stream, 'i' integer, 'f' float)
+    and the return kind, parsed from the header's FA_API declarations."""
+    text = re.sub(r"/\*.*?\*/", " ", open(HEADER).read(), flags=re.S)
+    out = {}
+    for ret, name, params in re.findall(r"FA_API\s+([\w\s\*]*?)\s*\b(fa_\w+)\s*\(([^)]*)\)\s*;",
+                                        text, flags=re.S):
+        kinds = []
+        for prm in (x.strip() for x in params.split(",")):
+            if not prm or prm == "void":
+                continue
+            if "*" in prm or prm.startswith("fa_stream_t"):
+                kinds.append("p")
+            elif prm.split()[0] in ("float", "double"):
+                kinds.append("f" if prm.split()[0] == "float" else "d")
+            else:
+                kinds.append("i")
+        out[name] = (kinds, "p" if "*" in ret else "i")
+    return out
+
+
+def _kind(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(t, ctypes._Pointer):
+        return "p"
+    return {ctypes.c_int: "i", ctypes.c_float: "f", ctypes.c_double: "d"}[t]
+
+
+def test_binding_argtypes_match_the_header(L):
+    """Each binding's ctypes signature has the header prototype's parameter
+    count and kinds, so a pointer never lands in an int slot (or a float in
+    an int) when the header changes and the binding does not."""
+    protos = _prototypes()
+    assert sorted(protos) == _declared()
+    for name, (kinds, ret) in protos.items():
+        fn = getattr(L, name)
+        assert [_kind(t) for t in fn.argtypes] == kinds, name
+        assert _kind(fn.restype) == ret, name
+
+
 def test_status_strings(L):
     codes = [fa.FA_OK, fa.FA_ERR_NULL, fa.FA_ERR_SHAPE, fa.FA_ERR_UNSUPPORTED, fa.FA_ERR_ALIGN,
              fa.FA_ERR_CUDA, fa.FA_ERR_DEVICE_TIMEOUT, fa.FA_ERR_NOMEM, fa.FA_ERR_DEVICE_BAD_INPUT]
