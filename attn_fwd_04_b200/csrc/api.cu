@@ -1,5 +1,5 @@
 // api.cu -- the extern "C" boundary of libfa.so (declared in include/fa.h):
-// argument checks, TMA tensor maps, the per-GPU library workspace and the
+// argument checks, TMA tensor maps, the per-(GPU, stream) library workspaces and the
 // device error word.  No kernel arithmetic lives here.
 #include <cmath>
 #include <cstdint>
