@@ -139,6 +139,54 @@ def prefill(L, q=A, kp=A, vp=A, pt=A, sl=A, cu=A, o=A, lse=A, B=2, H=8, H_kv=2, 
                               causal, scale, S)
 
 
+def bwd_gqa(L, q=A, k=A, v=A, o=A, lse=A, do=A, dq=A, dk=A, dv=A, B=1, H=8, H_kv=2, N=256,
+            d=128, causal=1, scale=0.1):
+    return L.fa_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, B, H, H_kv, N, d, causal, scale, S)
+
+
+def bwd_varlen(L, q=A, k=A, v=A, o=A, lse=A, do=A, dq=A, dk=A, dv=A, cu=A, B=2, H=8, H_kv=2,
+               total=100, maxlen=60, d=128, causal=1, scale=0.1):
+    return L.fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu, B, H, H_kv, total, maxlen, d,
+                           causal, scale, S)
+
+
+def varlen_gqa(L, q=A, k=A, v=A, o=A, lse=A, cu=A, B=2, H=8, H_kv=2, total=100, maxlen=60,
+               d=128, causal=1, scale=0.1):
+    return L.fa_fwd_varlen_gqa(q, k, v, o, lse, cu, B, H, H_kv, total, maxlen, d, causal, scale,
+                               S)
+
+
+def test_bwd_argument_errors(L):
+    assert L.fa_bwd(A, A, A, A, A, None, A, A, A, 1, 2, 256, 64, 1, 0.125, S) == fa.FA_ERR_NULL
+    assert bwd_gqa(L, dk=None) == fa.FA_ERR_NULL
+    assert bwd_gqa(L, N=0) == fa.FA_ERR_SHAPE
+    assert bwd_gqa(L, H=6, H_kv=4) == fa.FA_ERR_SHAPE       # H not a multiple of H_kv
+    assert bwd_gqa(L, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert bwd_gqa(L, scale=float("inf")) == fa.FA_ERR_SHAPE
+    assert bwd_gqa(L, dq=MIS) == fa.FA_ERR_ALIGN
+    assert bwd_gqa(L, lse=MIS) == fa.FA_ERR_ALIGN
+
+
+def test_bwd_varlen_argument_errors(L):
+    assert bwd_varlen(L, cu=None) == fa.FA_ERR_NULL
+    assert bwd_varlen(L, dv=None) == fa.FA_ERR_NULL
+    assert bwd_varlen(L, total=0) == fa.FA_ERR_SHAPE
+    assert bwd_varlen(L, maxlen=0) == fa.FA_ERR_SHAPE
+    assert bwd_varlen(L, H=8, H_kv=3) == fa.FA_ERR_SHAPE
+    assert bwd_varlen(L, d=32) == fa.FA_ERR_UNSUPPORTED
+    assert bwd_varlen(L, scale=float("nan")) == fa.FA_ERR_SHAPE
+    assert bwd_varlen(L, do=MIS) == fa.FA_ERR_ALIGN
+
+
+def test_varlen_gqa_argument_errors(L):
+    assert varlen_gqa(L, cu=None) == fa.FA_ERR_NULL
+    assert varlen_gqa(L, H_kv=0) == fa.FA_ERR_SHAPE
+    assert varlen_gqa(L, H=8, H_kv=3) == fa.FA_ERR_SHAPE
+    assert varlen_gqa(L, total=0) == fa.FA_ERR_SHAPE
+    assert varlen_gqa(L, d=256) == fa.FA_ERR_UNSUPPORTED
+    assert varlen_gqa(L, k=MIS) == fa.FA_ERR_ALIGN
+
+
 def test_append_and_prefill_argument_errors(L):
     assert append(L, cu=None) == fa.FA_ERR_NULL
     assert append(L, P=0) == fa.FA_ERR_SHAPE
