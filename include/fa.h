@@ -40,7 +40,10 @@
  *    stream are ordered by the stream.  The key is the stream handle: destroy
  *    a stream only after its calls have completed (a new stream may get the
  *    same handle), and call fa_release_workspace to return the memory of
- *    streams no longer used.
+ *    streams no longer used.  Under CUDA graph capture a call must not
+ *    allocate or grow its stream's workspace (the allocation would belong to
+ *    the graph): make one eager call of the largest size on that stream
+ *    before capturing, or use fa_decode_paged_noalloc.
  *  - Thread safety: the host entry points may be called from several host
  *    threads; the workspace bookkeeping is guarded by a mutex.
  */
