@@ -289,9 +289,10 @@ def attention_bwd_varlen(q, k, v, dout, cu_seqlens, causal: bool, scale: float):
 
 def rope(x, cos_t, sin_t, bf16_round: bool = True):
     """Rotary embedding of x [..., N, d] (positions 0..N-1) with the fp32 tables
-    cos_t, sin_t [>=N, d/2]; returns a new fp64 array.  With bf16_round the
-    rotated values are computed in fp32 and rounded to bf16 as the GPU path
-    does before its tensor cores; without it, exactly in fp64."""
+    cos_t, sin_t [>=N, d/2]; returns a new fp64 array.  Without bf16_round the
+    rotation is computed in fp64; with it, each rotated value is that fp64
+    rotation rounded once to the nearest bf16 (ties to even), the values the
+    bf16 tensor-core products consume."""
     xs = _f64(x).copy()
     N, d = xs.shape[-2], xs.shape[-1]
     c = np.ascontiguousarray(np.asarray(cos_t.cpu() if hasattr(cos_t, "cpu") else cos_t,

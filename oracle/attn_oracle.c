@@ -547,10 +547,14 @@ int oracle_prefill_paged(const double *q, const double *k_pages, const double *v
  *     x'_i       = x_i cos - x_{i+d/2} sin
  *     x'_{i+d/2} = x_{i+d/2} cos + x_i sin
  * x is [rows, N, d] (row r, position n at x + (r*N + n)*d), rotated in place.
- * oracle_rope_exact computes in fp64.  oracle_rope_bf16 takes the decision
- * the GPU path takes: the rotated values feed bf16 tensor cores, so they are
- * computed in fp32 (sin term first, then one fused multiply-add with the cos
- * term) and rounded to bf16, round-to-nearest-even. */
+ * oracle_rope_exact computes in fp64.  oracle_rope_bf16 is the rotation as
+ * the attention then consumes it: the rotated q and k are inputs of bf16
+ * tensor-core products, so each rotated value is the fp64 rotation (of the
+ * fp32 table entries) rounded once to the nearest bf16, ties to even.  It
+ * depends on no order of fp32 operations: any implementation that rotates in
+ * higher precision and rounds once gets these values, and one that rotates
+ * in fp32 differs from them only where its fp32 rounding error crosses a bf16
+ * rounding boundary (a rare one-ulp difference). */
 void oracle_rope_exact(double *x, const float *cos_t, const float *sin_t, int64_t rows,
                        int64_t N, int64_t d) {
     const int64_t half = d / 2;
@@ -566,36 +570,25 @@ void oracle_rope_exact(double *x, const float *cos_t, const float *sin_t, int64_
         }
 }
 
-static double round_bf16(float f) {
-    uint32_t u;
-    memcpy(&u, &f, 4);
-    if ((u & 0x7f800000u) == 0x7f800000u) { /* inf or nan: keep, quiet the nan */
-        if (u & 0x007fffffu) u |= 0x00400000u;
-        u &= 0xffff0000u;
-    } else {
-        u += 0x7fffu + ((u >> 16) & 1u);
-        u &= 0xffff0000u;
-    }
-    float g;
-    memcpy(&g, &u, 4);
-    return (double)g;
+/* Round a double to the nearest bf16 value (8 significant bits, the fp32
+ * exponent range), ties to even, in one step (no intermediate fp32 value, so
+ * no double rounding). */
+static double rne_bf16(double x) {
+    if (x == 0.0 || isnan(x) || isinf(x)) return x;
+    int e;
+    frexp(x, &e);                 /* |x| = m 2^e, 1/2 <= m < 1 */
+    int qe = e - 8;               /* weight of the last of 8 significant bits */
+    if (qe < -133) qe = -133;     /* bf16 subnormals: quantum 2^-133 */
+    const double r = ldexp(nearbyint(ldexp(x, -qe)), qe); /* default mode: ties to even */
+    if (fabs(r) >= 0x1p128) return x > 0 ? INFINITY : -INFINITY;
+    return r;
 }
 
 void oracle_rope_bf16(double *x, const float *cos_t, const float *sin_t, int64_t rows,
                       int64_t N, int64_t d) {
-    const int64_t half = d / 2;
-    for (int64_t r = 0; r < rows; ++r)
-        for (int64_t n = 0; n < N; ++n) {
-            double *v = x + (r * N + n) * d;
-            for (int64_t i = 0; i < half; ++i) {
-                const float c = cos_t[n * half + i], sn = sin_t[n * half + i];
-                const float a = (float)v[i], b = (float)v[i + half];
-                const float ta = fmaf(a, c, -(b * sn));
-                const float tb = fmaf(b, c, a * sn);
-                v[i] = round_bf16(ta);
-                v[i + half] = round_bf16(tb);
-            }
-        }
+    oracle_rope_exact(x, cos_t, sin_t, rows, N, d);
+    const int64_t n = rows * N * d;
+    for (int64_t i = 0; i < n; ++i) x[i] = rne_bf16(x[i]);
 }
 
 /* Gradients of the attention of one problem with respect to q, k and v,

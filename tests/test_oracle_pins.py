@@ -700,9 +700,21 @@ def test_rope_preserves_pair_norms_and_is_relative():
         assert abs(a - b) < 1e-5 * (1 + abs(a))
 
 
+def _rne_bf16_py(x: float) -> float:
+    """Nearest bf16 value (8 significant bits), ties to even: an independent
+    restatement with Python's own rounding (round() on a float rounds half to
+    even, and the power-of-two scalings are exact)."""
+    if x == 0.0 or not math.isfinite(x):
+        return x
+    _, e = math.frexp(x)
+    qe = max(e - 8, -133)
+    return math.ldexp(round(math.ldexp(x, -qe)), qe)
+
+
 def test_rope_bf16_is_the_rounded_rotation():
-    """The bf16 variant differs from the exact rotation by at most half a bf16
-    ulp (2^-9 relative) plus fp32 rounding, and its values are bf16 numbers."""
+    """The bf16 variant is the exact fp64 rotation rounded once to the nearest
+    bf16, element by element (checked against a Python rounding of the exact
+    rotation), and every value it returns is a bf16 number."""
     from attn_fwd_04_b200 import workloads as W
     torch = pytest.importorskip("torch")
     d, N = 64, 50
@@ -710,9 +722,45 @@ def test_rope_bf16_is_the_rounded_rotation():
     x = torch.randn((2, N, d), generator=torch.Generator().manual_seed(202)).to(torch.bfloat16)
     ex = oracle.rope(x, c, s, False)
     rb = oracle.rope(x, c, s, True)
+    want = np.vectorize(_rne_bf16_py)(ex)
+    np.testing.assert_array_equal(rb, want)
     assert np.all(np.abs(rb - ex) <= np.abs(ex) * 2.0 ** -8 + 1e-30)
     rt = torch.from_numpy(rb).float().to(torch.bfloat16).double().numpy()
     np.testing.assert_array_equal(rt, rb)
+
+
+def test_rope_bf16_hand_worked_d2():
+    """d = 2, the table of base 10000 (theta_0 = 1): (1, 0) at position 1 turns
+    to (cos 1, sin 1) = (0.540302..., 0.841470...).  In [1/2, 1) a bf16 step is
+    2^-8: 0.540302 * 256 = 138.32 -> 138/256 = 0.5390625 and 0.841471 * 256 =
+    215.42 -> 215/256 = 0.83984375.  (0, 1) at position 2 turns to
+    (-sin 2, cos 2) = (-0.909297..., -0.416147...): -232.78 -> -233/256 =
+    -0.91015625, and in [1/4, 1/2) the step is 2^-9: -213.07 -> -213/512 =
+    -0.416015625."""
+    from attn_fwd_04_b200 import workloads as W
+    c, s = W.rope_tables(3, 2)
+    x = np.array([[[0.0, 0.0], [1.0, 0.0], [0.0, 1.0]]])
+    y = oracle.rope(x, c, s, bf16_round=True)
+    np.testing.assert_array_equal(y[0, 1], [0.5390625, 0.83984375])
+    np.testing.assert_array_equal(y[0, 2], [-0.91015625, -0.416015625])
+    np.testing.assert_array_equal(y[0, 0], [0.0, 0.0])
+
+
+def test_rope_bf16_ties_to_even():
+    """A hand-made table (cos 1, sin 2^-8, exact in fp32) puts the rotation on
+    bf16 midpoints: with (a, b) = (1, -1), a cos - b sin = 1 + 2^-8, halfway
+    between 1 and 1 + 2^-7, goes to the even 1; with a = 1 + 2^-7 the value
+    1 + 2^-7 + 2^-8 goes up to the even 1 + 2^-6.  The second component
+    b cos + a sin = -1 + 2^-8 (resp. -1 + 2^-8 + 2^-15) is exact, resp. rounds
+    to -1 + 2^-8."""
+    cos_t = np.ones((2, 1), np.float32)
+    sin_t = np.full((2, 1), 2.0 ** -8, np.float32)
+    x = np.array([[[1.0, -1.0], [1.0 + 2.0 ** -7, -1.0]]])
+    y = oracle.rope(x, cos_t, sin_t, bf16_round=True)
+    np.testing.assert_array_equal(y[0, 0], [1.0, -1.0 + 2.0 ** -8])
+    np.testing.assert_array_equal(y[0, 1], [1.0 + 2.0 ** -6, -1.0 + 2.0 ** -8])
+    ex = oracle.rope(x, cos_t, sin_t, bf16_round=False)
+    np.testing.assert_array_equal(ex[0, 0], [1.0 + 2.0 ** -8, -1.0 + 2.0 ** -8])
 
 
 def test_rope_second_frequency_d4():
