@@ -96,8 +96,12 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+# device types the wrappers accept (the library reads device memory only)
+_DEVICE_TYPES = ("cuda",)
+
+
 def _check(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+    if not isinstance(t, torch.Tensor) or t.device.type not in _DEVICE_TYPES:
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
@@ -105,6 +109,32 @@ def _check(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
         raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _expect(t, name: str, dtype: torch.dtype, shape, device):
+    """t must be a contiguous CUDA tensor of this dtype and exact shape on
+    `device` (the device of the call's first input)."""
+    _check(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's inputs on {device}")
+
+
+def _same_device(device, **tensors):
+    for name, t in tensors.items():
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the call's inputs on {device}")
+
+
+def _pages(k_pages, v_pages, page_size: int, d: int, heads=None):
+    """k_pages, v_pages: the same [P, heads, page_size, d] shape."""
+    if v_pages.shape != k_pages.shape:
+        raise ValueError("k_pages and v_pages must have the same shape")
+    want = (heads if heads is not None else k_pages.shape[1], int(page_size), d)
+    if tuple(k_pages.shape[1:]) != want:
+        raise ValueError(f"pages must be [P, {want[0]}, {want[1]}, {want[2]}], got "
+                         f"{tuple(k_pages.shape)}")
 
 
 def _raise_if(status: int, what: str):
@@ -119,14 +149,15 @@ def fa_fwd(q, k, v, causal: bool, scale: Optional[float] = None, o=None, lse=Non
     B, H, N, d = q.shape
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must have the same [B,H,N,d] shape")
+    _same_device(q.device, k=k, v=v)
     if scale is None:
         scale = d ** -0.5
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _check(o, "o", torch.bfloat16, 4)
-    _check(lse, "lse", torch.float32, 3)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (B, H, N), q.device)
     rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                       B, H, N, d, int(bool(causal)), float(scale), _stream(stream))
     _raise_if(rc, "fa_fwd")
@@ -143,14 +174,15 @@ def fa_fwd_gqa(q, k, v, causal: bool, scale: Optional[float] = None, o=None, lse
     H_kv = k.shape[1]
     if k.shape != (B, H_kv, N, d) or v.shape != k.shape:
         raise ValueError("k, v must be [B,H_kv,N,d] with q's B, N, d")
+    _same_device(q.device, k=k, v=v)
     if scale is None:
         scale = d ** -0.5
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _check(o, "o", torch.bfloat16, 4)
-    _check(lse, "lse", torch.float32, 3)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (B, H, N), q.device)
     rc = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           B, H, H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
     _raise_if(rc, "fa_fwd_gqa")
@@ -172,12 +204,15 @@ def fa_fwd_rope(q, k, v, rope_cos, rope_sin, causal: bool, scale: Optional[float
         raise ValueError("k, v must be [B,H_kv,N,d] with q's B, N, d")
     if rope_cos.shape[1] != d // 2 or rope_sin.shape != rope_cos.shape:
         raise ValueError("rope tables must be [max_pos, d/2]")
+    _same_device(q.device, k=k, v=v, rope_cos=rope_cos, rope_sin=rope_sin)
     if scale is None:
         scale = d ** -0.5
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (B, H, N), q.device)
     rc = lib().fa_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                            rope_cos.data_ptr(), rope_sin.data_ptr(), rope_cos.shape[0], B, H,
                            H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
@@ -193,13 +228,16 @@ def fa_bwd(q, k, v, o, lse, dout, causal: bool, scale: Optional[float] = None, d
         _check(t, n, torch.bfloat16, 4)
         if t.shape != q.shape:
             raise ValueError(f"{n} must have q's shape")
-    _check(lse, "lse", torch.float32, 3)
     B, H, N, d = q.shape
+    _expect(lse, "lse", torch.float32, (B, H, N), q.device)
+    _same_device(q.device, k=k, v=v, o=o, dout=dout)
     if scale is None:
         scale = d ** -0.5
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _expect(t, n, torch.bfloat16, q.shape, q.device)
     rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                       dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
                       int(bool(causal)), float(scale), _stream(stream))
@@ -218,12 +256,16 @@ def fa_bwd_gqa(q, k, v, o, lse, dout, causal: bool, scale: Optional[float] = Non
     if o.shape != q.shape or dout.shape != q.shape or k.shape != (B, H_kv, N, d) or \
             v.shape != k.shape:
         raise ValueError("q, o, dout must be [B,H,N,d] and k, v [B,H_kv,N,d]")
-    _check(lse, "lse", torch.float32, 3)
+    _expect(lse, "lse", torch.float32, (B, H, N), q.device)
+    _same_device(q.device, k=k, v=v, o=o, dout=dout)
     if scale is None:
         scale = d ** -0.5
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _expect(dq, "dq", torch.bfloat16, q.shape, q.device)
+    _expect(dk, "dk", torch.bfloat16, k.shape, q.device)
+    _expect(dv, "dv", torch.bfloat16, k.shape, q.device)
     rc = lib().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H,
                           H_kv, N, d, int(bool(causal)), float(scale), _stream(stream))
@@ -239,18 +281,22 @@ def fa_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen: int, causal: bo
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _check(t, n, torch.bfloat16, 3)
     _check(cu_seqlens, "cu_seqlens", torch.int32, 1)
-    _check(lse, "lse", torch.float32, 2)
     total, H, d = q.shape
     H_kv = k.shape[1]
     if o.shape != q.shape or dout.shape != q.shape or k.shape != (total, H_kv, d) or \
             v.shape != k.shape:
         raise ValueError("q, o, dout must be [total,H,d] and k, v [total,H_kv,d]")
+    _expect(lse, "lse", torch.float32, (H, total), q.device)
+    _same_device(q.device, k=k, v=v, o=o, dout=dout, cu_seqlens=cu_seqlens)
     B = cu_seqlens.numel() - 1
     if scale is None:
         scale = d ** -0.5
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _expect(dq, "dq", torch.bfloat16, q.shape, q.device)
+    _expect(dk, "dk", torch.bfloat16, k.shape, q.device)
+    _expect(dv, "dv", torch.bfloat16, k.shape, q.device)
     rc = lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                              lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                              dv.data_ptr(), cu_seqlens.data_ptr(), B, H, H_kv, total,
@@ -266,6 +312,9 @@ def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
         _check(t, n, torch.bfloat16, 3)
     _check(cu_seqlens, "cu_seqlens", torch.int32, 1)
     total, H, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same [total,H,d] shape")
+    _same_device(q.device, k=k, v=v, cu_seqlens=cu_seqlens)
     B = cu_seqlens.numel() - 1
     if scale is None:
         scale = d ** -0.5
@@ -273,6 +322,8 @@ def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (H, total), q.device)
     rc = lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                              lse.data_ptr(), cu_seqlens.data_ptr(), B, H, total,
                              int(max_seqlen), d, int(bool(causal)), float(scale),
@@ -292,6 +343,7 @@ def fa_fwd_varlen_gqa(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
     H_kv = k.shape[1]
     if k.shape != (total, H_kv, d) or v.shape != k.shape:
         raise ValueError("k, v must be [total,H_kv,d]")
+    _same_device(q.device, k=k, v=v, cu_seqlens=cu_seqlens)
     B = cu_seqlens.numel() - 1
     if scale is None:
         scale = d ** -0.5
@@ -299,6 +351,8 @@ def fa_fwd_varlen_gqa(q, k, v, cu_seqlens, max_seqlen: int, causal: bool,
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (H, total), q.device)
     rc = lib().fa_fwd_varlen_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                  lse.data_ptr(), cu_seqlens.data_ptr(), B, H, H_kv, total,
                                  int(max_seqlen), d, int(bool(causal)), float(scale),
@@ -316,8 +370,16 @@ def fa_decode_paged(q, k_pages, v_pages, page_table, seq_lens, page_size: int = 
     _check(page_table, "page_table", torch.int32, 1)
     _check(seq_lens, "seq_lens", torch.int32, 1)
     B, H, d = q.shape
+    # the multi-head call takes no pool size, so the pool's layout is checked
+    # here: a cache of another head count or page size would be misread
+    _pages(k_pages, v_pages, page_size, d, heads=H)
+    if seq_lens.numel() != B:
+        raise ValueError(f"seq_lens must hold one length per sequence ({B})")
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, page_table=page_table,
+                 seq_lens=seq_lens)
     if o is None:
         o = torch.empty_like(q)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
     rc = lib().fa_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
                                B, H, d, int(page_size), _stream(stream))
@@ -336,8 +398,16 @@ def fa_decode_paged_gqa(q, k_pages, v_pages, page_table, seq_lens, page_size: in
     _check(seq_lens, "seq_lens", torch.int32, 1)
     B, H, d = q.shape
     H_kv = k_pages.shape[1]
+    _pages(k_pages, v_pages, page_size, d)
+    if H_kv == 0 or H % H_kv != 0:
+        raise ValueError(f"H ({H}) must be a multiple of the cache's K/V heads ({H_kv})")
+    if seq_lens.numel() != B:
+        raise ValueError(f"seq_lens must hold one length per sequence ({B})")
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, page_table=page_table,
+                 seq_lens=seq_lens)
     if o is None:
         o = torch.empty_like(q)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
     rc = lib().fa_decode_paged_gqa(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                    page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
                                    B, H, H_kv, k_pages.shape[0], d, int(page_size),
@@ -359,8 +429,16 @@ def fa_decode_paged_strided(q, k_pages, v_pages, block_table, seq_lens, page_siz
     H_kv = k_pages.shape[1]
     if block_table.shape[0] != B:
         raise ValueError("block_table must have one row per sequence")
+    _pages(k_pages, v_pages, page_size, d)
+    if H_kv == 0 or H % H_kv != 0:
+        raise ValueError(f"H ({H}) must be a multiple of the cache's K/V heads ({H_kv})")
+    if seq_lens.numel() != B:
+        raise ValueError(f"seq_lens must hold one length per sequence ({B})")
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens)
     if o is None:
         o = torch.empty_like(q)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
     rc = lib().fa_decode_paged_strided(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                        block_table.data_ptr(), block_table.shape[1],
                                        seq_lens.data_ptr(), o.data_ptr(), B, H, H_kv,
@@ -380,8 +458,16 @@ def fa_decode_paged_noalloc(q, k_pages, v_pages, page_table, seq_lens, page_size
     _check(page_table, "page_table", torch.int32, 1)
     _check(seq_lens, "seq_lens", torch.int32, 1)
     B, H, d = q.shape
+    # the multi-head call takes no pool size, so the pool's layout is checked
+    # here: a cache of another head count or page size would be misread
+    _pages(k_pages, v_pages, page_size, d, heads=H)
+    if seq_lens.numel() != B:
+        raise ValueError(f"seq_lens must hold one length per sequence ({B})")
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, page_table=page_table,
+                 seq_lens=seq_lens)
     if o is None:
         o = torch.empty_like(q)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
     rc = lib().fa_decode_paged_noalloc(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                        page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
                                        B, H, d, int(page_size), _stream(stream))
@@ -402,6 +488,13 @@ def fa_append_paged(k_new, v_new, cu_new, k_pages, v_pages, page_table, seq_lens
     _check(page_table, "page_table", torch.int32, 1)
     _check(seq_lens, "seq_lens", torch.int32, 1)
     total_new, H_kv, d = k_new.shape
+    if v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must have the same shape")
+    _pages(k_pages, v_pages, page_size, d, heads=H_kv)
+    if seq_lens.numel() != cu_new.numel() - 1:
+        raise ValueError("seq_lens must hold one length per sequence of cu_new")
+    _same_device(k_new.device, v_new=v_new, cu_new=cu_new, k_pages=k_pages, v_pages=v_pages,
+                 page_table=page_table, seq_lens=seq_lens)
     rc = lib().fa_append_paged(k_new.data_ptr(), v_new.data_ptr(), cu_new.data_ptr(),
                                k_pages.data_ptr(), v_pages.data_ptr(), page_table.data_ptr(),
                                seq_lens.data_ptr(), cu_new.numel() - 1, H_kv, total_new,
@@ -421,12 +514,22 @@ def fa_prefill_paged(q, k_pages, v_pages, page_table, seq_lens, cu_q, max_q: int
     _check(seq_lens, "seq_lens", torch.int32, 1)
     _check(cu_q, "cu_q", torch.int32, 1)
     total_q, H, d = q.shape
+    _pages(k_pages, v_pages, page_size, d)
+    if k_pages.shape[1] == 0 or H % k_pages.shape[1] != 0:
+        raise ValueError(f"H ({H}) must be a multiple of the cache's K/V heads "
+                         f"({k_pages.shape[1]})")
+    if seq_lens.numel() != cu_q.numel() - 1:
+        raise ValueError("seq_lens must hold one length per sequence of cu_q")
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, page_table=page_table,
+                 seq_lens=seq_lens, cu_q=cu_q)
     if scale is None:
         scale = d ** -0.5
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (H, total_q), q.device)
     rc = lib().fa_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                 page_table.data_ptr(), seq_lens.data_ptr(), cu_q.data_ptr(),
                                 o.data_ptr(), lse.data_ptr(), cu_q.numel() - 1, H,
@@ -443,9 +546,13 @@ def fa_gather_paged(pages, page_table, seq_lens, total_tokens: int, page_size: i
     _check(page_table, "page_table", torch.int32, 1)
     _check(seq_lens, "seq_lens", torch.int32, 1)
     _, H, _, d = pages.shape
+    if pages.shape[2] != int(page_size):
+        raise ValueError(f"pages must hold {page_size} tokens each, got {pages.shape[2]}")
     B = seq_lens.numel()
+    _same_device(pages.device, page_table=page_table, seq_lens=seq_lens)
     if out is None:
         out = torch.empty((total_tokens, H, d), dtype=torch.bfloat16, device=pages.device)
+    _expect(out, "out", torch.bfloat16, (total_tokens, H, d), pages.device)
     rc = lib().fa_gather_paged(pages.data_ptr(), page_table.data_ptr(), seq_lens.data_ptr(),
                                out.data_ptr(), B, H, d, int(page_size), _stream(stream))
     _raise_if(rc, "fa_gather_paged")

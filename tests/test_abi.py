@@ -307,3 +307,88 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(binding, "LIB_PATH", "/nonexistent/libfa.so")
     with pytest.raises(ImportError):
         binding.lib()
+
+
+# -- the Python wrappers reject inconsistent tensors before calling the library --
+# (meta tensors carry shapes, dtypes and devices without memory; the library
+# handle is replaced by one that fails the test if any call reaches it)
+
+@pytest.fixture
+def meta_binding(monkeypatch):
+    from attn_fwd_04_b200 import fa as binding
+
+    def no_library():
+        raise AssertionError("the library was called")
+
+    monkeypatch.setattr(binding, "_DEVICE_TYPES", ("cuda", "meta"))
+    monkeypatch.setattr(binding, "lib", no_library)
+    return binding
+
+
+def _m(*shape, dtype=torch.bfloat16):
+    return torch.empty(shape, dtype=dtype, device="meta")
+
+
+def _decode_args(B=3, H=4, P=5, Hc=None, PS=256, d=128, nlen=None):
+    Hc = H if Hc is None else Hc
+    return (_m(B, H, d), _m(P, Hc, PS, d), _m(P, Hc, PS, d), _m(7, dtype=torch.int32),
+            _m(B if nlen is None else nlen, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("name", ["fa_decode_paged", "fa_decode_paged_noalloc"])
+def test_multihead_decode_wrappers_check_the_pool(meta_binding, name):
+    f = getattr(meta_binding, name)
+    with pytest.raises(AssertionError, match="library was called"):
+        f(*_decode_args())                      # consistent: reaches the library
+    with pytest.raises(ValueError, match="pages"):
+        f(*_decode_args(Hc=2))                  # a grouped pool: other head count
+    q, kp, vp, pt, sl = _decode_args()
+    with pytest.raises(ValueError, match="pages"):
+        f(q, _m(5, 4, 128, 128), _m(5, 4, 128, 128), pt, sl)   # page size 128, not 256
+    with pytest.raises(ValueError, match="same shape"):
+        f(q, kp, _m(6, 4, 256, 128), pt, sl)    # k and v pools differ
+    with pytest.raises(ValueError, match="one length per sequence"):
+        f(*_decode_args(nlen=2))
+    with pytest.raises(ValueError, match="shape"):
+        f(q, kp, vp, pt, sl, o=_m(3, 4, 64))    # output of another shape
+    with pytest.raises(TypeError):
+        f(q, kp, vp, pt, sl, o=_m(3, 4, 128, dtype=torch.float32))
+
+
+def test_grouped_decode_wrappers_check_the_pool(meta_binding):
+    q, kp, vp, pt, sl = _decode_args(H=8, Hc=2)
+    with pytest.raises(AssertionError, match="library was called"):
+        meta_binding.fa_decode_paged_gqa(q, kp, vp, pt, sl)
+    q3, kp3, vp3, _, _ = _decode_args(H=8, Hc=3)
+    with pytest.raises(ValueError, match="multiple"):
+        meta_binding.fa_decode_paged_gqa(q3, kp3, vp3, pt, sl)
+    with pytest.raises(ValueError, match="one length per sequence"):
+        meta_binding.fa_decode_paged_gqa(q, kp, vp, pt, _m(4, dtype=torch.int32))
+    bt = _m(3, 6, dtype=torch.int32)
+    with pytest.raises(AssertionError, match="library was called"):
+        meta_binding.fa_decode_paged_strided(q, kp, vp, bt, sl)
+    with pytest.raises(ValueError, match="pages"):
+        meta_binding.fa_decode_paged_strided(q, kp, vp, bt, sl, page_size=128)
+
+
+def test_forward_and_backward_wrappers_check_outputs(meta_binding):
+    q = _m(1, 2, 64, 128)
+    with pytest.raises(AssertionError, match="library was called"):
+        meta_binding.fa_fwd(q, q, q, True)
+    with pytest.raises(ValueError, match="shape"):
+        meta_binding.fa_fwd(q, q, q, True, lse=_m(1, 2, 63, dtype=torch.float32))
+    with pytest.raises(ValueError, match="shape"):
+        meta_binding.fa_fwd(q, q, q, True, o=_m(1, 2, 64, 64))
+    lse = _m(1, 2, 64, dtype=torch.float32)
+    with pytest.raises(AssertionError, match="library was called"):
+        meta_binding.fa_bwd(q, q, q, q, lse, q, True)
+    with pytest.raises(ValueError, match="shape"):
+        meta_binding.fa_bwd(q, q, q, q, _m(1, 2, 32, dtype=torch.float32), q, True)
+    with pytest.raises(ValueError, match="shape"):
+        meta_binding.fa_bwd(q, q, q, q, lse, q, True, dk=_m(1, 1, 64, 128))
+    qp = _m(100, 4, 128)
+    cu = _m(3, dtype=torch.int32)
+    with pytest.raises(ValueError, match="shape"):
+        meta_binding.fa_fwd_varlen(qp, _m(100, 2, 128), _m(100, 2, 128), cu, 64, True)
+    with pytest.raises(ValueError, match="shape"):
+        meta_binding.fa_fwd_varlen(qp, qp, qp, cu, 64, True, lse=_m(100, 4, dtype=torch.float32))
