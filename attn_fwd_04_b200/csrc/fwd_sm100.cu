@@ -61,6 +61,12 @@ constexpr float kLazySum = 65536.f;
 // Exponentials of pairs (c/2) % 8 in [0, kPolyPairs) are evaluated with the
 // FMA-pipe polynomial below, the rest with the special-function unit.
 constexpr int kPolyPairs = 0;
+// The two softmax warpgroups take turns: warpgroup 1 starts the exponentials
+// of step j once warpgroup 0 has finished its own, and warpgroup 0 those of
+// step j + 1 once warpgroup 1 has finished step j, so one tile's exponentials
+// run while the other tile's products do, instead of both sharing the
+// special-function unit at the same time.
+constexpr bool kSoftmaxSeq = false;
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by
 // the Remez exchange in exp2_poly_remez.py beside this file.
 constexpr float kExp2P0 = 0.9999280571937561f, kExp2P1 = 0.6932609677314758f,
@@ -83,6 +89,7 @@ struct alignas(1024) FwdSmem {
     uint64_t q_full[2];
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
+    uint64_t sm_turn[2];  // warpgroup t finished the exponentials of a step
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
     uint64_t q_rot;      // RoPE: both Q tiles rotated
     uint64_t drain;
@@ -91,8 +98,8 @@ struct alignas(1024) FwdSmem {
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
-                                          volatile int* abort) {
-    bool ok = mbar_wait(bar, parity, err, FA_DEVERR_TIMEOUT, abort);
+                                          volatile int* abort, uint64_t limit_ns) {
+    bool ok = mbar_wait(bar, parity, err, FA_DEVERR_TIMEOUT, abort, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -190,7 +197,8 @@ __device__ __forceinline__ float exp_pairs(const uint32_t (&s)[BN], uint32_t (&p
 // (i, i + D/2) are turned by the angle whose cosine and sine are
 // cos_t[pos*(D/2) + i], sin_t[...] -- the precomputed table of the page
 // "“Flash”不是那个被时代淘汰的插件" (0539edu.com), section 3.  Computed in fp32
-// (sin term first, then one fused multiply-add) and rounded to bf16.
+// (x_i cos - x_{i+D/2} sin and x_{i+D/2} cos + x_i sin, every product and
+// sum rounded to fp32) and rounded to bf16 for the tensor cores.
 template <int D>
 __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const float* cos_t,
                                          const float* sin_t) {
@@ -221,9 +229,10 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const fl
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const float cc = cs[2 * e + k], ss = sn[2 * e + k];
-                const float bs = b[k] * ss, as = a[k] * ss;
-                ra[k] = fmaf(a[k], cc, -bs);
-                rb[k] = fmaf(b[k], cc, as);
+                // each product rounded to fp32, then the difference / sum
+                // (no fused multiply-add: a fixed, reproducible order)
+                ra[k] = __fsub_rn(__fmul_rn(a[k], cc), __fmul_rn(b[k], ss));
+                rb[k] = __fadd_rn(__fmul_rn(b[k], cc), __fmul_rn(a[k], ss));
             }
             oa[e] = pack_bf16x2(ra[0], ra[1]);
             ob[e] = pack_bf16x2(rb[0], rb[1]);
@@ -341,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t wg = warp / 4;
     unsigned int* err = p.err;
     volatile int* abort = &sm.abort;
+    const uint64_t wlim = p.wait_ns ? p.wait_ns : FA_WAIT_TIMEOUT_NS;
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
@@ -349,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.p_full[t], PAIR ? 8 : BM);  // pair: one arrival per softmax warp
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
+            mbar_init(&sm.sm_turn[t], 4);  // one arrival per softmax warp
         }
         mbar_init(&sm.vfix, 1);
         mbar_init(&sm.q_rot, BM);
@@ -428,9 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          bh);
                 }
                 for (int u = 0; u < 2 * n; ++u) {
+                    if (u + 1 == p.withhold_copy) break;  // failure-detection check
                     const int slot = u % R;
                     const uint32_t ph = (u / R) & 1;
-                    if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
+                    if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
                     if (crank == 0) mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
                     const uint32_t bar = mapa_rank(smem_u32(&sm.kv_full[slot]), 0);
                     const int j = u >> 1;
@@ -456,9 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             for (int u = 0; u < 2 * n; ++u) {
+                // failure-detection check: this copy (and every later one) is
+                // withheld, so its consumer's bounded wait runs out
+                if (u + 1 == p.withhold_copy) break;
                 const int slot = u % R;
                 const uint32_t ph = (u / R) & 1;
-                if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort)) break;
+                if (!mbar_wait(&sm.kv_empty[slot], ph ^ 1, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
                 mbar_arrive_expect_tx(&sm.kv_full[slot], BN * D * 2);
                 if constexpr (PAGED)
                     load_kv(sm.kv[slot], (u & 1) ? &tv : &tk, &sm.kv_full[slot], u >> 1);
@@ -475,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the sequence end (whole 128-byte rows, so the swizzle does not
                 // matter), make the writes visible to the tensor core, release
                 const int vs = ring_slot(n - 1, 1);
-                if (warp_wait(&sm.kv_full[vs], ring_phase(n - 1, 1), err, abort)) {
+                if (warp_wait(&sm.kv_full[vs], ring_phase(n - 1, 1), err, abort, wlim)) {
                     const int zr = klen - (n - 1) * BN;  // first row to clear
                     uint4* base = reinterpret_cast<uint4*>(sm.kv[vs]);
                     const int per_box = (BN - zr) * 8;   // 16-byte words per box
@@ -492,15 +507,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // every copy this CTA started must land before it exits
             if (crank == 0) {
                 for (int t = 0; t < 2; ++t)
-                    if (n_t[t] > 0) mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, nullptr);
+                    if (n_t[t] > 0) mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
                 for (int u = max(0, issued - R); u < issued; ++u)
-                    mbar_wait(&sm.kv_full[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, nullptr);
+                    mbar_wait(&sm.kv_full[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
             } else {
                 // the odd CTA of a pair cannot wait on the even CTA's barriers:
                 // a slot released by the MMAs has landed (and so has Q, read
                 // by earlier products)
                 for (int u = max(0, issued - R); u < issued; ++u)
-                    mbar_wait(&sm.kv_empty[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, abort);
+                    mbar_wait(&sm.kv_empty[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, abort, wlim);
             }
             }  // lane 0
         } else if (warp == 12 && lane == 0 && crank == 0) {
@@ -566,14 +581,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             auto wait_k = [&](int j) {
                 return mbar_wait(&sm.kv_full[ring_slot<R>(j, 0)], ring_phase<R>(j, 0), err,
-                                 FA_DEVERR_TIMEOUT, abort);
+                                 FA_DEVERR_TIMEOUT, abort, wlim);
             };
             if constexpr (ROPE) {
-                ok = mbar_wait(&sm.q_rot, 0, err, FA_DEVERR_TIMEOUT, abort);
+                ok = mbar_wait(&sm.q_rot, 0, err, FA_DEVERR_TIMEOUT, abort, wlim);
             } else {
                 for (int t = 0; t < 2 && ok; ++t)
                     if (n_t[t] > 0)
-                        ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort);
+                        ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort, wlim);
             }
             ok = ok && wait_k(0);
             if (ok) {
@@ -588,9 +603,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int j = 0; ok && j < n; ++j) {
                 if (zero_v_tail && j == n - 1) {
-                    if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort)) break;
+                    if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
                 } else if (!mbar_wait(&sm.kv_full[ring_slot<R>(j, 1)], ring_phase<R>(j, 1), err,
-                                      FA_DEVERR_TIMEOUT, abort)) {
+                                      FA_DEVERR_TIMEOUT, abort, wlim)) {
                     break;
                 }
                 const bool next_k = j + 1 < n;
@@ -598,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < 2; ++t) {
                     if (j >= n_t[t]) continue;
                     // a pair's P comes from both CTAs' softmax warps
-                    if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+                    if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort, wlim)) {
                         ok = false;
                         break;
                     }
@@ -617,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // every MMA this thread issued must be complete before TMEM is freed
             if constexpr (PAIR) tc_commit_pair(smem_u32(&sm.drain));
             else tc_commit(&sm.drain);
-            mbar_wait(&sm.drain, 0, err, FA_DEVERR_TIMEOUT, nullptr);
+            mbar_wait(&sm.drain, 0, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
         }
         __syncwarp();
     } else if (wg < 2) {
@@ -636,7 +651,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_t[t]; ++j) {
-            if (!warp_wait(&sm.s_full[t], j & 1, err, abort)) { ok = false; break; }
+            if (!warp_wait(&sm.s_full[t], j & 1, err, abort, wlim)) { ok = false; break; }
+            if constexpr (kSoftmaxSeq && !PAIR) {
+                // warpgroup 0 waits for warpgroup 1's step j - 1, warpgroup 1
+                // for warpgroup 0's step j (when the other tile has that step)
+                const bool turn = t == 0 ? (j >= 1 && j - 1 < n_t[1]) : (j < n_t[0]);
+                const uint32_t par = static_cast<uint32_t>(t == 0 ? j - 1 : j) & 1u;
+                if (turn && !warp_wait(&sm.sm_turn[t ^ 1], par, err, abort, wlim)) { ok = false; break; }
+            }
             tc_fence_after();
             // masked keys: past the sequence end, or after this row (causal)
             const int kbase = j * BN;
@@ -675,6 +697,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 rs = need_mask ? exp_pairs<true>(s, pk, sl2, m_used, lim)
                                : exp_pairs<false>(s, pk, sl2, m_used, BN);
                 if (pass == 1 || !__any_sync(0xffffffffu, !(rs <= kLazySum))) break;
+            }
+            if constexpr (kSoftmaxSeq && !PAIR) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sm_turn[t]);
             }
             l = l * alpha + rs;
             tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
@@ -728,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // fill and stay zero
             for (int t = 0; ok && t < 2; ++t) {
                 if (n_t[t] == 0) continue;
-                if (!warp_wait(&sm.q_full[t], 0, err, abort)) {
+                if (!warp_wait(&sm.q_full[t], 0, err, abort, wlim)) {
                     ok = false;
                     break;
                 }
@@ -741,8 +767,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // epilogue: O / l -> bf16, log-sum-exp
         for (int t = 0; ok && t < 2; ++t) {
             if (n_t[t] == 0) continue;
-            if (!warp_wait(&sm.stats_full[t], 0, err, abort) ||
-                !warp_wait(&sm.pv_done[t], 0, err, abort))
+            if (!warp_wait(&sm.stats_full[t], 0, err, abort, wlim) ||
+                !warp_wait(&sm.pv_done[t], 0, err, abort, wlim))
                 break;
             tc_fence_after();
             const int qrow = tile_row(t) + r;
@@ -840,9 +866,10 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const float cc = cs[2 * e + k], ss = sn[2 * e + k];
-                const float bs = b[k] * ss, as = a[k] * ss;
-                ra[k] = fmaf(a[k], cc, -bs);
-                rb[k] = fmaf(b[k], cc, as);
+                // each product rounded to fp32, then the difference / sum
+                // (no fused multiply-add: a fixed, reproducible order)
+                ra[k] = __fsub_rn(__fmul_rn(a[k], cc), __fmul_rn(b[k], ss));
+                rb[k] = __fadd_rn(__fmul_rn(b[k], cc), __fmul_rn(a[k], ss));
             }
             oa[e] = pack_bf16x2(ra[0], ra[1]);
             ob[e] = pack_bf16x2(rb[0], rb[1]);

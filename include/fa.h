@@ -129,7 +129,8 @@ FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, floa
  *                        (normally p * base^(-2i/d)); max_pos >= N
  * Position of row n is n.  Rotate-half pairs: for i < d/2,
  *   x'_i = x_i cos - x_{i+d/2} sin,  x'_{i+d/2} = x_{i+d/2} cos + x_i sin,
- * evaluated in fp32 and rounded to bf16 (the tensor cores' input), then
+ * evaluated in fp32 (each product rounded, then the difference or sum, no
+ * fused multiply-add) and rounded to bf16 (the tensor cores' input), then
  * attention as fa_fwd_gqa on the rotated q, k.  Both tables NULL or unaligned:
  * FA_ERR_NULL / FA_ERR_ALIGN; max_pos < N: FA_ERR_SHAPE.
  */
@@ -426,6 +427,25 @@ FA_API int fa_get_device_error(int* code, fa_stream_t stream);
  * Returns FA_OK once launched, or FA_ERR_CUDA.
  */
 FA_API int fa_selftest_bounded_wait(fa_stream_t stream);
+
+/*
+ * fa_selftest_fwd_stall -- the failure-detection path of the forward kernel
+ * itself: fa_fwd (causal, scale 1/sqrt(d), same arguments and layouts) with
+ * the K/V copy of ring use `withheld` (0: K of key tile 0, 1: V of tile 0,
+ * 2: K of tile 1, ...; every later copy too) never issued, and every wait of
+ * the kernel bounded by `wait_us` microseconds (1 .. 2,000,000) instead of
+ * the usual two seconds.  In each CTA with that many copies the MMA issuer's
+ * wait runs out, records FA_ERR_DEVICE_TIMEOUT and sets the CTA's abort flag;
+ * the other roles leave their loops, the copies already started land, the
+ * products already issued complete, TMEM is freed and the CTA returns (no
+ * trap, no fault: the GPU context stays usable).  o and lse are then partly
+ * unwritten.  The page "为什么“Flash”突然成了AI圈的高频词" (lqnn.cn), section 4,
+ * reports a kernel that stops on a device-side assertion; this call shows the
+ * stall is reported instead.  Returns the status of the launch (as fa_fwd);
+ * read the device error with fa_get_device_error.
+ */
+FA_API int fa_selftest_fwd_stall(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, int withheld, int wait_us, fa_stream_t stream);
 
 /* Free the library workspaces of every stream on the current GPU
  * (synchronises the device first).  Returns FA_OK or FA_ERR_CUDA. */

@@ -15,7 +15,7 @@ import torch
 import attn_fwd_04_b200 as fa
 import oracle
 from attn_fwd_04_b200 import workloads as W
-from helpers import assert_lse_close, assert_o_close, sample_rows, to64
+from helpers import assert_lse_close, assert_o_close, assert_o_close_scaled, sample_rows, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -121,6 +121,20 @@ def test_large_magnitude_scores_stay_finite():
     o_ref, lse_ref = oracle.attention(q, k, v, True, 1.0)
     assert_o_close(to64(o), o_ref, "large scores")
     # lse magnitudes are in the hundreds here; compare relative to them
+    np.testing.assert_allclose(to64(lse), lse_ref, rtol=2e-6, atol=1e-3)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_large_magnitude_values(causal):
+    """Large scores (q, k with std 4) and large values (V with std 4, |V| up
+    to ~18): O is compared with a max-abs gate relative to max |V|, the
+    log-sum-exp at the usual absolute tolerance scaled by its magnitude."""
+    q, k, v = W.custom_fwd_inputs(1, 2, 640, 128, seed=8, std=4.0)
+    o, lse = _fwd_gpu(q, k, v, causal, 1 / math.sqrt(128))
+    o_ref, lse_ref = oracle.attention(q, k, v, causal, 1 / math.sqrt(128))
+    vmax = float(v.float().abs().max())
+    assert vmax > 12
+    assert_o_close_scaled(to64(o), o_ref, vmax, f"large |V| causal={causal}")
     np.testing.assert_allclose(to64(lse), lse_ref, rtol=2e-6, atol=1e-3)
 
 
@@ -270,6 +284,26 @@ def test_bounded_wait_reports_timeout():
     assert_o_close(to64(o), o_ref, "after timeout")
 
 
+@pytest.mark.parametrize("withheld", [0, 3, 6])
+def test_forward_kernel_stall_is_reported_and_recovered(withheld):
+    """Failure detection inside the production forward kernel: one K/V copy
+    (K of tile 0, V of tile 1, or K of tile 3) is never issued and every wait
+    is bounded by 50 ms.  The stall comes back as FA_ERR_DEVICE_TIMEOUT (no
+    trap, no fault), and a normal call on the same stream right after it
+    computes correctly -- its CTAs allocate TMEM and use every barrier again,
+    which they could not if the stalled CTAs had leaked them."""
+    q, k, v = W.custom_fwd_inputs(1, 2, 1000, 128, seed=14)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    assert fa.fa_get_device_error() == fa.FA_OK
+    fa.fa_selftest_fwd_stall(qc, kc, vc, withheld, 50_000)
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_TIMEOUT
+    assert fa.fa_get_device_error() == fa.FA_OK
+    o, lse = _fwd_gpu(q, k, v, True, 1 / math.sqrt(128))
+    o_ref, lse_ref = oracle.attention(q, k, v, True, 1 / math.sqrt(128))
+    assert_o_close(to64(o), o_ref, "after a stalled forward")
+    assert_lse_close(to64(lse), lse_ref, "after a stalled forward")
+
+
 # -- grouped-query attention (fa_fwd_gqa) ----------------------------------------
 
 def _gqa_gpu(q, k, v, causal, scale):
@@ -337,8 +371,8 @@ def test_gqa_long_prefill_sampled():
 # -- rotary embedding fused into the forward pass (fa_fwd_rope) -------------------
 
 def _rope_ref(q, k, v, c, s, causal, scale):
-    """Oracle: rotate q and k (fp32 rotation rounded to bf16, the precision the
-    kernel feeds its tensor cores), then grouped-query attention in fp64."""
+    """Oracle: rotate q and k (the exact rotation rounded once to bf16, the
+    precision of the tensor-core inputs), then grouped-query attention in fp64."""
     qr = oracle.rope(q, c, s, bf16_round=True)
     kr = oracle.rope(k, c, s, bf16_round=True)
     return oracle.attention_gqa(qr, kr, v, causal, scale), qr, kr
@@ -364,23 +398,52 @@ def test_rope_full_compare(shape, causal):
     assert_lse_close(to64(lse), lse_ref, f"rope {shape}")
 
 
-def test_rope_equals_fwd_on_prerotated_inputs():
-    """The in-kernel rotation produces exactly the bf16 values of the oracle's
-    fp32 rotation, so fa_fwd_rope equals fa_fwd_gqa on pre-rotated q, k bit
-    for bit."""
+def _rope_torch_fp32(x, c, s):
+    """The rotation in the library's own fp32 operation order (each product
+    rounded to fp32, then the difference or sum, then bf16), written with
+    plain PyTorch ops on the GPU.  A self-consistency aid, not the oracle."""
+    h = x.shape[-1] // 2
+    N = x.shape[-2]
+    a, b = x[..., :h].float(), x[..., h:].float()
+    cc, ss = c[:N].float(), s[:N].float()
+    ra = a * cc - b * ss
+    rb = b * cc + a * ss
+    return torch.cat([ra, rb], dim=-1).to(torch.bfloat16).contiguous()
+
+
+def test_rope_self_consistent_with_fp32_rotation():
+    """GPU self-consistency, not an oracle check: the in-kernel rotation (Q in
+    shared memory, K by the row kernel) gives exactly the bf16 values of the
+    same fp32 formula evaluated by PyTorch on the GPU, so fa_fwd_rope equals
+    fa_fwd_gqa on inputs pre-rotated that way, bit for bit."""
     B, H, Hkv, N, d = 1, 4, 2, 777, 128
     q, k, v = W.gqa_fwd_inputs(B, H, Hkv, N, d, seed=410, device="cpu")
     c, s = W.rope_tables(N, d)
-    o, lse = fa.fa_fwd_rope(q.cuda(), k.cuda(), v.cuda(), c.cuda(), s.cuda(), True, 0.1)
-    qr = torch.from_numpy(oracle.rope(q, c, s, True)).to(torch.bfloat16).cuda()
-    kr = torch.from_numpy(oracle.rope(k, c, s, True)).to(torch.bfloat16).cuda()
+    q, k, v, c, s = q.cuda(), k.cuda(), v.cuda(), c.cuda(), s.cuda()
+    o, lse = fa.fa_fwd_rope(q, k, v, c, s, True, 0.1)
+    qr, kr = _rope_torch_fp32(q, c, s), _rope_torch_fp32(k, c, s)
     prev = fa.fa_fwd_set_cta_pairs(False)  # the kernel fa_fwd_rope runs on (the default)
     try:
-        o2, l2 = fa.fa_fwd_gqa(qr, kr, v.cuda(), True, 0.1)
+        o2, l2 = fa.fa_fwd_gqa(qr, kr, v, True, 0.1)
     finally:
         fa.fa_fwd_set_cta_pairs(prev)
     assert fa.fa_get_device_error() == fa.FA_OK
     assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+def test_rope_rotation_matches_oracle_rounding_almost_everywhere():
+    """The fp32 rotation (library order) against the oracle's exactly rounded
+    rotation: equal except where the fp32 rounding error crosses a bf16
+    rounding boundary, where they differ by one bf16 step."""
+    B, H, N, d = 1, 4, 2048, 128
+    q = W.gqa_fwd_inputs(B, H, H, N, d, seed=411, device="cpu")[0]
+    c, s = W.rope_tables(N, d)
+    got = _rope_torch_fp32(q.cuda(), c.cuda(), s.cuda()).cpu().double().numpy()
+    want = oracle.rope(q, c, s, True)
+    diff = got != want
+    assert diff.mean() < 1e-3, diff.mean()
+    step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(want[diff]), 1e-30))) - 7)
+    assert np.all(np.abs(got[diff] - want[diff]) <= step * 1.0000001)
 
 
 def test_rope_long_prefill_sampled():
