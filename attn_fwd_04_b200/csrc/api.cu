@@ -177,7 +177,7 @@ namespace {
 int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
               int H_kv, int N, int d, int causal, float scale, fa_stream_t stream,
               const float* rope_cos = nullptr, const float* rope_sin = nullptr,
-              int max_pos = 0) {
+              int max_pos = 0, int withhold_copy = 0, uint64_t wait_ns = 0) {
     if ((rope_cos == nullptr) != (rope_sin == nullptr)) return FA_ERR_NULL;
     if (rope_cos && (max_pos < N || !aligned16(rope_cos) || !aligned16(rope_sin)))
         return max_pos < N ? FA_ERR_SHAPE : FA_ERR_ALIGN;
@@ -233,6 +233,8 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     p.causal = causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = s->err;
+    p.withhold_copy = withhold_copy;
+    p.wait_ns = wait_ns;
     return fa::launch_fwd(p, tq, tk, tv, d, pair ? fa::kFixedPair : fa::kFixed, st);
 }
 
@@ -627,6 +629,19 @@ int fa_selftest_bounded_wait(fa_stream_t stream) {
     }
     fa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(s->err);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_selftest_fwd_stall(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, int withheld, int wait_us,
+                          fa_stream_t stream) {
+    if (withheld < 0 || wait_us < 1 || wait_us > 2000000) return FA_ERR_SHAPE;
+    // the single-CTA kernel (the CTA-pair variant is not selected here)
+    const int prev = g_fwd_pairs.exchange(0);
+    const int rc = fwd_fixed(q, k, v, o, lse, B, H, H, N, d, 1, 1.f / std::sqrt(float(d)),
+                             stream, nullptr, nullptr, 0, withheld + 1,
+                             static_cast<uint64_t>(wait_us) * 1000u);
+    g_fwd_pairs.store(prev);
+    return rc;
 }
 
 int fa_release_workspace(void) {

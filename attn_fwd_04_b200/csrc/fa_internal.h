@@ -32,6 +32,9 @@ struct FwdParams {
     int causal;
     float scale_log2;    // scale * log2(e)
     unsigned int* err;   // device error word
+    // failure-detection check only (fa_selftest_fwd_stall; 0 in every other call):
+    uint64_t wait_ns;    // bound of every wait in the kernel (0: FA_WAIT_TIMEOUT_NS)
+    int withhold_copy;   // 1 + the K/V ring use whose copy the producer withholds (0: none)
 };
 
 // rotary embedding of x [rows, N, d] into y (positions 0..N-1)

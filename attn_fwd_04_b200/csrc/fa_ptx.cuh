@@ -73,12 +73,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity);
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (after recording `code`) when the wait runs past the timeout or when another
-// role of the CTA has already aborted (`*abort` non-zero).  CLUSTER: acquire
-// at cluster scope, for barriers that threads of another CTA arrive on.
+// (after recording `code`) when the wait runs past `limit_ns` of global time
+// or when another role of the CTA has already aborted (`*abort` non-zero).
+// CLUSTER: acquire at cluster scope, for barriers that threads of another CTA
+// arrive on.
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
-                                          unsigned int code, volatile int* abort) {
+                                          unsigned int code, volatile int* abort,
+                                          uint64_t limit_ns = FA_WAIT_TIMEOUT_NS) {
     const uint32_t a = smem_u32(bar);
     auto poll = [&]() {
         if constexpr (CLUSTER) return mbar_try_wait_cluster(a, parity);
@@ -90,7 +92,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
         if (poll()) return true;
         if ((i & 63u) == 0u) {
             if (abort && *abort) return false;
-            if (global_timer_ns() - t0 > FA_WAIT_TIMEOUT_NS) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 record_error(err, code);
                 if (abort) *abort = 1;
                 return false;

@@ -30,8 +30,8 @@ EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_bw
            "fa_decode_paged_gqa", "fa_decode_paged_strided",
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
-           "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
-           "fa_status_str", "fa_version", "fa_fwd_set_cta_pairs")
+           "fa_get_device_error", "fa_selftest_bounded_wait", "fa_selftest_fwd_stall",
+           "fa_release_workspace", "fa_status_str", "fa_version", "fa_fwd_set_cta_pairs")
 
 _lib = None
 
@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.fa_prefill_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P]
         L.fa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
         L.fa_selftest_bounded_wait.argtypes = [P]
+        L.fa_selftest_fwd_stall.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_release_workspace.argtypes = []
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
@@ -79,8 +80,8 @@ def lib() -> ctypes.CDLL:
                      "fa_decode_paged_gqa", "fa_decode_paged_strided", "fa_decode_paged_noalloc",
                      "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
-                     "fa_get_device_error", "fa_selftest_bounded_wait", "fa_release_workspace",
-                     "fa_version", "fa_fwd_set_cta_pairs"):
+                     "fa_get_device_error", "fa_selftest_bounded_wait", "fa_selftest_fwd_stall",
+                     "fa_release_workspace", "fa_version", "fa_fwd_set_cta_pairs"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -570,6 +571,26 @@ def fa_get_device_error(stream=None) -> int:
 def fa_selftest_bounded_wait(stream=None) -> None:
     """Launch the bounded-wait self test; read the result with fa_get_device_error."""
     _raise_if(lib().fa_selftest_bounded_wait(_stream(stream)), "fa_selftest_bounded_wait")
+
+
+def fa_selftest_fwd_stall(q, k, v, withheld: int, wait_us: int, o=None, lse=None,
+                          stream=None):
+    """Launch the causal forward pass with K/V copy `withheld` never issued and
+    every wait bounded by wait_us; read the outcome with fa_get_device_error."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same [B,H,N,d] shape")
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    _expect(lse, "lse", torch.float32, (B, H, N), q.device)
+    rc = lib().fa_selftest_fwd_stall(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     lse.data_ptr(), B, H, N, d, int(withheld), int(wait_us),
+                                     _stream(stream))
+    _raise_if(rc, "fa_selftest_fwd_stall")
+    return o, lse
 
 
 def fa_release_workspace() -> None:
