@@ -12,9 +12,10 @@ solve the linear system p(x_i) - 2^x_i = (-1)^i E 2^x_i on n+2 reference
 points, move the references to the extrema of the new error curve, repeat
 until the equioscillation levels agree.
 
-The kernel's constants (kExp2Poly in fwd_sm100.cu) are this script's output
-rounded to fp32; tests/test_exp2_poly.py checks that they match and that the
-fp32 evaluation stays within the error bound printed here.
+The kernel's constants (kExp2P0 .. kExp2P3 in fwd_sm100.cu) are this script's
+output rounded to fp32; tests/test_exp2_poly.py checks that they match and
+that the fp32 evaluation, with the kernel's range reduction, stays within the
+error bound printed here.
 """
 import sys
 

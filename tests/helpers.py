@@ -39,6 +39,18 @@ def assert_o_close(o_gpu, o_ref, what=""):
     return max_abs, rel_rms
 
 
+def assert_o_close_scaled(o_gpu, o_ref, v_max_abs: float, what=""):
+    """O for values of any magnitude: the max-abs gate is taken relative to the
+    largest |V| (O is a convex combination of V's rows, and its error -- bf16
+    rounding of P and of O itself -- grows with |V|); relative RMS as usual."""
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
+    max_abs, rel_rms = o_errors(o_gpu, o_ref)
+    gate = O_MAX_ABS * max(1.0, v_max_abs)
+    assert max_abs <= gate, f"{what}: O max-abs {max_abs:.3e} > {gate:.3e}"
+    assert rel_rms <= O_REL_RMS, f"{what}: O rel-RMS {rel_rms:.3e} > {O_REL_RMS}"
+    return max_abs, rel_rms
+
+
 def assert_lse_close(lse_gpu, lse_ref, what=""):
     assert np.all(np.isfinite(lse_gpu)), f"{what}: non-finite lse"
     err = float(np.max(np.abs(lse_gpu - lse_ref))) if np.size(lse_ref) else 0.0
