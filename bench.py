@@ -42,7 +42,8 @@ METRIC = "attn fwd TFLOPS & % of BF16 tensor peak; paged-decode HBM GB/s (1×B20
 FWD = W.LONG_PREFILL
 DEC = W.PAGED_DECODE
 DATASHEET_BF16_TFLOPS = 2250.0
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0, "sustained_sm_mhz": 1300.0}
 
 
 # ---------------------------------------------------------------------------
@@ -68,12 +69,39 @@ def load_peaks():
     try:
         with open(p) as f:
             j = json.load(f)
+        cl = j.get("clocks_under_load") or {}
         return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
-                "bf16_tflops_sustained": float(j["bf16_tflops_sustained"]), "source": "measured"}
+                "bf16_tflops_sustained": float(j["bf16_tflops_sustained"]),
+                "sm_max_mhz": float(j.get("sm_max_mhz") or FALLBACK_PEAKS["sm_max_mhz"]),
+                "sustained_sm_mhz": float(cl.get("sm_mhz_median") or
+                                          FALLBACK_PEAKS["sustained_sm_mhz"]),
+                "source": "measured"}
     except Exception:
         d = dict(FALLBACK_PEAKS)
         d["source"] = "fallback"
         return d
+
+
+def tensor_peak_regime(peaks, sm_mhz, region_ms):
+    """Which measured GEMM peak a forward timing is compared with.
+
+    The pool's cuBLAS figures were taken in two regimes: a burst at the full
+    SM clock (bf16_tflops) and a seconds-long loop that settles at the power
+    cap with the clock near `sustained_sm_mhz` (bf16_tflops_sustained).  The
+    timed region is put in the regime its own sampled median SM clock is
+    closer to; without clock samples, by its length (under 2 s: burst).
+    Returns (regime, peak TFLOP/s, reason)."""
+    hi, lo = peaks["sm_max_mhz"], peaks["sustained_sm_mhz"]
+    if sm_mhz is not None:
+        burst = sm_mhz >= 0.5 * (hi + lo)
+        why = (f"median SM clock {sm_mhz:.0f} MHz during the timed region, against "
+               f"{hi:.0f} (burst GEMM) and {lo:.0f} (sustained GEMM)")
+    else:
+        burst = region_ms < 2000.0
+        why = f"no clock samples; timed region {region_ms / 1e3:.2f} s long"
+    if burst:
+        return "burst", peaks["bf16_tflops"], why
+    return "sustained", peaks["bf16_tflops_sustained"], why
 
 
 def kernel_source_sha(files):
@@ -101,55 +129,92 @@ def recorded_traffic(kernel: str, sha: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    """nvidia-smi clock / throttle-reason sampling around the timed region.
+
+    A reader thread stamps every sample with the host's monotonic clock when
+    it arrives, so that the samples taken while the timed region ran (between
+    mark_start() and mark_end(), the host enqueueing the region right after
+    the first mark and waiting for it to finish before the second) can be told
+    apart from those taken before and after it."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_ms: int = 50):
         self.gpu = gpu_index
+        self.period_ms = period_ms
         self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
 
     def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
         except Exception:
             self.proc = None
+            return
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, pw, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append((time.monotonic(), line))
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+
+    @classmethod
+    def parse(cls, stamped, t0=None, t1=None):
+        """Summary of (time, csv line) samples: the median SM clock, max clock,
+        the throttle reasons seen, over the samples inside [t0, t1] (all when
+        no sample falls inside)."""
+        rows = []
+        for t, line in stamped:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
+                sm, smax = float(f[1]), float(f[2])
             except ValueError:
                 continue
             try:
-                pw.append(float(f[3]))
+                pw = float(f[3])
             except ValueError:
-                pass
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+                pw = None
+            rows.append((t, sm, smax, pw, [n for n, v in zip(cls.REASONS, f[5:9])
+                                             if v.lower() == "active"]))
+        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        use = inside if inside else rows
+        sm = [r[1] for r in use]
+        pw = [r[3] for r in use if r[3] is not None]
+        reasons = sorted({n for r in use for n in r[4]})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons),
+                "sm_max_mhz": max(r[2] for r in use) if use else None,
+                "samples": len(use), "samples_in_timed_region": len(inside),
+                "window": "timed region" if inside else "around the timed region (none inside)",
+                "reasons": reasons,
                 "power_w_median": statistics.median(pw) if pw else None}
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(2 * self.period_ms / 1e3)  # let the last in-region sample arrive
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=10)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        return self.parse(list(self.lines), self.t0, self.t1)
 
 
 def dist_setup(args):
@@ -183,6 +248,16 @@ def job_rate(world: int, work_per_rank_step: float, steps: int, max_ms: float) -
     return world * work_per_rank_step * steps / (max_ms * 1e-3)
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -192,32 +267,78 @@ def barrier(world):
 # ---------------------------------------------------------------------------
 # CPU oracle samples (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_fwd_sample(q, k, v, target_s: float, seed: int, n_heads: int = 2):
-    """Time the oracle on seeded random query rows of the forward workload,
-    growing the sample until it has run about target_s seconds.  Rows come
-    from `n_heads` seeded heads, converted to fp64 once outside the timing.
-    Returns (TFLOP/s under the workload's FLOP convention, rows, seconds)."""
-    import numpy as np
-
+def oracle_rows_sample(slices, target_s: float, seed: int, causal: bool = True):
+    """Time the oracle on seeded random query rows of one-head problems,
+    growing the sample until it has run about target_s seconds.  `slices` are
+    (q, k, v) fp64 arrays [1, 1, L, d], converted once outside the timing.
+    FLOPs are counted like the GPU numbers: 4*L*d per row, halved when
+    causal.  Returns (TFLOP/s, rows, seconds)."""
     import oracle
-    B, H, N, d = q.shape
-    scale = 1 / math.sqrt(d)
     g = torch.Generator().manual_seed(seed)
-    heads = torch.randperm(H, generator=g)[:n_heads].tolist()
-    f64 = {h: tuple(np.ascontiguousarray(t[0, h].double().cpu().numpy())[None, None]
-                    for t in (q, k, v)) for h in heads}
-    per_row = (4.0 * N * d) / (2 if FWD.causal else 1)
-    done_rows, spent, count = 0, 0.0, 32
+    done_flops, done_rows, spent, count = 0.0, 0, 0.0, 32
     while spent < target_s:
-        for h in heads:
-            rows = sorted(set(torch.randint(0, N, (count,), generator=g).tolist()))
-            qh, kh, vh = f64[h]
+        for qh, kh, vh in slices:
+            L, d = qh.shape[2], qh.shape[3]
+            rows = sorted(set(torch.randint(0, L, (count,), generator=g).tolist()))
             t0 = time.perf_counter()
-            oracle.attention(qh, kh, vh, FWD.causal, scale, rows=rows)
+            oracle.attention(qh, kh, vh, causal, 1 / math.sqrt(d), rows=rows)
             spent += time.perf_counter() - t0
             done_rows += len(rows)
+            done_flops += len(rows) * 4.0 * L * d / (2 if causal else 1)
         count = min(count * 2, 4096)
-    return per_row * done_rows / spent / 1e12, done_rows, spent
+    return done_flops / spent / 1e12, done_rows, spent
+
+
+def _f64_slice(t):
+    import numpy as np
+    return np.ascontiguousarray(t.double().cpu().numpy())[None, None]
+
+
+def oracle_fwd_sample(q, k, v, target_s: float, seed: int, n_heads: int = 2):
+    """The oracle on seeded random rows of `n_heads` seeded heads of the
+    long-prefill workload (q, k, v [1, H, N, d]) -> (TFLOP/s, rows, seconds)."""
+    H = q.shape[1]
+    g = torch.Generator().manual_seed(seed)
+    heads = torch.randperm(H, generator=g)[:n_heads].tolist()
+    slices = [tuple(_f64_slice(t[0, h]) for t in (q, k, v)) for h in heads]
+    return oracle_rows_sample(slices, target_s, seed + 1, FWD.causal)
+
+
+def oracle_other_workloads(target_s: float):
+    """The oracle on the batched, variable-length and 128K-context forward
+    workloads: seeded random rows of two seeded (sequence, head) problems of
+    each, about target_s seconds apiece.  For the 128K context the full
+    launch's oracle time is extrapolated from the sampled rate by FLOPs."""
+    out = {}
+    for w in (W.BATCHED, W.CTX128K):
+        q, k, v = W.fwd_inputs(w, device="cuda")[:3]
+        g = torch.Generator().manual_seed(w.seed)
+        picks = [(int(torch.randint(0, w.B, (1,), generator=g)),
+                  int(torch.randint(0, w.H, (1,), generator=g))) for _ in range(2)]
+        slices = [tuple(_f64_slice(t[b, h]) for t in (q, k, v)) for b, h in picks]
+        del q, k, v
+        tf, rows, secs = oracle_rows_sample(slices, target_s, w.seed, w.causal)
+        d = {"value": tf, "unit": "TFLOP/s",
+             "sample": f"{rows} seeded random rows of (sequence, head) {picks}, {secs:.1f} s"}
+        if w is W.CTX128K:
+            d["extrapolated_full_launch_s"] = fwd_flops(w) / (tf * 1e12)
+            d["note"] = "full-launch time extrapolated from the sampled rate by FLOPs"
+        out[w.name] = d
+    w = W.BATCHED_VARLEN
+    q, k, v, cu = W.varlen_workload_inputs(w, device="cuda")
+    g = torch.Generator().manual_seed(w.seed)
+    picks = [(int(torch.randint(0, w.B, (1,), generator=g)),
+              int(torch.randint(0, w.H, (1,), generator=g))) for _ in range(2)]
+    slices = [tuple(_f64_slice(t[int(cu[b]):int(cu[b + 1]), h]) for t in (q, k, v))
+              for b, h in picks]
+    del q, k, v
+    tf, rows, secs = oracle_rows_sample(slices, target_s, w.seed, w.causal)
+    out[w.name] = {"value": tf, "unit": "TFLOP/s",
+                   "sample": f"{rows} seeded random rows of (sequence, head) {picks} "
+                             f"(lengths {[int(cu[b + 1] - cu[b]) for b, _ in picks]}), "
+                             f"{secs:.1f} s"}
+    torch.cuda.empty_cache()
+    return out
 
 
 def oracle_decode_sample(cache: W.PagedCache, target_s: float):
@@ -401,9 +522,11 @@ def decode_cache(batch: int, h_kv: int) -> W.PagedCache:
 
 
 def run_single_path(args, local):
-    """Profiling aid (--only prefill / rope / bwd): the paged-prefill workload,
-    or the RoPE forward pass or the backward pass on the long-prefill workload,
-    alone, timed with CUDA events; prints its own short JSON line."""
+    """Profiling aid (--only prefill / rope / bwd / batched / varlen): the
+    paged-prefill workload, the RoPE forward pass or the backward pass on the
+    long-prefill workload, or the forward pass on the batched or the
+    variable-length prefill workload, alone, timed with CUDA events; prints
+    its own short JSON line."""
     import attn_fwd_04_b200 as fa
     torch.cuda.set_device(local)
     stream = torch.cuda.current_stream()
@@ -420,6 +543,29 @@ def run_single_path(args, local):
         def fn():
             fa.fa_bwd(q, k, v, o, lse, g, True, 1 / math.sqrt(w.d), dq=dq, dk=dk, dv=dv,
                       stream=stream)
+    elif args.only == "batched":
+        w = W.BATCHED
+        q, k, v = W.fwd_inputs(w, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        flops = fwd_flops(w)
+        name = w.name
+
+        def fn():
+            fa.fa_fwd(q, k, v, w.causal, 1 / math.sqrt(w.d), o=o, lse=lse, stream=stream)
+    elif args.only == "varlen":
+        w = W.BATCHED_VARLEN
+        q, k, v, cu = W.varlen_workload_inputs(w, device="cuda")
+        lens = (cu[1:] - cu[:-1]).tolist()
+        cud = cu.cuda()
+        o = torch.empty_like(q)
+        lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=q.device)
+        flops = sum(4.0 * w.H * L * L * w.d / (2 if w.causal else 1) for L in lens)
+        name = w.name
+
+        def fn():
+            fa.fa_fwd_varlen(q, k, v, cud, max(lens), w.causal, 1 / math.sqrt(w.d), o=o, lse=lse,
+                             stream=stream)
     elif args.only == "prefill":
         w = W.PAGED_PREFILL
         cache, q, cu = W.prefill_workload_inputs(w, device="cuda")
@@ -513,11 +659,13 @@ def run_native(args, world, rank, local):
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)  # let the sampler take its first reading
+    sampler.mark_start()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
+    sampler.mark_end()
     barrier(world)
     clocks = sampler.stop()
     if fa.fa_get_device_error() != fa.FA_OK:
@@ -624,15 +772,17 @@ def run_native(args, world, rank, local):
             cpu_baseline["decode"] = {"value": gbs, "unit": "GB/s",
                                       "sample": f"{seqs} whole sequences (shortest first) of "
                                                 f"the paged-decode workload, {dsecs:.1f} s"}
+        if not args.no_secondary:
+            cpu_baseline["other_workloads"] = oracle_other_workloads(args.cpu_seconds / 3)
+        cpu_baseline["cpu_model"] = cpu_model()
 
     if rank != 0:
         return None
     fwd_sha = kernel_source_sha(["fwd_sm100.cu", "fa_ptx.cuh", "fa_internal.h"])
     dec_sha = kernel_source_sha(["decode_sm100.cu", "fa_ptx.cuh", "fa_internal.h"])
-    # The timed region is a seconds-long loop that runs the GPU at its power
-    # cap, like the sustained GEMM measurement; the burst figure is reported
-    # beside it in pct_of_bf16_peak.
-    peak_tf = peaks["bf16_tflops_sustained"]
+    # the forward's tensor peak is the measured GEMM figure of the regime the
+    # timed region ran in (burst at full clock, or sustained at the power cap)
+    regime, peak_tf, regime_why = tensor_peak_regime(peaks, clocks.get("sm_mhz"), total_ms)
     out = {
         "metric": METRIC,
         "value": fwd_tflops if do_fwd else dec_gbs,
@@ -662,13 +812,16 @@ def run_native(args, world, rank, local):
                                 "causal": FWD.causal, "scale": scale, "seed": FWD.seed}
         out["pct_of_bf16_peak"] = {
             "datasheet_2250": 100 * per_launch_tf / DATASHEET_BF16_TFLOPS,
-            "measured_burst": 100 * per_launch_tf / peak_tf,
+            "measured_burst": 100 * per_launch_tf / peaks["bf16_tflops"],
             "measured_sustained": 100 * per_launch_tf / peaks["bf16_tflops_sustained"]}
         out["fwd_ms_per_launch"] = fwd_sum / args.steps
+        sm_ghz = (clocks.get("sm_mhz") or 0) / 1e3
         out["roofline"] = {"bound": "tensor", "kernel": "fa_fwd_kernel", "achieved": per_launch_tf,
                            "peak": peak_tf, "unit": "TFLOP/s", "frac": per_launch_tf / peak_tf,
-                           "peak_source": f"{peaks['source']} bf16 sustained (seconds-long "
-                                          "GEMM loop at the power cap, as this timed region is)",
+                           "regime": regime,
+                           "peak_source": f"{peaks['source']} bf16 {regime} GEMM peak ({regime_why})",
+                           "timed_region_s": total_ms / 1e3,
+                           "tflops_per_sm_ghz": per_launch_tf / sm_ghz if sm_ghz else None,
                            "traffic": recorded_traffic("fa_fwd_kernel", fwd_sha),
                            "algorithmic_flops_per_launch": flops}
     if do_dec:
@@ -760,7 +913,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the forward pass on the other workloads")
-    ap.add_argument("--only", choices=["all", "fwd", "decode", "prefill", "rope", "bwd"],
+    ap.add_argument("--only", choices=["all", "fwd", "decode", "prefill", "rope", "bwd", "batched",
+                                       "varlen"],
                     default="all",
                     help="profiling aid: run one entry point only (the JSON line then "
                          "reports that part alone)")
@@ -779,7 +933,7 @@ def main(argv=None):
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    if args.only in ("prefill", "rope", "bwd"):
+    if args.only in ("prefill", "rope", "bwd", "batched", "varlen"):
         print(json.dumps(run_single_path(args, int(os.environ.get("LOCAL_RANK", "0")))),
               flush=True)
         return
