@@ -1,10 +1,10 @@
 // decode_noalloc.cu -- fa_decode_paged_noalloc: paged decode that allocates
 // nothing.
 //
-// Some callers cannot call cudaMalloc at all: code running while a CUDA graph
-// is being captured, a real-time serving loop whose memory was all reserved at
-// start-up, or an embedding program with its own device allocator that forbids
-// anyone else from allocating.  fa_decode_paged grows a library workspace on
+// Some callers cannot call cudaMalloc at all: a real-time serving loop whose
+// memory was all reserved at start-up (an allocation could fail, or stall the
+// loop while the allocator synchronises), or an embedding program with its own
+// device allocator that forbids anyone else from allocating.  fa_decode_paged grows a library workspace on
 // first use, which such callers cannot allow.  This entry point runs the same
 // decode kernels with their scratch (split offsets and per-split partial
 // outputs) in a fixed file-scope device array instead.

@@ -27,6 +27,8 @@
 // into the query).
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "fa_ptx.cuh"
 
 namespace fa {
@@ -461,10 +463,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // this one is done), which leaves room for more ring stages.
 // A unit holds gr <= GH query heads (GH, the template, is the capacity of
 // its registers and merge buffer).  Groups larger than 16 (multi-query
-// attention with many heads) are cut into sub equal sub-groups of gr <= 16
-// query heads, each a unit of its own with its K/V head's pages: Hk counts
-// the units per split (H / gr) and K/V head h / sub is read, once per
-// sub-group.
+// attention with many heads) are cut into equal sub-groups of gr <= 16 query
+// heads.  With teams == 2 a unit holds two sub-groups of the same K/V head:
+// each team of four warps takes every chunk for its own sub-group's rows, so
+// a staged K/V chunk serves 2 gr query heads and is read from memory once
+// for both (an even number of sub-groups is paired this way).  Otherwise
+// (teams == 1) each sub-group is a unit of its own and the two teams take
+// alternate chunks.  Hk counts the units per split (H / (teams gr)) and sub
+// the units per K/V head: the unit's K/V head is h / sub.
 // ---------------------------------------------------------------------------
 constexpr int kGqTok = 64;          // tokens per chunk
 constexpr int kGqWarps = 8;         // consumer warps (two teams of four)
@@ -504,7 +510,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
                          const __nv_bfloat16* __restrict__ q,
                          const int32_t* __restrict__ page_table,
                          const int32_t* __restrict__ seq_lens, int B, int H, int Hk, int gr, int sub,
-                         int num_pages, int max_splits, int min_pages,
+                         int teams, int num_pages, int max_splits, int min_pages,
                          const int32_t* __restrict__ page_off,
                          const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
                          float* __restrict__ part_o, float scale_log2, unsigned int* err) {
@@ -525,7 +531,9 @@ __global__ void __launch_bounds__(kGqThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], kGqWarps / 2);  // the four warps of the chunk's team
+            // the four warps of the chunk's team, or all eight when both
+            // teams read every chunk
+            mbar_init(&sm.empty[i], teams == 2 ? kGqWarps : kGqWarps / 2);
         }
         mbar_init(&sm.cmb, kGqWarps * 32);
         mbar_init(&sm.cfree, kGqWarps * 32);
@@ -592,6 +600,9 @@ __global__ void __launch_bounds__(kGqThreads, 1)
 
     // ================= consumers =================
     const int team = warp >> 2, wt = warp & 3;
+    const bool two = teams == 2;
+    const int rows = two ? 2 * gr : gr;      // query heads per unit
+    const int row_off = two ? team * gr : 0;  // this team's first one
     const int grp = lane >> 2, tig = lane & 3;    // fragment row, column pair
     const int lrow = lane & 7, lmat = lane >> 3;  // ldmatrix row and matrix
     int g = 0, k = 0;                             // ring uses, units done
@@ -608,7 +619,8 @@ __global__ void __launch_bounds__(kGqThreads, 1)
             const int row = grp + 8 * rr;
             const bool row_in = row < gr;
             const __nv_bfloat16* qr =
-                q + (static_cast<int64_t>(us.b) * H + us.h * gr + (row_in ? row : 0)) * D;
+                q + (static_cast<int64_t>(us.b) * H + us.h * rows + row_off + (row_in ? row : 0)) *
+                        D;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 qa[ks][rr] = row_in ? __ldg(reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tig)) : 0u;
@@ -623,7 +635,7 @@ __global__ void __launch_bounds__(kGqThreads, 1)
         for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
         const int nchunks = (us.ntok + kGqTok - 1) / kGqTok;
         for (int c = 0; c < nchunks; ++c, ++g) {
-            if ((g & 1) != team) continue;
+            if (!two && (g & 1) != team) continue;
             const int slot = g % STAGES;
             ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (g / STAGES) & 1, err,
                                                    FA_DEVERR_TIMEOUT, abort));
@@ -733,20 +745,27 @@ __global__ void __launch_bounds__(kGqThreads, 1)
         mbar_arrive(&sm.cmb);
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.cmb, k & 1, err, FA_DEVERR_TIMEOUT, abort));
         if (!ok) break;
-        for (int idx = threadIdx.x; idx < gr * D; idx += kGqWarps * 32) {
-            const int hi = idx / D, x = idx - hi * D;
-            float M = -INFINITY;
+        for (int idx = threadIdx.x; idx < rows * D; idx += kGqWarps * 32) {
+            const int ha = idx / D, x = idx - ha * D;  // the unit's query head, column
+            // the warps holding that head's states: its team's four, or all
+            const int tt = two ? ha / gr : 0;
+            const int hi = ha - tt * gr;
+            float M = -INFINITY, L = 0.f, o = 0.f;
+            auto combine = [&](int w0, auto nw_c) {
+                constexpr int NW = decltype(nw_c)::value;
 #pragma unroll
-            for (int w = 0; w < kGqWarps; ++w) M = fmaxf(M, sm.cm[hi][w]);
-            float L = 0.f, o = 0.f;
+                for (int w = 0; w < NW; ++w) M = fmaxf(M, sm.cm[hi][w0 + w]);
 #pragma unroll
-            for (int w = 0; w < kGqWarps; ++w) {
-                const float mw = sm.cm[hi][w];
-                const float wgt = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-                L += wgt * sm.cl[hi][w];
-                o += wgt * sm.co[hi][w][x];
-            }
-            const int64_t pu = static_cast<int64_t>(u) * gr + hi;
+                for (int w = 0; w < NW; ++w) {
+                    const float mw = sm.cm[hi][w0 + w];
+                    const float wgt = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+                    L += wgt * sm.cl[hi][w0 + w];
+                    o += wgt * sm.co[hi][w0 + w][x];
+                }
+            };
+            if (two) combine(4 * tt, std::integral_constant<int, kGqWarps / 2>{});
+            else combine(0, std::integral_constant<int, kGqWarps>{});
+            const int64_t pu = static_cast<int64_t>(u) * rows + ha;
             part_o[pu * D + x] = o / L;
             if (x == 0) part_lse[pu] = M + __log2f(L);
         }
@@ -872,15 +891,17 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// gr query heads per unit (gr <= GH, the kernel's capacity; GH == 1 is the
-// multi-head kernel), sub units per K/V head (a group of gr * sub)
+// gr query heads per team (gr <= GH, the kernel's capacity; GH == 1 is the
+// multi-head kernel), teams sub-groups per unit, sub units per K/V head (a
+// group of gr * teams * sub)
 template <int D, int GH>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
                        const int32_t* seq_lens, void* o, int B, int H, int num_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
-                       int num_sms, cudaStream_t stream, int gr, int sub) {
-    const int Hk = H / gr;  // units per split
+                       int num_sms, cudaStream_t stream, int gr, int sub, int teams = 1) {
+    const int rows = gr * teams;  // query heads per unit
+    const int Hk = H / rows;      // units per split
     // pages a split covers at least: with few units per split (few K/V heads),
     // larger splits keep the partials and per-unit merges down
     const int min_pages = Hk >= kDecodeManyUnits ? kDecodeChunkPages : kDecodeChunkPagesFew;
@@ -927,12 +948,12 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
             return FA_ERR_CUDA;
         split<<<num_sms * occ, kGqThreads, smem, stream>>>(
             *tk, *tv, static_cast<const __nv_bfloat16*>(q), page_table, seq_lens, B, H, Hk, gr, sub,
-            num_pages, max_splits, min_pages, page_off, unit_off, part_lse, part_o, scale_log2,
-            err);
+            teams, num_pages, max_splits, min_pages, page_off, unit_off, part_lse, part_o,
+            scale_log2, err);
     }
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
-        seq_lens, B, H, gr, page_size, max_splits, min_pages, unit_off, part_lse, part_o,
+        seq_lens, B, H, rows, page_size, max_splits, min_pages, unit_off, part_lse, part_o,
         static_cast<__nv_bfloat16*>(o));
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -1005,12 +1026,14 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
                     const int32_t* seq_lens, void* o, int B, int H, int Hk, int num_pages,
                     int page_size, int max_splits, void* workspace, unsigned int* err,
                     int num_sms, cudaStream_t stream) {
-    // a group of G query heads per K/V head runs as sub units of gr = G / sub
-    // heads, sub the fewest that leaves gr <= 16
+    // a group of G query heads per K/V head is cut into sub sub-groups of
+    // gr = G / sub heads, sub the fewest that leaves gr <= 16; an even number
+    // of sub-groups runs as pairs, one unit per pair (both read each chunk)
     const int G = H / Hk;
     int sub = (G + 15) / 16;
     while (G % sub != 0) ++sub;
     const int gr = G / sub;
+    const int teams = (sub % 2 == 0) ? 2 : 1;
     if (G == 1)
         return launch_decode_impl<D, 1>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, B,
                                         H, num_pages, page_size, max_splits, workspace, err,
@@ -1019,7 +1042,7 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
     if (gr <= GH)                                                                               \
         return launch_decode_impl<D, GH>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, \
                                          B, H, num_pages, page_size, max_splits, workspace,    \
-                                         err, num_sms, stream, gr, sub);
+                                         err, num_sms, stream, gr, sub / teams, teams);
     FA_DECODE_GH(2)
     FA_DECODE_GH(4)
     FA_DECODE_GH(8)

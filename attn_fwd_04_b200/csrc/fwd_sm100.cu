@@ -61,12 +61,6 @@ constexpr float kLazySum = 65536.f;
 // Exponentials of pairs (c/2) % 8 in [0, kPolyPairs) are evaluated with the
 // FMA-pipe polynomial below, the rest with the special-function unit.
 constexpr int kPolyPairs = 0;
-// The two softmax warpgroups take turns: warpgroup 1 starts the exponentials
-// of step j once warpgroup 0 has finished its own, and warpgroup 0 those of
-// step j + 1 once warpgroup 1 has finished step j, so one tile's exponentials
-// run while the other tile's products do, instead of both sharing the
-// special-function unit at the same time.
-constexpr bool kSoftmaxSeq = false;
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by
 // the Remez exchange in exp2_poly_remez.py beside this file.
 constexpr float kExp2P0 = 0.9999280571937561f, kExp2P1 = 0.6932609677314758f,
@@ -89,7 +83,6 @@ struct alignas(1024) FwdSmem {
     uint64_t q_full[2];
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
-    uint64_t sm_turn[2];  // warpgroup t finished the exponentials of a step
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
     uint64_t q_rot;      // RoPE: both Q tiles rotated
     uint64_t drain;
@@ -359,7 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.p_full[t], PAIR ? 8 : BM);  // pair: one arrival per softmax warp
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
-            mbar_init(&sm.sm_turn[t], 4);  // one arrival per softmax warp
         }
         mbar_init(&sm.vfix, 1);
         mbar_init(&sm.q_rot, BM);
@@ -652,13 +644,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; j < n_t[t]; ++j) {
             if (!warp_wait(&sm.s_full[t], j & 1, err, abort, wlim)) { ok = false; break; }
-            if constexpr (kSoftmaxSeq && !PAIR) {
-                // warpgroup 0 waits for warpgroup 1's step j - 1, warpgroup 1
-                // for warpgroup 0's step j (when the other tile has that step)
-                const bool turn = t == 0 ? (j >= 1 && j - 1 < n_t[1]) : (j < n_t[0]);
-                const uint32_t par = static_cast<uint32_t>(t == 0 ? j - 1 : j) & 1u;
-                if (turn && !warp_wait(&sm.sm_turn[t ^ 1], par, err, abort, wlim)) { ok = false; break; }
-            }
             tc_fence_after();
             // masked keys: past the sequence end, or after this row (causal)
             const int kbase = j * BN;
@@ -697,10 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 rs = need_mask ? exp_pairs<true>(s, pk, sl2, m_used, lim)
                                : exp_pairs<false>(s, pk, sl2, m_used, BN);
                 if (pass == 1 || !__any_sync(0xffffffffu, !(rs <= kLazySum))) break;
-            }
-            if constexpr (kSoftmaxSeq && !PAIR) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.sm_turn[t]);
             }
             l = l * alpha + rs;
             tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));

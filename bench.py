@@ -376,11 +376,16 @@ GQA_HKV = 8
 
 def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
     """Throughput on the other workloads (tiny, batched, variable-length, 128K
-    context; the grouped-query forward and decode), timed with CUDA events;
-    reported beside the headline number, not part of the timed step."""
+    context; the grouped-query forward and decode), timed with CUDA events,
+    each after a 0.5 s idle pause; reported beside the headline number, not
+    part of the timed step."""
     out = {}
 
     def timed(fn, flops, name, extra=None, n=steps):
+        # every workload starts from an idle GPU, so that none inherits the
+        # power-capped clock of the one before it
+        torch.cuda.synchronize()
+        time.sleep(0.5)
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize()
@@ -404,7 +409,6 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
     q, k, v = W.fwd_inputs(FWD, device="cuda")[:3]
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    time.sleep(0.5)
     timed(lambda: fa.fa_fwd(q, k, v, FWD.causal, 1 / math.sqrt(FWD.d), o=o, lse=lse,
                             stream=stream),
           fwd_flops(FWD), FWD.name + "_burst20", {"what": "20 launches after 0.5 s idle"}, n=20)

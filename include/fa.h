@@ -40,10 +40,11 @@
  *    stream are ordered by the stream.  The key is the stream handle: destroy
  *    a stream only after its calls have completed (a new stream may get the
  *    same handle), and call fa_release_workspace to return the memory of
- *    streams no longer used.  Under CUDA graph capture a call must not
- *    allocate or grow its stream's workspace (the allocation would belong to
- *    the graph): make one eager call of the largest size on that stream
- *    before capturing, or use fa_decode_paged_noalloc.
+ *    streams no longer used.
+ *  - Cached device state: the library caches, per GPU, the device addresses
+ *    of its error word and of the allocation-free decode's scratch array.
+ *    They belong to the GPU's primary context: do not keep using the library
+ *    across a cudaDeviceReset (which destroys that context).
  *  - Thread safety: the host entry points may be called from several host
  *    threads; the workspace bookkeeping is guarded by a mutex.
  */
@@ -383,11 +384,12 @@ FA_API int fa_gather_paged(const void* pages, const int32_t* page_table, const i
  * that must not allocate device memory (the pages have no counterpart: this
  * is a deployment variant of the decode entry point).
  *
- * Who needs it: code that runs while a CUDA graph is being captured, serving
- * loops that reserve all device memory up front, and hosts with their own
- * device allocator that forbid other allocations cannot let the library call
- * cudaMalloc, which fa_decode_paged does on its first call (and whenever it
- * needs a larger workspace).
+ * Who needs it: serving loops that reserve all device memory up front (so
+ * that a later allocation can fail, or stall the loop while the allocator
+ * synchronises), and host programs with their own device allocator that
+ * forbid any other allocation, cannot let the library call cudaMalloc, which
+ * fa_decode_paged does on its first call (and whenever it needs a larger
+ * workspace).
  *
  * Arguments, layouts and results are those of fa_decode_paged.  The scratch
  * (split offsets and per-split partial outputs) lives in one fixed 16 MiB
