@@ -172,8 +172,8 @@ int device_error_word(unsigned int** err, int* num_sms) {
 namespace {
 
 // Fixed-length forward pass with H query heads and H_kv K/V heads; with
-// rope_cos / rope_sin (tables of max_pos rows) Q and K are rotated first: K
-// once per position into the workspace, Q tile by tile inside the kernel.
+// rope_cos / rope_sin (tables of max_pos rows) Q and K are rotated first,
+// once per position, into the stream's workspace.
 int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
               int H_kv, int N, int d, int causal, float scale, fa_stream_t stream,
               const float* rope_cos = nullptr, const float* rope_sin = nullptr,
@@ -195,18 +195,25 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const void* k_use = k;
+    const void* q_use = q;
     if (rope_cos) {
+        // RoPE: Q and K rotated once per position by one row-kernel launch
+        // into the stream's workspace; the forward kernel then reads them
         void* ws = nullptr;
         const size_t kbytes = static_cast<size_t>(B) * H_kv * N * d * 2;
-        if ((rc = ensure_workspace(s, kbytes, st, &ws)) != FA_OK) return rc;
-        if ((rc = fa::launch_rope_rows(k, ws, rope_cos, rope_sin,
-                                       static_cast<int64_t>(B) * H_kv, N, d, s->num_sms, st)) !=
-            FA_OK)
+        const size_t qbytes = static_cast<size_t>(B) * H * N * d * 2;
+        if ((rc = ensure_workspace(s, kbytes + qbytes, st, &ws)) != FA_OK) return rc;
+        void* kr = ws;
+        void* qr = static_cast<uint8_t*>(ws) + kbytes;
+        if ((rc = fa::launch_rope_rows(k, kr, static_cast<int64_t>(B) * H_kv, q, qr,
+                                       static_cast<int64_t>(B) * H, rope_cos, rope_sin, N, d,
+                                       s->num_sms, st)) != FA_OK)
             return rc;
-        k_use = ws;
+        k_use = kr;
+        q_use = qr;
     }
     // CTA pairs (2-SM products) load K in halves of 64 keys
-    const bool pair = d == 128 && rope_cos == nullptr && g_fwd_pairs.load() != 0;
+    const bool pair = d == 128 && g_fwd_pairs.load() != 0;
     CUtensorMap tq, tk, tv;
     const cuuint64_t dims_q[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                   static_cast<cuuint64_t>(B) * H};
@@ -216,7 +223,7 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
                                    static_cast<cuuint64_t>(N) * d * 2};
     const cuuint32_t box[3] = {64, 128, 1};
     const cuuint32_t box_k[3] = {64, pair ? 64u : 128u, 1};
-    if ((rc = make_map(&tq, q, dims_q, strides, box)) != FA_OK) return rc;
+    if ((rc = make_map(&tq, q_use, dims_q, strides, box)) != FA_OK) return rc;
     if ((rc = make_map(&tk, k_use, dims_kv, strides, box_k)) != FA_OK) return rc;
     if ((rc = make_map(&tv, v, dims_kv, strides, box)) != FA_OK) return rc;
     fa::FwdParams p{};
@@ -226,8 +233,6 @@ int fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, 
     p.B = B;
     p.H = H;
     p.H_kv = H_kv;
-    p.rope_cos = rope_cos;
-    p.rope_sin = rope_sin;
     p.N = N;
     p.total = 0;
     p.causal = causal ? 1 : 0;

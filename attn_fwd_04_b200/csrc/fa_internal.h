@@ -26,8 +26,6 @@ struct FwdParams {
     int H_kv;            // K/V heads; query head h reads K/V head h / (H / H_kv)
     const int32_t* page_table;  // paged prefill: packed page table
     const int32_t* ctx_lens;    // paged prefill: cached tokens (keys) per sequence
-    const float* rope_cos;      // fixed-length RoPE: [>= N, d/2] tables, or null
-    const float* rope_sin;
     int total;           // varlen: packed rows
     int causal;
     float scale_log2;    // scale * log2(e)
@@ -37,9 +35,11 @@ struct FwdParams {
     int withhold_copy;   // 1 + the K/V ring use whose copy the producer withholds (0: none)
 };
 
-// rotary embedding of x [rows, N, d] into y (positions 0..N-1)
-int launch_rope_rows(const void* x, void* y, const float* cos_t, const float* sin_t, int64_t rows,
-                     int N, int d, int num_sms, cudaStream_t stream);
+// rotary embedding of x0 [rows0, N, d] into y0 and x1 [rows1, N, d] into y1
+// (positions 0..N-1), one launch
+int launch_rope_rows(const void* x0, void* y0, int64_t rows0, const void* x1, void* y1,
+                     int64_t rows1, const float* cos_t, const float* sin_t, int N, int d,
+                     int num_sms, cudaStream_t stream);
 // forward modes; kFixedPair: fixed length on CTA pairs (2-SM products; d = 128,
 // no RoPE), its K map with 64 x 64 boxes (tq, tv: 64 x 128 as for kFixed)
 constexpr int kFixed = 0, kVarlen = 1, kPaged = 2, kFixedPair = 3;

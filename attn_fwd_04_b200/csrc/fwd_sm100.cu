@@ -21,8 +21,7 @@
 //     the other tile's MMAs; each also rescales its own O accumulator when
 //     the running max grows; warpgroup 2 writes the epilogue; in warpgroup 3,
 //     warp 12 issues the MMAs and warp 13 the TMA loads.  Registers are moved
-//     to the softmax warpgroups with setmaxnreg (2 x 192 + 72 + 56 = 4 x 128
-//     per thread);
+//     to the softmax warpgroups with setmaxnreg (kRegsSoftmax etc. below);
 //   * exp is exp2 with scale*log2(e) folded in (the polynomial path below can
 //     take a share of the exponentials off the special-function unit; it is
 //     switched off because it measured slower here); O is rescaled only when
@@ -49,6 +48,13 @@ constexpr int BM = 128;       // query rows per tile (MMA M)
 constexpr int BN = 128;       // keys per K/V tile
 constexpr int kSlots = 4;     // K/V ring slots (each holds one K or one V tile)
 constexpr int kThreads = 512;
+// setmaxnreg shares (registers per thread) of the softmax warpgroups, the
+// epilogue warpgroup and warpgroup 3 (TMA and MMA warps).  They come out of
+// the 128 per thread the block launches with (65536 / 512): a split whose sum
+// exceeded 4 x 128 would make the increase wait forever.
+constexpr uint32_t kRegsSoftmax = 192, kRegsEpilogue = 72, kRegsIssue = 56;
+static_assert(2 * kRegsSoftmax + kRegsEpilogue + kRegsIssue <= 4 * 128,
+              "register split exceeds the launch share");
 constexpr int kHeadGroup = 4;  // (sequence, head) units scheduled together
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
@@ -61,6 +67,15 @@ constexpr float kLazySum = 65536.f;
 // Exponentials of pairs (c/2) % 8 in [0, kPolyPairs) are evaluated with the
 // FMA-pipe polynomial below, the rest with the special-function unit.
 constexpr int kPolyPairs = 0;
+// Single CTA: each tile's products issued by a thread of its own (warps 12
+// and 14), so that one tile's P V and next S do not wait behind the other
+// tile's issue.
+constexpr bool kDualIssue = false;
+// The softmax loads the two halves of a score row separately and starts the
+// exponentials of the first half while the second is still on its way.
+constexpr bool kSplitLoad = false;
+// The softmax signals P_t ready once per warp instead of once per thread.
+constexpr bool kWarpArrive = false;
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by
 // the Remez exchange in exp2_poly_remez.py beside this file.
 constexpr float kExp2P0 = 0.9999280571937561f, kExp2P1 = 0.6932609677314758f,
@@ -84,8 +99,7 @@ struct alignas(1024) FwdSmem {
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
-    uint64_t q_rot;      // RoPE: both Q tiles rotated
-    uint64_t drain;
+    uint64_t drain, drain2;
     uint32_t tmem_base;
     int abort;
 };
@@ -185,53 +199,32 @@ __device__ __forceinline__ float exp_pairs(const uint32_t (&s)[BN], uint32_t (&p
     return f2_lo(a2) + f2_hi(a2);
 }
 
-// Rotary position embedding of row r of a tile in shared memory (one or two
-// 128-row x 64-column boxes, 128-byte swizzle) at position pos: the pairs
-// (i, i + D/2) are turned by the angle whose cosine and sine are
-// cos_t[pos*(D/2) + i], sin_t[...] -- the precomputed table of the page
-// "“Flash”不是那个被时代淘汰的插件" (0539edu.com), section 3.  Computed in fp32
-// (x_i cos - x_{i+D/2} sin and x_{i+D/2} cos + x_i sin, every product and
-// sum rounded to fp32) and rounded to bf16 for the tensor cores.
-template <int D>
-__device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const float* cos_t,
-                                         const float* sin_t) {
-    constexpr int HALF = D / 2;
-    const float* ct = cos_t + static_cast<int64_t>(pos) * HALF;
-    const float* st = sin_t + static_cast<int64_t>(pos) * HALF;
-#pragma unroll 2
-    for (int c = 0; c < HALF / 8; ++c) {
-        const int i0 = 8 * c, i1 = 8 * c + HALF;  // first dims of the two chunks
-        uint4* pa = reinterpret_cast<uint4*>(tile + (i0 / 64) * kBoxBytes + r * 128 +
-                                             ((((i0 % 64) / 8) ^ (r & 7)) * 16));
-        uint4* pb = reinterpret_cast<uint4*>(tile + (i1 / 64) * kBoxBytes + r * 128 +
-                                             ((((i1 % 64) / 8) ^ (r & 7)) * 16));
-        const uint4 ua = *pa, ub = *pb;
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(ct + i0));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(ct + i0 + 4));
-        const float4 s0 = __ldg(reinterpret_cast<const float4*>(st + i0));
-        const float4 s1 = __ldg(reinterpret_cast<const float4*>(st + i0 + 4));
-        const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-        const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
-        uint32_t oa[4], ob[4];
+// exp_pairs over the columns [C0, C1) only, adding the pairs' p into the four
+// packed accumulators acc (the caller sums them).
+template <bool MASKED, int C0, int C1>
+__device__ __forceinline__ void exp_range(const uint32_t (&s)[BN], uint32_t (&pk)[BN / 2],
+                                          uint64_t (&acc)[4], uint64_t sl2, float m, int lim) {
+    const float mb = (m == -INFINITY) ? 0.f : m;
+    const uint64_t nm2 = f2_pack(-mb, -mb);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float a[2] = {__uint_as_float(wa[e] << 16), __uint_as_float(wa[e] & 0xffff0000u)};
-            float b[2] = {__uint_as_float(wb[e] << 16), __uint_as_float(wb[e] & 0xffff0000u)};
-            float ra[2], rb[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const float cc = cs[2 * e + k], ss = sn[2 * e + k];
-                // each product rounded to fp32, then the difference / sum
-                // (no fused multiply-add: a fixed, reproducible order)
-                ra[k] = __fsub_rn(__fmul_rn(a[k], cc), __fmul_rn(b[k], ss));
-                rb[k] = __fadd_rn(__fmul_rn(b[k], cc), __fmul_rn(a[k], ss));
-            }
-            oa[e] = pack_bf16x2(ra[0], ra[1]);
-            ob[e] = pack_bf16x2(rb[0], rb[1]);
+    for (int c = C0; c < C1; c += 2) {
+        const uint64_t x =
+            f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, nm2);
+        float p0, p1;
+        if ((c / 2) % 8 < kPolyPairs) {
+            const uint64_t e = exp2_poly2(x);
+            p0 = f2_lo(e);
+            p1 = f2_hi(e);
+        } else {
+            p0 = ex2_approx(f2_lo(x));
+            p1 = ex2_approx(f2_hi(x));
         }
-        *pa = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        *pb = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        if constexpr (MASKED) {
+            p0 = (c < lim) ? p0 : 0.f;
+            p1 = (c + 1 < lim) ? p1 : 0.f;
+        }
+        acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], f2_pack(p0, p1));
+        pk[c / 2] = pack_bf16x2(p0, p1);
     }
 }
 
@@ -239,9 +232,6 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const fl
 // kPaged (packed queries; keys and values read through the page table from a
 // pool of 256-token pages, the queries being the last positions of each
 // cached sequence).
-// ROPE (fixed-length only): the Q tiles are rotated in shared memory by the
-// epilogue warpgroup (idle until the last step) before their first score
-// product; K arrives rotated (fa_rope_rows_kernel, once per position).
 // PAIR (fixed-length, d = 128, no RoPE): CTAs run in clusters of two and a
 // pair shares one 512-row query block: CTA c of the pair holds 128-row tiles
 // 2t + c (t = 0, 1), and tile pair t (rows 256t .. 256t + 255 of the block) is
@@ -250,13 +240,15 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pos, const fl
 // from L2 once per 512 query rows instead of once per 256, and the B operand
 // is read from shared memory once for both SMs.  The even CTA issues every
 // MMA; both CTAs run the softmax and epilogue of their own tiles.
-template <int D, int MODE, bool ROPE, bool PAIR>
+template <int D, int MODE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
     constexpr bool VARLEN = MODE != kFixed;  // packed query rows
     constexpr bool PAGED = MODE == kPaged;
-    static_assert(!PAIR || (D == 128 && MODE == kFixed && !ROPE), "pair mode: fixed length, d=128");
+    static_assert(!PAIR || (D == 128 && MODE == kFixed), "pair mode: fixed length, d=128");
+    constexpr bool DUAL = kDualIssue && !PAIR;      // one MMA thread per tile
+    constexpr bool WARP_ARRIVE = kWarpArrive || PAIR;
     constexpr int R = ring_slots<PAIR>();          // K/V ring slots
     constexpr int kRows = PAIR ? 4 * BM : 2 * BM;  // query rows per work unit
     // ---- the work unit: (sequence/head, query block of kRows rows) ---------
@@ -349,17 +341,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm.q_full[t], 1);
             mbar_init(&sm.s_full[t], 1);
-            mbar_init(&sm.p_full[t], PAIR ? 8 : BM);  // pair: one arrival per softmax warp
+            // one arrival per softmax warp (of both CTAs, for a pair), or per thread
+            mbar_init(&sm.p_full[t], PAIR ? 8 : (WARP_ARRIVE ? 4 : BM));
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
         }
         mbar_init(&sm.vfix, 1);
-        mbar_init(&sm.q_rot, BM);
         for (int s = 0; s < R; ++s) {
             mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.kv_empty[s], DUAL ? 2 : 1);  // a release per MMA thread
         }
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain2, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -381,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = sm.tmem_base;
 
     if (wg == 3) {
-        regs_dec<56>();
+        regs_dec<kRegsIssue>();
         if (warp == 13) {
             // ================= TMA producer =================
             // paged: sequence b's pages start at entry sum_{b'<b} ceil(ctx_b'/256)
@@ -510,8 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait(&sm.kv_empty[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, abort, wlim);
             }
             }  // lane 0
-        } else if (warp == 12 && lane == 0 && crank == 0) {
-            // ================= MMA issuer =================
+        } else if ((warp == 12 || (DUAL && warp == 14)) && lane == 0 && crank == 0) {
+            // ================= MMA issuer(s) =================
+            // One thread issues both tiles' products, or (DUAL) warp 12's
+            // thread tile 0's and warp 14's tile 1's.
+            const int t_lo = DUAL ? (warp == 14 ? 1 : 0) : 0;
+            const int t_hi = DUAL ? t_lo + 1 : 2;
             // The tensor pipe runs this thread's MMAs in issue order, so
             // S_t(j+1), which overwrites the TMEM columns holding P_t(j), is
             // issued right behind P_t(j) V_j without waiting: P_t is read first.
@@ -575,17 +572,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return mbar_wait(&sm.kv_full[ring_slot<R>(j, 0)], ring_phase<R>(j, 0), err,
                                  FA_DEVERR_TIMEOUT, abort, wlim);
             };
-            if constexpr (ROPE) {
-                ok = mbar_wait(&sm.q_rot, 0, err, FA_DEVERR_TIMEOUT, abort, wlim);
-            } else {
-                for (int t = 0; t < 2 && ok; ++t)
-                    if (n_t[t] > 0)
-                        ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort, wlim);
-            }
+            for (int t = t_lo; t < t_hi && ok; ++t)
+                if (n_t[t] > 0)
+                    ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort, wlim);
             ok = ok && wait_k(0);
             if (ok) {
                 tc_fence_after();
-                for (int t = 0; t < 2; ++t) {
+                for (int t = t_lo; t < t_hi; ++t) {
                     if (n_t[t] > 0) {
                         issue_s(t, 0);
                         commit(&sm.s_full[t]);
@@ -593,43 +586,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 commit(&sm.kv_empty[ring_slot<R>(0, 0)]);
             }
+            // this thread's last step (DUAL: of its tile); past it, it only
+            // releases the slots the other thread still reads
+            const int n_own = DUAL ? n_t[t_lo] : n;
             for (int j = 0; ok && j < n; ++j) {
-                if (zero_v_tail && j == n - 1) {
-                    if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
-                } else if (!mbar_wait(&sm.kv_full[ring_slot<R>(j, 1)], ring_phase<R>(j, 1), err,
-                                      FA_DEVERR_TIMEOUT, abort, wlim)) {
-                    break;
-                }
                 const bool next_k = j + 1 < n;
-                if (next_k && !wait_k(j + 1)) break;
-                for (int t = 0; t < 2; ++t) {
-                    if (j >= n_t[t]) continue;
-                    // a pair's P comes from both CTAs' softmax warps
-                    if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort, wlim)) {
-                        ok = false;
+                if (j < n_own) {
+                    if (zero_v_tail && j == n - 1) {
+                        if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
+                    } else if (!mbar_wait(&sm.kv_full[ring_slot<R>(j, 1)], ring_phase<R>(j, 1),
+                                          err, FA_DEVERR_TIMEOUT, abort, wlim)) {
                         break;
                     }
-                    tc_fence_after();
-                    issue_pv(t, j);
-                    if (j + 1 == n_t[t]) commit(&sm.pv_done[t]);  // O_t final
-                    if (j + 1 < n_t[t]) {
-                        issue_s(t, j + 1);
-                        commit(&sm.s_full[t]);
+                    if (j + 1 < n_own && !wait_k(j + 1)) break;
+                    for (int t = t_lo; t < t_hi; ++t) {
+                        if (j >= n_t[t]) continue;
+                        // a pair's P comes from both CTAs' softmax warps
+                        if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort,
+                                             wlim)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_pv(t, j);
+                        if (j + 1 == n_t[t]) commit(&sm.pv_done[t]);  // O_t final
+                        if (j + 1 < n_t[t]) {
+                            issue_s(t, j + 1);
+                            commit(&sm.s_full[t]);
+                        }
                     }
+                    if (!ok) break;
                 }
-                if (!ok) break;
                 commit(&sm.kv_empty[ring_slot<R>(j, 1)]);
                 if (next_k) commit(&sm.kv_empty[ring_slot<R>(j + 1, 0)]);
             }
             // every MMA this thread issued must be complete before TMEM is freed
-            if constexpr (PAIR) tc_commit_pair(smem_u32(&sm.drain));
-            else tc_commit(&sm.drain);
-            mbar_wait(&sm.drain, 0, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
+            uint64_t* drain = (DUAL && warp == 14) ? &sm.drain2 : &sm.drain;
+            if constexpr (PAIR) tc_commit_pair(smem_u32(drain));
+            else tc_commit(drain);
+            mbar_wait(drain, 0, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
         }
         __syncwarp();
     } else if (wg < 2) {
         // ================= softmax of tile t (warpgroups 0 and 1) =================
-        regs_inc<192>();
+        regs_inc<kRegsSoftmax>();
         const int t = wg;
         const int r = threadIdx.x - t * BM;          // row within the tile == TMEM lane
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
@@ -661,6 +661,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             // row sum above kLazySum anywhere in the warp (or on the first
             // step), pass 2 reloads the scores and uses the true row max.
             for (int pass = (j == 0) ? 1 : 0; pass < 2; ++pass) {
+                if constexpr (kSplitLoad) {
+                    if (pass == 0) {
+                        // first half, then the second half's load overlaps
+                        // the first half's exponentials
+                        uint32_t (&h0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+                        uint32_t (&h1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
+                        uint32_t (&h2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
+                        uint32_t (&h3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
+                        tmem_ld32(s_addr, h0);
+                        tmem_ld32(s_addr + 32, h1);
+                        tmem_wait_ld_regs(h0);
+                        tmem_wait_ld_regs(h1);
+                        tmem_ld32(s_addr + 64, h2);
+                        tmem_ld32(s_addr + 96, h3);
+                        uint64_t acc[4] = {0, 0, 0, 0};
+                        if (need_mask) {
+                            const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
+#pragma unroll
+                            for (int c = 0; c < BN / 2; ++c) s[c] = (c < lim) ? s[c] : fill;
+                            exp_range<true, 0, BN / 2>(s, pk, acc, sl2, m_used, lim);
+                        } else {
+                            exp_range<false, 0, BN / 2>(s, pk, acc, sl2, m_used, BN);
+                        }
+                        tmem_wait_ld_regs(h2);
+                        tmem_wait_ld_regs(h3);
+                        if (need_mask) {
+                            const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
+#pragma unroll
+                            for (int c = BN / 2; c < BN; ++c) s[c] = (c < lim) ? s[c] : fill;
+                            exp_range<true, BN / 2, BN>(s, pk, acc, sl2, m_used, lim);
+                        } else {
+                            exp_range<false, BN / 2, BN>(s, pk, acc, sl2, m_used, BN);
+                        }
+                        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+                        rs = f2_lo(a2) + f2_hi(a2);
+                        if (!__any_sync(0xffffffffu, !(rs <= kLazySum))) break;
+                        continue;
+                    }
+                }
 #pragma unroll
                 for (int c = 0; c < BN / 32; ++c)
                     tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
@@ -715,6 +754,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (crank == 0) mbar_arrive(&sm.p_full[t]);
                     else mbar_arrive_cluster(mapa_rank(smem_u32(&sm.p_full[t]), 0));
                 }
+            } else if constexpr (WARP_ARRIVE) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.p_full[t]);
             } else {
                 mbar_arrive(&sm.p_full[t]);
             }
@@ -726,25 +768,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================= epilogue (warpgroup 2) =================
-        regs_dec<72>();
+        regs_dec<kRegsEpilogue>();
         const int r = threadIdx.x - 2 * BM;
         const uint32_t lane_off = ((warp & 3) * 32u) << 16;
         bool ok = true;
-        if constexpr (ROPE) {
-            // rotate both Q tiles; rows past the sequence end are TMA zero
-            // fill and stay zero
-            for (int t = 0; ok && t < 2; ++t) {
-                if (n_t[t] == 0) continue;
-                if (!warp_wait(&sm.q_full[t], 0, err, abort, wlim)) {
-                    ok = false;
-                    break;
-                }
-                const int pos = tile_row(t) + r;
-                if (pos < len) rope_row<D>(sm.q[t], r, pos, p.rope_cos, p.rope_sin);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            if (ok) mbar_arrive(&sm.q_rot);
-        }
         // epilogue: O / l -> bf16, log-sum-exp
         for (int t = 0; ok && t < 2; ++t) {
             if (n_t[t] == 0) continue;
@@ -809,24 +836,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Rotary embedding of whole rows in device memory (used for K, whose tiles
-// every query block of a head would otherwise rotate again): x [rows, N, D]
-// -> y, row n at position n, the same fp32 formula and bf16 rounding as
-// rope_row.  One thread per (row, 8 pairs).
+// Rotary position embedding of whole rows in device memory, applied once per
+// position before the attention (the page "“Flash”不是那个被时代淘汰的插件"
+// (0539edu.com): the kernel fuses RoPE, section 2, from a precomputed sin/cos
+// lookup table, section 3): rows x0 [rows0, N, D] -> y0 and x1 [rows1, N, D]
+// -> y1 in one launch, row n at position n.  Pairs (i, i + D/2) are turned by
+// the angle whose cosine and sine are cos_t[pos*(D/2) + i], sin_t[...]:
+// x_i cos - x_{i+D/2} sin and x_{i+D/2} cos + x_i sin, every product and sum
+// rounded to fp32 (no fused multiply-add: a fixed, reproducible order), then
+// rounded to bf16 for the tensor cores.  One thread per (row, 8 pairs).
 template <int D>
 __global__ void __launch_bounds__(256)
-    fa_rope_rows_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
-                        const float* __restrict__ cos_t, const float* __restrict__ sin_t,
-                        int64_t rows, int N) {
+    fa_rope_rows_kernel(const __nv_bfloat16* __restrict__ x0, __nv_bfloat16* __restrict__ y0,
+                        int64_t rows0, const __nv_bfloat16* __restrict__ x1,
+                        __nv_bfloat16* __restrict__ y1, int64_t rows1,
+                        const float* __restrict__ cos_t, const float* __restrict__ sin_t, int N) {
     constexpr int HALF = D / 2, G = HALF / 8;  // 8-pair groups per row
-    const int64_t total = rows * N * G;
-    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < total;
-         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n0 = rows0 * N * G;
+    const int64_t total = n0 + rows1 * N * G;
+    for (int64_t wi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; wi < total;
+         wi += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const bool second = wi >= n0;
+        const int64_t w = second ? wi - n0 : wi;
         const int g = static_cast<int>(w % G);
         const int64_t rn = w / G;  // flat (row, position)
         const int pos = static_cast<int>(rn % N);
-        const __nv_bfloat16* src = x + rn * D;
-        __nv_bfloat16* dst = y + rn * D;
+        const __nv_bfloat16* src = (second ? x1 : x0) + rn * D;
+        __nv_bfloat16* dst = (second ? y1 : y0) + rn * D;
         const uint4 ua = *reinterpret_cast<const uint4*>(src + 8 * g);
         const uint4 ub = *reinterpret_cast<const uint4*>(src + 8 * g + HALF);
         const float* ct = cos_t + static_cast<int64_t>(pos) * HALF + 8 * g;
@@ -847,8 +883,6 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const float cc = cs[2 * e + k], ss = sn[2 * e + k];
-                // each product rounded to fp32, then the difference / sum
-                // (no fused multiply-add: a fixed, reproducible order)
                 ra[k] = __fsub_rn(__fmul_rn(a[k], cc), __fmul_rn(b[k], ss));
                 rb[k] = __fadd_rn(__fmul_rn(b[k], cc), __fmul_rn(a[k], ss));
             }
@@ -860,14 +894,14 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <int D, int MODE, bool ROPE = false, bool PAIR = false>
+template <int D, int MODE, bool PAIR = false>
 int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, cudaStream_t stream) {
     // Every CTA allocates all 512 TMEM columns, so one CTA per SM: ask for
     // enough shared memory that a second CTA cannot be co-resident.
     constexpr size_t kSmemUse = sizeof(FwdSmem<D, PAIR>) + 1024;
     const size_t smem = kSmemUse > 120 * 1024 ? kSmemUse : 120 * 1024;
-    auto kern = fa_fwd_kernel<D, MODE, ROPE, PAIR>;
+    auto kern = fa_fwd_kernel<D, MODE, PAIR>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -902,16 +936,18 @@ int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk
 
 }  // namespace
 
-int launch_rope_rows(const void* x, void* y, const float* cos_t, const float* sin_t, int64_t rows,
-                     int N, int d, int num_sms, cudaStream_t stream) {
+int launch_rope_rows(const void* x0, void* y0, int64_t rows0, const void* x1, void* y1,
+                     int64_t rows1, const float* cos_t, const float* sin_t, int N, int d,
+                     int num_sms, cudaStream_t stream) {
+    using T = __nv_bfloat16;
     if (d == 128)
         fa_rope_rows_kernel<128><<<num_sms * 8, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), cos_t, sin_t,
-            rows, N);
+            static_cast<const T*>(x0), static_cast<T*>(y0), rows0, static_cast<const T*>(x1),
+            static_cast<T*>(y1), rows1, cos_t, sin_t, N);
     else if (d == 64)
         fa_rope_rows_kernel<64><<<num_sms * 8, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), cos_t, sin_t,
-            rows, N);
+            static_cast<const T*>(x0), static_cast<T*>(y0), rows0, static_cast<const T*>(x1),
+            static_cast<T*>(y1), rows1, cos_t, sin_t, N);
     else
         return FA_ERR_UNSUPPORTED;
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -922,12 +958,9 @@ int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     switch (mode) {
         case kFixedPair:
-            if (d != 128 || p.rope_cos) return FA_ERR_UNSUPPORTED;
-            return launch_impl<128, kFixed, false, true>(p, tq, tk, tv, stream);
+            if (d != 128) return FA_ERR_UNSUPPORTED;
+            return launch_impl<128, kFixed, true>(p, tq, tk, tv, stream);
         case kFixed:
-            if (p.rope_cos)
-                return d == 128 ? launch_impl<128, kFixed, true>(p, tq, tk, tv, stream)
-                                : launch_impl<64, kFixed, true>(p, tq, tk, tv, stream);
             return d == 128 ? launch_impl<128, kFixed>(p, tq, tk, tv, stream)
                             : launch_impl<64, kFixed>(p, tq, tk, tv, stream);
         case kVarlen:

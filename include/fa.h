@@ -121,10 +121,11 @@ FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, floa
  * kernel: the page "“Flash”不是那个被时代淘汰的插件" (0539edu.com) describes a
  * kernel that fuses RoPE (section 2) from a precomputed sin/cos lookup table
  * (section 3).  q and k are passed unrotated.  The page applies RoPE with the
- * QKV projection; here K, which every query block of a head reads, is rotated
- * once per position into the library workspace of the call's stream
- * (B*H_kv*N*d*2 bytes, grown on demand), and each Q tile is rotated in on-chip memory
- * after it is loaded, before its first score product.
+ * QKV projection, once per position; here one row-kernel launch rotates Q and
+ * K once per position into the library workspace of the call's stream
+ * ((B*H + B*H_kv)*N*d*2 bytes, grown on demand), and the forward kernel reads
+ * the rotated copies (every query block of a head reads K, so rotating tiles
+ * inside the forward kernel would repeat K's rotation once per block).
  *   rope_cos, rope_sin : DEVICE fp32 [max_pos, d/2], row-major; entry (p, i)
  *                        is cos / sin of the angle for position p and pair i
  *                        (normally p * base^(-2i/d)); max_pos >= N

@@ -1,6 +1,6 @@
 """fa_decode_paged_noalloc: paged decode for callers that cannot allocate
-device memory (graph capture, pre-reserved serving memory, foreign
-allocators).  Called straight through the C ABI and checked against the
+device memory (serving loops with all memory reserved up front, host programs
+whose own allocator forbids other allocations).  Called straight through the C ABI and checked against the
 allocating fa_decode_paged on the same inputs, twice in a row, within the
 tolerances the parity tests use.
 
@@ -66,6 +66,16 @@ def test_noalloc_matches_allocating_decode_twice_in_a_row():
     assert _noalloc_raw(c, o_again) == fa.FA_OK
     assert fa.fa_get_device_error() == fa.FA_OK
     assert torch.equal(o_again, results[0])
+    # through the Python wrapper, into a preallocated output, on a side stream
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    o_side = torch.full_like(c.q, float("nan"))
+    got = fa.fa_decode_paged_noalloc(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS,
+                                     o=o_side, stream=side)
+    assert got is o_side
+    assert fa.fa_get_device_error(stream=side) == fa.FA_OK
+    torch.cuda.current_stream().wait_stream(side)
+    assert torch.equal(o_side, results[0])
     # and against the fp64 oracle directly
     o64, _ = oracle.decode_paged(small.q, small.k_pages, small.v_pages, small.page_table,
                                  small.seq_lens, PS)
