@@ -67,15 +67,6 @@ constexpr float kLazySum = 65536.f;
 // Exponentials of pairs (c/2) % 8 in [0, kPolyPairs) are evaluated with the
 // FMA-pipe polynomial below, the rest with the special-function unit.
 constexpr int kPolyPairs = 0;
-// Single CTA: each tile's products issued by a thread of its own (warps 12
-// and 14), so that one tile's P V and next S do not wait behind the other
-// tile's issue.
-constexpr bool kDualIssue = false;
-// The softmax loads the two halves of a score row separately and starts the
-// exponentials of the first half while the second is still on its way.
-constexpr bool kSplitLoad = false;
-// The softmax signals P_t ready once per warp instead of once per thread.
-constexpr bool kWarpArrive = false;
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by
 // the Remez exchange in exp2_poly_remez.py beside this file.
 constexpr float kExp2P0 = 0.9999280571937561f, kExp2P1 = 0.6932609677314758f,
@@ -99,7 +90,7 @@ struct alignas(1024) FwdSmem {
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[2], p_full[2], pv_done[2], stats_full[2];
     uint64_t vfix;   // paged: the last V tile's rows past the sequence are zeroed
-    uint64_t drain, drain2;
+    uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -199,35 +190,6 @@ __device__ __forceinline__ float exp_pairs(const uint32_t (&s)[BN], uint32_t (&p
     return f2_lo(a2) + f2_hi(a2);
 }
 
-// exp_pairs over the columns [C0, C1) only, adding the pairs' p into the four
-// packed accumulators acc (the caller sums them).
-template <bool MASKED, int C0, int C1>
-__device__ __forceinline__ void exp_range(const uint32_t (&s)[BN], uint32_t (&pk)[BN / 2],
-                                          uint64_t (&acc)[4], uint64_t sl2, float m, int lim) {
-    const float mb = (m == -INFINITY) ? 0.f : m;
-    const uint64_t nm2 = f2_pack(-mb, -mb);
-#pragma unroll
-    for (int c = C0; c < C1; c += 2) {
-        const uint64_t x =
-            f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, nm2);
-        float p0, p1;
-        if ((c / 2) % 8 < kPolyPairs) {
-            const uint64_t e = exp2_poly2(x);
-            p0 = f2_lo(e);
-            p1 = f2_hi(e);
-        } else {
-            p0 = ex2_approx(f2_lo(x));
-            p1 = ex2_approx(f2_hi(x));
-        }
-        if constexpr (MASKED) {
-            p0 = (c < lim) ? p0 : 0.f;
-            p1 = (c + 1 < lim) ? p1 : 0.f;
-        }
-        acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], f2_pack(p0, p1));
-        pk[c / 2] = pack_bf16x2(p0, p1);
-    }
-}
-
 // MODE: kFixed ([B,H,N,d] tensors), kVarlen (packed [total,H,d] sequences),
 // kPaged (packed queries; keys and values read through the page table from a
 // pool of 256-token pages, the queries being the last positions of each
@@ -247,8 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool VARLEN = MODE != kFixed;  // packed query rows
     constexpr bool PAGED = MODE == kPaged;
     static_assert(!PAIR || (D == 128 && MODE == kFixed), "pair mode: fixed length, d=128");
-    constexpr bool DUAL = kDualIssue && !PAIR;      // one MMA thread per tile
-    constexpr bool WARP_ARRIVE = kWarpArrive || PAIR;
     constexpr int R = ring_slots<PAIR>();          // K/V ring slots
     constexpr int kRows = PAIR ? 4 * BM : 2 * BM;  // query rows per work unit
     // ---- the work unit: (sequence/head, query block of kRows rows) ---------
@@ -341,18 +301,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm.q_full[t], 1);
             mbar_init(&sm.s_full[t], 1);
-            // one arrival per softmax warp (of both CTAs, for a pair), or per thread
-            mbar_init(&sm.p_full[t], PAIR ? 8 : (WARP_ARRIVE ? 4 : BM));
+            mbar_init(&sm.p_full[t], PAIR ? 8 : BM);  // pair: one arrival per softmax warp
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.stats_full[t], BM);
         }
         mbar_init(&sm.vfix, 1);
         for (int s = 0; s < R; ++s) {
             mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], DUAL ? 2 : 1);  // a release per MMA thread
+            mbar_init(&sm.kv_empty[s], 1);
         }
         mbar_init(&sm.drain, 1);
-        mbar_init(&sm.drain2, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -503,12 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait(&sm.kv_empty[u % R], (u / R) & 1, err, FA_DEVERR_TIMEOUT, abort, wlim);
             }
             }  // lane 0
-        } else if ((warp == 12 || (DUAL && warp == 14)) && lane == 0 && crank == 0) {
-            // ================= MMA issuer(s) =================
-            // One thread issues both tiles' products, or (DUAL) warp 12's
-            // thread tile 0's and warp 14's tile 1's.
-            const int t_lo = DUAL ? (warp == 14 ? 1 : 0) : 0;
-            const int t_hi = DUAL ? t_lo + 1 : 2;
+        } else if (warp == 12 && lane == 0 && crank == 0) {
+            // ================= MMA issuer =================
             // The tensor pipe runs this thread's MMAs in issue order, so
             // S_t(j+1), which overwrites the TMEM columns holding P_t(j), is
             // issued right behind P_t(j) V_j without waiting: P_t is read first.
@@ -572,13 +526,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return mbar_wait(&sm.kv_full[ring_slot<R>(j, 0)], ring_phase<R>(j, 0), err,
                                  FA_DEVERR_TIMEOUT, abort, wlim);
             };
-            for (int t = t_lo; t < t_hi && ok; ++t)
+            for (int t = 0; t < 2 && ok; ++t)
                 if (n_t[t] > 0)
                     ok = mbar_wait(&sm.q_full[t], 0, err, FA_DEVERR_TIMEOUT, abort, wlim);
             ok = ok && wait_k(0);
             if (ok) {
                 tc_fence_after();
-                for (int t = t_lo; t < t_hi; ++t) {
+                for (int t = 0; t < 2; ++t) {
                     if (n_t[t] > 0) {
                         issue_s(t, 0);
                         commit(&sm.s_full[t]);
@@ -586,45 +540,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 commit(&sm.kv_empty[ring_slot<R>(0, 0)]);
             }
-            // this thread's last step (DUAL: of its tile); past it, it only
-            // releases the slots the other thread still reads
-            const int n_own = DUAL ? n_t[t_lo] : n;
             for (int j = 0; ok && j < n; ++j) {
+                if (zero_v_tail && j == n - 1) {
+                    if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
+                } else if (!mbar_wait(&sm.kv_full[ring_slot<R>(j, 1)], ring_phase<R>(j, 1), err,
+                                      FA_DEVERR_TIMEOUT, abort, wlim)) {
+                    break;
+                }
                 const bool next_k = j + 1 < n;
-                if (j < n_own) {
-                    if (zero_v_tail && j == n - 1) {
-                        if (!mbar_wait(&sm.vfix, 0, err, FA_DEVERR_TIMEOUT, abort, wlim)) break;
-                    } else if (!mbar_wait(&sm.kv_full[ring_slot<R>(j, 1)], ring_phase<R>(j, 1),
-                                          err, FA_DEVERR_TIMEOUT, abort, wlim)) {
+                if (next_k && !wait_k(j + 1)) break;
+                for (int t = 0; t < 2; ++t) {
+                    if (j >= n_t[t]) continue;
+                    // a pair's P comes from both CTAs' softmax warps
+                    if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort, wlim)) {
+                        ok = false;
                         break;
                     }
-                    if (j + 1 < n_own && !wait_k(j + 1)) break;
-                    for (int t = t_lo; t < t_hi; ++t) {
-                        if (j >= n_t[t]) continue;
-                        // a pair's P comes from both CTAs' softmax warps
-                        if (!mbar_wait<PAIR>(&sm.p_full[t], j & 1, err, FA_DEVERR_TIMEOUT, abort,
-                                             wlim)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        issue_pv(t, j);
-                        if (j + 1 == n_t[t]) commit(&sm.pv_done[t]);  // O_t final
-                        if (j + 1 < n_t[t]) {
-                            issue_s(t, j + 1);
-                            commit(&sm.s_full[t]);
-                        }
+                    tc_fence_after();
+                    issue_pv(t, j);
+                    if (j + 1 == n_t[t]) commit(&sm.pv_done[t]);  // O_t final
+                    if (j + 1 < n_t[t]) {
+                        issue_s(t, j + 1);
+                        commit(&sm.s_full[t]);
                     }
-                    if (!ok) break;
                 }
+                if (!ok) break;
                 commit(&sm.kv_empty[ring_slot<R>(j, 1)]);
                 if (next_k) commit(&sm.kv_empty[ring_slot<R>(j + 1, 0)]);
             }
             // every MMA this thread issued must be complete before TMEM is freed
-            uint64_t* drain = (DUAL && warp == 14) ? &sm.drain2 : &sm.drain;
-            if constexpr (PAIR) tc_commit_pair(smem_u32(drain));
-            else tc_commit(drain);
-            mbar_wait(drain, 0, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
+            if constexpr (PAIR) tc_commit_pair(smem_u32(&sm.drain));
+            else tc_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0, err, FA_DEVERR_TIMEOUT, nullptr, wlim);
         }
         __syncwarp();
     } else if (wg < 2) {
@@ -661,45 +608,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             // row sum above kLazySum anywhere in the warp (or on the first
             // step), pass 2 reloads the scores and uses the true row max.
             for (int pass = (j == 0) ? 1 : 0; pass < 2; ++pass) {
-                if constexpr (kSplitLoad) {
-                    if (pass == 0) {
-                        // first half, then the second half's load overlaps
-                        // the first half's exponentials
-                        uint32_t (&h0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-                        uint32_t (&h1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-                        uint32_t (&h2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-                        uint32_t (&h3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-                        tmem_ld32(s_addr, h0);
-                        tmem_ld32(s_addr + 32, h1);
-                        tmem_wait_ld_regs(h0);
-                        tmem_wait_ld_regs(h1);
-                        tmem_ld32(s_addr + 64, h2);
-                        tmem_ld32(s_addr + 96, h3);
-                        uint64_t acc[4] = {0, 0, 0, 0};
-                        if (need_mask) {
-                            const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
-#pragma unroll
-                            for (int c = 0; c < BN / 2; ++c) s[c] = (c < lim) ? s[c] : fill;
-                            exp_range<true, 0, BN / 2>(s, pk, acc, sl2, m_used, lim);
-                        } else {
-                            exp_range<false, 0, BN / 2>(s, pk, acc, sl2, m_used, BN);
-                        }
-                        tmem_wait_ld_regs(h2);
-                        tmem_wait_ld_regs(h3);
-                        if (need_mask) {
-                            const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
-#pragma unroll
-                            for (int c = BN / 2; c < BN; ++c) s[c] = (c < lim) ? s[c] : fill;
-                            exp_range<true, BN / 2, BN>(s, pk, acc, sl2, m_used, lim);
-                        } else {
-                            exp_range<false, BN / 2, BN>(s, pk, acc, sl2, m_used, BN);
-                        }
-                        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-                        rs = f2_lo(a2) + f2_hi(a2);
-                        if (!__any_sync(0xffffffffu, !(rs <= kLazySum))) break;
-                        continue;
-                    }
-                }
 #pragma unroll
                 for (int c = 0; c < BN / 32; ++c)
                     tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
@@ -754,9 +662,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (crank == 0) mbar_arrive(&sm.p_full[t]);
                     else mbar_arrive_cluster(mapa_rank(smem_u32(&sm.p_full[t]), 0));
                 }
-            } else if constexpr (WARP_ARRIVE) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.p_full[t]);
             } else {
                 mbar_arrive(&sm.p_full[t]);
             }
