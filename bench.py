@@ -82,17 +82,26 @@ def load_peaks():
         return d
 
 
-def tensor_peak_regime(peaks, sm_mhz, region_ms):
+def tensor_peak_regime(peaks, clocks, region_ms):
     """Which measured GEMM peak a forward timing is compared with.
 
     The pool's cuBLAS figures were taken in two regimes: a burst at the full
-    SM clock (bf16_tflops) and a seconds-long loop that settles at the power
-    cap with the clock near `sustained_sm_mhz` (bf16_tflops_sustained).  The
-    timed region is put in the regime its own sampled median SM clock is
-    closer to; without clock samples, by its length (under 2 s: burst).
-    Returns (regime, peak TFLOP/s, reason)."""
+    SM clock (bf16_tflops) and a seconds-long loop held at the 1000 W power
+    cap (bf16_tflops_sustained).  A timed region during which the power cap
+    was active (sw_power_cap among the reasons sampled inside it) is in the
+    sustained regime, one without it in the burst regime.  Without a reason
+    list, the median SM clock decides (nearer the burst GEMM's full clock or
+    the sustained GEMM's median); without clock samples, the region's length
+    (under 2 s: burst).  Returns (regime, peak TFLOP/s, reason)."""
     hi, lo = peaks["sm_max_mhz"], peaks["sustained_sm_mhz"]
-    if sm_mhz is not None:
+    clocks = clocks or {}
+    sm_mhz = clocks.get("sm_mhz")
+    reasons = clocks.get("reasons")
+    if sm_mhz is not None and isinstance(reasons, list):
+        burst = "sw_power_cap" not in reasons
+        why = (f"power cap {'not ' if burst else ''}active during the timed region "
+               f"(median SM clock {sm_mhz:.0f} MHz)")
+    elif sm_mhz is not None:
         burst = sm_mhz >= 0.5 * (hi + lo)
         why = (f"median SM clock {sm_mhz:.0f} MHz during the timed region, against "
                f"{hi:.0f} (burst GEMM) and {lo:.0f} (sustained GEMM)")
@@ -786,7 +795,7 @@ def run_native(args, world, rank, local):
     dec_sha = kernel_source_sha(["decode_sm100.cu", "fa_ptx.cuh", "fa_internal.h"])
     # the forward's tensor peak is the measured GEMM figure of the regime the
     # timed region ran in (burst at full clock, or sustained at the power cap)
-    regime, peak_tf, regime_why = tensor_peak_regime(peaks, clocks.get("sm_mhz"), total_ms)
+    regime, peak_tf, regime_why = tensor_peak_regime(peaks, clocks, total_ms)
     out = {
         "metric": METRIC,
         "value": fwd_tflops if do_fwd else dec_gbs,

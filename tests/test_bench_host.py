@@ -7,24 +7,27 @@ PEAKS = {"hbm_gbs": 6537.3, "bf16_tflops": 1647.8, "bf16_tflops_sustained": 1379
          "sm_max_mhz": 1965.0, "sustained_sm_mhz": 1252.0, "source": "measured"}
 
 
-def test_full_clock_region_takes_the_burst_peak():
-    regime, peak, why = bench.tensor_peak_regime(PEAKS, 1965.0, 87.0)
-    assert regime == "burst" and peak == 1647.8 and "1965" in why
+def test_region_without_power_cap_takes_the_burst_peak():
+    clocks = {"sm_mhz": 1965.0, "reasons": []}
+    regime, peak, why = bench.tensor_peak_regime(PEAKS, clocks, 87.0)
+    assert regime == "burst" and peak == 1647.8 and "not active" in why
     # 1250 TF/s in that regime is 0.76 of the measured burst GEMM
     assert abs(1250.0 / peak - 0.7586) < 1e-3
 
 
 def test_power_capped_region_takes_the_sustained_peak():
-    regime, peak, _ = bench.tensor_peak_regime(PEAKS, 1300.0, 5000.0)
+    # the forward pass at the cap keeps a higher clock than a GEMM at the cap:
+    # the cap, not the clock, names the regime
+    clocks = {"sm_mhz": 1661.0, "reasons": ["sw_power_cap"]}
+    regime, peak, _ = bench.tensor_peak_regime(PEAKS, clocks, 945.0)
     assert regime == "sustained" and peak == 1379.4
-    # the midpoint between the two regimes' clocks decides
-    assert bench.tensor_peak_regime(PEAKS, 1609.0, 900.0)[0] == "burst"
-    assert bench.tensor_peak_regime(PEAKS, 1600.0, 900.0)[0] == "sustained"
 
 
-def test_without_clock_samples_the_region_length_decides():
-    assert bench.tensor_peak_regime(PEAKS, None, 500.0)[0] == "burst"
-    assert bench.tensor_peak_regime(PEAKS, None, 4000.0)[0] == "sustained"
+def test_without_reasons_the_clock_decides_and_without_clocks_the_length():
+    assert bench.tensor_peak_regime(PEAKS, {"sm_mhz": 1609.0}, 900.0)[0] == "burst"
+    assert bench.tensor_peak_regime(PEAKS, {"sm_mhz": 1600.0}, 900.0)[0] == "sustained"
+    assert bench.tensor_peak_regime(PEAKS, {"sm_mhz": None}, 500.0)[0] == "burst"
+    assert bench.tensor_peak_regime(PEAKS, {}, 4000.0)[0] == "sustained"
 
 
 def _line(sm, reason_cap="Not Active"):
