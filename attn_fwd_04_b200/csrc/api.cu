@@ -514,8 +514,10 @@ int decode_impl(const void* q, const void* k_pages, const void* v_pages,
         if ((rc = make_map(&tv, v_pages, dims, strides, box)) != FA_OK) return rc;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const size_t dec_bytes =
-        (fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits) + 255) & ~static_cast<size_t>(255);
+    const size_t need = grouped ? fa::decode_gqa_workspace_bytes(B, H, H_kv, d,
+                                                                 fa::kDecodeMaxSplits, s->num_sms)
+                                : fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits);
+    const size_t dec_bytes = (need + 255) & ~static_cast<size_t>(255);
     // block table: the packed table and the cut lengths follow the decode's own workspace
     const size_t pack_bytes =
         max_pages > 0 ? (static_cast<size_t>(B) * max_pages + B) * sizeof(int32_t) : 0;
@@ -534,7 +536,8 @@ int decode_impl(const void* q, const void* k_pages, const void* v_pages,
     }
     return fa::launch_decode(q, k_pages, v_pages, grouped ? &tk : nullptr,
                              grouped ? &tv : nullptr, table, lens, o, B, H, H_kv, num_pages, d,
-                             page_size, fa::kDecodeMaxSplits, ws, s->err, s->num_sms, st);
+                             page_size, fa::kDecodeMaxSplits, ws, dec_bytes, s->err, s->num_sms,
+                             st);
 }
 }  // namespace
 

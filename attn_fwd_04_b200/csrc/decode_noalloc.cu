@@ -82,8 +82,8 @@ FA_API int fa_decode_paged_noalloc(const void* q, const void* k_pages, const voi
     if ((rc = fa::device_error_word(&err, &num_sms)) != FA_OK) return rc;
     // the signature carries no pool size: page indices are not bounded
     return fa::launch_decode(q, k_pages, v_pages, nullptr, nullptr, page_table, seq_lens, o, B, H,
-                             H, 0x7fffffff, d, page_size, splits, scratch, err, num_sms,
-                             reinterpret_cast<cudaStream_t>(stream));
+                             H, 0x7fffffff, d, page_size, splits, scratch, kScratchBytes, err,
+                             num_sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

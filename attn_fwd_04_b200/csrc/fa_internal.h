@@ -62,7 +62,9 @@ int launch_bwd(const void* o, const void* dout, const float* lse, void* dq, void
 // fastest on the paged-decode workload for 32 and 8 K/V heads (2: 2-3 %
 // slower, more partials and per-unit combines; 8: a longer tail).  With fewer
 // units per split the launch is short and 6 pages measured faster (4 K/V
-// heads: 6486-6518 GB/s against 6253-6296 with 4 pages).
+// heads: 6486-6518 GB/s against 6253-6296 with 4 pages; 8 pages 1 % slower).
+// The grouped decode with one or two units per split does not cut splits:
+// it divides the chunk stream evenly over the CTAs.
 constexpr int kDecodeChunkPages = 4;
 constexpr int kDecodeChunkPagesFew = 6;
 constexpr int kDecodeManyUnits = 8;
@@ -75,17 +77,21 @@ struct DecodePlan {
 };
 
 size_t decode_workspace_bytes(int B, int H, int d, int max_splits);
+// the grouped decode's workspace (H > Hk): a balanced partition over
+// num_sms CTAs for few unit heads, split units otherwise
+size_t decode_gqa_workspace_bytes(int B, int H, int Hk, int d, int max_splits, int num_sms);
 
 // H query heads over Hk K/V heads (any H % Hk == 0).  The grouped
 // kernels (H > Hk) read the pool through tk, tv: (d, 256, num_pages * Hk)
-// maps with 64 x 64 x 1 boxes and 128-byte swizzle; H == Hk reads it with
-// bulk copies and takes no maps (may be null).  Page indices outside
-// [0, num_pages) are reported.
+// maps with 64 x 64 x 1 boxes and 128-byte swizzle and need
+// decode_gqa_workspace_bytes of workspace (workspace_bytes is checked); H == Hk reads it with bulk copies, takes no
+// maps (may be null) and needs decode_workspace_bytes(B, H, d, max_splits).
+// Page indices outside [0, num_pages) are reported.
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
                   const int32_t* seq_lens, void* o, int B, int H, int Hk, int num_pages, int d,
-                  int page_size, int max_splits, void* workspace, unsigned int* err, int num_sms,
-                  cudaStream_t stream);
+                  int page_size, int max_splits, void* workspace, size_t workspace_bytes,
+                  unsigned int* err, int num_sms, cudaStream_t stream);
 bool decode_group_supported(int H, int Hk);
 
 // Block table [B, max_pages] -> packed table `packed` (at most B * max_pages

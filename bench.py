@@ -25,6 +25,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -114,10 +115,14 @@ def tensor_peak_regime(peaks, clocks, region_ms):
 
 
 def kernel_source_sha(files):
+    """Hash of the kernel's code: the files with their comments and white
+    space removed, so that a comment edit does not mark a capture stale."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "attn_fwd_04_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "attn_fwd_04_b200", "csrc", f), encoding="utf-8") as fh:
+            code = re.sub(r"/\*.*?\*/", " ", fh.read(), flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 
@@ -494,20 +499,22 @@ def secondary_workloads(fa, stream, steps: int = 5, warmup: int = 3):
                                    1 / math.sqrt(wv.d), dq=dq, dk=dk, dv=dv, stream=stream),
           2.5 * vflops, f"bwd_{wv.name}")
     del q, k, v, cu, cud, o, lse, g, dq, dk, dv
-    # grouped-query paged decode: the decode workload's lengths, 8 K/V heads
+    # grouped-query paged decode: the decode workload's lengths with 8, 2 and
+    # 1 K/V heads (the last two: the evenly split chunk stream)
     lengths = W.varlen_lengths(DEC.B, DEC.len_lo, DEC.len_hi, DEC.seed)
-    c = W.paged_inputs(DEC.B, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda",
-                       H_kv=GQA_HKV)
-    pt, sl = c.page_table.cuda(), c.seq_lens.cuda()
-    do = torch.empty_like(c.q)
-    nbytes = decode_bytes(lengths, DEC.H, DEC.d, DEC.B, H_kv=GQA_HKV)
-    name = f"gqa_paged_decode_b64_h32_hkv{GQA_HKV}_d128_len1024to32768_page256"
-    timed(lambda: fa.fa_decode_paged_gqa(c.q, c.k_pages, c.v_pages, pt, sl, DEC.page_size,
-                                         o=do, stream=stream), 0.0, name)
-    ms = out[name]["ms_per_launch"]
-    out[name] = {"ms_per_launch": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
-                 "bytes_per_launch": nbytes}
-    del c, pt, sl, do
+    for h_kv in (GQA_HKV, 2, 1):
+        c = W.paged_inputs(DEC.B, DEC.H, DEC.d, lengths, DEC.seed, DEC.page_size, device="cuda",
+                           H_kv=h_kv)
+        pt, sl = c.page_table.cuda(), c.seq_lens.cuda()
+        do = torch.empty_like(c.q)
+        nbytes = decode_bytes(lengths, DEC.H, DEC.d, DEC.B, H_kv=h_kv)
+        name = f"gqa_paged_decode_b64_h32_hkv{h_kv}_d128_len1024to32768_page256"
+        timed(lambda: fa.fa_decode_paged_gqa(c.q, c.k_pages, c.v_pages, pt, sl, DEC.page_size,
+                                             o=do, stream=stream), 0.0, name)
+        ms = out[name]["ms_per_launch"]
+        out[name] = {"ms_per_launch": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "bytes_per_launch": nbytes}
+        del c, pt, sl, do
     # paged prefill: 1024 new queries per sequence after 1024..8192 cached
     # tokens, K/V read through the page table; FLOPs count every attended
     # (query, key) pair (4*d per pair and head)

@@ -273,7 +273,11 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
  * slices once
  * (FA_ERR_UNSUPPORTED otherwise; FA_ERR_SHAPE if H is not a multiple of
  * H_kv, or num_pages < 1).  Each (page, K/V head) slice is read from device
- * memory once and serves all H / H_kv query heads of its group.  A page
+ * memory once and serves all H / H_kv query heads of its group.  With at
+ * most two work units per sequence (a unit is a group, or a pair of 16-head
+ * sub-groups: multi-query attention) the tokens of all sequences are
+ * divided evenly over the SMs, and the workspace grows with B and the SM
+ * count rather than with the sequence lengths.  A page
  * index outside [0, num_pages) is reported as FA_ERR_DEVICE_BAD_INPUT (see
  * fa_get_device_error); nothing outside the pool is read, and the output of
  * that sequence is unspecified.

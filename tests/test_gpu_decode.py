@@ -223,16 +223,45 @@ def test_decode_gqa_workload_sampled(H_kv):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("H,H_kv", [(8, 4), (8, 2), (16, 2), (16, 1)])
+@pytest.mark.parametrize("H,H_kv", [(8, 4), (8, 2), (16, 2), (16, 1), (32, 1), (40, 2)])
 def test_decode_gqa_chunk_and_warp_edges(d, H, H_kv):
-    """Lengths that end inside, and right at, the 16-token slices the warps own
-    and the 64-token chunks the two warp teams alternate on; the poisoned
+    """Lengths that end inside, and right at, the 16- or 32-token slices the
+    warps own (32 when two sub-groups share a unit: 32 and 40 query heads per
+    K/V head) and the 64-token chunks the crews take in turn; the poisoned
     (NaN) slots past each length must not reach the output."""
-    lens = [15, 16, 17, 48, 49, 64, 65, 127, 128, 129, 191, 320, 513, 767]
+    lens = [15, 16, 17, 31, 32, 33, 48, 49, 64, 65, 97, 127, 128, 129, 191, 320, 513, 767]
     c = W.paged_inputs(len(lens), H, d, lens, seed=90 + H + H_kv + d, device="cpu", H_kv=H_kv)
     o = _decode_gqa(_on_gpu(c))
     o_ref, _ = oracle.decode_paged_gqa(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
     assert_o_close(to64(o), o_ref, f"decode gqa edges d={d} H={H} H_kv={H_kv}")
+
+
+@pytest.mark.parametrize("H,H_kv", [(32, 1), (16, 2)])
+@pytest.mark.parametrize("lens", [[0, 0, 0], [5, 0, 64, 65], [131072], [0, 40000, 1]],
+                         ids=["all-empty", "fewer-chunks-than-ctas", "one-128k-sequence",
+                              "long-between-empty-and-short"])
+def test_decode_gqa_even_split_edges(H, H_kv, lens):
+    """Few unit heads per sequence (one or two) split the chunk stream evenly
+    over the CTAs: no work at all; fewer 64-token chunks than CTAs (only
+    some CTAs take part); one sequence whose chunks span every CTA (its
+    merge combines more than 32 pieces); a long sequence beside an empty and
+    a one-token one."""
+    # the pool must hold a page: with no tokens at all, one sequence's page is
+    # allocated and its length then set to 0
+    alloc = lens if sum(lens) else [1] + lens[1:]
+    c = W.paged_inputs(len(lens), H, 128, alloc, seed=7 + len(lens) + H_kv, device="cpu",
+                       H_kv=H_kv)
+    c = W.PagedCache(c.q, c.k_pages, c.v_pages, c.page_table,
+                     torch.tensor(lens, dtype=torch.int32), c.page_size, c.pages_per_seq)
+    o = _decode_gqa(_on_gpu(c))
+    assert bool(torch.isfinite(o).all())
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(o[b] == 0)
+    if sum(lens) == 0:
+        return
+    o_ref, _ = oracle.decode_paged_gqa(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, PS)
+    assert_o_close(to64(o), o_ref, f"decode gqa even split H={H} H_kv={H_kv} lens={lens}")
 
 
 @pytest.mark.parametrize("H,H_kv", [(8, 2), (4, 4)])
