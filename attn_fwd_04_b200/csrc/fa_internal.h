@@ -30,6 +30,9 @@ struct FwdParams {
     int causal;
     float scale_log2;    // scale * log2(e)
     unsigned int* err;   // device error word
+    // packed sequences: the sequences in the order their CTAs run, heaviest
+    // first (launch_seq_order; paged prefill); null: 0, 1, ..., B-1
+    const int32_t* seq_order;
     // failure-detection check only (fa_selftest_fwd_stall; 0 in every other call):
     uint64_t wait_ns;    // bound of every wait in the kernel (0: FA_WAIT_TIMEOUT_NS)
     int withhold_copy;   // 1 + the K/V ring use whose copy the producer withholds (0: none)
@@ -45,6 +48,13 @@ int launch_rope_rows(const void* x0, void* y0, int64_t rows0, const void* x1, vo
 constexpr int kFixed = 0, kVarlen = 1, kPaged = 2, kFixedPair = 3;
 int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, int d, int mode, cudaStream_t stream);
+// order[0..B) <- the packed sequences sorted by the forward pass's work on
+// them, heaviest first (ties by index): query rows from cu_seqlens, keys from
+// ctx_lens (paged prefill, the queries ending the sequence) or the rows
+// themselves.  Up to kSeqOrderMax sequences (more: leave the order alone).
+constexpr int kSeqOrderMax = 4096;
+int launch_seq_order(const int32_t* cu_seqlens, const int32_t* ctx_lens, int B, int causal,
+                     int32_t* order, cudaStream_t stream);
 
 // ---- backward ------------------------------------------------------------
 size_t bwd_workspace_bytes(int B, int H, int N, int d);

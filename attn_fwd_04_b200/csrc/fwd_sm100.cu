@@ -233,8 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // prefill, whose queries end the sequence; 0 otherwise)
     int len, klen, kshift = 0, seq_start = 0, bh = 0, h = 0, bkv = 0, b = 0;
     if constexpr (VARLEN) {
-        b = unit / p.H;
-        h = unit - b * p.H;
+        const int bi = unit / p.H;  // the bi-th sequence to run, heaviest first
+        b = p.seq_order ? p.seq_order[bi] : bi;
+        h = unit - bi * p.H;
         const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
         // keep every access inside the [total, H, d] tensors whatever the offsets say
         const int c0 = min(max(s0, 0), p.total), c1 = min(max(s1, c0), p.total);
@@ -839,6 +840,40 @@ int launch_impl(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk
     }
 }
 
+// The packed sequences by decreasing work, one CTA: work = attended (query,
+// key) pairs (causal: row i sees kshift + i + 1 keys); rank = how many
+// sequences come before (more work, or as much and a lower index).  The
+// forward pass then starts its heaviest sequences first, and the lighter ones
+// fill the last wave (longest-processing-time-first list scheduling).
+__global__ void __launch_bounds__(1024)
+    fa_seq_order_kernel(const int32_t* __restrict__ cu_seqlens,
+                        const int32_t* __restrict__ ctx_lens, int B, int causal,
+                        int32_t* __restrict__ order) {
+    __shared__ long long work[kSeqOrderMax];
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const long long len = max(0, cu_seqlens[b + 1] - cu_seqlens[b]);
+        const long long klen = ctx_lens ? max(0, ctx_lens[b]) : len;
+        long long w;
+        if (!causal) {
+            w = len * klen;
+        } else {
+            const long long kshift = klen - len;  // < 0 only for bad input (not computed)
+            w = kshift < 0 ? 0 : len * kshift + len * (len + 1) / 2;
+        }
+        work[b] = w;
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const long long w = work[b];
+        int r = 0;
+        for (int j = 0; j < B; ++j) {
+            const long long x = work[j];
+            r += (x > w || (x == w && j < b)) ? 1 : 0;
+        }
+        order[r] = b;
+    }
+}
+
 }  // namespace
 
 int launch_rope_rows(const void* x0, void* y0, int64_t rows0, const void* x1, void* y1,
@@ -876,6 +911,13 @@ int launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                             : launch_impl<64, kPaged>(p, tq, tk, tv, stream);
         default: return FA_ERR_UNSUPPORTED;
     }
+}
+
+int launch_seq_order(const int32_t* cu_seqlens, const int32_t* ctx_lens, int B, int causal,
+                     int32_t* order, cudaStream_t stream) {
+    if (B < 1 || B > kSeqOrderMax) return FA_ERR_SHAPE;
+    fa_seq_order_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, ctx_lens, B, causal, order);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // namespace fa

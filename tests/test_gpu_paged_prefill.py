@@ -81,6 +81,29 @@ def test_prefill_whole_sequences_equal_varlen_bitwise():
     assert torch.equal(o, ov) and torch.equal(lse, lv)
 
 
+def test_prefill_heaviest_first_keeps_each_sequence():
+    """Paged prefill runs its sequences heaviest first (a device-side ranking
+    by attended pairs): a batch whose cached lengths are not in that order,
+    with a tie, gives each sequence bit for bit what a call on that sequence
+    alone gives."""
+    ctx = [700, 3000, 257, 3000, 1200]
+    ql = [128, 64, 257, 64, 300]
+    H, d = 4, 128
+    cache, q, cu = W.prefill_inputs(len(ctx), H, H, d, ctx, ql, seed=313, device="cpu")
+    o, lse = _prefill(cache, q, cu, max(ql), True, 0.1)
+    for b in range(len(ctx)):
+        pages = cache.pages_per_seq
+        p0 = sum(pages[:b])
+        one = W.PagedCache(cache.q, cache.k_pages, cache.v_pages,
+                           cache.page_table[p0:p0 + pages[b]].contiguous(),
+                           cache.seq_lens[b:b + 1].contiguous(), cache.page_size, [pages[b]])
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        cu1 = torch.tensor([0, s1 - s0], dtype=torch.int32)
+        o1, l1 = _prefill(one, q[s0:s1].contiguous(), cu1, s1 - s0, True, 0.1)
+        assert torch.equal(o1, o[s0:s1]), f"sequence {b}"
+        assert torch.equal(l1, lse[:, s0:s1]), f"sequence {b}"
+
+
 def test_prefill_more_queries_than_tokens_reported():
     lens, nq = [100, 50], [10, 60]
     cache, q, cu = W.prefill_inputs(2, 2, 2, 64, lens, [10, 50], seed=312, device="cpu")
