@@ -12,6 +12,6 @@ from .fa import (EXPORTS, FA_ERR_ALIGN, FA_ERR_CUDA, FA_ERR_DEVICE_BAD_INPUT,  #
                  fa_fwd_set_cta_pairs, fa_fwd_varlen_gqa,
                  fa_fwd_varlen,
                  fa_gather_paged, fa_get_device_error, fa_release_workspace, fa_selftest_bounded_wait,
-                 fa_selftest_fwd_stall,
+                 fa_selftest_decode_stall, fa_selftest_fwd_stall,
                  fa_status_str,
                  fa_version, lib)

@@ -674,6 +674,31 @@ int fa_selftest_fwd_stall(const void* q, const void* k, const void* v, void* o, 
     return rc;
 }
 
+int fa_selftest_decode_stall(const void* q, const void* k_pages, const void* v_pages,
+                             const int32_t* page_table, const int32_t* seq_lens, void* o, int B,
+                             int H, int d, int page_size, int withheld, int wait_us,
+                             fa_stream_t stream) {
+    if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !o) return FA_ERR_NULL;
+    if (withheld < 0 || wait_us < 1 || wait_us > 2000000) return FA_ERR_SHAPE;
+    if (B < 1 || H < 1 || static_cast<int64_t>(B) * H * fa::kDecodeMaxSplits > 0x7fffffff)
+        return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (page_size != 256) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
+        return FA_ERR_ALIGN;
+    DeviceState* s = nullptr;
+    int rc = lookup_device(&s);
+    if (rc != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if ((rc = ensure_workspace(s, fa::decode_workspace_bytes(B, H, d, fa::kDecodeMaxSplits), st,
+                               &ws)) != FA_OK)
+        return rc;
+    return fa::launch_decode_stall(q, k_pages, v_pages, page_table, seq_lens, o, B, H, d,
+                                   page_size, ws, s->err, s->num_sms, st,
+                                   static_cast<uint64_t>(wait_us) * 1000u, withheld + 1);
+}
+
 int fa_release_workspace(void) {
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;

@@ -384,7 +384,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                            int page_size, int max_splits, int min_pages,
                            const int32_t* __restrict__ page_off,
                            const int32_t* __restrict__ unit_off, float* __restrict__ part_lse,
-                           float* __restrict__ part_o, float scale_log2, unsigned int* err) {
+                           float* __restrict__ part_o, float scale_log2, unsigned int* err,
+                           uint64_t wait_ns, int withhold) {
+    // wait_ns, withhold: the failure-detection check only (0 in every other
+    // call): the bound of every wait (0: FA_WAIT_TIMEOUT_NS), and 1 + the ring
+    // use at which the producer stops issuing copies (0: none)
     using Sm = DecSmem<D>;
     constexpr int LPT = Sm::LPT, G = Sm::G;
     constexpr int kDecStages = Sm::STAGES;
@@ -395,6 +399,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                     ~static_cast<uintptr_t>(127));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &sm.abort;
+    const uint64_t wlim = wait_ns ? wait_ns : FA_WAIT_TIMEOUT_NS;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecStages; ++i) {
             mbar_init(&sm.full[i], 1);
@@ -429,9 +434,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     }
                 }
                 const int slot = g % kDecStages;
+                if (g + 1 == withhold) {  // failure-detection check: no more copies
+                    ok = false;
+                    break;
+                }
                 if (lane == 0) {
                     if (!mbar_wait(&sm.empty[slot], ((g / kDecStages) & 1) ^ 1, err,
-                                   FA_DEVERR_TIMEOUT, abort)) {
+                                   FA_DEVERR_TIMEOUT, abort, wlim)) {
                         ok = false;
                     } else {
                         const int64_t row = (static_cast<int64_t>(page) * H + us.h) * page_size +
@@ -449,7 +458,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (lane == 0)
             for (int i = max(0, g - kDecStages); i < g; ++i)
                 mbar_wait(&sm.full[i % kDecStages], (i / kDecStages) & 1, err, FA_DEVERR_TIMEOUT,
-                          nullptr);
+                          nullptr, wlim);
         __syncwarp();
     } else {
         // ================= consumers =================
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             for (int c = 0; c < nchunks; ++c, ++g) {
                 const int slot = g % kDecStages;
                 if (!mbar_wait(&sm.full[slot], (g / kDecStages) & 1, err, FA_DEVERR_TIMEOUT,
-                               abort)) {
+                               abort, wlim)) {
                     ok = false;
                     break;
                 }
@@ -535,7 +544,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) sm.co[par][grp][gl * 8 + i] = acc[i];
             mbar_arrive(&sm.cmb[par]);
-            if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort)) {
+            if (!mbar_wait(&sm.cmb[par], (k >> 1) & 1, err, FA_DEVERR_TIMEOUT, abort, wlim)) {
                 ok = false;
                 break;
             }
@@ -1313,7 +1322,8 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
                        const int32_t* seq_lens, void* o, int B, int H, int num_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
-                       int num_sms, cudaStream_t stream) {
+                       int num_sms, cudaStream_t stream, uint64_t wait_ns = 0,
+                       int withhold = 0) {
     const int rows = 1;  // query heads per unit
     const int Hk = H;    // units per split
     // pages a split covers at least: with few units per split (few K/V heads),
@@ -1347,7 +1357,7 @@ int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
             static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pages),
             static_cast<const __nv_bfloat16*>(v_pages), page_table, seq_lens, B, H, num_pages,
             page_size, max_splits, min_pages, page_off, unit_off, part_lse, part_o, scale_log2,
-            err);
+            err, wait_ns, withhold);
     }
     const int warps = B * H;
     fa_decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(
@@ -1551,6 +1561,21 @@ size_t decode_gqa_workspace_bytes(int B, int H, int Hk, int d, int max_splits, i
     const GroupShape gs = group_shape(H, Hk);
     const int rows = gs.gr * gs.teams;
     return gqa_workspace_bytes(B, H / rows, rows, d, max_splits, num_sms);
+}
+
+int launch_decode_stall(const void* q, const void* k_pages, const void* v_pages,
+                        const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                        int d, int page_size, void* workspace, unsigned int* err, int num_sms,
+                        cudaStream_t stream, uint64_t wait_ns, int withhold) {
+    if (d == 128)
+        return launch_decode_impl<128>(q, k_pages, v_pages, nullptr, nullptr, page_table,
+                                       seq_lens, o, B, H, 0x7fffffff, page_size, kDecodeMaxSplits,
+                                       workspace, err, num_sms, stream, wait_ns, withhold);
+    if (d == 64)
+        return launch_decode_impl<64>(q, k_pages, v_pages, nullptr, nullptr, page_table, seq_lens,
+                                      o, B, H, 0x7fffffff, page_size, kDecodeMaxSplits, workspace,
+                                      err, num_sms, stream, wait_ns, withhold);
+    return FA_ERR_UNSUPPORTED;
 }
 
 int launch_decode(const void* q, const void* k_pages, const void* v_pages,

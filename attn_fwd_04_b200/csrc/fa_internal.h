@@ -103,6 +103,13 @@ int launch_decode(const void* q, const void* k_pages, const void* v_pages,
                   int page_size, int max_splits, void* workspace, size_t workspace_bytes,
                   unsigned int* err, int num_sms, cudaStream_t stream);
 bool decode_group_supported(int H, int Hk);
+// The multi-head decode with the failure-detection check's settings: every
+// wait bounded by wait_ns, and the producer stops issuing copies at ring use
+// withhold - 1 (workspace: decode_workspace_bytes(B, H, d, kDecodeMaxSplits)).
+int launch_decode_stall(const void* q, const void* k_pages, const void* v_pages,
+                        const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                        int d, int page_size, void* workspace, unsigned int* err, int num_sms,
+                        cudaStream_t stream, uint64_t wait_ns, int withhold);
 
 // Block table [B, max_pages] -> packed table `packed` (at most B * max_pages
 // entries) and lengths `lens` [B] cut to each row, for launch_decode.

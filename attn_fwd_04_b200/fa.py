@@ -31,6 +31,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_rope", "fa_bwd", "fa_bwd_gqa", "fa_bw
            "fa_decode_paged_noalloc", "fa_append_paged", "fa_prefill_paged",
            "fa_gather_paged",
            "fa_get_device_error", "fa_selftest_bounded_wait", "fa_selftest_fwd_stall",
+           "fa_selftest_decode_stall",
            "fa_release_workspace", "fa_status_str", "fa_version", "fa_fwd_set_cta_pairs")
 
 _lib = None
@@ -69,6 +70,7 @@ def lib() -> ctypes.CDLL:
         L.fa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
         L.fa_selftest_bounded_wait.argtypes = [P]
         L.fa_selftest_fwd_stall.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
+        L.fa_selftest_decode_stall.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.fa_release_workspace.argtypes = []
         L.fa_status_str.argtypes = [I]
         L.fa_status_str.restype = ctypes.c_char_p
@@ -81,6 +83,7 @@ def lib() -> ctypes.CDLL:
                      "fa_append_paged",
                      "fa_prefill_paged", "fa_gather_paged",
                      "fa_get_device_error", "fa_selftest_bounded_wait", "fa_selftest_fwd_stall",
+                     "fa_selftest_decode_stall",
                      "fa_release_workspace", "fa_version", "fa_fwd_set_cta_pairs"):
             getattr(L, name).restype = I
         _lib = L
@@ -591,6 +594,32 @@ def fa_selftest_fwd_stall(q, k, v, withheld: int, wait_us: int, o=None, lse=None
                                      _stream(stream))
     _raise_if(rc, "fa_selftest_fwd_stall")
     return o, lse
+
+
+def fa_selftest_decode_stall(q, k_pages, v_pages, page_table, seq_lens, withheld: int,
+                             wait_us: int, page_size: int = 256, o=None, stream=None):
+    """Launch the paged decode with no copy issued from ring use `withheld` on
+    and every wait bounded by wait_us; read the outcome with
+    fa_get_device_error."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 1)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, H, d = q.shape
+    _pages(k_pages, v_pages, page_size, d, heads=H)
+    if seq_lens.numel() != B:
+        raise ValueError(f"seq_lens must hold one length per sequence ({B})")
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, page_table=page_table,
+                 seq_lens=seq_lens)
+    o = torch.empty_like(q) if o is None else o
+    _expect(o, "o", torch.bfloat16, q.shape, q.device)
+    rc = lib().fa_selftest_decode_stall(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                        page_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
+                                        B, H, d, int(page_size), int(withheld), int(wait_us),
+                                        _stream(stream))
+    _raise_if(rc, "fa_selftest_decode_stall")
+    return o
 
 
 def fa_release_workspace() -> None:

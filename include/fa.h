@@ -454,6 +454,22 @@ FA_API int fa_selftest_bounded_wait(fa_stream_t stream);
 FA_API int fa_selftest_fwd_stall(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int H, int N, int d, int withheld, int wait_us, fa_stream_t stream);
 
+/*
+ * fa_selftest_decode_stall -- the failure-detection path of the paged decode
+ * kernel: fa_decode_paged (same arguments and layouts; page indices are not
+ * bounded, as there) with the producer issuing no copy from ring use
+ * `withheld` on (ring use u: the K and V slices of the u-th 64-token chunk a
+ * CTA streams), and every wait bounded by `wait_us` microseconds (1 ..
+ * 2,000,000).  In each CTA with that many chunks the consumers' wait runs
+ * out, records FA_ERR_DEVICE_TIMEOUT and sets the CTA's abort flag; the other
+ * warps leave their loops, the copies already started land and the CTA
+ * returns (no trap, no fault).  o is then unspecified.  Returns the status of
+ * the launch; read the device error with fa_get_device_error.
+ */
+FA_API int fa_selftest_decode_stall(const void* q, const void* k_pages, const void* v_pages,
+           const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H, int d,
+           int page_size, int withheld, int wait_us, fa_stream_t stream);
+
 /* Free the library workspaces of every stream on the current GPU
  * (synchronises the device first).  Returns FA_OK or FA_ERR_CUDA. */
 FA_API int fa_release_workspace(void);

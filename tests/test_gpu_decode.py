@@ -172,6 +172,27 @@ def test_paged_gather_workload_sampled_bit_exact():
                            torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16))
 
 
+@pytest.mark.parametrize("withheld", [0, 5, 20])
+def test_decode_kernel_stall_is_reported_and_recovered(withheld):
+    """Failure detection inside the production decode kernel: from one ring
+    use on (the first chunk, the sixth, the 21st: the longest units here hold
+    24 chunks of 64 tokens) the producer issues no copy
+    and every wait is bounded by 50 ms.  The stall comes back as
+    FA_ERR_DEVICE_TIMEOUT (no trap, no fault), and a normal decode on the same
+    stream right after it computes correctly."""
+    lens = [1000, 4103, 9000, 257]
+    c = _on_gpu(W.paged_inputs(len(lens), 4, 128, lens, seed=23, device="cpu"))
+    assert fa.fa_get_device_error() == fa.FA_OK
+    fa.fa_selftest_decode_stall(c.q, c.k_pages, c.v_pages, c.page_table, c.seq_lens, withheld,
+                                50_000)
+    assert fa.fa_get_device_error() == fa.FA_ERR_DEVICE_TIMEOUT
+    assert fa.fa_get_device_error() == fa.FA_OK
+    o = _decode(c)
+    o_ref, _ = oracle.decode_paged(c.q.cpu(), c.k_pages.cpu(), c.v_pages.cpu(),
+                                   c.page_table.cpu(), c.seq_lens.cpu(), PS)
+    assert_o_close(to64(o), o_ref, "decode after a stalled decode")
+
+
 # -- grouped K/V heads (fa_decode_paged_gqa) ---------------------------------------
 
 def _decode_gqa(c: W.PagedCache):
