@@ -568,39 +568,41 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 
 // ---------------------------------------------------------------------------
-// Grouped query heads (groups of 2 or more; see below for the sizes).  A
-// unit is (split, K/V head); the GH query heads of its group are the rows of
-// a 16-row MMA tile (rows GH..15 are zero), so each staged K/V byte serves
-// all of them and the dot products run as two small matrix products per
-// chunk on the tensor cores (warp-level m16n8k16: a tcgen05 tile has at least
-// 64 rows, 8x-32x more than the group has).  K/V chunks of 64 tokens arrive
-// by TMA in the 128-byte-swizzled layout, so the ldmatrix reads of 8 token
-// rows at one column fall in 8 distinct bank groups.  A warp takes WT
-// consecutive tokens of a chunk (16 or 32, the template), so 64 / WT warps
-// cover a chunk for one set of rows:
+// Grouped query heads (groups of 2 or more; see below for the sizes).  The
+// GH query heads of a unit are the rows of a 16-row MMA tile (rows GH..15 are
+// zero), so each staged K/V byte serves all of them and the dot products run
+// as small matrix products on the tensor cores (warp-level m16n8k16; a
+// tcgen05 form, S^T = K Q^T with the chunk as M, measured slower: with 32
+// heads as N its operand reads outrun shared memory).  K/V chunks of 64
+// tokens arrive by TMA in the 128-byte-swizzled layout, so the ldmatrix reads
+// of 8 token rows at one column fall in 8 distinct bank groups.  A warp takes
+// WT consecutive tokens of a chunk, so 64 / WT warps cover a chunk for one
+// set of rows:
 //   S  = Q_g K^T   WT/8 8-token n-tiles over D/16 k-steps (fp32)
 //   online softmax per query row (rows lane / 4 and, for groups of 16,
 //   lane / 4 + 8; the 4 lanes of a quad share them), base 2 with
 //   scale * log2(e) applied to S
 //   O += P V       P from S's accumulators as the A operand, V through
 //                  ldmatrix.trans, D/8 n-tiles over WT/16 k-steps
-// and the 8 warps' (m, l, O) are merged per unit through one shared buffer
-// (a second barrier tells the writers of the next unit that every reader of
-// this one is done), which leaves room for more ring stages.  With 32 tokens
-// per warp the row bookkeeping of the softmax (max shuffles, the rescale of
-// the D/4 accumulators of a row pair) is paid once per 32 tokens, not 16.
-// A unit holds gr <= GH query heads (GH, the template, is the capacity of
-// its registers and merge buffer).  Groups larger than 16 (multi-query
-// attention with many heads) are cut into equal sub-groups of gr <= 16 query
-// heads.  With teams == 2 a unit holds two sub-groups of the same K/V head:
-// warps 0-3 take the first sub-group's rows and warps 4-7 the second's, each
-// half covering every chunk, so a staged K/V chunk serves 2 gr query heads
-// and is read from memory once for both (an even number of sub-groups is
-// paired this way).  Otherwise (teams == 1) each sub-group is a unit of its
-// own.  The warps covering one chunk for one set of rows form a crew, and the
-// crews of a set of rows take the chunks in turn.  Hk counts the units per
-// split (H / (teams gr)) and sub the units per K/V head: the unit's K/V head
-// is h / sub.
+// The warps covering one chunk for one set of rows form a crew, and two
+// crews per set of rows take the chunks in turn.
+// Groups larger than 16 (multi-query attention with many heads) are cut into
+// equal sub-groups of gr <= 16 query heads (GH, the template, is the capacity
+// of the registers and merge slots).  An even number of sub-groups is paired:
+// a unit then holds two sub-groups of the same K/V head (warps 0-3 the first
+// one's rows, warps 4-7 the second's, each half covering every chunk), so a
+// staged chunk serves 2 gr query heads and is read from memory once for both,
+// and a warp takes 32 tokens (its softmax row bookkeeping -- max shuffles,
+// the rescale of the D/4 accumulators of a row pair -- is paid once per 32
+// tokens, not 16).  Otherwise a unit holds one sub-group and a warp 16
+// tokens.  Hk counts the unit heads per sequence (H / rows) and sub the unit
+// heads per K/V head: a unit head h reads K/V head h / sub.
+// At the end of a unit the 8 warps' (m, l, O) are merged in two rounds
+// through 4 slots (crew 1 into crew 0, then the slots of each set of rows),
+// which leaves room for 6 ring stages.  The producer warp walks the units --
+// split units taken in turn, or the pieces of the evenly split chunk stream
+// for one or two unit heads (see launch_decode_gqa) -- and hands each one's
+// shape to the consumers.
 // ---------------------------------------------------------------------------
 constexpr int kGqTok = 64;          // tokens per chunk
 constexpr int kGqWarps = 8;         // consumer warps
