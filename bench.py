@@ -542,11 +542,12 @@ def decode_cache(batch: int, h_kv: int) -> W.PagedCache:
 
 
 def run_single_path(args, local):
-    """Profiling aid (--only prefill / rope / bwd / batched / varlen): the
-    paged-prefill workload, the RoPE forward pass or the backward pass on the
-    long-prefill workload, or the forward pass on the batched or the
-    variable-length prefill workload, alone, timed with CUDA events; prints
-    its own short JSON line."""
+    """Profiling aid (--only prefill / rope / bwd / batched / varlen /
+    bwd_varlen): the paged-prefill workload, the RoPE forward pass or the
+    backward pass on the long-prefill workload, the forward pass on the
+    batched or the variable-length prefill workload, or the backward pass on
+    the latter, alone, timed with CUDA events; prints its own short JSON
+    line."""
     import attn_fwd_04_b200 as fa
     torch.cuda.set_device(local)
     stream = torch.cuda.current_stream()
@@ -586,6 +587,22 @@ def run_single_path(args, local):
         def fn():
             fa.fa_fwd_varlen(q, k, v, cud, max(lens), w.causal, 1 / math.sqrt(w.d), o=o, lse=lse,
                              stream=stream)
+    elif args.only == "bwd_varlen":
+        w = W.BATCHED_VARLEN
+        q, k, v, cu = W.varlen_workload_inputs(w, device="cuda")
+        lens = (cu[1:] - cu[:-1]).tolist()
+        cud = cu.cuda()
+        o, lse = fa.fa_fwd_varlen(q, k, v, cud, max(lens), w.causal, 1 / math.sqrt(w.d),
+                                  stream=stream)
+        g = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(8),
+                        device="cuda").to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        flops = 2.5 * sum(4.0 * w.H * L * L * w.d / (2 if w.causal else 1) for L in lens)
+        name = f"bwd_{w.name}"
+
+        def fn():
+            fa.fa_bwd_varlen(q, k, v, o, lse, g, cud, max(lens), w.causal, 1 / math.sqrt(w.d),
+                             dq=dq, dk=dk, dv=dv, stream=stream)
     elif args.only == "prefill":
         w = W.PAGED_PREFILL
         cache, q, cu = W.prefill_workload_inputs(w, device="cuda")
@@ -934,7 +951,7 @@ def main(argv=None):
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the forward pass on the other workloads")
     ap.add_argument("--only", choices=["all", "fwd", "decode", "prefill", "rope", "bwd", "batched",
-                                       "varlen"],
+                                       "varlen", "bwd_varlen"],
                     default="all",
                     help="profiling aid: run one entry point only (the JSON line then "
                          "reports that part alone)")
@@ -953,7 +970,7 @@ def main(argv=None):
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    if args.only in ("prefill", "rope", "bwd", "batched", "varlen"):
+    if args.only in ("prefill", "rope", "bwd", "batched", "varlen", "bwd_varlen"):
         print(json.dumps(run_single_path(args, int(os.environ.get("LOCAL_RANK", "0")))),
               flush=True)
         return
