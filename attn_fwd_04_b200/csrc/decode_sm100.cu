@@ -1321,8 +1321,8 @@ __global__ void __launch_bounds__(256)
 // Multi-head decode (one query head per K/V head): plan, split, merge.
 template <int D>
 int launch_decode_impl(const void* q, const void* k_pages, const void* v_pages,
-                       const CUtensorMap* tk, const CUtensorMap* tv, const int32_t* page_table,
-                       const int32_t* seq_lens, void* o, int B, int H, int num_pages,
+                       const int32_t* page_table, const int32_t* seq_lens, void* o, int B, int H,
+                       int num_pages,
                        int page_size, int max_splits, void* workspace, unsigned int* err,
                        int num_sms, cudaStream_t stream, uint64_t wait_ns = 0,
                        int withhold = 0) {
@@ -1532,7 +1532,7 @@ int launch_decode_d(const void* q, const void* k_pages, const void* v_pages,
                     int page_size, int max_splits, void* workspace, size_t workspace_bytes,
                     unsigned int* err, int num_sms, cudaStream_t stream) {
     if (H == Hk)
-        return launch_decode_impl<D>(q, k_pages, v_pages, tk, tv, page_table, seq_lens, o, B, H,
+        return launch_decode_impl<D>(q, k_pages, v_pages, page_table, seq_lens, o, B, H,
                                      num_pages, page_size, max_splits, workspace, err, num_sms,
                                      stream);
     const GroupShape gs = group_shape(H, Hk);
@@ -1570,11 +1570,11 @@ int launch_decode_stall(const void* q, const void* k_pages, const void* v_pages,
                         int d, int page_size, void* workspace, unsigned int* err, int num_sms,
                         cudaStream_t stream, uint64_t wait_ns, int withhold) {
     if (d == 128)
-        return launch_decode_impl<128>(q, k_pages, v_pages, nullptr, nullptr, page_table,
+        return launch_decode_impl<128>(q, k_pages, v_pages, page_table,
                                        seq_lens, o, B, H, 0x7fffffff, page_size, kDecodeMaxSplits,
                                        workspace, err, num_sms, stream, wait_ns, withhold);
     if (d == 64)
-        return launch_decode_impl<64>(q, k_pages, v_pages, nullptr, nullptr, page_table, seq_lens,
+        return launch_decode_impl<64>(q, k_pages, v_pages, page_table, seq_lens,
                                       o, B, H, 0x7fffffff, page_size, kDecodeMaxSplits, workspace,
                                       err, num_sms, stream, wait_ns, withhold);
     return FA_ERR_UNSUPPORTED;
